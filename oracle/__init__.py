@@ -308,17 +308,20 @@ def fixed_block_bounds(n: int, block_size: int):
 
 def decode_fixed_segment(q_grp, K_seg, V_seg, n_sel: int, n_now: int, kind: int,
                          block_size: int, topk: int, budget_tokens: int, sink: int,
-                         window: int, keep_current: bool, scale: float):
+                         window: int, keep_current: bool, scale: float, q_sel=None):
     """One (batch, KV head) segment of a decode step over fixed-size blocks.
 
-    Selection happens for a cache of n_sel tokens (the last refresh); between
-    refreshes the window keeps growing, so attention reads the selected
+    Selection happens at the last refresh, for a cache of n_sel tokens and
+    with that step's queries q_sel (default: q_grp, a refresh now); the pages
+    it picked stay selected until the next refresh while the window keeps
+    growing, so attention of the current queries q_grp reads the selected
     ranges with the last one extended to the n_now tokens present now
-    ("Sparse attention in hybrid LLMs": selection is refreshed every 32
-    steps and the window is extended in between)."""
+    ("Sparse attention in hybrid LLMs", "Which parts of the context each
+    layer reads": selection is refreshed every 32 steps and the window is
+    extended in between)."""
     beg, end = fixed_block_bounds(n_sel, block_size)
     summ = block_summaries(K_seg, beg, end, kind)
-    s32, s64 = block_scores(q_grp, summ, kind)
+    s32, s64 = block_scores(q_grp if q_sel is None else q_sel, summ, kind)
     sel, ranges, ties = select_fixed(s32, s64, n_sel, block_size, topk, budget_tokens,
                                      sink, window, keep_current)
     if ranges and n_now > ranges[-1][1]:

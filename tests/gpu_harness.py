@@ -1,0 +1,126 @@
+"""Shared driver for the GPU parity tests: runs a decode workload through the
+C ABI and through the CPU oracle on the same seeded inputs and compares.
+
+Bars (from the method's statement): selected block ids and token ranges
+bit-exact; outputs and log-sum-exp within max-abs 2e-3 of the fp64 oracle.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle
+from block_sparse_long_build_b200 import native as N
+from block_sparse_long_build_b200.session import DecodeSession
+from block_sparse_long_build_b200.workloads import Workload
+
+ATOL = 2e-3
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    """Device tensor -> numpy: bf16 as uint16 bit patterns, fp32 as float32."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def gpu_summaries(sess: DecodeSession, s: int, nb: int):
+    c = sess.cfg
+    raw = sess.summaries.cpu().numpy()
+    if sess.kind == N.BSA_SUM_MINMAX:
+        esz = 2 if c.kv_dtype == torch.bfloat16 else 4
+        row = 2 * c.D * esz
+        seg = raw[s * sess.nb * row:(s * sess.nb + nb) * row]
+        if esz == 2:
+            x = oracle.bf16_bits_to_f32(seg.view(np.uint16)).reshape(nb, 2, c.D)
+        else:
+            x = seg.view(np.float32).reshape(nb, 2, c.D)
+        return x[:, 0], x[:, 1]
+    row = c.D * 4
+    return raw[s * sess.nb * row:(s * sess.nb + nb) * row].view(np.float32).reshape(nb, c.D)
+
+
+class FixedDecodeCheck:
+    """Runs fixed-block decode steps on both sides and compares."""
+
+    def __init__(self, cfg, device="cuda"):
+        self.cfg = cfg
+        self.wl = Workload(cfg, device)
+        self.sess = DecodeSession(self.wl)
+        self.K = host(self.wl.K)     # the oracle's own copy of the cache
+        self.V = host(self.wl.V)
+        self.n = [int(x) for x in self.wl.cur_len.cpu()]
+        self.n_sel = list(self.n)
+        self.q_sel = None       # queries of the last refresh step
+
+    def run(self, steps: int, check_summaries=True):
+        c, sess = self.cfg, self.sess
+        sess.build_summaries()
+        torch.cuda.synchronize()
+        worst = 0.0
+        for t in range(steps):
+            q = self.wl.decode_query(t)
+            if t > 0 or c.name != "tiny":
+                k, v = self.wl.decode_new_kv(t)
+                kh, vh = host(k), host(v)
+                for b in range(c.B):
+                    if self.n[b] < c.L_max:
+                        self.K[b, :, self.n[b]] = kh[b]
+                        self.V[b, :, self.n[b]] = vh[b]
+                        self.n[b] += 1
+            else:
+                k = v = None
+            sess.step(t, q, k, v)
+            torch.cuda.synchronize()
+            refresh = t % c.refresh == 0
+            if refresh:
+                self.n_sel = list(self.n)
+                self.q_sel = host(q)
+            worst = max(worst, self.compare(q, refresh, check_summaries and refresh))
+        return worst
+
+    def compare(self, q, check_sel: bool, check_summaries: bool) -> float:
+        c, sess = self.cfg, self.sess
+        qh = host(q)
+        out, lse = host(sess.out), host(sess.lse)
+        assert np.all(host(self.wl.cur_len) == np.array(self.n))
+        sel_blocks, sel_count = host(sess.sel_blocks), host(sess.sel_count)
+        ranges, n_ranges = host(sess.ranges), host(sess.n_ranges)
+        worst = 0.0
+        for b in range(c.B):
+            for g in range(c.Hkv):
+                s = b * c.Hkv + g
+                qg = qh[b, g * c.G:(g + 1) * c.G]
+                qs = self.q_sel[b, g * c.G:(g + 1) * c.G] if self.q_sel is not None else qg
+                ref = oracle.decode_fixed_segment(
+                    qg, self.K[b, g], self.V[b, g], self.n_sel[b], self.n[b], c.kind,
+                    c.block_size, c.topk, c.budget_tokens, c.sink, c.window, c.keep_current,
+                    1.0 / math.sqrt(c.D), q_sel=qs)
+                if check_summaries:
+                    nb = self.n_sel[b] // c.block_size
+                    beg, end = oracle.fixed_block_bounds(self.n_sel[b], c.block_size)
+                    want = oracle.block_summaries(self.K[b, g], beg, end, c.kind)
+                    got = gpu_summaries(sess, s, nb)
+                    if c.kind == N.BSA_SUM_MINMAX:
+                        assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1]), \
+                            f"minmax summaries differ (segment {s})"
+                    else:
+                        assert np.array_equal(got, want), f"centroid summaries differ (segment {s})"
+                if check_sel:
+                    gs = sel_blocks[s, :sel_count[s]].tolist()
+                    assert gs == ref["sel"], (
+                        f"segment {s}: selection differs; near-ties {ref['ties']}")
+                    sel_r, sel_rr, _ = oracle.select_fixed(
+                        ref["s32"], ref["s64"], self.n_sel[b], c.block_size, c.topk,
+                        c.budget_tokens, c.sink, c.window, c.keep_current)
+                    gr = [tuple(x) for x in ranges[s, :n_ranges[s]].tolist()]
+                    assert gr == sel_rr, f"segment {s}: ranges differ"
+                err = np.abs(out[b, g * c.G:(g + 1) * c.G] - ref["out"]).max()
+                lerr = np.abs(lse[b, g * c.G:(g + 1) * c.G] - ref["lse"]).max()
+                worst = max(worst, float(err), float(lerr))
+                assert err <= ATOL, f"segment {s}: max |out - oracle| = {err:.3e}"
+                assert lerr <= ATOL, f"segment {s}: max |lse - oracle| = {lerr:.3e}"
+        return worst

@@ -1,0 +1,119 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, sizes buffers, and rejects bad arguments on the host before
+touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_long_build_b200 import build as B
+from block_sparse_long_build_b200 import native as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return N.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(N.EXPORTED) == set(names)
+
+
+def test_version_and_status_strings(lib):
+    assert N.bsa_version() >= 100
+    for s in (0, -1, -2, -3, -4, -5):
+        assert N.status_string(s)
+
+
+def _desc(**kw):
+    d = dict(B=4, Hq=32, Hkv=8, D=128, kv_dtype=N.BSA_BF16, L_max=65664, stride_b=8 * 65664 * 128,
+             stride_h=65664 * 128, stride_t=128)
+    d.update(kw)
+    return N.KvDesc(**d)
+
+
+def test_sizes(lib):
+    d = _desc()
+    p = N.sel_params(16, topk=-1, budget_tokens=4096, sink=256, window=1024)
+    assert N.bsa_summary_blocks(d, p) == 65664 // 16
+    assert N.bsa_summary_bytes(d, p, N.BSA_SUM_MINMAX) == 32 * (65664 // 16) * 2 * 128 * 2
+    assert N.bsa_summary_bytes(d, p, N.BSA_SUM_CENTROID) == 32 * (65664 // 16) * 128 * 4
+    assert N.bsa_max_selected(d, p) == 256
+    assert N.bsa_max_ranges(d, p) >= 256 + 3
+    assert N.bsa_workspace_size(d, p, N.BSA_OP_SELECT) > 0
+    assert N.bsa_workspace_size(d, p, N.BSA_OP_DECODE, 0, 5500) > 0
+
+
+@pytest.mark.parametrize("bad", [dict(D=96), dict(Hq=12), dict(kv_dtype=7), dict(L_max=0),
+                                 dict(stride_t=100), dict(B=0)])
+def test_bad_descriptor_rejected_on_host(lib, bad):
+    d = _desc(**bad)
+    p = N.sel_params(16, topk=8)
+    fake = 1 << 20   # never dereferenced: validation fails first
+    L = N.lib()
+    st = L.bsa_decode(ctypes.byref(d), fake, fake, fake, fake, fake, 16, fake, 100, 0.1, fake,
+                      None, fake, 1 << 30, None)
+    assert st == N.BSA_ERR_ARG
+    st = L.bsa_build_summaries(ctypes.byref(d), fake, ctypes.byref(p), 0, 0, 1, fake, None)
+    assert st == N.BSA_ERR_ARG
+
+
+def test_bad_arguments_rejected_on_host(lib):
+    L = N.lib()
+    d = _desc()
+    p = N.sel_params(16, topk=8, sink=4, window=16)
+    fake = 1 << 20
+    # null output
+    assert L.bsa_decode(ctypes.byref(d), fake, fake, fake, fake, fake, 16, fake, 100, 0.1, None,
+                        None, fake, 1 << 30, None) == N.BSA_ERR_ARG
+    # misaligned K
+    assert L.bsa_decode(ctypes.byref(d), fake, fake + 2, fake, fake, fake, 16, fake, 100, 0.1,
+                        fake, None, fake, 1 << 30, None) == N.BSA_ERR_ARG
+    # non-positive scale
+    assert L.bsa_decode(ctypes.byref(d), fake, fake, fake, fake, fake, 16, fake, 100, 0.0, fake,
+                        None, fake, 1 << 30, None) == N.BSA_ERR_ARG
+    # workspace too small
+    assert L.bsa_decode(ctypes.byref(d), fake, fake, fake, fake, fake, 16, fake, 100, 0.1, fake,
+                        None, fake, 16, None) == N.BSA_ERR_WORKSPACE
+    # summaries past the end of the cache
+    assert L.bsa_build_summaries(ctypes.byref(d), fake, ctypes.byref(p), 2, 4100, 10, fake,
+                                 None) == N.BSA_ERR_ARG
+    # selection buffers smaller than the bound
+    assert L.bsa_select(ctypes.byref(d), fake, fake, 2, ctypes.byref(p), fake, 4, fake, fake,
+                        64, fake, fake, fake, 1 << 30, None) == N.BSA_ERR_ARG
+    # negative sink
+    p2 = N.sel_params(16, topk=8, sink=-1)
+    assert L.bsa_select(ctypes.byref(d), fake, fake, 2, ctypes.byref(p2), fake, 8, fake, fake,
+                        64, fake, fake, fake, 1 << 30, None) == N.BSA_ERR_ARG
+    # variable blocks without offsets
+    p3 = N.sel_params(0, n_blocks=16, topk=-1, budget_tokens=100)
+    assert L.bsa_summary_blocks(ctypes.byref(d), ctypes.byref(p3)) == -1
+    # grouped prefill outside its domain (fixed blocks)
+    assert L.bsa_prefill_grouped(ctypes.byref(d), fake, fake, ctypes.byref(p), fake,
+                                 ctypes.byref(d), fake, fake, fake, 0, 16, 0.1, fake, None, fake,
+                                 1 << 30, None) in (N.BSA_ERR_ARG, N.BSA_ERR_UNSUPPORTED)
+
+
+def test_product_path_has_no_oracle_import():
+    """The package never imports the oracle (independence of the two sides)."""
+    pkg = os.path.join(ROOT, "block_sparse_long_build_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), f
+                assert "oracle.c" not in src and "_oracle.so" not in src, f

@@ -330,6 +330,17 @@ def test_refresh_extends_window():
     assert set(range(300 - 16, 317)) <= rows and max(rows) == 316
     b = oracle.decode_fixed_segment(q, K, V, 300, 300, oracle.MINMAX, S, 3, 0, 8, 16, False, 0.25)
     assert a["sel"] == b["sel"]
+    # between refreshes the pages are the ones the refresh step's queries
+    # picked, whatever the current queries would pick
+    q2 = -q
+    c = oracle.decode_fixed_segment(q2, K, V, 300, 317, oracle.MINMAX, S, 3, 0, 8, 16, False,
+                                    0.25, q_sel=q)
+    d = oracle.decode_fixed_segment(q2, K, V, 300, 317, oracle.MINMAX, S, 3, 0, 8, 16, False, 0.25)
+    assert c["sel"] == a["sel"] and c["ranges"] == a["ranges"]
+    assert d["sel"] != a["sel"]
+    rows = oracle.ranges_to_rows(c["ranges"])
+    ref, _ = _dense_reference(q2[0], K, V, np.isin(np.arange(400), rows), 0.25)
+    np.testing.assert_allclose(c["out"][0], ref, atol=1e-12)
 
 
 def test_needle_blocks_are_recalled():
