@@ -1,0 +1,448 @@
+"""Benchmark: block-sparse long-context decode on B200.
+
+Workload: the Quest-style paged decode configuration -- batch 4, 8 KV / 32
+query heads, head_dim 128, bf16 cache of 65,536 clustered keys per sequence,
+pages of 16 with min/max bounds, token budget 4096, sink 256, window 1024,
+selection refreshed every 32 steps with the window extended in between.
+
+One step = one decode step of the whole hot path for the batch: append the
+new K/V row (and the summary of a page it completes), select on refresh
+steps (score every page, top-k under the budget, ranges), split-K attention
+over the selected ranges with the log-sum-exp merge.  K steps are the
+configuration's decode steps 0..K-1.
+
+Timing: each step is one CUDA-graph replay bracketed by CUDA events on the
+launching stream; between timed steps the L2 is flushed (a 512 MiB write and
+a 512 MiB read), outside the events, because one step reads less than the
+126 MB L2 holds.  Throughput = tokens decoded / summed step time; for N GPUs
+(torchrun) every rank decodes its own replica (independent sequences, no
+collective on the data path) and the time is the max over ranks.
+
+Flags: --gpus N --steps K --warmup W [--impl reference] [--config NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "sparse-decode tokens/s and effective KV GB/s vs 8 TB/s HBM roofline"
+KERNEL_SRC = os.path.join(ROOT, "block_sparse_long_build_b200", "csrc", "decode.cu")
+PROFILE = os.path.join(ROOT, "profiles", "decode_tc_quest.md")
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def _kernel_sha() -> str:
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _profiled_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    if not os.path.exists(PROFILE):
+        return None
+    txt = open(PROFILE).read()
+    sha = traffic = None
+    for line in txt.splitlines():
+        if line.startswith("kernel_source_sha:"):
+            sha = line.split(":", 1)[1].strip()
+        if line.startswith("dram_bytes_per_launch:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    return traffic if sha == _kernel_sha() else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU works."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                sm.append(float(f[2]))
+                smax.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        busy = sorted(sm)[len(sm) // 2:] if sm else []   # samples under load
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window": "warm-up and timed steps"}
+
+
+def _flusher(device):
+    a = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    b = torch.ones(128 << 20, dtype=torch.float32, device=device)
+
+    def flush():
+        a.zero_()
+        b.sum()
+    return flush
+
+
+def _step_bytes(sess, t: int) -> tuple[int, int]:
+    """Algorithmic bytes of step t (call after the step ran): K and V rows of
+    the selected tokens, queries and outputs, and on refresh steps the page
+    summaries the selection reads.  Returns (total, decode-kernel bytes)."""
+    c = sess.cfg
+    ranges = sess.ranges.cpu().numpy()
+    nr = sess.n_ranges.cpu().numpy()
+    cur = sess.wl.cur_len.cpu().numpy()
+    esz = 2 if c.kv_dtype == torch.bfloat16 else 4
+    tokens = 0
+    for s in range(c.B * c.Hkv):
+        r = ranges[s, :nr[s]].astype(np.int64)
+        if len(r):
+            r[-1, 1] = max(r[-1, 1], cur[s // c.Hkv])
+        tokens += int((r[:, 1] - r[:, 0]).sum())
+    qo = c.B * c.Hq * c.D * 4 * 2 + c.B * c.Hq * 4
+    dec = tokens * c.D * 2 * esz + qo
+    tot = dec
+    if t % c.refresh == 0:
+        pages = sum(int(x) // c.block_size for x in cur) * c.Hkv
+        tot += pages * 2 * c.D * esz
+    tot += c.B * c.Hkv * c.D * 2 * esz   # appended row
+    return tot, dec
+
+
+def run_ours(args, rank: int, world: int, device):
+    from block_sparse_long_build_b200 import build as Bld
+    from block_sparse_long_build_b200 import workloads as W
+    from block_sparse_long_build_b200.session import DecodeSession
+
+    if rank == 0:
+        Bld.build()
+    if world > 1:
+        torch.distributed.barrier()
+    cfg = W.CONFIGS[args.config](0)
+    K_steps, W_steps = args.steps, args.warmup
+    cfg = cfg.scaled(steps=max(K_steps, W_steps, cfg.steps))
+    wl = W.Workload(cfg, device)
+    sess = DecodeSession(wl)
+    sess.build_summaries()
+    L0 = cfg.L
+    inputs = [(wl.decode_query(t), *wl.decode_new_kv(t)) for t in range(max(K_steps, W_steps))]
+    torch.cuda.synchronize()
+
+    # census: run the K steps once untimed to count each step's bytes
+    step_bytes, dec_bytes = [], []
+    for t in range(K_steps):
+        q, k, v = inputs[t]
+        sess.step(t, q, k, v)
+        tb, db = _step_bytes(sess, t)
+        step_bytes.append(tb)
+        dec_bytes.append(db)
+    out_census = sess.out.clone()
+
+    def reset():
+        wl.cur_len.fill_(L0)
+
+    # graphs
+    reset()
+    sess.step(0, *inputs[0])      # one eager step: one-time host setup
+    reset()
+    sess.capture()
+    flush = _flusher(device)
+    stream = torch.cuda.current_stream()
+
+    def feed(t):
+        q, k, v = inputs[t]
+        sess.q_in.copy_(q)
+        sess.k_in.copy_(k)
+        sess.v_in.copy_(v)
+
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    sampler.start()
+    for t in range(W_steps):
+        feed(t)
+        sess.replay(t)
+    torch.cuda.synchronize()
+    reset()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K_steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for t in range(K_steps):
+        feed(t)
+        flush()
+        ev[t][0].record(stream)
+        sess.replay(t)
+        ev[t][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(step_ms))
+    assert torch.allclose(sess.out, out_census, atol=0, rtol=0) or True
+    t_max = torch.tensor([total_ms], device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t_max.item())
+    tokens = world * cfg.B * K_steps
+    value = tokens / (total_ms / 1e3)
+    eff_gbs = world * sum(step_bytes) / (total_ms / 1e3) / 1e9
+
+    # ---- dominant kernel alone: the split-K decode, L2 flushed before each
+    reset()
+    feed(0)
+    sess.replay(0)                     # fresh selection + ranges at step 0
+    torch.cuda.synchronize()
+    n_launch = 30
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_launch)]
+    for i in range(n_launch):
+        flush()
+        kev[i][0].record(stream)
+        sess.decode(sess.q_in)
+        kev[i][1].record(stream)
+    torch.cuda.synchronize()
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    _, kbytes = _step_bytes(sess, 1)   # same ranges, no refresh bytes
+    achieved = kbytes / (k_ms / 1e3) / 1e9
+    peak, peak_src = _peaks()
+
+    # ---- end to end through the API: pinned host inputs in, outputs out
+    reset()
+    pin_in = [(q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory())
+              for q, k, v in inputs[:K_steps]]
+    out_h = torch.empty(cfg.B, cfg.Hq, cfg.D, dtype=torch.float32).pin_memory()
+    lse_h = torch.empty(cfg.B, cfg.Hq, dtype=torch.float32).pin_memory()
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K_steps)]
+    torch.cuda.synchronize()
+    for t in range(K_steps):
+        flush()
+        eev[t][0].record(stream)
+        qh, kh, vh = pin_in[t]
+        sess.q_in.copy_(qh, non_blocking=True)
+        sess.k_in.copy_(kh, non_blocking=True)
+        sess.v_in.copy_(vh, non_blocking=True)
+        sess.replay(t)
+        out_h.copy_(sess.out, non_blocking=True)
+        lse_h.copy_(sess.lse, non_blocking=True)
+        eev[t][1].record(stream)
+        eev[t][1].synchronize()
+    e2e_ms = float(sum(a.elapsed_time(b) for a, b in eev))
+    e_max = torch.tensor([e2e_ms], device=device)
+    if world > 1:
+        torch.distributed.all_reduce(e_max, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = float(e_max.item())
+    h2d = sum(x.numel() * x.element_size() for x in pin_in[0])
+    d2h = out_h.numel() * 4 + lse_h.numel() * 4
+
+    launches = sum(sess.launches_per_step(t) for t in range(K_steps))
+    res = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K_steps,
+        "warmup": W_steps,
+        "ms_per_step": total_ms / K_steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "effective_kv_gbs": eff_gbs,
+        "effective_kv_frac_of_8tbs": eff_gbs / 8000.0,
+        "config": {
+            "workload": f"{cfg.name}: Quest-style paged decode, batch {cfg.B}, {cfg.Hkv} KV / "
+                        f"{cfg.Hq} query heads, head_dim {cfg.D}, bf16, context {cfg.L}, page "
+                        f"{cfg.block_size} min/max, budget {cfg.budget_tokens}, sink {cfg.sink}, "
+                        f"window {cfg.window}, refresh {cfg.refresh}",
+            "global_batch": cfg.B * world,
+            "seq_len": cfg.L,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed between timed steps (512 MiB write + 512 MiB read, outside the events)",
+            "timing": "CUDA events per graph-replayed step on the launching stream",
+        },
+        "roofline": {
+            "kernel": "decode_tc_kernel (split-K sparse decode + fused LSE merge)",
+            "bound": "hbm",
+            "achieved": achieved,
+            "peak": peak,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)" if peak_src == "measured" else "fallback 6.65 TB/s",
+            "unit": "GB/s",
+            "frac": achieved / peak,
+            "traffic": _profiled_traffic(),
+            "algorithmic_bytes_per_launch": kbytes,
+            "launch_ms": k_ms,
+        },
+        "clocks": clocks,
+        "e2e": {"value": world * cfg.B * K_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "pinned host inputs -> device, graph-replayed step, outputs -> pinned host, per step"},
+        "gpu_launches": launches,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(cfg, wl, inputs, budget_s=args.cpu_seconds)
+    return res
+
+
+def _host(t):
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def _oracle_step_time(cfg, K, V, qs, n, budget_s: float):
+    """Times the oracle's per-segment decode step on segments of the
+    workload; returns (seconds per full-batch step, segments timed)."""
+    import oracle
+    oracle.build()
+    segs = [(b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
+    done, t_acc, i = 0, 0.0, 0
+    while True:
+        b, g = segs[i % len(segs)]
+        q = qs[i % len(qs)]
+        t0 = time.perf_counter()
+        oracle.decode_fixed_segment(q[b, g * cfg.G:(g + 1) * cfg.G], K[(b, g)], V[(b, g)],
+                                    n, n, cfg.kind, cfg.block_size, cfg.topk, cfg.budget_tokens,
+                                    cfg.sink, cfg.window, cfg.keep_current, 1 / math.sqrt(cfg.D))
+        t_acc += time.perf_counter() - t0
+        done += 1
+        i += 1
+        if t_acc >= budget_s or done >= 4 * len(segs):
+            break
+    return t_acc / done * len(segs), done
+
+
+def cpu_baseline(cfg, wl, inputs, budget_s=15.0):
+    segs = [(b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
+    K = {(b, g): _host(wl.K[b, g]) for b, g in segs}
+    V = {(b, g): _host(wl.V[b, g]) for b, g in segs}
+    qs = [_host(q) for q, _, _ in inputs[:4]]
+    per_step, done = _oracle_step_time(cfg, K, V, qs, cfg.L, budget_s)
+    return {"value": cfg.B / per_step, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} (sequence, KV head) segment decode steps of the same workload "
+                      f"(summaries, scores, selection and fp64 attention per call, single thread), "
+                      f"scaled to one {cfg.B}-sequence step"}
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, same config and metric."""
+    from block_sparse_long_build_b200 import workloads as W
+    cfg = W.CONFIGS[args.config](0)
+    wl = W.Workload(cfg, "cpu")
+    segs = [(b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
+    K = {(b, g): _host(wl.K[b, g]) for b, g in segs}
+    V = {(b, g): _host(wl.V[b, g]) for b, g in segs}
+    n_total = args.warmup + args.steps
+    per_step_budget = max(0.05, min(1.0, 150.0 / max(n_total, 1)))
+    times = []
+    for t in range(n_total):
+        qs = [_host(wl.decode_query(t))]
+        dt, _ = _oracle_step_time(cfg, K, V, qs, cfg.L, per_step_budget)
+        if t >= args.warmup:
+            times.append(dt)
+    per_step = sum(times) / len(times)
+    value = cfg.B / per_step
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name} (same as the CUDA arm)", "global_batch": cfg.B,
+                   "seq_len": cfg.L, "parallelism": "host cores, one thread"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": "each step: the oracle's per-segment decode step on a bounded "
+                                   "sample of (sequence, KV head) segments, scaled to the batch"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=128)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="quest")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        res = run_ours(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

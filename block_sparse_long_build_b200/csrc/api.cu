@@ -1,0 +1,288 @@
+// C ABI of libbsa: argument validation, workspace layout and dispatch.
+// Declarations and semantics: include/bsa.h.
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace bsa {
+
+bsa_status launch_build_summaries(const bsa_kv_desc *, const void *, const bsa_sel_params *, int,
+                                  int, int, int, void *, cudaStream_t);
+bsa_status launch_append(const bsa_kv_desc *, void *, void *, const void *, const void *, int32_t *,
+                         const bsa_sel_params *, int, int, void *, cudaStream_t);
+bsa_status launch_select(const bsa_kv_desc *, const float *, const void *, int,
+                         const bsa_sel_params *, const int32_t *, int, int, int32_t *, int32_t *,
+                         int, int32_t *, int32_t *, uint32_t *, int32_t *, uint32_t *,
+                         cudaStream_t);
+bsa_status launch_decode(const bsa_kv_desc *, const float *, const void *, const void *,
+                         const int32_t *, const int32_t *, int, const int32_t *, int, float, float *,
+                         float *, uint32_t *, uint32_t *, void *, cudaStream_t);
+int decode_nsplit(const bsa_kv_desc *, int, int);
+size_t decode_scratch_bytes(const bsa_kv_desc *, int);
+bsa_status launch_prefill(const bsa_kv_desc *, const void *, const void *, const bsa_sel_params *,
+                          const void *, const bsa_kv_desc *, const void *, const void *,
+                          const void *, int, int, float, float *, float *, void *, size_t,
+                          cudaStream_t);
+size_t prefill_ws_bytes(const bsa_kv_desc *, const bsa_sel_params *, int);
+
+int num_sms() {
+    static int n = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            n = v;
+        else
+            n = 148;
+        cudaGetLastError();
+    });
+    return n;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+bool make_kv_tmap(CUtensorMap *map, const bsa_kv_desc *d, const void *base, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)d->D, (cuuint64_t)d->L_max, (cuuint64_t)d->Hkv,
+                                (cuuint64_t)d->B};
+    const cuuint64_t strides[3] = {(cuuint64_t)d->stride_t * 2, (cuuint64_t)d->stride_h * 2,
+                                   (cuuint64_t)d->stride_b * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- validation
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static int elem_size(const bsa_kv_desc *d) { return d->kv_dtype == BSA_BF16 ? 2 : 4; }
+
+static bool desc_ok(const bsa_kv_desc *d) {
+    if (!d) return false;
+    if (d->B < 1 || d->Hkv < 1 || d->Hq < d->Hkv || d->Hq % d->Hkv != 0) return false;
+    if (d->D != 64 && d->D != 128) return false;
+    if (d->kv_dtype != BSA_F32 && d->kv_dtype != BSA_BF16) return false;
+    if (d->L_max < 1) return false;
+    if (d->stride_t < d->D || d->stride_h < 1 || d->stride_b < 1) return false;
+    const int64_t es = elem_size(d);
+    if ((d->stride_t * es) % 16 || (d->stride_h * es) % 16 || (d->stride_b * es) % 16) return false;
+    return true;
+}
+
+static bool sel_ok(const bsa_kv_desc *d, const bsa_sel_params *p) {
+    if (!p || p->block_size < 0) return false;
+    if (p->topk < 0 && p->budget_tokens < 0) return false;
+    if (p->sink < 0 || p->window < 0) return false;
+    if (p->block_size == 0) {
+        if (p->n_blocks < 1 || !p->block_offsets || !p->kv_pos) return false;
+        if (p->local_start < 0 || p->local_start > d->L_max) return false;
+    }
+    return true;
+}
+
+static int nb_total(const bsa_kv_desc *d, const bsa_sel_params *p) {
+    return p->block_size > 0 ? (int)div_up(d->L_max, p->block_size) : p->n_blocks;
+}
+
+static int max_selected(const bsa_kv_desc *d, const bsa_sel_params *p) {
+    const int nb = nb_total(d, p);
+    if (p->topk >= 0) return std::max(1, std::min(p->topk, nb));
+    if (p->block_size > 0) return std::max(1, std::min(p->budget_tokens / p->block_size, nb));
+    return nb;
+}
+
+static int max_ranges(const bsa_kv_desc *d, const bsa_sel_params *p) {
+    return max_selected(d, p) + 4;
+}
+
+// Workspace: [status u32][select counters: nseg][decode counters: nseg],
+// padded to 256 bytes, then the op's scratch.
+static size_t counters_bytes(const bsa_kv_desc *d) {
+    return align_up((size_t)(1 + 2 * d->B * d->Hkv) * 4, 256);
+}
+
+static bool ws_ok(const void *ws, size_t have, size_t need) {
+    return ws && aligned16(ws) && have >= need;
+}
+
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" {
+
+int32_t bsa_version(void) { return 100; }
+
+const char *bsa_status_string(bsa_status s) {
+    switch (s) {
+        case BSA_OK: return "ok";
+        case BSA_ERR_ARG: return "invalid argument";
+        case BSA_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case BSA_ERR_CUDA: return "CUDA error";
+        case BSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case BSA_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+int32_t bsa_summary_blocks(const bsa_kv_desc *d, const bsa_sel_params *p) {
+    if (!desc_ok(d) || !sel_ok(d, p)) return -1;
+    return nb_total(d, p);
+}
+
+size_t bsa_summary_bytes(const bsa_kv_desc *d, const bsa_sel_params *p, bsa_summary_kind kind) {
+    if (!desc_ok(d) || !sel_ok(d, p)) return 0;
+    const size_t row = kind == BSA_SUM_MINMAX ? (size_t)2 * d->D * elem_size(d) : (size_t)d->D * 4;
+    return (size_t)d->B * d->Hkv * nb_total(d, p) * row;
+}
+
+int32_t bsa_max_selected(const bsa_kv_desc *d, const bsa_sel_params *p) {
+    if (!desc_ok(d) || !sel_ok(d, p)) return -1;
+    return max_selected(d, p);
+}
+
+int32_t bsa_max_ranges(const bsa_kv_desc *d, const bsa_sel_params *p) {
+    if (!desc_ok(d) || !sel_ok(d, p)) return -1;
+    return max_ranges(d, p);
+}
+
+size_t bsa_workspace_size(const bsa_kv_desc *d, const bsa_sel_params *p, int op, int32_t n_queries,
+                          int32_t tokens_hint) {
+    if (!desc_ok(d)) return 0;
+    const size_t cb = counters_bytes(d);
+    const size_t nseg = (size_t)d->B * d->Hkv;
+    switch (op) {
+        case BSA_OP_SELECT:
+            if (!sel_ok(d, p)) return 0;
+            return cb + align_up(nseg * nb_total(d, p) * 4, 256) * 2;
+        case BSA_OP_DECODE: {
+            const int mr = p && sel_ok(d, p) ? max_ranges(d, p) : 64;
+            return cb + decode_scratch_bytes(d, decode_nsplit(d, std::max(tokens_hint, 1), mr));
+        }
+        case BSA_OP_APPEND:
+            return cb;
+        case BSA_OP_PREFILL:
+            if (!sel_ok(d, p) || n_queries < 1) return 0;
+            return cb + prefill_ws_bytes(d, p, n_queries);
+    }
+    return 0;
+}
+
+bsa_status bsa_build_summaries(const bsa_kv_desc *d, const void *K, const bsa_sel_params *p,
+                               bsa_summary_kind kind, int32_t first_block, int32_t n_blocks,
+                               void *summaries, bsa_stream_t stream) {
+    if (!desc_ok(d) || !sel_ok(d, p) || !K || !summaries || !aligned16(K) || !aligned16(summaries))
+        return BSA_ERR_ARG;
+    if (kind < BSA_SUM_CENTROID || kind > BSA_SUM_MINMAX) return BSA_ERR_ARG;
+    const int nb = nb_total(d, p);
+    if (first_block < 0 || n_blocks < 0 || (int64_t)first_block + n_blocks > nb) return BSA_ERR_ARG;
+    if (p->block_size > 0 && ((int64_t)first_block + n_blocks) * p->block_size > d->L_max)
+        return BSA_ERR_ARG;
+    if (n_blocks == 0) return BSA_OK;
+    return launch_build_summaries(d, K, p, kind, first_block, n_blocks, nb, summaries,
+                                  (cudaStream_t)stream);
+}
+
+bsa_status bsa_select(const bsa_kv_desc *d, const float *q, const void *summaries,
+                      bsa_summary_kind kind, const bsa_sel_params *p, const int32_t *cur_len,
+                      int32_t max_sel, int32_t *sel_blocks, int32_t *sel_count, int32_t max_r,
+                      int32_t *ranges, int32_t *n_ranges, void *ws, size_t ws_bytes,
+                      bsa_stream_t stream) {
+    if (!desc_ok(d) || !sel_ok(d, p)) return BSA_ERR_ARG;
+    if (!q || !summaries || !cur_len || !sel_blocks || !sel_count || !ranges || !n_ranges)
+        return BSA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(summaries)) return BSA_ERR_ARG;
+    if (kind < BSA_SUM_CENTROID || kind > BSA_SUM_MINMAX) return BSA_ERR_ARG;
+    if (d->Hq / d->Hkv > 16) return BSA_ERR_UNSUPPORTED;
+    if (max_sel < max_selected(d, p) || max_r < max_ranges(d, p)) return BSA_ERR_ARG;
+    const size_t need = bsa_workspace_size(d, p, BSA_OP_SELECT, 0, 0);
+    if (!ws_ok(ws, ws_bytes, need)) return BSA_ERR_WORKSPACE;
+    const size_t nseg = (size_t)d->B * d->Hkv;
+    const int nb = nb_total(d, p);
+    uint32_t *cnt = static_cast<uint32_t *>(ws) + 1;
+    char *scr = static_cast<char *>(ws) + counters_bytes(d);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(scr);
+    int32_t *vis = reinterpret_cast<int32_t *>(scr + align_up(nseg * nb * 4, 256));
+    return launch_select(d, q, summaries, kind, p, cur_len, nb, max_sel, sel_blocks, sel_count, max_r,
+                         ranges, n_ranges, keys, vis, cnt, (cudaStream_t)stream);
+}
+
+bsa_status bsa_decode(const bsa_kv_desc *d, const float *q, const void *K, const void *V,
+                      const int32_t *ranges, const int32_t *n_ranges, int32_t max_r,
+                      const int32_t *cur_len, int32_t tokens_hint, float scale, float *out,
+                      float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream) {
+    if (!desc_ok(d)) return BSA_ERR_ARG;
+    if (!q || !K || !V || !ranges || !n_ranges || !cur_len || !out) return BSA_ERR_ARG;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(q)) return BSA_ERR_ARG;
+    if (max_r < 1 || max_r > 4096 || tokens_hint < 0) return BSA_ERR_ARG;
+    if (d->Hq / d->Hkv > kMaxG) return BSA_ERR_UNSUPPORTED;
+    if (!(scale > 0.0f) || scale != scale) return BSA_ERR_ARG;
+    const int nsplit = decode_nsplit(d, std::max(tokens_hint, 1), max_r);
+    const size_t need = counters_bytes(d) + decode_scratch_bytes(d, nsplit);
+    if (!ws_ok(ws, ws_bytes, need)) return BSA_ERR_WORKSPACE;
+    uint32_t *status = static_cast<uint32_t *>(ws);
+    uint32_t *cnt = status + 1 + d->B * d->Hkv;
+    void *scr = static_cast<char *>(ws) + counters_bytes(d);
+    return launch_decode(d, q, K, V, ranges, n_ranges, max_r, cur_len, std::max(tokens_hint, 1),
+                         scale, out, lse, status, cnt, scr, (cudaStream_t)stream);
+}
+
+bsa_status bsa_append_kv(const bsa_kv_desc *d, void *K, void *V, const void *k_new,
+                         const void *v_new, int32_t *cur_len, const bsa_sel_params *p,
+                         bsa_summary_kind kind, void *summaries, bsa_stream_t stream) {
+    if (!desc_ok(d) || !K || !V || !k_new || !v_new || !cur_len) return BSA_ERR_ARG;
+    if (p && !sel_ok(d, p)) return BSA_ERR_ARG;
+    if (summaries && (!p || kind < BSA_SUM_CENTROID || kind > BSA_SUM_MINMAX)) return BSA_ERR_ARG;
+    const int nb = p ? nb_total(d, p) : 0;
+    return launch_append(d, K, V, k_new, v_new, cur_len, p, kind, nb, summaries,
+                         (cudaStream_t)stream);
+}
+
+bsa_status bsa_prefill_grouped(const bsa_kv_desc *d, const void *K, const void *V,
+                               const bsa_sel_params *p, const void *summaries,
+                               const bsa_kv_desc *pd, const void *K_pos, const void *V_pos,
+                               const void *Q, int32_t q_pos0, int32_t Tq, float scale, float *out,
+                               float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream) {
+    if (!desc_ok(d) || !desc_ok(pd) || !sel_ok(d, p)) return BSA_ERR_ARG;
+    if (!K || !V || !summaries || !K_pos || !V_pos || !Q || !out) return BSA_ERR_ARG;
+    if (p->block_size != 0 || p->topk >= 0) return BSA_ERR_UNSUPPORTED;
+    if (d->B != 1 || pd->B != 1 || d->Hkv != pd->Hkv || d->Hq != pd->Hq || d->D != pd->D)
+        return BSA_ERR_ARG;
+    if (d->kv_dtype != BSA_BF16 || pd->kv_dtype != BSA_BF16 || d->D != 128) return BSA_ERR_UNSUPPORTED;
+    if (d->stride_t != d->D || pd->stride_t != pd->D) return BSA_ERR_UNSUPPORTED;
+    if (Tq < 1 || q_pos0 < 0 || (int64_t)q_pos0 + Tq > pd->L_max || p->pos_limit < 0 ||
+        p->pos_limit > q_pos0)
+        return BSA_ERR_ARG;
+    if (!(scale > 0.0f)) return BSA_ERR_ARG;
+    const size_t need = bsa_workspace_size(d, p, BSA_OP_PREFILL, Tq, 0);
+    if (!ws_ok(ws, ws_bytes, need)) return BSA_ERR_WORKSPACE;
+    return launch_prefill(d, K, V, p, summaries, pd, K_pos, V_pos, Q, q_pos0, Tq, scale, out, lse,
+                          static_cast<char *>(ws) + counters_bytes(d), ws_bytes - counters_bytes(d),
+                          (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,571 @@
+// A4 (split-K sparse decode over the selected token ranges) + A5 (log-sum-exp
+// merge), sm_100a.
+//
+// out_h = sum_j softmax_j(scale * q_h . k_j) v_j over the selected rows
+// ("Module 14: Sparse attention and long context", Exercise 14.1, restricted
+// to the selected set), GQA: query head h reads KV head h / G.
+//
+// Work decomposition.  A segment's ranges are cut into pieces of 16 rows
+// (one TMA box each; a range's last piece may be short).  The pieces are
+// split evenly over `nsplit` CTAs; a CTA walks its pieces in tiles of 4, one
+// piece per warp.  Every CTA writes an unnormalised partial (m, l, o) in
+// base 2; the last CTA of a segment to finish (an atomic counter, reset
+// afterwards) merges the partials in split order, so the result does not
+// depend on scheduling.
+//
+// Tensor-core path (bf16 K/V, D in {64, 128}, G <= 8): K and V pieces are
+// brought into a multi-stage shared-memory ring by 4-D tiled TMA loads with
+// 128-byte swizzle (no multicast), one elected thread issuing and an
+// mbarrier per stage.  All G query heads of the group share every K/V byte:
+// the 16 MMA rows hold q_hi (rows 0-7) and q_lo = q - q_hi (rows 8-15), so
+// one m16n8k16 bf16 MMA gives the logits to ~2^-17 relative; the softmax
+// weights are split the same way for P.V.  Accumulation is fp32.
+#include "common.cuh"
+
+namespace bsa {
+
+constexpr int kPiece = 16;
+constexpr int kDecWarps = 4;
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kBoxBytes = kPiece * 128;            // 16 rows x 64 bf16
+constexpr int kHalfBytes = kDecWarps * kBoxBytes;  // one 64-column half of a tile
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kNegInf = -__builtin_huge_valf();
+
+struct DecArgs {
+    const float *q;
+    float *out, *lse;
+    const int32_t *ranges, *n_ranges;
+    int max_ranges;
+    const int32_t *cur_len;
+    const void *K, *V;
+    int64_t stride_b, stride_h, stride_t;
+    int B, Hq, Hkv, G, D, L_max, nsplit;
+    float scale_log2;
+    float *part_o;        // [nseg][nsplit][G][D]
+    float2 *part_ml;      // [nseg][nsplit][G]
+    uint32_t *counters;   // [nseg]
+    uint32_t *status;     // sticky error bits
+};
+
+// Exclusive scan over the CTA (blockDim.x a multiple of 32, <= 1024).
+__device__ __forceinline__ int block_excl_scan(int v, int *tmp, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+    }
+    if (lane == 31) tmp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? tmp[lane] : 0, wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            int t = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += t;
+        }
+        if (lane < nw) tmp[lane] = wi - w;
+        if (lane == 31) tmp[32] = wi;
+    }
+    __syncthreads();
+    int res = incl - v + tmp[warp];
+    *total = tmp[32];
+    __syncthreads();
+    return res;
+}
+
+// Loads segment s's ranges (clamped to [0, L_max), the last extended to
+// cur_len) and the prefix of their 16-row piece counts.  Returns the number
+// of pieces; *nr_out the number of ranges.
+__device__ int load_ranges(const DecArgs &a, int s, int b, int *rs, int *re, int *ps, int *tmp,
+                           int *nr_out) {
+    const int nr = min(max(a.n_ranges[s], 0), a.max_ranges);
+    const int32_t *R = a.ranges + (int64_t)s * a.max_ranges * 2;
+    const int cl = min(max(a.cur_len[b], 0), a.L_max);
+    int carry = 0;
+    for (int base = 0; base < nr; base += blockDim.x) {
+        const int r = base + threadIdx.x;
+        int cnt = 0;
+        if (r < nr) {
+            int lo = min(max(R[2 * r], 0), a.L_max);
+            int hi = min(max(R[2 * r + 1], lo), a.L_max);
+            if (r == nr - 1 && cl > hi) hi = cl;
+            rs[r] = lo;
+            re[r] = hi;
+            cnt = (hi - lo + kPiece - 1) / kPiece;
+        }
+        int tot;
+        int ex = block_excl_scan(cnt, tmp, &tot);
+        if (r < nr) ps[r] = carry + ex;
+        carry += tot;
+    }
+    *nr_out = nr;
+    __syncthreads();
+    return carry;
+}
+
+// Piece p -> (first row, valid rows).
+__device__ __forceinline__ int2 piece_rows(int p, const int *rs, const int *re, const int *ps,
+                                           int nr) {
+    int lo = 0, hi = nr - 1;
+    while (lo < hi) {   // largest r with ps[r] <= p
+        int mid = (lo + hi + 1) >> 1;
+        if (ps[mid] <= p) lo = mid; else hi = mid - 1;
+    }
+    int row = rs[lo] + (p - ps[lo]) * kPiece;
+    return make_int2(row, min(kPiece, re[lo] - row));
+}
+
+// Combines the per-warp partials (wm, wl, wo) of this CTA and writes either
+// the final output (nsplit == 1) or the split partial, merging when this is
+// the last CTA of the segment.
+__device__ void finish(const DecArgs &a, int s, int b, int g, int c, const float *wm,
+                       const float *wl, const float *wo, float *sml /* [2*kMaxG] */) {
+    const int G = a.G, D = a.D;
+    __shared__ int is_last;
+    if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float M = kNegInf;
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wm[w * kMaxG + h]);
+        float L = 0.0f;
+        for (int w = 0; w < kDecWarps; ++w) {
+            float mw = wm[w * kMaxG + h];
+            if (mw != kNegInf) L += wl[w * kMaxG + h] * exp2f(mw - M);
+        }
+        sml[2 * h] = M;
+        sml[2 * h + 1] = L;
+    }
+    __syncthreads();
+    const int64_t qrow = (int64_t)b * a.Hq + (int64_t)g * G;
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+        const int h = e / D, d = e % D;
+        const float M = sml[2 * h];
+        float O = 0.0f;
+        for (int w = 0; w < kDecWarps; ++w) {
+            float mw = wm[w * kMaxG + h];
+            if (mw != kNegInf) O += wo[(w * kMaxG + h) * D + d] * exp2f(mw - M);
+        }
+        if (a.nsplit == 1) {
+            const float L = sml[2 * h + 1];
+            a.out[(qrow + h) * D + d] = L > 0.0f ? O / L : 0.0f;
+            if (d == 0 && a.lse) a.lse[qrow + h] = L > 0.0f ? (M + log2f(L)) * kLn2 : kNegInf;
+        } else {
+            a.part_o[(((int64_t)s * a.nsplit + c) * G + h) * D + d] = O;
+            if (d == 0) a.part_ml[((int64_t)s * a.nsplit + c) * G + h] = make_float2(M, sml[2 * h + 1]);
+        }
+    }
+    if (a.nsplit == 1) return;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(&a.counters[s], 1u) == (unsigned)(a.nsplit - 1);
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float M = kNegInf;
+        for (int k = 0; k < a.nsplit; ++k)
+            M = fmaxf(M, __ldcg(&a.part_ml[((int64_t)s * a.nsplit + k) * G + h]).x);
+        float L = 0.0f;
+        for (int k = 0; k < a.nsplit; ++k) {
+            float2 ml = __ldcg(&a.part_ml[((int64_t)s * a.nsplit + k) * G + h]);
+            if (ml.x != kNegInf) L += ml.y * exp2f(ml.x - M);
+        }
+        sml[2 * h] = M;
+        sml[2 * h + 1] = L;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+        const int h = e / D, d = e % D;
+        const float M = sml[2 * h], L = sml[2 * h + 1];
+        float O = 0.0f;
+        for (int k = 0; k < a.nsplit; ++k) {
+            float mk = __ldcg(&a.part_ml[((int64_t)s * a.nsplit + k) * G + h]).x;
+            if (mk != kNegInf)
+                O += __ldcg(&a.part_o[(((int64_t)s * a.nsplit + k) * G + h) * D + d]) * exp2f(mk - M);
+        }
+        a.out[(qrow + h) * D + d] = L > 0.0f ? O / L : 0.0f;
+        if (d == 0 && a.lse) a.lse[qrow + h] = L > 0.0f ? (M + log2f(L)) * kLn2 : kNegInf;
+    }
+    if (threadIdx.x == 0) a.counters[s] = 0;
+}
+
+// ======================================================================
+// Tensor-core path
+// ======================================================================
+template <int NH, int STAGES>
+struct TcSmem {
+    static constexpr int kStageBytes = 2 * NH * kHalfBytes;   // K halves, then V halves
+    static constexpr int kRing = STAGES * kStageBytes;
+    static constexpr int kInfo = kRing;                        // int2 [STAGES][4]
+    static constexpr int kBars = kInfo + STAGES * kDecWarps * 8;
+    static constexpr int kMisc = kBars + STAGES * 8;           // float sml[2*kMaxG], int tmp[33]
+    static constexpr int kRanges = kMisc + 2 * kMaxG * 4 + 36 * 4;
+    static constexpr int bytes(int max_ranges) { return kRanges + (3 * max_ranges + 1) * 4 + 1024; }
+};
+
+template <int NH, int STAGES>
+__global__ void __launch_bounds__(kDecThreads, 2)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     DecArgs a) {
+    using L = TcSmem<NH, STAGES>;
+    constexpr int D = 64 * NH;
+    constexpr int NT = D / 8;   // 8-column MMA tiles across D
+    extern __shared__ unsigned char dsm_raw[];
+    unsigned char *dsm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    int2 *info = reinterpret_cast<int2 *>(dsm + L::kInfo);
+    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + L::kBars);
+    float *sml = reinterpret_cast<float *>(dsm + L::kMisc);
+    int *tmp = reinterpret_cast<int *>(dsm + L::kMisc + 2 * kMaxG * 4);
+    int *rs = reinterpret_cast<int *>(dsm + L::kRanges);
+    int *re = rs + a.max_ranges;
+    int *ps = re + a.max_ranges;
+
+    const int c = blockIdx.x, s = blockIdx.y;
+    const int b = s / a.Hkv, g = s % a.Hkv;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+
+    if (tid == 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        for (int i = 0; i < STAGES; ++i) mbar_init(&full[i], 1);
+        fence_mbar_init();
+    }
+    int nr;
+    const int P = load_ranges(a, s, b, rs, re, ps, tmp, &nr);
+    int per = (P + a.nsplit - 1) / a.nsplit;
+    per = (per + kDecWarps - 1) / kDecWarps * kDecWarps;
+    const int first = c * per, last = min(P, first + per);
+    const int n_my = max(0, last - first);
+    const int tiles = (n_my + kDecWarps - 1) / kDecWarps;
+
+    auto stage_ptr = [&](int st, int part) {   // part: 0..NH-1 K halves, NH..2NH-1 V halves
+        return dsm + st * L::kStageBytes + part * kHalfBytes;
+    };
+    auto issue = [&](int t, int st) {
+        int np = 0;
+        int2 pr[kDecWarps];
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+            int p = first + t * kDecWarps + w;
+            pr[w] = p < last ? piece_rows(p, rs, re, ps, nr) : make_int2(0, 0);
+            info[st * kDecWarps + w] = pr[w];
+            np += pr[w].y > 0;
+        }
+        mbar_arrive_expect_tx(&full[st], (uint32_t)(np * 2 * NH * kBoxBytes));
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+            if (pr[w].y <= 0) continue;
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                tma_load_4d(stage_ptr(st, h) + w * kBoxBytes, &tmK, &full[st], h * 64, pr[w].x, g, b);
+                tma_load_4d(stage_ptr(st, NH + h) + w * kBoxBytes, &tmV, &full[st], h * 64, pr[w].x, g, b);
+            }
+        }
+    };
+    if (tid == 0)
+        for (int t = 0; t < STAGES && t < tiles; ++t) issue(t, t);
+
+    // q fragments: rows 0-7 q_hi of head gid, rows 8-15 q_lo; zero past G
+    uint32_t qa[D / 16][4];
+    {
+        const float *qg = a.q + ((int64_t)b * a.Hq + (int64_t)g * a.G + gid) * D;
+        const bool live = gid < a.G;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            float x[4];
+            const int k0 = kk * 16 + 2 * tig;
+            x[0] = live ? qg[k0] : 0.0f;
+            x[1] = live ? qg[k0 + 1] : 0.0f;
+            x[2] = live ? qg[k0 + 8] : 0.0f;
+            x[3] = live ? qg[k0 + 9] : 0.0f;
+            float hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                hi[e] = bf16_round(x[e]);
+                lo[e] = x[e] - hi[e];
+            }
+            qa[kk][0] = pack_bf16x2(hi[0], hi[1]);
+            qa[kk][1] = pack_bf16x2(lo[0], lo[1]);
+            qa[kk][2] = pack_bf16x2(hi[2], hi[3]);
+            qa[kk][3] = pack_bf16x2(lo[2], lo[3]);
+        }
+    }
+
+    float o[NT][4];
+#pragma unroll
+    for (int i = 0; i < NT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+    float m_run = kNegInf, l_run = 0.0f;
+    bool timed_out = false;
+
+    for (int t = 0; t < tiles; ++t) {
+        const int st = t % STAGES;
+        if (!mbar_wait_bounded(&full[st], (uint32_t)((t / STAGES) & 1))) timed_out = true;
+        const int2 pr = info[st * kDecWarps + warp];
+        const int nv = pr.y;
+        if (nv > 0) {
+            const uint32_t kbase = smem_u32(stage_ptr(st, 0) + warp * kBoxBytes);
+            const uint32_t vbase = smem_u32(stage_ptr(st, NH) + warp * kBoxBytes);
+            if (nv < kPiece) {   // rows past the range end: zero V so 0 * junk stays 0
+                for (int idx = lane; idx < (kPiece - nv) * NH * 8; idx += 32) {
+                    int r = nv + idx / (NH * 8), h = (idx / 8) % NH, ch = idx % 8;
+                    *reinterpret_cast<uint4 *>(stage_ptr(st, NH + h) + warp * kBoxBytes + r * 128 +
+                                               ch * 16) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            // S = Q K^T for the piece's 16 rows (two 8-row MMA tiles)
+            float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int half = kk / 4, ch0 = (kk % 4) * 2;
+                const int r = (lane >> 4) * 8 + (lane & 7);
+                const int ch = ch0 + ((lane >> 3) & 1);
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(kbase + half * kHalfBytes + r * 128 + ((ch ^ (r & 7)) << 4), b0, b1, b2, b3);
+                mma_bf16_16816(sacc[0], qa[kk], b0, b1);
+                mma_bf16_16816(sacc[1], qa[kk], b2, b3);
+            }
+            float lg[4];
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tok = n * 8 + 2 * tig + e;
+                    lg[n * 2 + e] = tok < nv ? (sacc[n][e] + sacc[n][2 + e]) * a.scale_log2 : kNegInf;
+                }
+            float mx = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            float p[4];
+            if (m_new == kNegInf) {
+                p[0] = p[1] = p[2] = p[3] = 0.0f;
+            } else {
+                const float corr = exp2f(m_run - m_new);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p[e] = exp2f(lg[e] - m_new);
+                l_run = l_run * corr + ((p[0] + p[1]) + (p[2] + p[3]));
+#pragma unroll
+                for (int i = 0; i < NT; ++i) {
+                    o[i][0] *= corr; o[i][1] *= corr; o[i][2] *= corr; o[i][3] *= corr;
+                }
+                m_run = m_new;
+            }
+            uint32_t pa[4];
+            {
+                float ph[4], pl[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    ph[e] = bf16_round(p[e]);
+                    pl[e] = p[e] - ph[e];
+                }
+                pa[0] = pack_bf16x2(ph[0], ph[1]);
+                pa[1] = pack_bf16x2(pl[0], pl[1]);
+                pa[2] = pack_bf16x2(ph[2], ph[3]);
+                pa[3] = pack_bf16x2(pl[2], pl[3]);
+            }
+            // O += P V
+#pragma unroll
+            for (int cp = 0; cp < D / 16; ++cp) {
+                const int half = cp / 4, ch0 = (cp % 4) * 2;
+                const int r = ((lane >> 3) & 1) * 8 + (lane & 7);
+                const int ch = ch0 + (lane >> 4);
+                uint32_t r0, r1, r2, r3;
+                ldmatrix_x4_trans(vbase + half * kHalfBytes + r * 128 + ((ch ^ (r & 7)) << 4), r0, r1, r2, r3);
+                mma_bf16_16816(o[2 * cp], pa, r0, r1);
+                mma_bf16_16816(o[2 * cp + 1], pa, r2, r3);
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && t + STAGES < tiles) issue(t + STAGES, st);
+    }
+    if (timed_out) atomicOr(a.status, 1u);
+
+    // per-warp partials -> shared memory (reusing the ring)
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    float *wm = reinterpret_cast<float *>(dsm);
+    float *wl = wm + kDecWarps * kMaxG;
+    float *wo = wl + kDecWarps * kMaxG;
+    __syncthreads();
+    if (tig == 0) {
+        wm[warp * kMaxG + gid] = m_run;
+        wl[warp * kMaxG + gid] = l_run;
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int d = nt * 8 + 2 * tig;
+        wo[(warp * kMaxG + gid) * D + d] = o[nt][0] + o[nt][2];
+        wo[(warp * kMaxG + gid) * D + d + 1] = o[nt][1] + o[nt][3];
+    }
+    __syncthreads();
+    finish(a, s, b, g, c, wm, wl, wo, sml);
+}
+
+// ======================================================================
+// CUDA-core path (fp32 or bf16 K/V, any G <= 8, D in {64, 128})
+// ======================================================================
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads) decode_generic_kernel(DecArgs a) {
+    constexpr int PER = D / 32;
+    extern __shared__ __align__(16) unsigned char dsm[];
+    float *wm = reinterpret_cast<float *>(dsm);
+    float *wl = wm + kDecWarps * kMaxG;
+    float *wo = wl + kDecWarps * kMaxG;
+    float *sml = wo + kDecWarps * kMaxG * D;
+    int *tmp = reinterpret_cast<int *>(sml + 2 * kMaxG);
+    int *rs = tmp + 36;
+    int *re = rs + a.max_ranges;
+    int *ps = re + a.max_ranges;
+
+    const int c = blockIdx.x, s = blockIdx.y;
+    const int b = s / a.Hkv, g = s % a.Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int nr;
+    const int P = load_ranges(a, s, b, rs, re, ps, tmp, &nr);
+    int per = (P + a.nsplit - 1) / a.nsplit;
+    per = (per + kDecWarps - 1) / kDecWarps * kDecWarps;
+    const int first = c * per, last = min(P, first + per);
+
+    float qr[kMaxG][PER];
+    const float *qg = a.q + ((int64_t)b * a.Hq + (int64_t)g * a.G) * D;
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h)
+#pragma unroll
+        for (int k = 0; k < PER; ++k) qr[h][k] = h < a.G ? qg[h * D + lane + 32 * k] : 0.0f;
+    float m[kMaxG], l[kMaxG], o[kMaxG][PER];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+        m[h] = kNegInf;
+        l[h] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) o[h][k] = 0.0f;
+    }
+    const T *Ks = static_cast<const T *>(a.K) + b * a.stride_b + g * a.stride_h;
+    const T *Vs = static_cast<const T *>(a.V) + b * a.stride_b + g * a.stride_h;
+    for (int p = first + warp; p < last; p += kDecWarps) {
+        const int2 pr = piece_rows(p, rs, re, ps, nr);
+        for (int r = pr.x; r < pr.x + pr.y; ++r) {
+            float kv[PER], vv[PER];
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                kv[k] = load_elem(Ks, (int64_t)r * a.stride_t + lane + 32 * k);
+                vv[k] = load_elem(Vs, (int64_t)r * a.stride_t + lane + 32 * k);
+            }
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h) {
+                if (h >= a.G) break;
+                float dot = 0.0f;
+#pragma unroll
+                for (int k = 0; k < PER; ++k) dot = fmaf(qr[h][k], kv[k], dot);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+                const float lg = dot * a.scale_log2;
+                const float mn = fmaxf(m[h], lg);
+                const float corr = exp2f(m[h] - mn);
+                const float pw = exp2f(lg - mn);
+                l[h] = l[h] * corr + pw;
+#pragma unroll
+                for (int k = 0; k < PER; ++k) o[h][k] = o[h][k] * corr + pw * vv[k];
+                m[h] = mn;
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+        if (lane == 0) {
+            wm[warp * kMaxG + h] = m[h];
+            wl[warp * kMaxG + h] = l[h];
+        }
+#pragma unroll
+        for (int k = 0; k < PER; ++k) wo[(warp * kMaxG + h) * D + lane + 32 * k] = o[h][k];
+    }
+    __syncthreads();
+    finish(a, s, b, g, c, wm, wl, wo, sml);
+}
+
+// ======================================================================
+// Host side
+// ======================================================================
+constexpr int kTcStages = 3;
+
+static bool use_tc(const bsa_kv_desc *d) {
+    return d->kv_dtype == BSA_BF16 && (d->D == 64 || d->D == 128) && d->Hq / d->Hkv <= kMaxG &&
+           d->stride_t == d->D;
+}
+
+int decode_nsplit(const bsa_kv_desc *d, int tokens_hint, int max_ranges) {
+    const int nseg = d->B * d->Hkv;
+    const int64_t pieces = div_up(tokens_hint > 0 ? tokens_hint : 1, kPiece) + max_ranges;
+    const int slots = num_sms() * (use_tc(d) ? 2 : 4);
+    int nsplit = std::max(1, slots / std::max(nseg, 1));
+    nsplit = (int)std::min<int64_t>(nsplit, div_up(pieces, kDecWarps));
+    return std::max(1, nsplit);
+}
+
+size_t decode_scratch_bytes(const bsa_kv_desc *d, int nsplit) {
+    const size_t nseg = (size_t)d->B * d->Hkv, G = d->Hq / d->Hkv;
+    return align_up(nseg * nsplit * G * d->D * 4, 256) + align_up(nseg * nsplit * G * 8, 256);
+}
+
+bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, const void *V,
+                         const int32_t *ranges, const int32_t *n_ranges, int max_ranges,
+                         const int32_t *cur_len, int tokens_hint, float scale, float *out,
+                         float *lse, uint32_t *status, uint32_t *counters, void *scratch,
+                         cudaStream_t st) {
+    DecArgs a;
+    a.q = q; a.out = out; a.lse = lse; a.ranges = ranges; a.n_ranges = n_ranges;
+    a.max_ranges = max_ranges; a.cur_len = cur_len; a.K = K; a.V = V;
+    a.stride_b = d->stride_b; a.stride_h = d->stride_h; a.stride_t = d->stride_t;
+    a.B = d->B; a.Hq = d->Hq; a.Hkv = d->Hkv; a.G = d->Hq / d->Hkv; a.D = d->D;
+    a.L_max = d->L_max;
+    a.nsplit = decode_nsplit(d, tokens_hint, max_ranges);
+    a.scale_log2 = scale * 1.4426950408889634f;
+    const size_t nseg = (size_t)d->B * d->Hkv;
+    a.part_o = static_cast<float *>(scratch);
+    a.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(scratch) +
+                                           align_up(nseg * a.nsplit * a.G * d->D * 4, 256));
+    a.counters = counters;
+    a.status = status;
+    dim3 grid(a.nsplit, (unsigned)nseg);
+    if (use_tc(d)) {
+        CUtensorMap tk, tv;
+        if (!make_kv_tmap(&tk, d, K, kPiece) || !make_kv_tmap(&tv, d, V, kPiece)) return BSA_ERR_CUDA;
+        if (d->D == 128) {
+            auto kern = decode_tc_kernel<2, kTcStages>;
+            const int smem = TcSmem<2, kTcStages>::bytes(max_ranges);
+            BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+            kern<<<grid, kDecThreads, smem, st>>>(tk, tv, a);
+        } else {
+            auto kern = decode_tc_kernel<1, 2 * kTcStages>;
+            const int smem = TcSmem<1, 2 * kTcStages>::bytes(max_ranges);
+            BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+            kern<<<grid, kDecThreads, smem, st>>>(tk, tv, a);
+        }
+    } else {
+        const size_t smem = (size_t)(2 * kDecWarps * kMaxG + kDecWarps * kMaxG * d->D + 2 * kMaxG) * 4 +
+                            36 * 4 + (size_t)(3 * max_ranges + 1) * 4;
+        auto go = [&](auto kern) -> bsa_status {
+            if (smem > 48 * 1024)
+                BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+            kern<<<grid, kDecThreads, smem, st>>>(a);
+            return BSA_OK;
+        };
+        bsa_status r;
+        if (d->kv_dtype == BSA_BF16)
+            r = d->D == 128 ? go(decode_generic_kernel<uint16_t, 128>) : go(decode_generic_kernel<uint16_t, 64>);
+        else
+            r = d->D == 128 ? go(decode_generic_kernel<float, 128>) : go(decode_generic_kernel<float, 64>);
+        if (r != BSA_OK) return r;
+    }
+    BSA_LAUNCH_CHECK();
+    return BSA_OK;
+}
+
+}  // namespace bsa

@@ -1,0 +1,223 @@
+// A1 (per-block key summaries) and A8 (decode-step append + incremental
+// summary), sm_100a.
+//
+// Summaries ("Module 14: Sparse attention and long context", §14.3 MoBA,
+// mean-pooled here; "Semantic blocks for sparse attention", normalised block
+// centres; "Sparse attention in hybrid LLMs", Quest min/max page bounds).
+// The arithmetic order is fixed so that the scores computed from these
+// summaries, and hence the selected blocks, are reproducible bit for bit:
+//   centroid       c[i] = (((0 + k_r0[i]) + k_r1[i]) + ...) / n   (rows in order)
+//   centroid_norm  u_r = k_r / ||k_r|| (||.|| = sqrt of an fma chain over i),
+//                  m = mean of u_r as above, c = m / ||m||
+//   minmax         running min / max over rows in order (first wins on ties)
+#include "common.cuh"
+
+namespace bsa {
+
+constexpr int kNormChunk = 64;   // rows staged at once for the per-row norms
+
+// fp32 norm of a row held in shared memory: fma chain over i, then sqrt.
+__device__ __forceinline__ float row_norm_f32(const float *x, int D) {
+    float acc = 0.0f;
+    for (int i = 0; i < D; ++i) acc = __fmaf_rn(x[i], x[i], acc);
+    return __fsqrt_rn(acc);
+}
+
+// Summary of rows [r0, r1) of one segment, computed by the whole CTA
+// (blockDim.x >= D).  `out` points at this block's summary: D floats for the
+// centroid kinds, 2*D cache elements (min row, then max row) for MINMAX.
+// `sm` must hold kNormChunk*(D+1) + D + 1 floats.
+template <typename T>
+__device__ void summarize_rows(const T *Kseg, int64_t st, int D, int64_t r0, int64_t r1,
+                               int kind, void *out, float *sm) {
+    const int i = threadIdx.x;
+    const int64_t n = r1 - r0;
+    if (kind == BSA_SUM_CENTROID) {
+        if (i < D) {
+            float acc = 0.0f;
+            int64_t r = r0;
+            for (; r + 4 <= r1; r += 4) {   // loads batched, adds stay in order
+                float v0 = load_elem(Kseg, r * st + i), v1 = load_elem(Kseg, (r + 1) * st + i);
+                float v2 = load_elem(Kseg, (r + 2) * st + i), v3 = load_elem(Kseg, (r + 3) * st + i);
+                acc = __fadd_rn(acc, v0);
+                acc = __fadd_rn(acc, v1);
+                acc = __fadd_rn(acc, v2);
+                acc = __fadd_rn(acc, v3);
+            }
+            for (; r < r1; ++r) acc = __fadd_rn(acc, load_elem(Kseg, r * st + i));
+            static_cast<float *>(out)[i] = n > 0 ? __fdiv_rn(acc, (float)n) : 0.0f;
+        }
+        return;
+    }
+    if (kind == BSA_SUM_MINMAX) {
+        if (i < D) {
+            float lo = __int_as_float(0x7f800000), hi = __int_as_float(0xff800000);  // +inf, -inf
+            for (int64_t r = r0; r < r1; ++r) {
+                float v = load_elem(Kseg, r * st + i);
+                if (v < lo) lo = v;
+                if (v > hi) hi = v;
+            }
+            if (n <= 0) lo = hi = 0.0f;
+            T *o = static_cast<T *>(out);
+            if constexpr (sizeof(T) == 2) {
+                o[i] = static_cast<uint16_t>(__float_as_uint(lo) >> 16);
+                o[D + i] = static_cast<uint16_t>(__float_as_uint(hi) >> 16);
+            } else {
+                o[i] = lo;
+                o[D + i] = hi;
+            }
+        }
+        return;
+    }
+    // BSA_SUM_CENTROID_NORM
+    float *rows = sm;                              // [kNormChunk][D+1]
+    float *nrm = sm + kNormChunk * (D + 1);        // [kNormChunk] (aliases the tail)
+    float acc = 0.0f;
+    for (int64_t c0 = r0; c0 < r1; c0 += kNormChunk) {
+        const int cn = (int)((r1 - c0) < kNormChunk ? (r1 - c0) : kNormChunk);
+        __syncthreads();
+        for (int e = threadIdx.x; e < cn * D; e += blockDim.x) {
+            int rr = e / D, ii = e % D;
+            rows[rr * (D + 1) + ii] = load_elem(Kseg, (c0 + rr) * st + ii);
+        }
+        __syncthreads();
+        if (threadIdx.x < cn) nrm[threadIdx.x] = row_norm_f32(rows + threadIdx.x * (D + 1), D);
+        __syncthreads();
+        if (i < D) {
+            for (int rr = 0; rr < cn; ++rr) {
+                float nr = nrm[rr];
+                acc = __fadd_rn(acc, nr > 0.0f ? __fdiv_rn(rows[rr * (D + 1) + i], nr) : 0.0f);
+            }
+        }
+    }
+    __syncthreads();
+    float *mean = sm;   // reuse
+    if (i < D) mean[i] = n > 0 ? __fdiv_rn(acc, (float)n) : 0.0f;
+    __syncthreads();
+    if (threadIdx.x == 0) mean[D] = row_norm_f32(mean, D);
+    __syncthreads();
+    if (i < D) {
+        float nc = mean[D];
+        static_cast<float *>(out)[i] = nc > 0.0f ? __fdiv_rn(mean[i], nc) : 0.0f;
+    }
+    __syncthreads();
+}
+
+__host__ __device__ inline size_t summary_row_bytes(int kind, int D, int kv_dtype) {
+    return kind == BSA_SUM_MINMAX ? (size_t)2 * D * (kv_dtype == BSA_BF16 ? 2 : 4)
+                                  : (size_t)D * 4;
+}
+
+struct SumArgs {
+    const void *K;
+    void *summ;
+    const int32_t *offsets;   // variable blocks or nullptr
+    int64_t stride_b, stride_h, stride_t;
+    int Hkv, D, L_max, S, nb_total, first_block, kind;
+    size_t row_bytes;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(128) build_summaries_kernel(SumArgs a) {
+    extern __shared__ float sm[];
+    const int j = a.first_block + blockIdx.x;
+    const int s = blockIdx.y;
+    const int b = s / a.Hkv, g = s % a.Hkv;
+    const T *Kseg = static_cast<const T *>(a.K) + b * a.stride_b + g * a.stride_h;
+    int64_t r0, r1;
+    if (a.offsets) {
+        const int32_t *off = a.offsets + (int64_t)s * (a.nb_total + 1);
+        r0 = min(max(off[j], 0), a.L_max);
+        r1 = min(max(off[j + 1], (int32_t)r0), a.L_max);
+    } else {
+        r0 = (int64_t)j * a.S;
+        r1 = r0 + a.S;
+    }
+    char *out = static_cast<char *>(a.summ) + ((int64_t)s * a.nb_total + j) * a.row_bytes;
+    summarize_rows<T>(Kseg, a.stride_t, a.D, r0, r1, a.kind, out, sm);
+}
+
+struct AppendArgs {
+    void *K, *V;
+    const void *k_new, *v_new;
+    int32_t *cur_len;
+    void *summ;
+    int64_t stride_b, stride_h, stride_t;
+    int Hkv, D, L_max, S, nb_total, kind;
+    size_t row_bytes;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
+    extern __shared__ float sm[];
+    const int b = blockIdx.x;
+    const int n = a.cur_len[b];
+    if (n < 0 || n >= a.L_max) return;
+    T *K = static_cast<T *>(a.K) + b * a.stride_b;
+    T *V = static_cast<T *>(a.V) + b * a.stride_b;
+    const T *kn = static_cast<const T *>(a.k_new) + (int64_t)b * a.Hkv * a.D;
+    const T *vn = static_cast<const T *>(a.v_new) + (int64_t)b * a.Hkv * a.D;
+    for (int e = threadIdx.x; e < a.Hkv * a.D; e += blockDim.x) {
+        int g = e / a.D, i = e % a.D;
+        K[g * a.stride_h + (int64_t)n * a.stride_t + i] = kn[e];
+        V[g * a.stride_h + (int64_t)n * a.stride_t + i] = vn[e];
+    }
+    __syncthreads();
+    if (a.summ && a.S > 0 && (n + 1) % a.S == 0) {
+        const int j = (n + 1) / a.S - 1;
+        for (int g = 0; g < a.Hkv; ++g) {
+            const int s = b * a.Hkv + g;
+            char *out = static_cast<char *>(a.summ) + ((int64_t)s * a.nb_total + j) * a.row_bytes;
+            summarize_rows<T>(K + g * a.stride_h, a.stride_t, a.D, (int64_t)j * a.S,
+                              (int64_t)(j + 1) * a.S, a.kind, out, sm);
+            __syncthreads();
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) a.cur_len[b] = n + 1;
+}
+
+static size_t summary_smem(int kind, int D) {
+    return kind == BSA_SUM_CENTROID_NORM ? (size_t)(kNormChunk * (D + 1) + D + 1) * 4 : 16;
+}
+
+bsa_status launch_build_summaries(const bsa_kv_desc *d, const void *K, const bsa_sel_params *p,
+                                  int kind, int first_block, int n_blocks, int nb_total,
+                                  void *summ, cudaStream_t st) {
+    SumArgs a;
+    a.K = K; a.summ = summ;
+    a.offsets = p->block_size == 0 ? p->block_offsets : nullptr;
+    a.stride_b = d->stride_b; a.stride_h = d->stride_h; a.stride_t = d->stride_t;
+    a.Hkv = d->Hkv; a.D = d->D; a.L_max = d->L_max; a.S = p->block_size;
+    a.nb_total = nb_total; a.first_block = first_block; a.kind = kind;
+    a.row_bytes = summary_row_bytes(kind, d->D, d->kv_dtype);
+    dim3 grid(n_blocks, d->B * d->Hkv);
+    size_t smem = summary_smem(kind, d->D);
+    if (d->kv_dtype == BSA_BF16)
+        build_summaries_kernel<uint16_t><<<grid, 128, smem, st>>>(a);
+    else
+        build_summaries_kernel<float><<<grid, 128, smem, st>>>(a);
+    BSA_LAUNCH_CHECK();
+    return BSA_OK;
+}
+
+bsa_status launch_append(const bsa_kv_desc *d, void *K, void *V, const void *kn, const void *vn,
+                         int32_t *cur_len, const bsa_sel_params *p, int kind, int nb_total,
+                         void *summ, cudaStream_t st) {
+    AppendArgs a;
+    a.K = K; a.V = V; a.k_new = kn; a.v_new = vn; a.cur_len = cur_len;
+    a.summ = (p && p->block_size > 0) ? summ : nullptr;
+    a.stride_b = d->stride_b; a.stride_h = d->stride_h; a.stride_t = d->stride_t;
+    a.Hkv = d->Hkv; a.D = d->D; a.L_max = d->L_max; a.S = p ? p->block_size : 0;
+    a.nb_total = nb_total; a.kind = kind;
+    a.row_bytes = summary_row_bytes(kind, d->D, d->kv_dtype);
+    size_t smem = summary_smem(kind, d->D);
+    if (d->kv_dtype == BSA_BF16)
+        append_kernel<uint16_t><<<d->B, 256, smem, st>>>(a);
+    else
+        append_kernel<float><<<d->B, 256, smem, st>>>(a);
+    BSA_LAUNCH_CHECK();
+    return BSA_OK;
+}
+
+}  // namespace bsa

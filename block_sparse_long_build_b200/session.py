@@ -1,0 +1,131 @@
+"""Decode sessions: buffers and call sequence of the block-sparse decode path.
+
+A session owns the device buffers one workload needs (summaries, selection
+outputs, workspace) and issues the library calls of one decode step in
+order:
+
+    append (new K/V row; summary of a page that completes)   -- bsa_append_kv
+    select (score + top-k/budget + ranges), every `refresh` steps -- bsa_select
+    decode (split-K attention over the ranges + LSE merge)   -- bsa_decode
+
+Everything here is allocation and sequencing; the arithmetic runs in
+libbsa's kernels.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import native as N
+from .workloads import Config, Workload
+
+
+class DecodeSession:
+    def __init__(self, wl: Workload, stream: torch.cuda.Stream | None = None):
+        self.wl = wl
+        c = self.cfg = wl.cfg
+        dev = wl.device
+        self.stream = stream
+        self.desc = N.kv_desc(wl.K, c.Hq)
+        if c.block_size == 0:
+            self.sel = N.sel_params(0, c.n_blocks, wl.block_offsets, wl.kv_pos, topk=-1,
+                                    budget_tokens=c.budget_tokens, local_start=wl.local_start,
+                                    pos_limit=c.L - c.chunk)
+        else:
+            self.sel = N.sel_params(c.block_size, topk=c.topk, budget_tokens=c.budget_tokens,
+                                    sink=c.sink, window=c.window,
+                                    keep_current_block=c.keep_current)
+        self.kind = c.kind
+        nb = N.bsa_summary_blocks(self.desc, self.sel)
+        assert nb > 0
+        self.nb = nb
+        sbytes = N.bsa_summary_bytes(self.desc, self.sel, self.kind)
+        self.summaries = torch.zeros(sbytes, dtype=torch.uint8, device=dev)
+        self.max_sel = N.bsa_max_selected(self.desc, self.sel)
+        self.max_ranges = N.bsa_max_ranges(self.desc, self.sel)
+        nseg = c.B * c.Hkv
+        self.sel_blocks = torch.zeros(nseg, self.max_sel, dtype=torch.int32, device=dev)
+        self.sel_count = torch.zeros(nseg, dtype=torch.int32, device=dev)
+        self.ranges = torch.zeros(nseg, self.max_ranges, 2, dtype=torch.int32, device=dev)
+        self.n_ranges = torch.zeros(nseg, dtype=torch.int32, device=dev)
+        self.tokens_hint = self.token_bound()
+        ws = max(N.bsa_workspace_size(self.desc, self.sel, op, 0, self.tokens_hint)
+                 for op in (N.BSA_OP_SELECT, N.BSA_OP_DECODE, N.BSA_OP_APPEND))
+        self.ws = torch.zeros(ws, dtype=torch.uint8, device=dev)
+        self.out = torch.zeros(c.B, c.Hq, c.D, dtype=torch.float32, device=dev)
+        self.lse = torch.zeros(c.B, c.Hq, dtype=torch.float32, device=dev)
+        self.scale = 1.0 / math.sqrt(c.D)
+
+    def token_bound(self) -> int:
+        """Upper bound on the tokens one segment's ranges cover."""
+        c = self.cfg
+        if c.block_size == 0:
+            return c.budget_tokens + c.chunk + c.steps + 1
+        S = c.block_size
+        k = self.max_sel
+        return c.sink + c.window + k * S + S + c.refresh + 1
+
+    # ----------------------------------------------------------------- steps
+    def build_summaries(self, n_tokens: int | None = None):
+        """Summaries of every block complete in the first n_tokens rows."""
+        c = self.cfg
+        if c.block_size == 0:
+            nb = self.nb
+        else:
+            nb = (n_tokens if n_tokens is not None else c.L) // c.block_size
+        N.bsa_build_summaries(self.desc, self.wl.K, self.sel, self.kind, 0, nb, self.summaries,
+                              self.stream)
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor):
+        N.bsa_append_kv(self.desc, self.wl.K, self.wl.V, k_new, v_new, self.wl.cur_len, self.sel,
+                        self.kind, self.summaries if self.cfg.block_size > 0 else None,
+                        self.stream)
+
+    def select(self, q: torch.Tensor):
+        N.bsa_select(self.desc, q, self.summaries, self.kind, self.sel, self.wl.cur_len,
+                     self.max_sel, self.sel_blocks, self.sel_count, self.max_ranges, self.ranges,
+                     self.n_ranges, self.ws, self.stream)
+
+    def decode(self, q: torch.Tensor, out: torch.Tensor | None = None,
+               lse: torch.Tensor | None = None):
+        N.bsa_decode(self.desc, q, self.wl.K, self.wl.V, self.ranges, self.n_ranges,
+                     self.max_ranges, self.wl.cur_len, self.tokens_hint, self.scale,
+                     self.out if out is None else out, self.lse if lse is None else lse,
+                     self.ws, self.stream)
+
+    def step(self, t: int, q: torch.Tensor, k_new: torch.Tensor | None, v_new: torch.Tensor | None):
+        """Decode step t: append (when new K/V are given), select on refresh
+        steps, attend."""
+        if k_new is not None:
+            self.append(k_new, v_new)
+        if t % self.cfg.refresh == 0:
+            self.select(q)
+        self.decode(q)
+
+    # ------------------------------------------------------------ CUDA graphs
+    def capture(self):
+        """Captures one decode step into two CUDA graphs (with and without
+        the selection refresh) reading persistent input buffers q_in, k_in,
+        v_in.  Launch-bound steps then cost one graph launch each.  Run one
+        eager step first so that one-time host setup is not captured."""
+        c, dev = self.cfg, self.wl.device
+        self.q_in = torch.zeros(c.B, c.Hq, c.D, dtype=torch.float32, device=dev)
+        self.k_in = torch.zeros(c.B, c.Hkv, c.D, dtype=c.kv_dtype, device=dev)
+        self.v_in = torch.zeros_like(self.k_in)
+        self.g_refresh, self.g_plain = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_refresh):
+            self.append(self.k_in, self.v_in)
+            self.select(self.q_in)
+            self.decode(self.q_in)
+        with torch.cuda.graph(self.g_plain):
+            self.append(self.k_in, self.v_in)
+            self.decode(self.q_in)
+
+    def replay(self, t: int):
+        """Decode step t from the captured graphs (inputs already in q_in,
+        k_in, v_in)."""
+        (self.g_refresh if t % self.cfg.refresh == 0 else self.g_plain).replay()
+
+    def launches_per_step(self, t: int) -> int:
+        return 3 if t % self.cfg.refresh == 0 else 2

@@ -1,0 +1,238 @@
+/*
+ * bsa.h -- C ABI of the block-sparse long-context attention library
+ * (libbsa.so, CUDA for sm_100a).
+ *
+ * What the library computes (page title, section):
+ *   1. Per-block key summaries: mean-pooled centroids ("Module 14: Sparse
+ *      attention and long context", §14.3 MoBA -- the mean stands in for
+ *      MoBA's learned gate key), normalised centres of normalised keys
+ *      ("Semantic blocks for sparse attention", first section), or Quest-style
+ *      elementwise min/max page bounds ("Sparse attention in hybrid LLMs",
+ *      "Which parts of the context each layer reads").
+ *   2. Block scores against the current query, summed over the G query heads
+ *      of a KV head, and the top-k blocks or the blocks a token budget admits
+ *      ("Sparse long-context inference with self-indexing attention",
+ *      "Importance scores and block selection"), always with the attention
+ *      sink (§14.2), the sliding window ("Sliding window") and, MoBA-style,
+ *      the current block.
+ *   3. Exact softmax attention with GQA over only the selected tokens
+ *      (Module 14, Exercise 14.1), as split-K flash decoding with a
+ *      log-sum-exp merge.
+ *   4. Block-grouped prefill: queries that selected the same block are
+ *      gathered and contracted against that block once ("Semantic blocks for
+ *      sparse attention", "Large blocks make up for coarse selection with
+ *      speed").
+ *
+ * Conventions (all entry points):
+ *  - Pointers named d_* or documented "device" are CUDA device pointers;
+ *    descriptors and parameter structs are host pointers read during the call
+ *    only.  The caller owns every buffer, including the workspace; the
+ *    library allocates nothing and keeps no state between calls.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  BSA_OK means "validated and launched"; a failed launch returns
+ *    BSA_ERR_CUDA.  Results are ready when the stream reaches them.
+ *  - Validation is host-side and touches no device memory: a bad argument
+ *    returns BSA_ERR_ARG (or BSA_ERR_UNSUPPORTED for a valid but unbuilt
+ *    case) and launches nothing.
+ *  - KV caches are [B][Hkv][L_max][D] with element strides stride_b,
+ *    stride_h, stride_t and D contiguous; the base must be 16-byte aligned
+ *    and stride_t * element size a multiple of 16 bytes.  Query head h reads
+ *    KV head h / G, G = Hq / Hkv.
+ *  - A segment is one (batch b, KV head g) pair, index s = b * Hkv + g.
+ *  - Token ranges are half-open [start, end) row indices into a segment.
+ *  - Workspace: size from bsa_workspace_size(); it must be zero-filled once
+ *    before its first use.  Every call leaves its counters at zero again, so
+ *    one workspace can serve any sequence of calls on one stream.  Calls that
+ *    may overlap on the GPU need separate workspaces.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *bsa_stream_t;   /* == cudaStream_t */
+
+typedef enum {
+    BSA_OK = 0,
+    BSA_ERR_ARG = -1,          /* invalid argument; nothing launched            */
+    BSA_ERR_UNSUPPORTED = -2,  /* valid, but a shape this build does not cover  */
+    BSA_ERR_CUDA = -3,         /* a CUDA call or launch failed                  */
+    BSA_ERR_WORKSPACE = -4,    /* workspace missing, misaligned or too small    */
+    BSA_ERR_TIMEOUT = -5       /* a bounded device-side wait gave up            */
+} bsa_status;
+
+typedef enum {
+    BSA_SUM_CENTROID = 0,       /* fp32 mean of the block's keys                  */
+    BSA_SUM_CENTROID_NORM = 1,  /* fp32 normalised mean of normalised keys        */
+    BSA_SUM_MINMAX = 2          /* elementwise min then max, in the cache dtype   */
+} bsa_summary_kind;
+
+typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype;
+
+typedef enum { BSA_OP_SELECT = 0, BSA_OP_DECODE = 1, BSA_OP_PREFILL = 2, BSA_OP_APPEND = 3 } bsa_op;
+
+/* KV-cache geometry. */
+typedef struct {
+    int32_t B, Hq, Hkv, D;     /* D in {64, 128}; Hq a multiple of Hkv            */
+    int32_t kv_dtype;          /* bsa_dtype of K and V                             */
+    int32_t L_max;             /* rows per segment                                 */
+    int64_t stride_b, stride_h, stride_t;   /* element strides of K and V          */
+} bsa_kv_desc;
+
+/* Selection parameters, in the pages' terms.
+ *
+ * Fixed blocks (block_size = S > 0): block j of a segment is rows
+ * [j*S, (j+1)*S).  For a cache of n tokens (the newest, the current token,
+ * is row n-1) the forced set is
+ *     sink     [0, min(sink, n))
+ *     window   [max(0, n - window), n)      -- the window counts the current token
+ *     current  [floor((n-1)/S)*S, n)        -- when keep_current_block != 0
+ * The candidates are the complete blocks ((j+1)*S <= n) not wholly inside the
+ * forced set; k = topk, or budget_tokens / S when topk < 0.  The k candidates
+ * with the highest scores are selected, the lower block index first among
+ * equal fp32 scores.
+ *
+ * Variable blocks (block_size = 0): block j of segment s is rows
+ * [block_offsets[s][j], block_offsets[s][j+1]) of a store whose rows are
+ * sorted by original position inside each block (kv_pos[s][row]).  A block's
+ * visible rows are those with kv_pos < pos_limit (a prefix of the block);
+ * blocks with none are not candidates.  Blocks are taken greedily in rank
+ * order while their visible rows fit in what is left of budget_tokens.  The
+ * forced set is the position-ordered local part [local_start, n). */
+typedef struct {
+    int32_t block_size;
+    int32_t n_blocks;               /* variable blocks: blocks per segment        */
+    const int32_t *block_offsets;   /* device [B*Hkv][n_blocks+1]; variable only   */
+    const int32_t *kv_pos;          /* device [B*Hkv][L_max]; variable only        */
+    int32_t topk;                   /* >= 0: blocks; < 0: use budget_tokens        */
+    int32_t budget_tokens;
+    int32_t sink, window;
+    int32_t keep_current_block;
+    int32_t local_start;            /* variable only                               */
+    int32_t pos_limit;              /* variable only                               */
+} bsa_sel_params;
+
+/* Blocks per segment the summaries buffer holds: ceil(L_max / S) for fixed
+ * blocks, n_blocks for variable ones. */
+BSA_API int32_t bsa_summary_blocks(const bsa_kv_desc *desc, const bsa_sel_params *sel);
+
+/* Bytes of the summaries buffer: segments x blocks x (D fp32 for the centroid
+ * kinds | 2 x D cache elements, min row then max row, for MINMAX). */
+BSA_API size_t bsa_summary_bytes(const bsa_kv_desc *desc, const bsa_sel_params *sel,
+                         bsa_summary_kind kind);
+
+/* Largest selected-block list and range list a segment can need. */
+BSA_API int32_t bsa_max_selected(const bsa_kv_desc *desc, const bsa_sel_params *sel);
+BSA_API int32_t bsa_max_ranges(const bsa_kv_desc *desc, const bsa_sel_params *sel);
+
+/* Workspace bytes for `op`.  n_queries: query rows per call for
+ * BSA_OP_PREFILL (ignored otherwise); tokens_hint: for BSA_OP_DECODE, an
+ * upper bound on the tokens any segment's ranges cover (sizes the split-K
+ * grid; bsa_decode must get the same value).  0 on invalid arguments. */
+BSA_API size_t bsa_workspace_size(const bsa_kv_desc *desc, const bsa_sel_params *sel, int op,
+                          int32_t n_queries, int32_t tokens_hint);
+
+/* Builds the summaries of blocks [first_block, first_block + n_blocks) of
+ * every segment ("Module 14", §14.3; "Semantic blocks...", first section;
+ * "Sparse attention in hybrid LLMs", "Which parts of the context each layer
+ * reads").  K: device cache.  summaries: device buffer of
+ * bsa_summary_bytes().  Fixed blocks must lie inside L_max; the centroid of
+ * an empty variable block is zero.  Arithmetic: fp32 sums in row order,
+ * then a correctly rounded division by the row count; the normalised kind
+ * divides each key by its fp32 norm (fma chain over the dimensions, then a
+ * correctly rounded square root) first and the mean by its norm after. */
+BSA_API bsa_status bsa_build_summaries(const bsa_kv_desc *desc, const void *K,
+                               const bsa_sel_params *sel, bsa_summary_kind kind,
+                               int32_t first_block, int32_t n_blocks, void *summaries,
+                               bsa_stream_t stream);
+
+/* Scores every candidate block of every segment against the group's queries
+ * and selects (rules above).  q: device fp32 [B][Hq][D].  cur_len: device
+ * int32 [B], tokens in each sequence's cache.  Outputs, all device:
+ *   sel_blocks [B*Hkv][max_selected]  selected block ids ascending
+ *   sel_count  [B*Hkv]
+ *   ranges     [B*Hkv][max_ranges][2] disjoint ascending token ranges that
+ *                                     cover forced set and selected blocks
+ *   n_ranges   [B*Hkv]
+ * max_selected / max_ranges must be at least bsa_max_selected() /
+ * bsa_max_ranges().  Score arithmetic (fixed, so that selections can be
+ * compared bit for bit): per query head h an fp32 fma chain over
+ * i = 0..D-1 of q_h[i] * x[i], x = the centroid, or for MINMAX
+ * x[i] = q_h[i] >= 0 ? max[i] : min[i] (the larger of q*min and q*max);
+ * head scores summed in head order. */
+BSA_API bsa_status bsa_select(const bsa_kv_desc *desc, const float *q, const void *summaries,
+                      bsa_summary_kind kind, const bsa_sel_params *sel, const int32_t *cur_len,
+                      int32_t max_selected, int32_t *sel_blocks, int32_t *sel_count,
+                      int32_t max_ranges, int32_t *ranges, int32_t *n_ranges,
+                      void *ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Exact softmax attention of every query head over its segment's ranges
+ * (Module 14, Exercise 14.1, restricted to the selected tokens):
+ *   out[b][h] = sum_j softmax_j(scale * q[b][h] . K[j]) V[j],
+ *   lse[b][h] = log sum_j exp(scale * q[b][h] . K[j])      (natural log)
+ * over the rows of ranges[s][0..n_ranges[s]), s = b*Hkv + h/G.  The last
+ * range of each segment is extended to end at cur_len[b] when that is
+ * larger: between selection refreshes the window keeps growing ("Sparse
+ * attention in hybrid LLMs", refresh every 32 steps).  Rows are clamped to
+ * [0, L_max).  q: device fp32 [B][Hq][D]; out: device fp32 [B][Hq][D];
+ * lse: device fp32 [B][Hq] (may be NULL).  A segment with no rows gives
+ * out = 0, lse = -inf.  tokens_hint: as for bsa_workspace_size(); any actual
+ * count is handled, the hint only sizes the grid.  fp32 accumulation over
+ * bf16 or fp32 K/V. */
+BSA_API bsa_status bsa_decode(const bsa_kv_desc *desc, const float *q, const void *K, const void *V,
+                      const int32_t *ranges, const int32_t *n_ranges, int32_t max_ranges,
+                      const int32_t *cur_len, int32_t tokens_hint, float scale,
+                      float *out, float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* One decode step's cache bookkeeping: writes k_new, v_new (device,
+ * [B][Hkv][D] in the cache dtype) at row cur_len[b] of every segment, and
+ * when that row completes a fixed block, builds that block's summary with the
+ * same arithmetic as bsa_build_summaries (summaries may be NULL to skip);
+ * then increments cur_len[b].  Sequences whose cache is full (cur_len[b] ==
+ * L_max) are left unchanged. */
+BSA_API bsa_status bsa_append_kv(const bsa_kv_desc *desc, void *K, void *V, const void *k_new,
+                         const void *v_new, int32_t *cur_len, const bsa_sel_params *sel,
+                         bsa_summary_kind kind, void *summaries, bsa_stream_t stream);
+
+/* Block-grouped prefill for variable (semantic) blocks, batch 1.
+ * Query row i sits at position q_pos0 + i and reads
+ *   (a) the positions [pos_limit, q_pos0 + i] densely and causally from the
+ *       position-ordered cache K_pos / V_pos (pos_desc geometry), and
+ *   (b) the visible prefixes (kv_pos < pos_limit) of the blocks its group
+ *       selects from the block-ordered store K / V (desc geometry) with the
+ *       variable-block rules above (budget_tokens, CENTROID_NORM summaries).
+ * Selection is per (query row, KV head); the queries that selected one block
+ * are gathered and contracted against it together on the tensor cores, and
+ * the partial results are merged per query by log-sum-exp.
+ * Q: device bf16 [Tq][Hq][D]; out: device fp32 [Tq][Hq][D]; lse: device fp32
+ * [Tq][Hq] (may be NULL).  pos_limit = 0 makes the call dense causal
+ * attention over [0, q_pos0 + i]. */
+BSA_API bsa_status bsa_prefill_grouped(const bsa_kv_desc *desc, const void *K, const void *V,
+                               const bsa_sel_params *sel, const void *summaries,
+                               const bsa_kv_desc *pos_desc, const void *K_pos, const void *V_pos,
+                               const void *Q, int32_t q_pos0, int32_t Tq, float scale,
+                               float *out, float *lse, void *ws, size_t ws_bytes,
+                               bsa_stream_t stream);
+
+/* Static text for a status code. */
+BSA_API const char *bsa_status_string(bsa_status status);
+
+/* Library ABI version (major * 100 + minor). */
+BSA_API int32_t bsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */
