@@ -29,6 +29,7 @@ constexpr int kDecWarps = 4;
 constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kBoxBytes = kPiece * 128;            // 16 rows x 64 bf16
 constexpr int kHalfBytes = kDecWarps * kBoxBytes;  // one 64-column half of a tile
+constexpr int kPieceCap = 512;                     // CTA piece table held in shared memory
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kNegInf = -__builtin_huge_valf();
 
@@ -120,9 +121,11 @@ __device__ __forceinline__ int2 piece_rows(int p, const int *rs, const int *re, 
 
 // Combines the per-warp partials (wm, wl, wo) of this CTA and writes either
 // the final output (nsplit == 1) or the split partial, merging when this is
-// the last CTA of the segment.
+// the last CTA of the segment.  `scr` is shared scratch of at least
+// 2 * nsplit * G floats that does not alias wm / wl / wo.
 __device__ void finish(const DecArgs &a, int s, int b, int g, int c, const float *wm,
-                       const float *wl, const float *wo, float *sml /* [2*kMaxG] */) {
+                       const float *wl, const float *wo, float *sml /* [2*kMaxG] */,
+                       float *scr) {
     const int G = a.G, D = a.D;
     __shared__ int is_last;
     if (threadIdx.x < G) {
@@ -163,29 +166,38 @@ __device__ void finish(const DecArgs &a, int s, int b, int g, int c, const float
     __syncthreads();
     if (!is_last) return;
     __threadfence();
+    // every split's (m, l) into shared memory with independent loads
+    const int nsg = a.nsplit * G;
+    const float2 *pml = a.part_ml + (int64_t)s * nsg;
+    float *sm_m = scr, *sm_w = scr + nsg;
+    for (int i = threadIdx.x; i < nsg; i += blockDim.x) {
+        float2 ml = __ldcg(&pml[i]);
+        sm_m[i] = ml.x;
+        sm_w[i] = ml.y;
+    }
+    __syncthreads();
     if (threadIdx.x < G) {
         const int h = threadIdx.x;
         float M = kNegInf;
-        for (int k = 0; k < a.nsplit; ++k)
-            M = fmaxf(M, __ldcg(&a.part_ml[((int64_t)s * a.nsplit + k) * G + h]).x);
+        for (int k = 0; k < a.nsplit; ++k) M = fmaxf(M, sm_m[k * G + h]);
         float L = 0.0f;
         for (int k = 0; k < a.nsplit; ++k) {
-            float2 ml = __ldcg(&a.part_ml[((int64_t)s * a.nsplit + k) * G + h]);
-            if (ml.x != kNegInf) L += ml.y * exp2f(ml.x - M);
+            const float mk = sm_m[k * G + h];
+            const float f = mk != kNegInf ? exp2f(mk - M) : 0.0f;
+            L += sm_w[k * G + h] * f;
+            sm_w[k * G + h] = f;   // now the split's scale factor
         }
         sml[2 * h] = M;
         sml[2 * h + 1] = L;
     }
     __syncthreads();
+    const float *po = a.part_o + (int64_t)s * nsg * D;
     for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
         const int h = e / D, d = e % D;
         const float M = sml[2 * h], L = sml[2 * h + 1];
         float O = 0.0f;
-        for (int k = 0; k < a.nsplit; ++k) {
-            float mk = __ldcg(&a.part_ml[((int64_t)s * a.nsplit + k) * G + h]).x;
-            if (mk != kNegInf)
-                O += __ldcg(&a.part_o[(((int64_t)s * a.nsplit + k) * G + h) * D + d]) * exp2f(mk - M);
-        }
+#pragma unroll 8
+        for (int k = 0; k < a.nsplit; ++k) O += __ldcg(&po[(k * G + h) * D + d]) * sm_w[k * G + h];
         a.out[(qrow + h) * D + d] = L > 0.0f ? O / L : 0.0f;
         if (d == 0 && a.lse) a.lse[qrow + h] = L > 0.0f ? (M + log2f(L)) * kLn2 : kNegInf;
     }
@@ -202,7 +214,8 @@ struct TcSmem {
     static constexpr int kInfo = kRing;                        // int2 [STAGES][4]
     static constexpr int kBars = kInfo + STAGES * kDecWarps * 8;
     static constexpr int kMisc = kBars + STAGES * 8;           // float sml[2*kMaxG], int tmp[33]
-    static constexpr int kRanges = kMisc + 2 * kMaxG * 4 + 36 * 4;
+    static constexpr int kPtab = kMisc + 2 * kMaxG * 4 + 36 * 4;   // int2 [kPieceCap]
+    static constexpr int kRanges = kPtab + kPieceCap * 8;
     static constexpr int bytes(int max_ranges) { return kRanges + (3 * max_ranges + 1) * 4 + 1024; }
 };
 
@@ -243,6 +256,13 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     const int n_my = max(0, last - first);
     const int tiles = (n_my + kDecWarps - 1) / kDecWarps;
 
+    // this CTA's pieces, looked up in parallel once (the producer then only
+    // reads the table)
+    int2 *ptab = reinterpret_cast<int2 *>(dsm + L::kPtab);
+    for (int i = tid; i < min(n_my, kPieceCap); i += kDecThreads)
+        ptab[i] = piece_rows(first + i, rs, re, ps, nr);
+    __syncthreads();
+
     auto stage_ptr = [&](int st, int part) {   // part: 0..NH-1 K halves, NH..2NH-1 V halves
         return dsm + st * L::kStageBytes + part * kHalfBytes;
     };
@@ -252,7 +272,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 #pragma unroll
         for (int w = 0; w < kDecWarps; ++w) {
             int p = first + t * kDecWarps + w;
-            pr[w] = p < last ? piece_rows(p, rs, re, ps, nr) : make_int2(0, 0);
+            pr[w] = p >= last ? make_int2(0, 0)
+                    : (p - first < kPieceCap ? ptab[p - first] : piece_rows(p, rs, re, ps, nr));
             info[st * kDecWarps + w] = pr[w];
             np += pr[w].y > 0;
         }
@@ -405,7 +426,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         wo[(warp * kMaxG + gid) * D + d + 1] = o[nt][1] + o[nt][3];
     }
     __syncthreads();
-    finish(a, s, b, g, c, wm, wl, wo, sml);
+    finish(a, s, b, g, c, wm, wl, wo, sml, reinterpret_cast<float *>(dsm + 32768));
 }
 
 // ======================================================================
@@ -423,6 +444,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_generic_kernel(DecArgs a) 
     int *rs = tmp + 36;
     int *re = rs + a.max_ranges;
     int *ps = re + a.max_ranges;
+    float *mscr = reinterpret_cast<float *>(ps + a.max_ranges + 1);   // [2 * nsplit * G]
 
     const int c = blockIdx.x, s = blockIdx.y;
     const int b = s / a.Hkv, g = s % a.Hkv;
@@ -487,7 +509,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_generic_kernel(DecArgs a) 
         for (int k = 0; k < PER; ++k) wo[(warp * kMaxG + h) * D + lane + 32 * k] = o[h][k];
     }
     __syncthreads();
-    finish(a, s, b, g, c, wm, wl, wo, sml);
+    finish(a, s, b, g, c, wm, wl, wo, sml, mscr);
 }
 
 // ======================================================================
@@ -550,7 +572,8 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
         }
     } else {
         const size_t smem = (size_t)(2 * kDecWarps * kMaxG + kDecWarps * kMaxG * d->D + 2 * kMaxG) * 4 +
-                            36 * 4 + (size_t)(3 * max_ranges + 1) * 4;
+                            36 * 4 + (size_t)(3 * max_ranges + 1) * 4 +
+                            (size_t)2 * a.nsplit * a.G * 4;
         auto go = [&](auto kern) -> bsa_status {
             if (smem > 48 * 1024)
                 BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));

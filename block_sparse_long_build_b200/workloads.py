@@ -167,7 +167,7 @@ class Workload:
         self.cur_len = torch.full((B,), c.L, dtype=torch.int32, device=dev)
         if c.n_clusters:
             self.centres = _unit(torch.randn(B, H, c.n_clusters, D, generator=g, device=dev))
-        if c.n_needles and c.name != "tiny":
+        if c.name == "moba":
             self.needle_dir = _unit(torch.randn(B, H, D, generator=g, device=dev))
         for b in range(B):
             for h in range(H):
@@ -187,13 +187,14 @@ class Workload:
             needle = 3.0 * _unit(self.q0[0, 0])
             self.K[0, 0, pos] = needle.to(c.kv_dtype)
             self.needle_pos = pos
-        elif c.n_needles:
+        elif c.name == "moba":
             # needle blocks among the complete blocks before the current one
             S = c.block_size
-            nb = c.L // S - 1
+            nb = max(c.L // S - 1, 0)
+            n_need = min(c.n_needles, nb)
             self.needle_blocks = torch.stack([
-                torch.randperm(nb, generator=g, device=dev)[: c.n_needles] for _ in range(B * H)
-            ]).view(B, H, c.n_needles)
+                torch.randperm(max(nb, 1), generator=g, device=dev)[:n_need] for _ in range(B * H)
+            ]).view(B, H, n_need)
             for b in range(B):
                 for h in range(H):
                     add = (math.sqrt(D) * self.needle_dir[b, h]).to(torch.float32)
@@ -248,7 +249,7 @@ class Workload:
             return self.q0.clone()
         g = _gen(dev, c.seed + 1 + step)
         eps = torch.randn(c.B, c.Hq, c.D, generator=g, device=dev)
-        if c.n_needles:
+        if c.name == "moba":
             aim = self.needle_dir
         else:
             n_c = self.centres.shape[2]
