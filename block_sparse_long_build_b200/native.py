@@ -23,7 +23,8 @@ BSA_OP_SELECT, BSA_OP_DECODE, BSA_OP_PREFILL, BSA_OP_APPEND = 0, 1, 2, 3
 
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_summary_blocks", "bsa_summary_bytes",
             "bsa_max_selected", "bsa_max_ranges", "bsa_workspace_size", "bsa_build_summaries",
-            "bsa_select", "bsa_decode", "bsa_append_kv", "bsa_prefill_grouped")
+            "bsa_select", "bsa_decode", "bsa_decode_noalloc", "bsa_append_kv",
+            "bsa_prefill_grouped")
 
 
 class BsaError(RuntimeError):
@@ -73,6 +74,7 @@ def lib() -> ctypes.CDLL:
             "bsa_select": (ctypes.c_int, [pd, P, P, ctypes.c_int, pp, P, I32, P, P, I32, P, P, P,
                                           SZ, P]),
             "bsa_decode": (ctypes.c_int, [pd, P, P, P, P, P, I32, P, I32, F, P, P, P, SZ, P]),
+            "bsa_decode_noalloc": (ctypes.c_int, [pd, P, P, P, P, P, I32, P, I32, F, P, P, P]),
             "bsa_append_kv": (ctypes.c_int, [pd, P, P, P, P, P, pp, ctypes.c_int, P, P]),
             "bsa_prefill_grouped": (ctypes.c_int, [pd, P, P, pp, P, pd, P, P, P, I32, I32, F, P, P,
                                                    P, SZ, P]),
@@ -169,6 +171,16 @@ def bsa_decode(desc, q, K, V, ranges, n_ranges, max_ranges, cur_len, tokens_hint
            lib().bsa_decode(ctypes.byref(desc), _p(q), _p(K), _p(V), _p(ranges), _p(n_ranges),
                             max_ranges, _p(cur_len), tokens_hint, scale, _p(out), _p(lse), _p(ws),
                             ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def bsa_decode_noalloc(desc, q, K, V, ranges, n_ranges, max_ranges, cur_len, tokens_hint, scale,
+                       out, lse, stream=None):
+    """bsa_decode with the library's built-in scratch instead of a workspace,
+    for callers that cannot allocate one (see include/bsa.h)."""
+    _check("bsa_decode_noalloc",
+           lib().bsa_decode_noalloc(ctypes.byref(desc), _p(q), _p(K), _p(V), _p(ranges),
+                                    _p(n_ranges), max_ranges, _p(cur_len), tokens_hint, scale,
+                                    _p(out), _p(lse), _stream(stream)))
 
 
 def bsa_append_kv(desc, K, V, k_new, v_new, cur_len, sel, kind, summaries, stream=None):

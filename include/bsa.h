@@ -195,6 +195,32 @@ BSA_API bsa_status bsa_decode(const bsa_kv_desc *desc, const float *q, const voi
                       const int32_t *cur_len, int32_t tokens_hint, float scale,
                       float *out, float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream);
 
+/* bsa_decode without a caller workspace.  The source pages have no
+ * counterpart: this is a deployment convenience, not part of the method.
+ *
+ * For callers that cannot allocate device memory for a workspace -- code
+ * embedded in an application that owns every device allocation and forbids
+ * new ones once it is running (fixed budgets, pre-planned pools), or code
+ * that cannot afford cudaMalloc's implicit synchronisation.  It computes
+ * exactly what bsa_decode computes, with the same arguments minus ws and
+ * ws_bytes, using a 4 MiB scratch array built into the library (a
+ * file-scope device array: every GPU that loads the library holds it until
+ * the process exits).  It allocates nothing.
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress (with that device current) and caches it; make
+ *    that first call before any stream capture.
+ *  - Every call shares the one array and zeroes its counters first, on
+ *    `stream`.  Calls that may overlap on the GPU (other streams, other host
+ *    threads) race on it and give wrong results: serialise them.
+ *  - A problem that needs more scratch than 4 MiB (what bsa_workspace_size
+ *    reports for BSA_OP_DECODE with these sizes) is rejected with
+ *    BSA_ERR_WORKSPACE before anything is launched. */
+BSA_API bsa_status bsa_decode_noalloc(const bsa_kv_desc *desc, const float *q, const void *K,
+                                      const void *V, const int32_t *ranges,
+                                      const int32_t *n_ranges, int32_t max_ranges,
+                                      const int32_t *cur_len, int32_t tokens_hint, float scale,
+                                      float *out, float *lse, bsa_stream_t stream);
+
 /* One decode step's cache bookkeeping: writes k_new, v_new (device,
  * [B][Hkv][D] in the cache dtype) at row cur_len[b] of every segment, and
  * when that row completes a fixed block, builds that block's summary with the
