@@ -13,7 +13,7 @@ bsa_status launch_append(const bsa_kv_desc *, void *, void *, const void *, cons
                          const bsa_sel_params *, int, int, void *, cudaStream_t);
 bsa_status launch_select(const bsa_kv_desc *, const float *, const void *, int,
                          const bsa_sel_params *, const int32_t *, int, int, int32_t *, int32_t *,
-                         int, int32_t *, int32_t *, uint32_t *, int32_t *, uint32_t *,
+                         int, int32_t *, int32_t *, uint32_t *, int32_t *, uint32_t *, uint32_t *,
                          cudaStream_t);
 bsa_status launch_decode(const bsa_kv_desc *, const float *, const void *, const void *,
                          const int32_t *, const int32_t *, int, const int32_t *, int, float, float *,
@@ -72,6 +72,20 @@ bool make_kv_tmap(CUtensorMap *map, const bsa_kv_desc *d, const void *base, int 
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool make_rows_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int esize, const void *base,
+                    int64_t cols, int64_t rows, int64_t row_bytes, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / esize), (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -228,7 +242,8 @@ bsa_status bsa_select(const bsa_kv_desc *d, const float *q, const void *summarie
     uint32_t *keys = reinterpret_cast<uint32_t *>(scr);
     int32_t *vis = reinterpret_cast<int32_t *>(scr + align_up(nseg * nb * 4, 256));
     return launch_select(d, q, summaries, kind, p, cur_len, nb, max_sel, sel_blocks, sel_count, max_r,
-                         ranges, n_ranges, keys, vis, cnt, (cudaStream_t)stream);
+                         ranges, n_ranges, keys, vis, cnt, static_cast<uint32_t *>(ws),
+                         (cudaStream_t)stream);
 }
 
 bsa_status bsa_decode(const bsa_kv_desc *d, const float *q, const void *K, const void *V,
@@ -238,6 +253,7 @@ bsa_status bsa_decode(const bsa_kv_desc *d, const float *q, const void *K, const
     if (!desc_ok(d)) return BSA_ERR_ARG;
     if (!q || !K || !V || !ranges || !n_ranges || !cur_len || !out) return BSA_ERR_ARG;
     if (!aligned16(K) || !aligned16(V) || !aligned16(q)) return BSA_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(ranges) % 8) return BSA_ERR_ARG;
     if (max_r < 1 || max_r > 4096 || tokens_hint < 0) return BSA_ERR_ARG;
     if (d->Hq / d->Hkv > kMaxG) return BSA_ERR_UNSUPPORTED;
     if (!(scale > 0.0f) || scale != scale) return BSA_ERR_ARG;

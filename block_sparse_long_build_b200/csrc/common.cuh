@@ -129,7 +129,101 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// CTA-wide scans (blockDim.x a multiple of 32, at most 1024).  `tmp` holds at
+// least 33 ints (or floats).  Every thread of the CTA must call them.
+__device__ __forceinline__ int cta_excl_sum(int v, int *tmp, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+    }
+    if (lane == 31) tmp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? tmp[lane] : 0, wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            int t = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += t;
+        }
+        if (lane < nw) tmp[lane] = wi - w;
+        if (lane == 31) tmp[32] = wi;
+    }
+    __syncthreads();
+    const int res = incl - v + tmp[warp];
+    *total = tmp[32];
+    __syncthreads();
+    return res;
+}
+
+// Inclusive prefix maximum; *total receives the CTA-wide maximum.
+__device__ __forceinline__ int cta_incl_max(int v, int *tmp, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl = max(incl, t);
+    }
+    if (lane == 31) tmp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int lo = -0x7fffffff - 1;
+        int w = lane < nw ? tmp[lane] : lo, wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            int t = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi = max(wi, t);
+        }
+        int ex = __shfl_up_sync(0xffffffffu, wi, 1);
+        if (lane < nw) tmp[lane] = lane == 0 ? lo : ex;
+        if (lane == 31) tmp[32] = wi;
+    }
+    __syncthreads();
+    const int res = max(incl, tmp[warp]);
+    *total = tmp[32];
+    __syncthreads();
+    return res;
+}
+
+// 2-D tiled TMA load (no multicast) completing on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Programmatic dependent launch: a kernel launched with launch_pdl() may be
+// scheduled before the previous kernel on its stream has finished; it must
+// call pdl_wait() before touching anything that kernel writes.  pdl_trigger()
+// lets this kernel's own dependents be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- host side
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Error-code plumbing for the entry points.
 #define BSA_CUDA_TRY(expr)                                          \
     do {                                                            \
@@ -152,6 +246,12 @@ int num_sms();
 // Encodes a 4-D bf16 tensor map over a KV cache: dims (D, L_max, Hkv, B),
 // box (64, rows, 1, 1), 128-byte swizzle, zero fill out of bounds.
 bool make_kv_tmap(CUtensorMap *map, const bsa_kv_desc *desc, const void *base, int box_rows);
+
+// Encodes a 2-D tensor map over `rows` rows of `row_bytes` bytes holding
+// `cols` elements of `dtype`; box = (128 bytes of columns) x box_rows,
+// 128-byte swizzle, zero fill out of bounds.
+bool make_rows_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int esize, const void *base,
+                    int64_t cols, int64_t rows, int64_t row_bytes, int box_rows);
 
 // Workspace layout shared by all ops: a zeroed counter area first, then the
 // op's scratch.

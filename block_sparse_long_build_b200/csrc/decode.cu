@@ -6,20 +6,25 @@
 // to the selected set), GQA: query head h reads KV head h / G.
 //
 // Work decomposition.  A segment's ranges are cut into pieces of 16 rows
-// (one TMA box each; a range's last piece may be short).  The pieces are
-// split evenly over `nsplit` CTAs; a CTA walks its pieces in tiles of 4, one
-// piece per warp.  Every CTA writes an unnormalised partial (m, l, o) in
-// base 2; the last CTA of a segment to finish (an atomic counter, reset
-// afterwards) merges the partials in split order, so the result does not
-// depend on scheduling.
+// (one TMA box row-block each; a range's last piece may be short).  The
+// pieces are split evenly over `nsplit` CTAs; inside a CTA, warp w takes the
+// pieces w, w+4, w+8, ... and streams them through its own shared-memory ring
+// (lane 0 issues the loads, one mbarrier per stage, no CTA-wide barrier in
+// the loop).  Each CTA combines its warps and writes an unnormalised partial
+// (m, l, o) in base 2; lse_merge_kernel, launched as a programmatic dependent
+// of the decode grid, merges the partials in split order, so the result does
+// not depend on scheduling.  With one split the decode writes the output.
 //
-// Tensor-core path (bf16 K/V, D in {64, 128}, G <= 8): K and V pieces are
-// brought into a multi-stage shared-memory ring by 4-D tiled TMA loads with
-// 128-byte swizzle (no multicast), one elected thread issuing and an
-// mbarrier per stage.  All G query heads of the group share every K/V byte:
-// the 16 MMA rows hold q_hi (rows 0-7) and q_lo = q - q_hi (rows 8-15), so
-// one m16n8k16 bf16 MMA gives the logits to ~2^-17 relative; the softmax
-// weights are split the same way for P.V.  Accumulation is fp32.
+// Tensor-core path (bf16 K/V, D in {64, 128}, G <= 8): pieces arrive by 4-D
+// tiled TMA loads with 128-byte swizzle (no multicast).  All G query heads of
+// the group share every K/V byte: the 16 MMA rows hold q_hi (rows 0-7) and
+// q_lo = q - q_hi (rows 8-15), so one m16n8k16 bf16 MMA gives the logits to
+// ~2^-17 relative; the softmax weights are split the same way for P.V.
+// Accumulation is fp32.
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include "common.cuh"
 
 namespace bsa {
@@ -30,6 +35,7 @@ constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kBoxBytes = kPiece * 128;            // 16 rows x 64 bf16
 constexpr int kHalfBytes = kDecWarps * kBoxBytes;  // one 64-column half of a tile
 constexpr int kPieceCap = 512;                     // CTA piece table held in shared memory
+constexpr int kMaxClusterSplits = 16;              // splits merged inside one cluster
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kNegInf = -__builtin_huge_valf();
 
@@ -82,16 +88,25 @@ __device__ __forceinline__ int block_excl_scan(int v, int *tmp, int *total) {
 // of pieces; *nr_out the number of ranges.
 __device__ int load_ranges(const DecArgs &a, int s, int b, int *rs, int *re, int *ps, int *tmp,
                            int *nr_out) {
-    const int nr = min(max(a.n_ranges[s], 0), a.max_ranges);
+    // One round trip: the count, the length and every slot of the range table
+    // are requested together (slots past the count are ignored).
     const int32_t *R = a.ranges + (int64_t)s * a.max_ranges * 2;
-    const int cl = min(max(a.cur_len[b], 0), a.L_max);
+    const int nr_raw = a.n_ranges[s];
+    const int cl_raw = a.cur_len[b];
+    for (int r = threadIdx.x; r < a.max_ranges; r += blockDim.x) {
+        const int2 v = *reinterpret_cast<const int2 *>(R + 2 * r);
+        rs[r] = v.x;
+        re[r] = v.y;
+    }
+    const int nr = min(max(nr_raw, 0), a.max_ranges);
+    const int cl = min(max(cl_raw, 0), a.L_max);
     int carry = 0;
     for (int base = 0; base < nr; base += blockDim.x) {
         const int r = base + threadIdx.x;
         int cnt = 0;
         if (r < nr) {
-            int lo = min(max(R[2 * r], 0), a.L_max);
-            int hi = min(max(R[2 * r + 1], lo), a.L_max);
+            int lo = min(max(rs[r], 0), a.L_max);
+            int hi = min(max(re[r], lo), a.L_max);
             if (r == nr - 1 && cl > hi) hi = cl;
             rs[r] = lo;
             re[r] = hi;
@@ -120,14 +135,10 @@ __device__ __forceinline__ int2 piece_rows(int p, const int *rs, const int *re, 
 }
 
 // Combines the per-warp partials (wm, wl, wo) of this CTA and writes either
-// the final output (nsplit == 1) or the split partial, merging when this is
-// the last CTA of the segment.  `scr` is shared scratch of at least
-// 2 * nsplit * G floats that does not alias wm / wl / wo.
+// the final output (nsplit == 1) or the split's partial for the merge kernel.
 __device__ void finish(const DecArgs &a, int s, int b, int g, int c, const float *wm,
-                       const float *wl, const float *wo, float *sml /* [2*kMaxG] */,
-                       float *scr) {
+                       const float *wl, const float *wo, float *sml /* [2*kMaxG] */) {
     const int G = a.G, D = a.D;
-    __shared__ int is_last;
     if (threadIdx.x < G) {
         const int h = threadIdx.x;
         float M = kNegInf;
@@ -159,71 +170,143 @@ __device__ void finish(const DecArgs &a, int s, int b, int g, int c, const float
             if (d == 0) a.part_ml[((int64_t)s * a.nsplit + c) * G + h] = make_float2(M, sml[2 * h + 1]);
         }
     }
-    if (a.nsplit == 1) return;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) is_last = atomicAdd(&a.counters[s], 1u) == (unsigned)(a.nsplit - 1);
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    // every split's (m, l) into shared memory with independent loads
-    const int nsg = a.nsplit * G;
-    const float2 *pml = a.part_ml + (int64_t)s * nsg;
-    float *sm_m = scr, *sm_w = scr + nsg;
-    for (int i = threadIdx.x; i < nsg; i += blockDim.x) {
-        float2 ml = __ldcg(&pml[i]);
-        sm_m[i] = ml.x;
-        sm_w[i] = ml.y;
-    }
-    __syncthreads();
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+
+// Reads a float from the shared memory of CTA `rank` of this cluster at the
+// address `local` has in this CTA.
+__device__ __forceinline__ float ld_peer(uint32_t local, uint32_t rank) {
+    uint32_t remote;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+// The split-K merge inside a thread-block cluster (the segment's splits):
+// every CTA leaves its partial (m, l per head in sml, o in `part`) in its own
+// shared memory; after a cluster barrier each CTA merges a slice of the
+// output elements reading its peers' partials through distributed shared
+// memory, in split order; a second barrier keeps the partials alive until
+// every peer has read them.  All threads of all CTAs reach both barriers.
+__device__ void cluster_finish(const DecArgs &a, int b, int g, const float *wm, const float *wl,
+                               const float *wo, float *sml, float *part) {
+    const int G = a.G, D = a.D;
     if (threadIdx.x < G) {
         const int h = threadIdx.x;
         float M = kNegInf;
-        for (int k = 0; k < a.nsplit; ++k) M = fmaxf(M, sm_m[k * G + h]);
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wm[w * kMaxG + h]);
         float L = 0.0f;
-        for (int k = 0; k < a.nsplit; ++k) {
-            const float mk = sm_m[k * G + h];
-            const float f = mk != kNegInf ? exp2f(mk - M) : 0.0f;
-            L += sm_w[k * G + h] * f;
-            sm_w[k * G + h] = f;   // now the split's scale factor
+        for (int w = 0; w < kDecWarps; ++w) {
+            const float mw = wm[w * kMaxG + h];
+            if (mw != kNegInf) L += wl[w * kMaxG + h] * exp2f(mw - M);
         }
         sml[2 * h] = M;
         sml[2 * h + 1] = L;
     }
     __syncthreads();
-    const float *po = a.part_o + (int64_t)s * nsg * D;
     for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
         const int h = e / D, d = e % D;
-        const float M = sml[2 * h], L = sml[2 * h + 1];
+        const float M = sml[2 * h];
         float O = 0.0f;
-#pragma unroll 8
-        for (int k = 0; k < a.nsplit; ++k) O += __ldcg(&po[(k * G + h) * D + d]) * sm_w[k * G + h];
-        a.out[(qrow + h) * D + d] = L > 0.0f ? O / L : 0.0f;
-        if (d == 0 && a.lse) a.lse[qrow + h] = L > 0.0f ? (M + log2f(L)) * kLn2 : kNegInf;
+        for (int w = 0; w < kDecWarps; ++w) {
+            const float mw = wm[w * kMaxG + h];
+            if (mw != kNegInf) O += wo[(w * kMaxG + h) * D + d] * exp2f(mw - M);
+        }
+        part[e] = O;
     }
-    if (threadIdx.x == 0) a.counters[s] = 0;
+    cluster_sync_all();
+    const uint32_t rank = cluster_ctarank(), n = (uint32_t)a.nsplit;
+    const uint32_t sml_a = smem_u32(sml), part_a = smem_u32(part);
+    const int64_t qrow = (int64_t)b * a.Hq + (int64_t)g * G;
+    for (int e = rank * blockDim.x + threadIdx.x; e < G * D; e += n * blockDim.x) {
+        const int h = e / D, d = e % D;
+        float m = kNegInf, l = 0.0f, o = 0.0f;
+        for (uint32_t k = 0; k < n; ++k) {
+            const float mk = ld_peer(sml_a + 8 * h, k);
+            const float lk = ld_peer(sml_a + 8 * h + 4, k);
+            const float ok = ld_peer(part_a + 4 * e, k);
+            if (mk != kNegInf) {
+                const float mn = fmaxf(m, mk);
+                const float c_old = exp2f(m - mn), c_new = exp2f(mk - mn);
+                l = l * c_old + lk * c_new;
+                o = o * c_old + ok * c_new;
+                m = mn;
+            }
+        }
+        a.out[(qrow + h) * D + d] = l > 0.0f ? o / l : 0.0f;
+        if (d == 0 && a.lse) a.lse[qrow + h] = l > 0.0f ? (m + log2f(l)) * kLn2 : kNegInf;
+    }
+    cluster_sync_all();
+}
+
+// Log-sum-exp merge of the split partials (A5), one CTA per (segment, query
+// head), one thread per output element.  Launched as a programmatic
+// dependent of the decode kernel: it waits for the decode grid to complete
+// (and its writes to be visible) before reading the partials, so its launch
+// overlaps the decode's tail.  Splits are merged in split order.
+__global__ void __launch_bounds__(128) lse_merge_kernel(DecArgs a) {
+    pdl_wait();
+    const int s = blockIdx.x, h = blockIdx.y, G = a.G, D = a.D;
+    const int b = s / a.Hkv, g = s % a.Hkv;
+    const float2 *pml = a.part_ml + (int64_t)s * a.nsplit * G + h;
+    const float *po = a.part_o + ((int64_t)s * a.nsplit * G + h) * D;
+    const int64_t qrow = (int64_t)b * a.Hq + (int64_t)g * G + h;
+    // Every thread merges its output element over the splits in split order
+    // with a running maximum; all loads are independent of one another.
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        float m = kNegInf, l = 0.0f, o = 0.0f;
+#pragma unroll 16
+        for (int k = 0; k < a.nsplit; ++k) {
+            const float2 ml = __ldcg(&pml[(int64_t)k * G]);
+            const float ov = __ldcg(&po[(int64_t)k * G * D + d]);
+            if (ml.x != kNegInf) {
+                const float mn = fmaxf(m, ml.x);
+                const float c_old = exp2f(m - mn), c_new = exp2f(ml.x - mn);
+                l = l * c_old + ml.y * c_new;
+                o = o * c_old + ov * c_new;
+                m = mn;
+            }
+        }
+        a.out[qrow * D + d] = l > 0.0f ? o / l : 0.0f;
+        if (d == 0 && a.lse) a.lse[qrow] = l > 0.0f ? (m + log2f(l)) * kLn2 : kNegInf;
+    }
 }
 
 // ======================================================================
 // Tensor-core path
 // ======================================================================
-template <int NH, int STAGES>
+// Shared memory: one ring per warp, NST stages of one piece each (K then V,
+// NH boxes of 16 rows x 64 columns apiece).
+template <int NH, int NST>
 struct TcSmem {
-    static constexpr int kStageBytes = 2 * NH * kHalfBytes;   // K halves, then V halves
-    static constexpr int kRing = STAGES * kStageBytes;
-    static constexpr int kInfo = kRing;                        // int2 [STAGES][4]
-    static constexpr int kBars = kInfo + STAGES * kDecWarps * 8;
-    static constexpr int kMisc = kBars + STAGES * 8;           // float sml[2*kMaxG], int tmp[33]
-    static constexpr int kPtab = kMisc + 2 * kMaxG * 4 + 36 * 4;   // int2 [kPieceCap]
+    static constexpr int kPieceBytes = 2 * NH * kBoxBytes;
+    static constexpr int kRing = kDecWarps * NST * kPieceBytes;
+    static constexpr int kInfo = kRing;                               // int2 [warps][NST]
+    static constexpr int kBars = kInfo + kDecWarps * NST * 8;         // u64  [warps][NST]
+    static constexpr int kMisc = kBars + kDecWarps * NST * 8;         // float sml[2*kMaxG], int tmp[36]
+    static constexpr int kPtab = kMisc + 2 * kMaxG * 4 + 36 * 4;      // int2 [kPieceCap]
     static constexpr int kRanges = kPtab + kPieceCap * 8;
     static constexpr int bytes(int max_ranges) { return kRanges + (3 * max_ranges + 1) * 4 + 1024; }
+    static_assert(kRing >= kDecWarps * kMaxG * (2 + 64 * NH) * 4,
+                  "per-warp partials must fit in the ring");
 };
 
-template <int NH, int STAGES>
+template <int NH, int NST, bool CLUSTER>
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      DecArgs a) {
-    using L = TcSmem<NH, STAGES>;
+    using L = TcSmem<NH, NST>;
     constexpr int D = 64 * NH;
     constexpr int NT = D / 8;   // 8-column MMA tiles across D
     extern __shared__ unsigned char dsm_raw[];
@@ -233,6 +316,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     uint64_t *full = reinterpret_cast<uint64_t *>(dsm + L::kBars);
     float *sml = reinterpret_cast<float *>(dsm + L::kMisc);
     int *tmp = reinterpret_cast<int *>(dsm + L::kMisc + 2 * kMaxG * 4);
+    int2 *ptab = reinterpret_cast<int2 *>(dsm + L::kPtab);
     int *rs = reinterpret_cast<int *>(dsm + L::kRanges);
     int *re = rs + a.max_ranges;
     int *ps = re + a.max_ranges;
@@ -245,51 +329,39 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (tid == 0) {
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
-        for (int i = 0; i < STAGES; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < kDecWarps * NST; ++i) mbar_init(&full[i], 1);
         fence_mbar_init();
     }
+    pdl_wait();   // ranges, lengths and the cache come from earlier kernels
     int nr;
     const int P = load_ranges(a, s, b, rs, re, ps, tmp, &nr);
     int per = (P + a.nsplit - 1) / a.nsplit;
     per = (per + kDecWarps - 1) / kDecWarps * kDecWarps;
     const int first = c * per, last = min(P, first + per);
     const int n_my = max(0, last - first);
-    const int tiles = (n_my + kDecWarps - 1) / kDecWarps;
-
-    // this CTA's pieces, looked up in parallel once (the producer then only
-    // reads the table)
-    int2 *ptab = reinterpret_cast<int2 *>(dsm + L::kPtab);
     for (int i = tid; i < min(n_my, kPieceCap); i += kDecThreads)
         ptab[i] = piece_rows(first + i, rs, re, ps, nr);
     __syncthreads();
 
-    auto stage_ptr = [&](int st, int part) {   // part: 0..NH-1 K halves, NH..2NH-1 V halves
-        return dsm + st * L::kStageBytes + part * kHalfBytes;
-    };
-    auto issue = [&](int t, int st) {
-        int np = 0;
-        int2 pr[kDecWarps];
+    // this warp's pieces: local indices warp, warp + 4, warp + 8, ...
+    const int my_count = n_my > warp ? (n_my - warp + kDecWarps - 1) / kDecWarps : 0;
+    unsigned char *ring = dsm + warp * NST * L::kPieceBytes;
+    uint64_t *wfull = full + warp * NST;
+    int2 *winfo = info + warp * NST;
+    auto issue = [&](int idx, int st) {   // lane 0 only
+        const int i = warp + idx * kDecWarps;
+        const int2 pr = i < kPieceCap ? ptab[i] : piece_rows(first + i, rs, re, ps, nr);
+        winfo[st] = pr;
+        mbar_arrive_expect_tx(&wfull[st], (uint32_t)(2 * NH * kBoxBytes));
+        unsigned char *dst = ring + st * L::kPieceBytes;
 #pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) {
-            int p = first + t * kDecWarps + w;
-            pr[w] = p >= last ? make_int2(0, 0)
-                    : (p - first < kPieceCap ? ptab[p - first] : piece_rows(p, rs, re, ps, nr));
-            info[st * kDecWarps + w] = pr[w];
-            np += pr[w].y > 0;
-        }
-        mbar_arrive_expect_tx(&full[st], (uint32_t)(np * 2 * NH * kBoxBytes));
-#pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) {
-            if (pr[w].y <= 0) continue;
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                tma_load_4d(stage_ptr(st, h) + w * kBoxBytes, &tmK, &full[st], h * 64, pr[w].x, g, b);
-                tma_load_4d(stage_ptr(st, NH + h) + w * kBoxBytes, &tmV, &full[st], h * 64, pr[w].x, g, b);
-            }
+        for (int h = 0; h < NH; ++h) {
+            tma_load_4d(dst + h * kBoxBytes, &tmK, &wfull[st], h * 64, pr.x, g, b);
+            tma_load_4d(dst + (NH + h) * kBoxBytes, &tmV, &wfull[st], h * 64, pr.x, g, b);
         }
     };
-    if (tid == 0)
-        for (int t = 0; t < STAGES && t < tiles; ++t) issue(t, t);
+    if (lane == 0)
+        for (int j = 0; j < NST && j < my_count; ++j) issue(j, j);
 
     // q fragments: rows 0-7 q_hi of head gid, rows 8-15 q_lo; zero past G
     uint32_t qa[D / 16][4];
@@ -323,92 +395,102 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     float m_run = kNegInf, l_run = 0.0f;
     bool timed_out = false;
 
-    for (int t = 0; t < tiles; ++t) {
-        const int st = t % STAGES;
-        if (!mbar_wait_bounded(&full[st], (uint32_t)((t / STAGES) & 1))) timed_out = true;
-        const int2 pr = info[st * kDecWarps + warp];
-        const int nv = pr.y;
-        if (nv > 0) {
-            const uint32_t kbase = smem_u32(stage_ptr(st, 0) + warp * kBoxBytes);
-            const uint32_t vbase = smem_u32(stage_ptr(st, NH) + warp * kBoxBytes);
-            if (nv < kPiece) {   // rows past the range end: zero V so 0 * junk stays 0
-                for (int idx = lane; idx < (kPiece - nv) * NH * 8; idx += 32) {
-                    int r = nv + idx / (NH * 8), h = (idx / 8) % NH, ch = idx % 8;
-                    *reinterpret_cast<uint4 *>(stage_ptr(st, NH + h) + warp * kBoxBytes + r * 128 +
-                                               ch * 16) = make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
+    for (int idx = 0; idx < my_count; ++idx) {
+        const int st = idx % NST;
+        if (!mbar_wait_bounded(&wfull[st], (uint32_t)((idx / NST) & 1))) timed_out = true;
+        const int nv = winfo[st].y;
+        unsigned char *kp = ring + st * L::kPieceBytes;
+        unsigned char *vp = kp + NH * kBoxBytes;
+        if (nv < kPiece) {   // rows past the range end: zero V so 0 * junk stays 0
+            for (int e = lane; e < (kPiece - nv) * NH * 8; e += 32) {
+                const int r = nv + e / (NH * 8), h = (e / 8) % NH, ch = e % 8;
+                *reinterpret_cast<uint4 *>(vp + h * kBoxBytes + r * 128 + ch * 16) =
+                    make_uint4(0, 0, 0, 0);
             }
-            // S = Q K^T for the piece's 16 rows (two 8-row MMA tiles)
-            float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
+        const uint32_t kbase = smem_u32(kp), vbase = smem_u32(vp);
+        // S = Q K^T for the piece's 16 rows: two 8-row MMA tiles, even and odd
+        // k-steps in separate accumulators (shorter dependency chains)
+        float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const int half = kk / 4, ch0 = (kk % 4) * 2;
-                const int r = (lane >> 4) * 8 + (lane & 7);
-                const int ch = ch0 + ((lane >> 3) & 1);
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4(kbase + half * kHalfBytes + r * 128 + ((ch ^ (r & 7)) << 4), b0, b1, b2, b3);
-                mma_bf16_16816(sacc[0], qa[kk], b0, b1);
-                mma_bf16_16816(sacc[1], qa[kk], b2, b3);
-            }
-            float lg[4];
-#pragma unroll
-            for (int n = 0; n < 2; ++n)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int tok = n * 8 + 2 * tig + e;
-                    lg[n * 2 + e] = tok < nv ? (sacc[n][e] + sacc[n][2 + e]) * a.scale_log2 : kNegInf;
-                }
-            float mx = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m_run, mx);
-            float p[4];
-            if (m_new == kNegInf) {
-                p[0] = p[1] = p[2] = p[3] = 0.0f;
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int half = kk / 4, ch0 = (kk % 4) * 2;
+            const int r = (lane >> 4) * 8 + (lane & 7);
+            const int ch = ch0 + ((lane >> 3) & 1);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(kbase + half * kBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4), b0, b1, b2, b3);
+            if (kk & 1) {
+                mma_bf16_16816(sb[0], qa[kk], b0, b1);
+                mma_bf16_16816(sb[1], qa[kk], b2, b3);
             } else {
-                const float corr = exp2f(m_run - m_new);
+                mma_bf16_16816(sa[0], qa[kk], b0, b1);
+                mma_bf16_16816(sa[1], qa[kk], b2, b3);
+            }
+        }
+        float lg[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) p[e] = exp2f(lg[e] - m_new);
-                l_run = l_run * corr + ((p[0] + p[1]) + (p[2] + p[3]));
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int tok = n * 8 + 2 * tig + e;
+                const float v = (sa[n][e] + sb[n][e]) + (sa[n][2 + e] + sb[n][2 + e]);
+                lg[n * 2 + e] = tok < nv ? v * a.scale_log2 : kNegInf;
+            }
+        float mx = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float m_new = fmaxf(m_run, mx);
+        float p[4];
+        if (m_new == kNegInf) {
+            p[0] = p[1] = p[2] = p[3] = 0.0f;
+        } else {
+            const float corr = exp2f(m_run - m_new);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) p[e] = exp2f(lg[e] - m_new);
+            l_run = l_run * corr + ((p[0] + p[1]) + (p[2] + p[3]));
+            if (corr != 1.0f) {
 #pragma unroll
                 for (int i = 0; i < NT; ++i) {
                     o[i][0] *= corr; o[i][1] *= corr; o[i][2] *= corr; o[i][3] *= corr;
                 }
-                m_run = m_new;
             }
-            uint32_t pa[4];
-            {
-                float ph[4], pl[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    ph[e] = bf16_round(p[e]);
-                    pl[e] = p[e] - ph[e];
-                }
-                pa[0] = pack_bf16x2(ph[0], ph[1]);
-                pa[1] = pack_bf16x2(pl[0], pl[1]);
-                pa[2] = pack_bf16x2(ph[2], ph[3]);
-                pa[3] = pack_bf16x2(pl[2], pl[3]);
-            }
-            // O += P V
-#pragma unroll
-            for (int cp = 0; cp < D / 16; ++cp) {
-                const int half = cp / 4, ch0 = (cp % 4) * 2;
-                const int r = ((lane >> 3) & 1) * 8 + (lane & 7);
-                const int ch = ch0 + (lane >> 4);
-                uint32_t r0, r1, r2, r3;
-                ldmatrix_x4_trans(vbase + half * kHalfBytes + r * 128 + ((ch ^ (r & 7)) << 4), r0, r1, r2, r3);
-                mma_bf16_16816(o[2 * cp], pa, r0, r1);
-                mma_bf16_16816(o[2 * cp + 1], pa, r2, r3);
-            }
+            m_run = m_new;
         }
-        __syncthreads();
-        if (tid == 0 && t + STAGES < tiles) issue(t + STAGES, st);
+        uint32_t pa[4];
+        {
+            float ph[4], pl[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ph[e] = bf16_round(p[e]);
+                pl[e] = p[e] - ph[e];
+            }
+            pa[0] = pack_bf16x2(ph[0], ph[1]);
+            pa[1] = pack_bf16x2(pl[0], pl[1]);
+            pa[2] = pack_bf16x2(ph[2], ph[3]);
+            pa[3] = pack_bf16x2(pl[2], pl[3]);
+        }
+        // O += P V
+#pragma unroll
+        for (int cp = 0; cp < D / 16; ++cp) {
+            const int half = cp / 4, ch0 = (cp % 4) * 2;
+            const int r = ((lane >> 3) & 1) * 8 + (lane & 7);
+            const int ch = ch0 + (lane >> 4);
+            uint32_t r0, r1, r2, r3;
+            ldmatrix_x4_trans(vbase + half * kBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4), r0, r1, r2, r3);
+            mma_bf16_16816(o[2 * cp], pa, r0, r1);
+            mma_bf16_16816(o[2 * cp + 1], pa, r2, r3);
+        }
+        __syncwarp();
+        if (lane == 0 && idx + NST < my_count) issue(idx + NST, st);
     }
     if (timed_out) atomicOr(a.status, 1u);
+    // the merge kernel may be scheduled now; it waits for this grid to finish
+    pdl_trigger();
 
-    // per-warp partials -> shared memory (reusing the ring)
+    // per-warp partials -> shared memory (reusing the rings once all are idle)
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     float *wm = reinterpret_cast<float *>(dsm);
@@ -426,7 +508,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         wo[(warp * kMaxG + gid) * D + d + 1] = o[nt][1] + o[nt][3];
     }
     __syncthreads();
-    finish(a, s, b, g, c, wm, wl, wo, sml, reinterpret_cast<float *>(dsm + 32768));
+    if constexpr (CLUSTER)
+        cluster_finish(a, b, g, wm, wl, wo, sml, reinterpret_cast<float *>(dsm + 32768));
+    else
+        finish(a, s, b, g, c, wm, wl, wo, sml);
 }
 
 // ======================================================================
@@ -444,11 +529,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_generic_kernel(DecArgs a) 
     int *rs = tmp + 36;
     int *re = rs + a.max_ranges;
     int *ps = re + a.max_ranges;
-    float *mscr = reinterpret_cast<float *>(ps + a.max_ranges + 1);   // [2 * nsplit * G]
 
     const int c = blockIdx.x, s = blockIdx.y;
     const int b = s / a.Hkv, g = s % a.Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
     int nr;
     const int P = load_ranges(a, s, b, rs, re, ps, tmp, &nr);
     int per = (P + a.nsplit - 1) / a.nsplit;
@@ -499,6 +584,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_generic_kernel(DecArgs a) 
             }
         }
     }
+    pdl_trigger();
 #pragma unroll
     for (int h = 0; h < kMaxG; ++h) {
         if (lane == 0) {
@@ -509,13 +595,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_generic_kernel(DecArgs a) 
         for (int k = 0; k < PER; ++k) wo[(warp * kMaxG + h) * D + lane + 32 * k] = o[h][k];
     }
     __syncthreads();
-    finish(a, s, b, g, c, wm, wl, wo, sml, mscr);
+    finish(a, s, b, g, c, wm, wl, wo, sml);
 }
 
 // ======================================================================
 // Host side
 // ======================================================================
-constexpr int kTcStages = 3;
+constexpr int kTcStages = 3;   // pieces in flight per warp
 
 static bool use_tc(const bsa_kv_desc *d) {
     return d->kv_dtype == BSA_BF16 && (d->D == 64 || d->D == 128) && d->Hq / d->Hkv <= kMaxG &&
@@ -527,8 +613,40 @@ int decode_nsplit(const bsa_kv_desc *d, int tokens_hint, int max_ranges) {
     const int64_t pieces = div_up(tokens_hint > 0 ? tokens_hint : 1, kPiece) + max_ranges;
     const int slots = num_sms() * (use_tc(d) ? 2 : 4);
     int nsplit = std::max(1, slots / std::max(nseg, 1));
+    if (use_tc(d)) nsplit = std::min(nsplit, kMaxClusterSplits);   // one cluster per segment
     nsplit = (int)std::min<int64_t>(nsplit, div_up(pieces, kDecWarps));
     return std::max(1, nsplit);
+}
+
+// Largest cluster size c <= max_c (c >= 2) for which all nseg clusters of the
+// decode kernel can be resident at once, or 0.  Cached per configuration.
+static int cluster_splits(const void *kern, int smem, int nseg, int max_c, cudaLaunchConfig_t cfg) {
+    struct Key {
+        const void *k;
+        int smem, nseg, max_c, dev;
+    };
+    static std::mutex mu;
+    static std::vector<std::pair<Key, int>> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto &e : cache)
+        if (e.first.k == kern && e.first.smem == smem && e.first.nseg == nseg &&
+            e.first.max_c == max_c && e.first.dev == dev)
+            return e.second;
+    int best = 0;
+    cudaLaunchAttribute attr = cfg.attrs[0];
+    for (int c = std::min(max_c, kMaxClusterSplits); c >= 2 && !best; --c) {
+        attr.val.clusterDim.x = c;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(c, (unsigned)nseg);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= nseg) best = c;
+        cudaGetLastError();
+    }
+    cache.push_back({{kern, smem, nseg, max_c, dev}, best});
+    return best;
 }
 
 size_t decode_scratch_bytes(const bsa_kv_desc *d, int nsplit) {
@@ -559,25 +677,57 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
     if (use_tc(d)) {
         CUtensorMap tk, tv;
         if (!make_kv_tmap(&tk, d, K, kPiece) || !make_kv_tmap(&tv, d, V, kPiece)) return BSA_ERR_CUDA;
-        if (d->D == 128) {
-            auto kern = decode_tc_kernel<2, kTcStages>;
-            const int smem = TcSmem<2, kTcStages>::bytes(max_ranges);
-            BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-            kern<<<grid, kDecThreads, smem, st>>>(tk, tv, a);
-        } else {
-            auto kern = decode_tc_kernel<1, 2 * kTcStages>;
-            const int smem = TcSmem<1, 2 * kTcStages>::bytes(max_ranges);
-            BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-            kern<<<grid, kDecThreads, smem, st>>>(tk, tv, a);
-        }
+        // The splits of a segment form one thread-block cluster when they fit
+        // (merge through distributed shared memory, no second kernel).
+        bool clustered = false;
+        auto go_tc = [&](auto kern_plain, auto kern_cluster, int smem) -> bsa_status {
+            BSA_CUDA_TRY(cudaFuncSetAttribute(kern_plain, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+            if (a.nsplit > 1) {
+                BSA_CUDA_TRY(cudaFuncSetAttribute(kern_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+                BSA_CUDA_TRY(cudaFuncSetAttribute(kern_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+                cudaLaunchConfig_t cfg = {};
+                cfg.blockDim = dim3(kDecThreads);
+                cfg.dynamicSmemBytes = smem;
+                cfg.stream = st;
+                cudaLaunchAttribute attr[2];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+                attr[1].val.programmaticStreamSerializationAllowed = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 2;
+                const int c = cluster_splits(reinterpret_cast<const void *>(kern_cluster), smem,
+                                             (int)nseg, a.nsplit, cfg);
+                if (c > 1) {
+                    a.nsplit = c;
+                    cfg.gridDim = dim3(c, (unsigned)nseg);
+                    attr[0].val.clusterDim.x = c;
+                    BSA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern_cluster, tk, tv, a));
+                    clustered = true;
+                    return BSA_OK;
+                }
+            }
+            BSA_CUDA_TRY(launch_pdl(kern_plain, grid, dim3(kDecThreads), smem, st, tk, tv, a));
+            return BSA_OK;
+        };
+        bsa_status r;
+        if (d->D == 128)
+            r = go_tc(decode_tc_kernel<2, kTcStages, false>, decode_tc_kernel<2, kTcStages, true>,
+                      TcSmem<2, kTcStages>::bytes(max_ranges));
+        else   // D = 64
+            r = go_tc(decode_tc_kernel<1, 2 * kTcStages, false>, decode_tc_kernel<1, 2 * kTcStages, true>,
+                      TcSmem<1, 2 * kTcStages>::bytes(max_ranges));
+        if (r != BSA_OK) return r;
+        BSA_LAUNCH_CHECK();
+        if (clustered) return BSA_OK;
     } else {
         const size_t smem = (size_t)(2 * kDecWarps * kMaxG + kDecWarps * kMaxG * d->D + 2 * kMaxG) * 4 +
-                            36 * 4 + (size_t)(3 * max_ranges + 1) * 4 +
-                            (size_t)2 * a.nsplit * a.G * 4;
+                            36 * 4 + (size_t)(3 * max_ranges + 1) * 4;
         auto go = [&](auto kern) -> bsa_status {
             if (smem > 48 * 1024)
                 BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-            kern<<<grid, kDecThreads, smem, st>>>(a);
+            BSA_CUDA_TRY(launch_pdl(kern, grid, dim3(kDecThreads), smem, st, a));
             return BSA_OK;
         };
         bsa_status r;
@@ -588,6 +738,11 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
         if (r != BSA_OK) return r;
     }
     BSA_LAUNCH_CHECK();
+    if (a.nsplit > 1) {
+        // the merge, as a programmatic dependent launch of the decode kernel
+        BSA_CUDA_TRY(launch_pdl(lse_merge_kernel, dim3((unsigned)nseg, (unsigned)a.G), dim3(128),
+                                0, st, a));
+    }
     return BSA_OK;
 }
 

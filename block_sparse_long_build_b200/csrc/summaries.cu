@@ -150,6 +150,8 @@ struct AppendArgs {
 template <typename T>
 __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
     extern __shared__ float sm[];
+    pdl_trigger();
+    pdl_wait();
     const int b = blockIdx.x;
     const int n = a.cur_len[b];
     if (n < 0 || n >= a.L_max) return;
@@ -213,9 +215,9 @@ bsa_status launch_append(const bsa_kv_desc *d, void *K, void *V, const void *kn,
     a.row_bytes = summary_row_bytes(kind, d->D, d->kv_dtype);
     size_t smem = summary_smem(kind, d->D);
     if (d->kv_dtype == BSA_BF16)
-        append_kernel<uint16_t><<<d->B, 256, smem, st>>>(a);
+        BSA_CUDA_TRY(launch_pdl(append_kernel<uint16_t>, dim3(d->B), dim3(256), smem, st, a));
     else
-        append_kernel<float><<<d->B, 256, smem, st>>>(a);
+        BSA_CUDA_TRY(launch_pdl(append_kernel<float>, dim3(d->B), dim3(256), smem, st, a));
     BSA_LAUNCH_CHECK();
     return BSA_OK;
 }

@@ -181,7 +181,8 @@ BSA_API bsa_status bsa_select(const bsa_kv_desc *desc, const float *q, const voi
  * (Module 14, Exercise 14.1, restricted to the selected tokens):
  *   out[b][h] = sum_j softmax_j(scale * q[b][h] . K[j]) V[j],
  *   lse[b][h] = log sum_j exp(scale * q[b][h] . K[j])      (natural log)
- * over the rows of ranges[s][0..n_ranges[s]), s = b*Hkv + h/G.  The last
+ * over the rows of ranges[s][0..n_ranges[s]), s = b*Hkv + h/G (ranges must
+ * be 8-byte aligned; slots past n_ranges[s] may hold anything).  The last
  * range of each segment is extended to end at cur_len[b] when that is
  * larger: between selection refreshes the window keeps growing ("Sparse
  * attention in hybrid LLMs", refresh every 32 steps).  Rows are clamped to
