@@ -22,8 +22,8 @@ int decode_nsplit(const bsa_kv_desc *, int, int);
 size_t decode_scratch_bytes(const bsa_kv_desc *, int);
 bsa_status launch_prefill(const bsa_kv_desc *, const void *, const void *, const bsa_sel_params *,
                           const void *, const bsa_kv_desc *, const void *, const void *,
-                          const void *, int, int, float, float *, float *, void *, size_t,
-                          cudaStream_t);
+                          const void *, int, int, float, float *, float *, uint32_t *, void *,
+                          size_t, cudaStream_t);
 size_t prefill_ws_bytes(const bsa_kv_desc *, const bsa_sel_params *, int);
 
 int num_sms() {
@@ -297,8 +297,8 @@ bsa_status bsa_prefill_grouped(const bsa_kv_desc *d, const void *K, const void *
     const size_t need = bsa_workspace_size(d, p, BSA_OP_PREFILL, Tq, 0);
     if (!ws_ok(ws, ws_bytes, need)) return BSA_ERR_WORKSPACE;
     return launch_prefill(d, K, V, p, summaries, pd, K_pos, V_pos, Q, q_pos0, Tq, scale, out, lse,
-                          static_cast<char *>(ws) + counters_bytes(d), ws_bytes - counters_bytes(d),
-                          (cudaStream_t)stream);
+                          static_cast<uint32_t *>(ws), static_cast<char *>(ws) + counters_bytes(d),
+                          ws_bytes - counters_bytes(d), (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -1,15 +1,558 @@
-// A6/A7: block-grouped prefill (placeholder until the tensor-core kernels land).
+// A6 (per-query block selection and grouping) + A7 (block-grouped contraction
+// on tcgen05 tensor cores) for the semantic-block prefill, sm_100a.
+//
+// "Semantic blocks for sparse attention": during prefill, neighbouring
+// queries pick different blocks; instead of taking the union, the queries
+// that need the same block are gathered and the block's keys and values are
+// loaded once for the whole group.  The current fragment is attended densely
+// and causally, and while the prefix is short the whole prefix is dense.
+//
+// Per call (one chunk of Tq queries at positions q_pos0 .. q_pos0+Tq-1):
+//   P1 prefill_select_kernel  one warp per (query, KV head): scores the
+//      KV head's block centres in the fixed fp32 order (as bsa_select) and
+//      walks them greedily under the token budget; writes a selection bitmap
+//      and appends the query to each selected block's list.
+//   P2 prefill_tiles_kernel   prefix of 128-row tiles over (KV head, block).
+//   P3 prefill_attend_kernel  persistent; work items are 128-row tiles:
+//      local (32 queries x 4 heads against the position-ordered keys
+//      [pos_limit, q], causal) and grouped (the gathered rows of one block
+//      against its visible prefix).  Q rows are gathered into 128-byte-
+//      swizzled shared memory, K/V tiles arrive by TMA (no multicast),
+//      S = Q K^T accumulates in TMEM (tcgen05.mma, bf16 in, fp32 out), one
+//      thread per row runs the online softmax and writes P (bf16) back to
+//      TMEM, O += P V reads P from TMEM.  Each item leaves an unnormalised
+//      partial (o, m, l) in its (query, KV head, slot) record.
+//   P4 prefill_merge_kernel   log-sum-exp merge of a query's slots (local
+//      first, then blocks in index order).
 #include "common.cuh"
 
 namespace bsa {
 
-size_t prefill_ws_bytes(const bsa_kv_desc *, const bsa_sel_params *, int) { return 256; }
+constexpr int kPfMaxBlocks = 256;          // blocks per KV head (bitmap of 8 words)
+constexpr int kPfWords = kPfMaxBlocks / 32;
+constexpr int kPfMaxSel = 64;              // selected blocks kept per (query, KV head)
+constexpr int kPfSlots = kPfMaxSel + 1;    // slot 0 = local part
+constexpr int kPfRowsPerCta = 64;          // P1 query rows per CTA
+constexpr int kTile = 128;                 // rows per MMA tile, keys per key tile
+constexpr int kPfThreads = 128;
+constexpr float kPfNegInf = -__builtin_huge_valf();
+constexpr float kPfLn2 = 0.69314718055994530942f;
 
-bsa_status launch_prefill(const bsa_kv_desc *, const void *, const void *, const bsa_sel_params *,
-                          const void *, const bsa_kv_desc *, const void *, const void *,
-                          const void *, int, int, float, float *, float *, void *, size_t,
-                          cudaStream_t) {
-    return BSA_ERR_UNSUPPORTED;
+struct PfArgs {
+    int Hq, Hkv, G, D, nb, L_max, Lpos;
+    int Tq, q_pos0, pos_limit, budget;
+    float scale_log2;
+    const uint16_t *Q;         // [Tq][Hq][D] bf16
+    const float *cent;         // [Hkv][nb][D]
+    const int32_t *offsets;    // [Hkv][nb + 1]
+    const int32_t *kv_pos;     // [Hkv][L_max]
+    uint32_t *bitmap;          // [Tq][Hkv][kPfWords]
+    int32_t *vis;              // [Hkv][nb]
+    int32_t *qcount;           // [Hkv][nb]          (zeroed per call)
+    int32_t *qlist;            // [Hkv][nb][Tq]
+    int32_t *tile_prefix;      // [Hkv * nb + 1]
+    int32_t *work;             // [1]                (zeroed per call)
+    float *part_o;             // [Tq][Hkv][kPfSlots][G][D]
+    float2 *part_ml;           // [Tq][Hkv][kPfSlots][G]
+    uint32_t *status;
+    float *out, *lse;          // [Tq][Hq][D], [Tq][Hq]
+    int n_local;               // local work items
+};
+
+__device__ __forceinline__ int pf_visible(const int32_t *pos, int r0, int r1, int lim) {
+    int lo = r0, hi = r1;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (pos[mid] < lim) lo = mid + 1; else hi = mid;
+    }
+    return lo - r0;
+}
+
+// ---------------------------------------------------------------- P1
+__global__ void __launch_bounds__(256) prefill_select_kernel(PfArgs a) {
+    extern __shared__ float psm[];
+    const int D = a.D, G = a.G, nb = a.nb;
+    float *cs = psm;                                   // [nb][D+1]
+    float *qv = cs + nb * (D + 1);                     // [8 warps][G][D]
+    int *visS = reinterpret_cast<int *>(qv + 8 * G * D);   // [nb]
+    __shared__ int min_vis_sh;
+    const int g = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_wait();
+    const float *cg = a.cent + (int64_t)g * nb * D;
+    for (int e = tid; e < nb * D; e += blockDim.x) cs[(e / D) * (D + 1) + e % D] = cg[e];
+    const int32_t *off = a.offsets + (int64_t)g * (nb + 1);
+    const int32_t *pos = a.kv_pos + (int64_t)g * a.L_max;
+    if (tid == 0) min_vis_sh = 0x7fffffff;
+    __syncthreads();
+    for (int j = tid; j < nb; j += blockDim.x) {
+        const int r0 = min(max(off[j], 0), a.L_max), r1 = min(max(off[j + 1], r0), a.L_max);
+        const int v = pf_visible(pos, r0, r1, a.pos_limit);
+        visS[j] = v;
+        if (blockIdx.x == 0) a.vis[g * nb + j] = v;
+        if (v > 0) atomicMin(&min_vis_sh, v);
+    }
+    __syncthreads();
+    const int min_vis = min_vis_sh;
+    float *qw = qv + warp * G * D;
+    for (int r = 0; r < kPfRowsPerCta / 8; ++r) {
+        const int i = blockIdx.x * kPfRowsPerCta + warp * (kPfRowsPerCta / 8) + r;
+        if (i >= a.Tq) break;
+        const uint16_t *qi = a.Q + ((int64_t)i * a.Hq + (int64_t)g * G) * D;
+        for (int e = lane; e < G * D; e += 32) qw[e] = bf16_to_f32(qi[e]);
+        __syncwarp();
+        // lane owns blocks lane + 32 t; composite keys (orderable score, ~index)
+        unsigned long long key[kPfWords];
+#pragma unroll
+        for (int t = 0; t < kPfWords; ++t) {
+            key[t] = 0ull;
+            const int j = lane + 32 * t;
+            if (j < nb && visS[j] > 0) {
+                const float *c = cs + j * (D + 1);
+                float tot = 0.0f;
+                for (int h = 0; h < G; ++h) {
+                    const float *qh = qw + h * D;
+                    float acc = 0.0f;
+                    for (int d = 0; d < D; ++d) acc = __fmaf_rn(qh[d], c[d], acc);
+                    tot = h == 0 ? acc : __fadd_rn(tot, acc);
+                }
+                uint32_t k32 = f32_order_key(__fadd_rn(tot, 0.0f));
+                if (k32 == 0) k32 = 1;
+                key[t] = ((unsigned long long)k32 << 32) | (0xffffffffu - (uint32_t)j);
+            }
+        }
+        // greedy walk in rank order: take a block when its visible rows fit
+        uint32_t selbits = 0;   // bit t: block lane + 32 t selected
+        int remaining = a.budget, nsel = 0;
+        while (remaining >= min_vis && nsel < kPfMaxSel) {
+            unsigned long long best = 0ull;
+#pragma unroll
+            for (int t = 0; t < kPfWords; ++t) best = key[t] > best ? key[t] : best;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+                best = other > best ? other : best;
+            }
+            if (best == 0ull) break;
+            const int j = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
+            const int v = visS[j];
+            const bool take = v <= remaining;
+            if (lane == (j & 31)) {
+#pragma unroll
+                for (int t = 0; t < kPfWords; ++t)
+                    if (t == (j >> 5)) {
+                        key[t] = 0ull;
+                        if (take) selbits |= 1u << t;
+                    }
+            }
+            if (take) {
+                remaining -= v;
+                ++nsel;
+                if (lane == 0) {
+                    const int p = atomicAdd(&a.qcount[g * nb + j], 1);
+                    a.qlist[((int64_t)g * nb + j) * a.Tq + p] = i;
+                }
+            }
+        }
+        if (nsel >= kPfMaxSel && lane == 0) atomicOr(a.status, 4u);
+        uint32_t *bm = a.bitmap + ((int64_t)i * a.Hkv + g) * kPfWords;
+#pragma unroll
+        for (int t = 0; t < kPfWords; ++t) {
+            const uint32_t word = __ballot_sync(0xffffffffu, (selbits >> t) & 1u);
+            if (lane == 0) bm[t] = word;
+        }
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------- P2
+__global__ void __launch_bounds__(1024) prefill_tiles_kernel(PfArgs a) {
+    __shared__ int tmp[40];
+    const int n = a.Hkv * a.nb;
+    int carry = 0;
+    for (int base = 0; base < n; base += blockDim.x) {
+        const int e = base + threadIdx.x;
+        const int t = e < n ? (a.qcount[e] * a.G + kTile - 1) / kTile : 0;
+        int tot;
+        const int ex = cta_excl_sum(t, tmp, &tot);
+        if (e < n) a.tile_prefix[e] = carry + ex;
+        carry += tot;
+    }
+    if (threadIdx.x == 0) a.tile_prefix[n] = carry;
+}
+
+// ---------------------------------------------------------------- P3
+struct PfSmem {
+    static constexpr int kQ = 0;                         // 2 boxes x 16 KiB
+    static constexpr int kStage = 32768;                 // 2 stages x (K 32 KiB + V 32 KiB)
+    static constexpr int kStageBytes = 65536;
+    static constexpr int kRowQ = kStage + 2 * kStageBytes;   // int [128] query index
+    static constexpr int kRowPos = kRowQ + kTile * 4;        // int [128] query position
+    static constexpr int kBars = kRowPos + kTile * 4;        // u64 full[2], mma_s, mma_o
+    static constexpr int kMisc = kBars + 4 * 8;              // int item, tmem base
+    static constexpr int kBytes = kMisc + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_attend_kernel(const __grid_constant__ CUtensorMap tmKp, const __grid_constant__ CUtensorMap tmVp,
+                          const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVl,
+                          PfArgs a) {
+    extern __shared__ unsigned char praw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(praw) + 1023) & ~uintptr_t(1023));
+    unsigned char *Qs = sm + PfSmem::kQ;
+    int *rowq = reinterpret_cast<int *>(sm + PfSmem::kRowQ);
+    int *rowpos = reinterpret_cast<int *>(sm + PfSmem::kRowPos);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + PfSmem::kBars);
+    uint64_t *bar_s = full + 2, *bar_o = full + 3;
+    int *item_sh = reinterpret_cast<int *>(sm + PfSmem::kMisc);
+    uint32_t *tmem_sh = reinterpret_cast<uint32_t *>(sm + PfSmem::kMisc + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int G = a.G, D = a.D;
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+            smem_u32(tmem_sh)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (tid == 0) {
+        prefetch_tmap(&tmKp); prefetch_tmap(&tmVp); prefetch_tmap(&tmKl); prefetch_tmap(&tmVl);
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+        fence_mbar_init();
+    }
+    pdl_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_sh;
+    const uint32_t tS = tmem, tO = tmem + 128;        // S (and P over its first 64 columns), O
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int n_group = a.tile_prefix[a.Hkv * a.nb];
+    const int n_items = a.n_local + n_group;
+    uint32_t full_use[2] = {0, 0}, s_use = 0, o_use = 0;
+    bool timed_out = false;
+    constexpr uint32_t kIdescQK = umma_idesc_bf16(128, 128, 0, 0);
+    constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 128, 0, 1);
+    const int qpt = kTile / G;   // queries per tile
+
+    for (;;) {
+        if (tid == 0) *item_sh = atomicAdd(a.work, 1);
+        __syncthreads();
+        const int item = *item_sh;
+        if (item >= n_items) break;
+        // ---- decode the work item
+        int g, kbeg, kend, jblk = -1, mtile = 0;
+        bool local = item < a.n_local;
+        const int tiles_per_head = (a.Tq + qpt - 1) / qpt;
+        if (local) {
+            g = item / tiles_per_head;
+            const int i0 = (item % tiles_per_head) * qpt;
+            const int ilast = min(a.Tq, i0 + qpt) - 1;
+            kbeg = a.pos_limit;
+            kend = a.q_pos0 + ilast + 1;
+            const int r = tid, i = i0 + r / G;
+            rowq[r] = i < a.Tq ? i : -1;
+            rowpos[r] = a.q_pos0 + i;
+            mtile = i0;
+        } else {
+            const int u = item - a.n_local;
+            int lo = 0, hi = a.Hkv * a.nb - 1;   // largest e with prefix[e] <= u
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (a.tile_prefix[mid] <= u) lo = mid; else hi = mid - 1;
+            }
+            g = lo / a.nb;
+            jblk = lo % a.nb;
+            mtile = u - a.tile_prefix[lo];
+            const int r0 = min(max(a.offsets[(int64_t)g * (a.nb + 1) + jblk], 0), a.L_max);
+            kbeg = r0;
+            kend = r0 + a.vis[g * a.nb + jblk];
+            const int cnt = a.qcount[g * a.nb + jblk];
+            const int idx = mtile * kTile + tid, qi = idx / G;
+            rowq[tid] = qi < cnt ? a.qlist[((int64_t)g * a.nb + jblk) * a.Tq + qi] : -1;
+            rowpos[tid] = 0x7fffffff;   // every key of the visible prefix is earlier
+        }
+        __syncthreads();
+        // ---- gather Q rows (bf16) into the swizzled K-major layout
+        for (int c = tid; c < kTile * 16; c += kPfThreads) {
+            const int r = c >> 4, ch = c & 15, half = ch >> 3, cc = ch & 7;
+            const int qi = rowq[r];
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (qi >= 0) {
+                const int hh = local ? (r % G) : ((mtile * kTile + r) % G);
+                v = *reinterpret_cast<const uint4 *>(
+                    a.Q + ((int64_t)qi * a.Hq + (int64_t)g * G + hh) * D + ch * 8);
+            }
+            *reinterpret_cast<uint4 *>(Qs + half * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        const int ntiles = max(0, (kend - kbeg + kTile - 1) / kTile);
+        auto issue_kv = [&](int t, int st) {
+            unsigned char *base = sm + PfSmem::kStage + st * PfSmem::kStageBytes;
+            mbar_arrive_expect_tx(&full[st], 4 * 16384);
+            const CUtensorMap *mk = local ? &tmKl : &tmKp;
+            const CUtensorMap *mv = local ? &tmVl : &tmVp;
+            const int row = kbeg + t * kTile;
+            tma_load_4d(base, mk, &full[st], 0, row, g, 0);
+            tma_load_4d(base + 16384, mk, &full[st], 64, row, g, 0);
+            tma_load_4d(base + 32768, mv, &full[st], 0, row, g, 0);
+            tma_load_4d(base + 49152, mv, &full[st], 64, row, g, 0);
+        };
+        if (tid == 0 && ntiles > 0) issue_kv(0, 0);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        float m_run = kPfNegInf, l_run = 0.0f;
+        const int my_pos = rowpos[tid];
+        for (int t = 0; t < ntiles; ++t) {
+            const int st = t & 1;
+            if (tid == 0) {
+                if (t + 1 < ntiles) issue_kv(t + 1, st ^ 1);
+                if (!mbar_wait_bounded(&full[st], full_use[st] & 1)) timed_out = true;
+                tc_fence_after();
+                const uint32_t q0 = smem_u32(Qs);
+                const uint32_t k0 = smem_u32(sm + PfSmem::kStage + st * PfSmem::kStageBytes);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                    umma_ss(tS, umma_sdesc_sw128(q0 + off, 16, 1024), umma_sdesc_sw128(k0 + off, 16, 1024),
+                            kIdescQK, k > 0);
+                }
+                umma_commit(bar_s);
+            }
+            ++full_use[st];
+            if (!mbar_wait_bounded(bar_s, s_use & 1)) timed_out = true;
+            ++s_use;
+            tc_fence_after();
+            // ---- online softmax, one thread per row
+            uint32_t sv[4][32];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + lane_base + c4 * 32, sv[c4]);
+            tmem_ld_wait();
+            const int key0 = kbeg + t * kTile;
+            float mx = kPfNegInf;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int kr = key0 + c4 * 32 + e;
+                    const bool ok = kr < kend && kr <= my_pos;
+                    const float v = ok ? __uint_as_float(sv[c4][e]) * a.scale_log2 : kPfNegInf;
+                    sv[c4][e] = __float_as_uint(v);
+                    mx = fmaxf(mx, v);
+                }
+            const float m_new = fmaxf(m_run, mx);
+            const float corr = m_new == kPfNegInf ? 1.0f : exp2f(m_run - m_new);
+            // P = P_hi + P_lo, both bf16: columns 0..63 of S take P_hi, 64..127
+            // P_lo (the row's S values are all in registers by now), so the
+            // weights carry ~2^-17 relative error instead of 2^-9
+            float lsum = 0.0f;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t ph[16], pl[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = m_new == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[c4][e]) - m_new);
+                    const float p1 = m_new == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[c4][e + 1]) - m_new);
+                    lsum += p0 + p1;
+                    const float h0 = bf16_round(p0), h1 = bf16_round(p1);
+                    ph[e / 2] = pack_bf16x2(h0, h1);
+                    pl[e / 2] = pack_bf16x2(p0 - h0, p1 - h1);
+                }
+                tmem_st16(tS + lane_base + c4 * 16, ph);
+                tmem_st16(tS + lane_base + 64 + c4 * 16, pl);
+            }
+            l_run = l_run * corr + lsum;
+            // rescale the O accumulator; tcgen05.ld/st are warp-collective, so
+            // the whole warp takes the branch when any of its rows needs it
+            if (t > 0 && __any_sync(0xffffffffu, corr != 1.0f)) {
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + lane_base + c4 * 32, ov);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+                    tmem_st32(tO + lane_base + c4 * 32, ov);
+                }
+            }
+            m_run = m_new;
+            tmem_st_wait();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t v0 = smem_u32(sm + PfSmem::kStage + st * PfSmem::kStageBytes + 32768);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t vd = umma_sdesc_sw128(v0 + k * 2048, 16384, 1024);
+                    umma_ts(tO, tS + k * 8, vd, kIdescPV, (t > 0 || k > 0) ? 1u : 0u);   // P_hi
+                    umma_ts(tO, tS + 64 + k * 8, vd, kIdescPV, 1u);                       // P_lo
+                }
+                umma_commit(bar_o);
+            }
+            if (!mbar_wait_bounded(bar_o, o_use & 1)) timed_out = true;
+            ++o_use;
+            tc_fence_after();
+        }
+        // ---- epilogue: this item's partial for every live row (the TMEM loads
+        // are warp-collective and run for every row; dead rows drop them)
+        const int qi = rowq[tid];
+        int64_t rec = -1;
+        if (qi >= 0) {
+            const int hh = local ? (tid % G) : ((mtile * kTile + tid) % G);
+            int slot = 0;
+            if (!local) {
+                const uint32_t *bm = a.bitmap + ((int64_t)qi * a.Hkv + g) * kPfWords;
+                for (int w = 0; w < (jblk >> 5); ++w) slot += __popc(bm[w]);
+                slot += __popc(bm[jblk >> 5] & ((1u << (jblk & 31)) - 1u)) + 1;
+            }
+            if (slot < kPfSlots) rec = (((int64_t)qi * a.Hkv + g) * kPfSlots + slot) * G + hh;
+        }
+        float *po = rec >= 0 ? a.part_o + rec * D : nullptr;
+        if (ntiles > 0) {
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t ov[32];
+                tmem_ld32(tO + lane_base + c4 * 32, ov);
+                tmem_ld_wait();
+                if (po) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(po + c4 * 32 + e) =
+                            make_float4(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1]),
+                                        __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
+                }
+            }
+        } else if (po) {
+            for (int d = 0; d < D; ++d) po[d] = 0.0f;
+        }
+        if (rec >= 0) a.part_ml[rec] = make_float2(m_run, l_run);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    if (timed_out) atomicOr(a.status, 8u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+}
+
+// ---------------------------------------------------------------- P4
+__global__ void __launch_bounds__(128) prefill_merge_kernel(PfArgs a) {
+    pdl_wait();
+    const int i = blockIdx.x, g = blockIdx.y, G = a.G, D = a.D;
+    const uint32_t *bm = a.bitmap + ((int64_t)i * a.Hkv + g) * kPfWords;
+    int nsel = 0;
+    for (int w = 0; w < kPfWords; ++w) nsel += __popc(bm[w]);
+    const int nslot = min(1 + nsel, kPfSlots);
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+        const int hh = e / D, d = e % D;
+        float m = kPfNegInf, l = 0.0f, o = 0.0f;
+        for (int s = 0; s < nslot; ++s) {
+            const int64_t rec = (((int64_t)i * a.Hkv + g) * kPfSlots + s) * G + hh;
+            const float2 ml = __ldcg(&a.part_ml[rec]);
+            const float ov = __ldcg(&a.part_o[rec * D + d]);
+            if (ml.x != kPfNegInf) {
+                const float mn = fmaxf(m, ml.x);
+                const float c_old = exp2f(m - mn), c_new = exp2f(ml.x - mn);
+                l = l * c_old + ml.y * c_new;
+                o = o * c_old + ov * c_new;
+                m = mn;
+            }
+        }
+        const int64_t orow = (int64_t)i * a.Hq + (int64_t)g * G + hh;
+        a.out[orow * D + d] = l > 0.0f ? o / l : 0.0f;
+        if (d == 0 && a.lse) a.lse[orow] = l > 0.0f ? (m + log2f(l)) * kPfLn2 : kPfNegInf;
+    }
+}
+
+// ---------------------------------------------------------------- host
+struct PfLayout {
+    size_t bitmap, vis, qcount, qlist, prefix, work, part_o, part_ml, total;
+};
+
+static PfLayout pf_layout(const bsa_kv_desc *d, const bsa_sel_params *p, int Tq) {
+    PfLayout L;
+    const size_t G = d->Hq / d->Hkv, nb = p->n_blocks, H = d->Hkv;
+    size_t o = 0;
+    L.bitmap = o;  o += align_up((size_t)Tq * H * kPfWords * 4, 256);
+    L.vis = o;     o += align_up(H * nb * 4, 256);
+    L.qcount = o;  o += align_up(H * nb * 4, 256);
+    L.work = o;    o += 256;
+    L.qlist = o;   o += align_up(H * nb * (size_t)Tq * 4, 256);
+    L.prefix = o;  o += align_up((H * nb + 1) * 4, 256);
+    L.part_o = o;  o += align_up((size_t)Tq * H * kPfSlots * G * d->D * 4, 256);
+    L.part_ml = o; o += align_up((size_t)Tq * H * kPfSlots * G * 8, 256);
+    L.total = o;
+    return L;
+}
+
+size_t prefill_ws_bytes(const bsa_kv_desc *d, const bsa_sel_params *p, int Tq) {
+    return pf_layout(d, p, Tq).total;
+}
+
+bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
+                          const bsa_sel_params *p, const void *summaries, const bsa_kv_desc *pd,
+                          const void *K_pos, const void *V_pos, const void *Q, int q_pos0, int Tq,
+                          float scale, float *out, float *lse, uint32_t *status, void *ws,
+                          size_t ws_bytes, cudaStream_t st) {
+    const int G = d->Hq / d->Hkv;
+    if (p->n_blocks > kPfMaxBlocks || kTile % G != 0 || G > 16) return BSA_ERR_UNSUPPORTED;
+    const PfLayout L = pf_layout(d, p, Tq);
+    if (ws_bytes < L.total) return BSA_ERR_WORKSPACE;
+    char *w = static_cast<char *>(ws);
+    PfArgs a;
+    a.Hq = d->Hq; a.Hkv = d->Hkv; a.G = G; a.D = d->D; a.nb = p->n_blocks;
+    a.L_max = d->L_max; a.Lpos = pd->L_max;
+    a.Tq = Tq; a.q_pos0 = q_pos0; a.pos_limit = p->pos_limit; a.budget = p->budget_tokens;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.Q = static_cast<const uint16_t *>(Q);
+    a.cent = static_cast<const float *>(summaries);
+    a.offsets = p->block_offsets;
+    a.kv_pos = p->kv_pos;
+    a.bitmap = reinterpret_cast<uint32_t *>(w + L.bitmap);
+    a.vis = reinterpret_cast<int32_t *>(w + L.vis);
+    a.qcount = reinterpret_cast<int32_t *>(w + L.qcount);
+    a.qlist = reinterpret_cast<int32_t *>(w + L.qlist);
+    a.tile_prefix = reinterpret_cast<int32_t *>(w + L.prefix);
+    a.work = reinterpret_cast<int32_t *>(w + L.work);
+    a.part_o = reinterpret_cast<float *>(w + L.part_o);
+    a.part_ml = reinterpret_cast<float2 *>(w + L.part_ml);
+    a.status = status;
+    a.out = out; a.lse = lse;
+    const int qpt = kTile / G;
+    a.n_local = d->Hkv * ((Tq + qpt - 1) / qpt);
+
+    CUtensorMap kp, vp, kl, vl;
+    if (!make_kv_tmap(&kp, d, K, kTile) || !make_kv_tmap(&vp, d, V, kTile) ||
+        !make_kv_tmap(&kl, pd, K_pos, kTile) || !make_kv_tmap(&vl, pd, V_pos, kTile))
+        return BSA_ERR_CUDA;
+    // zero the per-block counts and the work counter
+    BSA_CUDA_TRY(cudaMemsetAsync(w + L.qcount, 0, (size_t)d->Hkv * p->n_blocks * 4, st));
+    BSA_CUDA_TRY(cudaMemsetAsync(w + L.work, 0, 4, st));
+    // P1: selection
+    const size_t smem1 = ((size_t)a.nb * (a.D + 1) + (size_t)8 * G * a.D + a.nb) * 4;
+    BSA_CUDA_TRY(cudaFuncSetAttribute(prefill_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem1));
+    BSA_CUDA_TRY(launch_pdl(prefill_select_kernel,
+                            dim3((unsigned)div_up(Tq, kPfRowsPerCta), (unsigned)d->Hkv), dim3(256),
+                            smem1, st, a));
+    // P2: tile prefix over (KV head, block)
+    prefill_tiles_kernel<<<1, 1024, 0, st>>>(a);
+    BSA_LAUNCH_CHECK();
+    // P3: persistent tensor-core attention over local and grouped tiles
+    BSA_CUDA_TRY(cudaFuncSetAttribute(prefill_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      PfSmem::kBytes));
+    prefill_attend_kernel<<<num_sms(), kPfThreads, PfSmem::kBytes, st>>>(kp, vp, kl, vl, a);
+    BSA_LAUNCH_CHECK();
+    // P4: merge of every query's slots
+    BSA_CUDA_TRY(launch_pdl(prefill_merge_kernel, dim3((unsigned)Tq, (unsigned)d->Hkv), dim3(128), 0,
+                            st, a));
+    return BSA_OK;
 }
 
 }  // namespace bsa

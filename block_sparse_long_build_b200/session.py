@@ -103,6 +103,28 @@ class DecodeSession:
             self.select(q)
         self.decode(q)
 
+    # ---------------------------------------------------------------- prefill
+    def prefill_chunk(self, Q: torch.Tensor, q_pos0: int, out: torch.Tensor, lse: torch.Tensor,
+                      ws: torch.Tensor | None = None) -> torch.Tensor:
+        """Block-grouped prefill of the query rows Q [Tq, Hq, D] (bf16) at
+        positions q_pos0.. of a semantic-block workload: dense causal while
+        the prefix is shorter than the configured dense limit, otherwise the
+        chunk densely and causally plus the blocks each query selects under a
+        budget of 1/16 of the prefix.  Returns the workspace used."""
+        c, wl = self.cfg, self.wl
+        Tq = Q.shape[0]
+        sparse = q_pos0 >= c.dense_below
+        sel = N.sel_params(0, c.n_blocks, wl.block_offsets, wl.kv_pos, topk=-1,
+                           budget_tokens=q_pos0 // 16 if sparse else 0,
+                           local_start=wl.local_start, pos_limit=q_pos0 if sparse else 0)
+        pos_desc = N.kv_desc(wl.Kpos, c.Hq)
+        need = N.bsa_workspace_size(self.desc, sel, N.BSA_OP_PREFILL, Tq, 0)
+        if ws is None or ws.numel() < need:
+            ws = torch.zeros(need, dtype=torch.uint8, device=wl.device)
+        N.bsa_prefill_grouped(self.desc, wl.K, wl.V, sel, self.summaries, pos_desc, wl.Kpos,
+                              wl.Vpos, Q, q_pos0, Tq, self.scale, out, lse, ws, self.stream)
+        return ws
+
     # ------------------------------------------------------------ CUDA graphs
     def capture(self):
         """Captures one decode step into two CUDA graphs (with and without
