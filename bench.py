@@ -151,8 +151,12 @@ def _step_bytes(sess, t: int) -> tuple[int, int]:
     dec = tokens * c.D * 2 * esz + qo
     tot = dec
     if t % c.refresh == 0:
-        pages = sum(int(x) // c.block_size for x in cur) * c.Hkv
-        tot += pages * 2 * c.D * esz
+        if c.block_size:
+            rows = sum(int(x) // c.block_size for x in cur) * c.Hkv
+        else:
+            rows = c.n_blocks * c.B * c.Hkv
+        row_bytes = 2 * c.D * esz if c.kind == 2 else c.D * 4
+        tot += rows * row_bytes
     tot += c.B * c.Hkv * c.D * 2 * esz   # appended row
     return tot, dec
 
@@ -172,8 +176,8 @@ def run_ours(args, rank: int, world: int, device):
     wl = W.Workload(cfg, device)
     sess = DecodeSession(wl)
     sess.build_summaries()
-    L0 = cfg.L
-    inputs = [(wl.decode_query(t), *wl.decode_new_kv(t)) for t in range(max(K_steps, W_steps))]
+    L0 = int(wl.cur_len[0].item())   # rows in each cache when decoding starts
+    inputs =[(wl.decode_query(t), *wl.decode_new_kv(t)) for t in range(max(K_steps, W_steps))]
     torch.cuda.synchronize()
 
     # census: run the K steps once untimed to count each step's bytes
@@ -296,15 +300,12 @@ def run_ours(args, rank: int, world: int, device):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16" if cfg.kv_dtype == torch.bfloat16 else "f32",
         "data": "synthetic",
         "effective_kv_gbs": eff_gbs,
         "effective_kv_frac_of_8tbs": eff_gbs / 8000.0,
         "config": {
-            "workload": f"{cfg.name}: Quest-style paged decode, batch {cfg.B}, {cfg.Hkv} KV / "
-                        f"{cfg.Hq} query heads, head_dim {cfg.D}, bf16, context {cfg.L}, page "
-                        f"{cfg.block_size} min/max, budget {cfg.budget_tokens}, sink {cfg.sink}, "
-                        f"window {cfg.window}, refresh {cfg.refresh}",
+            "workload": f"{cfg.name}: " + " ".join((W.CONFIGS[cfg.name].__doc__ or "").split()),
             "global_batch": cfg.B * world,
             "seq_len": cfg.L,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -312,7 +313,8 @@ def run_ours(args, rank: int, world: int, device):
             "timing": "CUDA events per graph-replayed step on the launching stream",
         },
         "roofline": {
-            "kernel": "decode_tc_kernel (split-K sparse decode + fused LSE merge)",
+            "kernel": "bsa_decode: split-K sparse decode with the split merge inside a "
+                      "thread-block cluster (or the merge kernel when the splits do not fit one)",
             "bound": "hbm",
             "achieved": achieved,
             "peak": peak,
@@ -375,6 +377,92 @@ def cpu_baseline(cfg, wl, inputs, budget_s=15.0):
                       f"scaled to one {cfg.B}-sequence step"}
 
 
+def run_prefill(args, device):
+    """Block-grouped prefill of the semantic-block configuration: every
+    4096-query chunk of the 524,288-token context (dense while the prefix is
+    under 16k), one bsa_prefill_grouped call per chunk, each timed with CUDA
+    events; L2 is flushed before each chunk."""
+    from block_sparse_long_build_b200 import build as Bld
+    from block_sparse_long_build_b200 import native as N
+    from block_sparse_long_build_b200 import workloads as W
+    from block_sparse_long_build_b200.session import DecodeSession
+
+    Bld.build()
+    cfg = W.semantic(0)
+    if args.prefill_context:
+        cfg = cfg.scaled(L=args.prefill_context, budget_tokens=args.prefill_context // 16)
+    wl = W.Workload(cfg, device)
+    sess = DecodeSession(wl)
+    sess.build_summaries()
+    Tq = cfg.chunk
+    out = torch.empty(Tq, cfg.Hq, cfg.D, dtype=torch.float32, device=device)
+    lse = torch.empty(Tq, cfg.Hq, dtype=torch.float32, device=device)
+    flush = _flusher(device)
+    vis_all = None
+    chunks = list(range(0, cfg.L, Tq))
+    times, pairs = [], 0
+    ws = None
+    # warm-up on the first sparse chunk (one-time host setup, caches)
+    warm = next((p for p in chunks if p >= cfg.dense_below), 0)
+    ws = sess.prefill_chunk(wl.prefill_queries(warm, Tq), warm, out, lse, ws)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    sampler.start()
+    for p in chunks:
+        n = min(Tq, cfg.L - p)
+        Q = wl.prefill_queries(p, n)
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ws = sess.prefill_chunk(Q, p, out[:n], lse[:n], ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+        # (query head, key) pairs this chunk attends: local causal part plus
+        # the visible rows of every selected block
+        sparse = p >= cfg.dense_below
+        lo = p if sparse else 0
+        local = sum(p + i + 1 - lo for i in range(n)) * cfg.Hq
+        grouped = 0
+        if sparse:
+            cb = 256
+            words = ws[cb:cb + n * cfg.Hkv * 8 * 4].view(torch.int32).view(n, cfg.Hkv, 8)
+            bits = ((words.unsqueeze(-1) >> torch.arange(32, device=device)) & 1).reshape(n, cfg.Hkv, 256)
+            vis_off = cb + n * cfg.Hkv * 8 * 4
+            vis_off = (vis_off + 255) // 256 * 256
+            vis = ws[vis_off:vis_off + cfg.Hkv * cfg.n_blocks * 4].view(torch.int32).view(cfg.Hkv, cfg.n_blocks)
+            grouped = int((bits[:, :, :cfg.n_blocks].long() * vis.long()[None]).sum().item()) * cfg.G
+        pairs += local + grouped
+    clocks = sampler.stop()
+    total_ms = float(sum(times))
+    flops = 4.0 * pairs * cfg.D
+    tflops = flops / (total_ms / 1e3) / 1e12
+    peak = _bf16_peak()
+    return {
+        "metric": "block-grouped prefill, algorithmic TFLOP/s (4 x attended pairs x head_dim)",
+        "value": tflops, "unit": "TFLOP/s", "n_gpus": 1, "steps": len(chunks), "warmup": 1,
+        "ms_total": total_ms, "ms_per_chunk": total_ms / len(chunks),
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "prefill_tokens_per_s": cfg.L / (total_ms / 1e3),
+        "algorithmic_tflop": flops / 1e12,
+        "config": {"workload": f"semantic blocks: batch 1, {cfg.Hkv} KV / {cfg.Hq} query heads, "
+                               f"head_dim {cfg.D}, context {cfg.L}, {cfg.n_blocks} blocks, chunks of "
+                               f"{Tq}, dense below {cfg.dense_below}, budget prefix/16",
+                   "l2": "flushed before each chunk"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak[0], "unit": "TFLOP/s",
+                     "frac": tflops / peak[0], "peak_source": peak[1], "traffic": None},
+        "clocks": clocks,
+    }
+
+
+def _bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured (bf16_tflops_sustained)"
+    return 1400.0, "fallback 1.4 PFLOP/s sustained"
+
+
 def run_reference(args):
     """The oracle as it stands, on the host cores, same config and metric."""
     from block_sparse_long_build_b200 import workloads as W
@@ -411,17 +499,31 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=128)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="decode steps to time (default: the configuration's own count)")
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="quest")
+    ap.add_argument("--config", default="quest", help="tiny | quest | moba | largebatch | semantic")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the block-grouped prefill of the semantic configuration instead")
+    ap.add_argument("--prefill-context", type=int, default=0,
+                    help="context of the prefill run (default: the configuration's 524,288)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.steps is None:
+        from block_sparse_long_build_b200 import workloads as W
+        args.steps = W.CONFIGS[args.config](0).steps
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.prefill:
+        if rank == 0:
+            local = int(os.environ.get("LOCAL_RANK", "0"))
+            torch.cuda.set_device(local)
+            print(json.dumps(run_prefill(args, torch.device("cuda", local))), flush=True)
+        return 0
     if args.impl == "reference":
         if rank != 0:
             return 0
