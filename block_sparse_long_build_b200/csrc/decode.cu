@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
     for (int idx = 0; idx < my_count; ++idx) {
         const int st = idx % NST;
-        if (!mbar_wait_bounded(&wfull[st], (uint32_t)((idx / NST) & 1))) timed_out = true;
+        if (!timed_out && !mbar_wait_bounded(&wfull[st], (uint32_t)((idx / NST) & 1))) timed_out = true;
         const int nv = winfo[st].y;
         unsigned char *kp = ring + st * L::kPieceBytes;
         unsigned char *vp = kp + NH * kBoxBytes;

@@ -181,18 +181,39 @@ __global__ void __launch_bounds__(1024) prefill_tiles_kernel(PfArgs a) {
 }
 
 // ---------------------------------------------------------------- P3
+// Warp-specialised: warps 0..7 run the softmax, two threads per row (warp w
+// owns TMEM lanes 32*(w%4).. and the column half w/4); lane 0 of warp 8
+// issues every TMA load and every tcgen05.mma.  S is double-buffered in TMEM
+// so that S(t+1) = Q K(t+1)^T runs on the tensor cores while the softmax of
+// tile t runs; P.V of tile t follows the softmax.  O is rescaled only when a
+// row's running maximum grows by more than 2^8 (the exponentials then stay
+// below 256), so P.V rarely sits on the softmax's critical path.
+constexpr int kPfSoftWarps = 8;
+constexpr int kPfAttThreads = 32 * (kPfSoftWarps + 1);
+constexpr float kPfRescale = 8.0f;   // log2 of the largest exponential kept without rescaling
+
 struct PfSmem {
-    static constexpr int kQ = 0;                         // 2 boxes x 16 KiB
-    static constexpr int kStage = 32768;                 // 2 stages x (K 32 KiB + V 32 KiB)
-    static constexpr int kStageBytes = 65536;
-    static constexpr int kRowQ = kStage + 2 * kStageBytes;   // int [128] query index
-    static constexpr int kRowPos = kRowQ + kTile * 4;        // int [128] query position
-    static constexpr int kBars = kRowPos + kTile * 4;        // u64 full[2], mma_s, mma_o
-    static constexpr int kMisc = kBars + 4 * 8;              // int item, tmem base
+    static constexpr int kQ = 0;                          // 2 boxes x 16 KiB
+    static constexpr int kK = 32768;                      // 2 stages x 32 KiB
+    static constexpr int kV = kK + 2 * 32768;             // 2 stages x 32 KiB
+    static constexpr int kRowQ = kV + 2 * 32768;          // int [128] query index
+    static constexpr int kRowPos = kRowQ + kTile * 4;     // int [128] query position
+    static constexpr int kPair = kRowPos + kTile * 4;     // float [2][128] half-row maxima / sums
+    static constexpr int kBars = kPair + 2 * kTile * 4;   // u64: kfull[2] vfull[2] sfull[2] pfull[2] odone[2]
+    static constexpr int kMisc = kBars + 10 * 8;          // int item, tmem base
     static constexpr int kBytes = kMisc + 16 + 1024;
 };
 
-__global__ void __launch_bounds__(kPfThreads, 1)
+struct PfItem {
+    int g, kbeg, kend, jblk, mtile, ntiles;
+    bool local;
+};
+
+__device__ __forceinline__ void pair_sync(int q) {   // the two warps holding rows 32q..32q+31
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+}
+
+__global__ void __launch_bounds__(kPfAttThreads, 1)
     prefill_attend_kernel(const __grid_constant__ CUtensorMap tmKp, const __grid_constant__ CUtensorMap tmVp,
                           const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVl,
                           PfArgs a) {
@@ -202,24 +223,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     unsigned char *Qs = sm + PfSmem::kQ;
     int *rowq = reinterpret_cast<int *>(sm + PfSmem::kRowQ);
     int *rowpos = reinterpret_cast<int *>(sm + PfSmem::kRowPos);
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + PfSmem::kBars);
-    uint64_t *bar_s = full + 2, *bar_o = full + 3;
+    float *pairv = reinterpret_cast<float *>(sm + PfSmem::kPair);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PfSmem::kBars);
+    uint64_t *kfull = bars, *vfull = bars + 2, *sfull = bars + 4, *pfull = bars + 6, *odone = bars + 8;   // odone[2]
     int *item_sh = reinterpret_cast<int *>(sm + PfSmem::kMisc);
     uint32_t *tmem_sh = reinterpret_cast<uint32_t *>(sm + PfSmem::kMisc + 4);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = a.G, D = a.D;
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
             smem_u32(tmem_sh)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (tid == 0) {
         prefetch_tmap(&tmKp); prefetch_tmap(&tmVp); prefetch_tmap(&tmKl); prefetch_tmap(&tmVl);
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        mbar_init(bar_s, 1);
-        mbar_init(bar_o, 1);
+        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        mbar_init(&pfull[0], kPfSoftWarps);
+        mbar_init(&pfull[1], kPfSoftWarps);
+        mbar_init(&odone[0], 1);
+        mbar_init(&odone[1], 1);
         fence_mbar_init();
     }
     pdl_wait();
@@ -227,35 +250,33 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_sh;
-    const uint32_t tS = tmem, tO = tmem + 128;        // S (and P over its first 64 columns), O
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t tO = tmem + 256;                 // S0 = cols 0..127, S1 = 128..255, O = 256..383
     const int n_group = a.tile_prefix[a.Hkv * a.nb];
     const int n_items = a.n_local + n_group;
-    uint32_t full_use[2] = {0, 0}, s_use = 0, o_use = 0;
-    bool timed_out = false;
+    const int qpt = kTile / G;
+    const int tiles_per_head = (a.Tq + qpt - 1) / qpt;
     constexpr uint32_t kIdescQK = umma_idesc_bf16(128, 128, 0, 0);
     constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 128, 0, 1);
-    const int qpt = kTile / G;   // queries per tile
+    // phase counters (every role tracks the barriers it waits on)
+    uint32_t kuse[2] = {0, 0}, vuse[2] = {0, 0}, puse[2] = {0, 0};   // issuing lane only
+    uint32_t sbase[2] = {0, 0}, obase[2] = {0, 0};                       // every thread
+    bool timed_out = false;
 
     for (;;) {
         if (tid == 0) *item_sh = atomicAdd(a.work, 1);
         __syncthreads();
         const int item = *item_sh;
         if (item >= n_items) break;
-        // ---- decode the work item
-        int g, kbeg, kend, jblk = -1, mtile = 0;
-        bool local = item < a.n_local;
-        const int tiles_per_head = (a.Tq + qpt - 1) / qpt;
-        if (local) {
-            g = item / tiles_per_head;
+        // ---- decode the work item (every thread, same result)
+        PfItem it;
+        it.local = item < a.n_local;
+        it.jblk = -1;
+        if (it.local) {
+            it.g = item / tiles_per_head;
             const int i0 = (item % tiles_per_head) * qpt;
-            const int ilast = min(a.Tq, i0 + qpt) - 1;
-            kbeg = a.pos_limit;
-            kend = a.q_pos0 + ilast + 1;
-            const int r = tid, i = i0 + r / G;
-            rowq[r] = i < a.Tq ? i : -1;
-            rowpos[r] = a.q_pos0 + i;
-            mtile = i0;
+            it.mtile = i0;
+            it.kbeg = a.pos_limit;
+            it.kend = a.q_pos0 + min(a.Tq, i0 + qpt);
         } else {
             const int u = item - a.n_local;
             int lo = 0, hi = a.Hkv * a.nb - 1;   // largest e with prefix[e] <= u
@@ -263,174 +284,248 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 const int mid = (lo + hi + 1) >> 1;
                 if (a.tile_prefix[mid] <= u) lo = mid; else hi = mid - 1;
             }
-            g = lo / a.nb;
-            jblk = lo % a.nb;
-            mtile = u - a.tile_prefix[lo];
-            const int r0 = min(max(a.offsets[(int64_t)g * (a.nb + 1) + jblk], 0), a.L_max);
-            kbeg = r0;
-            kend = r0 + a.vis[g * a.nb + jblk];
-            const int cnt = a.qcount[g * a.nb + jblk];
-            const int idx = mtile * kTile + tid, qi = idx / G;
-            rowq[tid] = qi < cnt ? a.qlist[((int64_t)g * a.nb + jblk) * a.Tq + qi] : -1;
-            rowpos[tid] = 0x7fffffff;   // every key of the visible prefix is earlier
+            it.g = lo / a.nb;
+            it.jblk = lo % a.nb;
+            it.mtile = u - a.tile_prefix[lo];
+            it.kbeg = min(max(a.offsets[(int64_t)it.g * (a.nb + 1) + it.jblk], 0), a.L_max);
+            it.kend = it.kbeg + a.vis[it.g * a.nb + it.jblk];
+        }
+        it.ntiles = max(0, (it.kend - it.kbeg + kTile - 1) / kTile);
+        const int g = it.g;
+        if (tid < kTile) {
+            const int r = tid;
+            if (it.local) {
+                const int i = it.mtile + r / G;
+                rowq[r] = i < a.Tq ? i : -1;
+                rowpos[r] = a.q_pos0 + i;
+            } else {
+                const int cnt = a.qcount[g * a.nb + it.jblk];
+                const int idx = it.mtile * kTile + r, qi = idx / G;
+                rowq[r] = qi < cnt ? a.qlist[((int64_t)g * a.nb + it.jblk) * a.Tq + qi] : -1;
+                rowpos[r] = 0x7fffffff;   // every key of a visible prefix is earlier
+            }
         }
         __syncthreads();
         // ---- gather Q rows (bf16) into the swizzled K-major layout
-        for (int c = tid; c < kTile * 16; c += kPfThreads) {
+        for (int c = tid; c < kTile * 16; c += kPfAttThreads) {
             const int r = c >> 4, ch = c & 15, half = ch >> 3, cc = ch & 7;
             const int qi = rowq[r];
             uint4 v = make_uint4(0, 0, 0, 0);
             if (qi >= 0) {
-                const int hh = local ? (r % G) : ((mtile * kTile + r) % G);
+                const int hh = r % G;
                 v = *reinterpret_cast<const uint4 *>(
                     a.Q + ((int64_t)qi * a.Hq + (int64_t)g * G + hh) * D + ch * 8);
             }
             *reinterpret_cast<uint4 *>(Qs + half * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
         }
         fence_proxy_async_smem();
-        const int ntiles = max(0, (kend - kbeg + kTile - 1) / kTile);
-        auto issue_kv = [&](int t, int st) {
-            unsigned char *base = sm + PfSmem::kStage + st * PfSmem::kStageBytes;
-            mbar_arrive_expect_tx(&full[st], 4 * 16384);
-            const CUtensorMap *mk = local ? &tmKl : &tmKp;
-            const CUtensorMap *mv = local ? &tmVl : &tmVp;
-            const int row = kbeg + t * kTile;
-            tma_load_4d(base, mk, &full[st], 0, row, g, 0);
-            tma_load_4d(base + 16384, mk, &full[st], 64, row, g, 0);
-            tma_load_4d(base + 32768, mv, &full[st], 0, row, g, 0);
-            tma_load_4d(base + 49152, mv, &full[st], 64, row, g, 0);
-        };
-        if (tid == 0 && ntiles > 0) issue_kv(0, 0);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        const int T = it.ntiles;
 
-        float m_run = kPfNegInf, l_run = 0.0f;
-        const int my_pos = rowpos[tid];
-        for (int t = 0; t < ntiles; ++t) {
-            const int st = t & 1;
-            if (tid == 0) {
-                if (t + 1 < ntiles) issue_kv(t + 1, st ^ 1);
-                if (!mbar_wait_bounded(&full[st], full_use[st] & 1)) timed_out = true;
+        // Barrier protocol.  kfull/vfull/pfull are waited by the issuing lane
+        // for every phase (plain counters).  S(t) completes on sfull[t&1] and
+        // P.V(t) on odone[t&1]; a wait for one of them is for a specific MMA
+        // whose predecessor on the same barrier is already known complete, so
+        // the parity follows from the MMA's index: base[b] (MMAs on barrier b
+        // in earlier items) + t/2.
+        auto par = [](uint32_t base, int t) { return (base + (uint32_t)(t >> 1)) & 1u; };
+        if (warp == kPfSoftWarps) {
+            // ================= TMA + MMA issue (one lane)
+            if (lane == 0) {
+                const CUtensorMap *mk = it.local ? &tmKl : &tmKp;
+                const CUtensorMap *mv = it.local ? &tmVl : &tmVp;
+                auto load_k = [&](int t) {
+                    unsigned char *dst = sm + PfSmem::kK + (t & 1) * 32768;
+                    mbar_arrive_expect_tx(&kfull[t & 1], 32768);
+                    tma_load_4d(dst, mk, &kfull[t & 1], 0, it.kbeg + t * kTile, g, 0);
+                    tma_load_4d(dst + 16384, mk, &kfull[t & 1], 64, it.kbeg + t * kTile, g, 0);
+                };
+                auto load_v = [&](int t) {
+                    unsigned char *dst = sm + PfSmem::kV + (t & 1) * 32768;
+                    mbar_arrive_expect_tx(&vfull[t & 1], 32768);
+                    tma_load_4d(dst, mv, &vfull[t & 1], 0, it.kbeg + t * kTile, g, 0);
+                    tma_load_4d(dst + 16384, mv, &vfull[t & 1], 64, it.kbeg + t * kTile, g, 0);
+                };
+                auto pv = [&](int t) {   // O (+)= P(t) V(t), P read from S(t & 1)
+                    if (!timed_out && !mbar_wait_bounded(&pfull[t & 1], puse[t & 1] & 1)) timed_out = true;
+                    ++puse[t & 1];
+                    if (!timed_out && !mbar_wait_bounded(&vfull[t & 1], vuse[t & 1] & 1)) timed_out = true;
+                    ++vuse[t & 1];
+                    tc_fence_after();
+                    const uint32_t v0 = smem_u32(sm + PfSmem::kV + (t & 1) * 32768);
+                    const uint32_t tP = tmem + (t & 1) * 128;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint64_t vd = umma_sdesc_sw128(v0 + k * 2048, 16384, 1024);
+                        umma_ts(tO, tP + k * 8, vd, kIdescPV, (t > 0 || k > 0) ? 1u : 0u);
+                        umma_ts(tO, tP + 64 + k * 8, vd, kIdescPV, 1u);
+                    }
+                    umma_commit(&odone[t & 1]);
+                };
+                for (int t = 0; t < 2 && t < T; ++t) { load_k(t); load_v(t); }
+                for (int t = 0; t < T; ++t) {
+                    if (!timed_out && !mbar_wait_bounded(&kfull[t & 1], kuse[t & 1] & 1)) timed_out = true;
+                    ++kuse[t & 1];
+                    if (t >= 2) {   // S(t&1) and V stage t&1 are free once P.V(t-2) is done
+                        if (!timed_out && !mbar_wait_bounded(&odone[t & 1], par(obase[t & 1], t - 2))) timed_out = true;
+                        load_v(t);
+                    }
+                    tc_fence_after();
+                    const uint32_t q0 = smem_u32(Qs);
+                    const uint32_t k0 = smem_u32(sm + PfSmem::kK + (t & 1) * 32768);
+                    const uint32_t tS = tmem + (t & 1) * 128;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                        umma_ss(tS, umma_sdesc_sw128(q0 + off, 16, 1024),
+                                umma_sdesc_sw128(k0 + off, 16, 1024), kIdescQK, k > 0);
+                    }
+                    umma_commit(&sfull[t & 1]);
+                    if (t + 2 < T) {   // K stage t&1 is free once S(t) is done
+                        if (!timed_out && !mbar_wait_bounded(&sfull[t & 1], par(sbase[t & 1], t))) timed_out = true;
+                        load_k(t + 2);
+                    }
+                    if (t >= 1) pv(t - 1);
+                }
+                if (T >= 1) pv(T - 1);
+            }
+            __syncwarp();
+        } else {
+            // ================= softmax warps
+            const int q = warp & 3, half = warp >> 2;
+            const int r = q * 32 + lane;                 // this thread's row
+            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+            const int my_pos = rowpos[r];
+            float m_used = kPfNegInf, l_part = 0.0f;
+            for (int t = 0; t < T; ++t) {
+                if (!timed_out && !mbar_wait_bounded(&sfull[t & 1], par(sbase[t & 1], t))) timed_out = true;
                 tc_fence_after();
-                const uint32_t q0 = smem_u32(Qs);
-                const uint32_t k0 = smem_u32(sm + PfSmem::kStage + st * PfSmem::kStageBytes);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                    umma_ss(tS, umma_sdesc_sw128(q0 + off, 16, 1024), umma_sdesc_sw128(k0 + off, 16, 1024),
-                            kIdescQK, k > 0);
-                }
-                umma_commit(bar_s);
-            }
-            ++full_use[st];
-            if (!mbar_wait_bounded(bar_s, s_use & 1)) timed_out = true;
-            ++s_use;
-            tc_fence_after();
-            // ---- online softmax, one thread per row
-            uint32_t sv[4][32];
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + lane_base + c4 * 32, sv[c4]);
-            tmem_ld_wait();
-            const int key0 = kbeg + t * kTile;
-            float mx = kPfNegInf;
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4)
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int kr = key0 + c4 * 32 + e;
-                    const bool ok = kr < kend && kr <= my_pos;
-                    const float v = ok ? __uint_as_float(sv[c4][e]) * a.scale_log2 : kPfNegInf;
-                    sv[c4][e] = __float_as_uint(v);
-                    mx = fmaxf(mx, v);
-                }
-            const float m_new = fmaxf(m_run, mx);
-            const float corr = m_new == kPfNegInf ? 1.0f : exp2f(m_run - m_new);
-            // P = P_hi + P_lo, both bf16: columns 0..63 of S take P_hi, 64..127
-            // P_lo (the row's S values are all in registers by now), so the
-            // weights carry ~2^-17 relative error instead of 2^-9
-            float lsum = 0.0f;
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t ph[16], pl[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float p0 = m_new == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[c4][e]) - m_new);
-                    const float p1 = m_new == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[c4][e + 1]) - m_new);
-                    lsum += p0 + p1;
-                    const float h0 = bf16_round(p0), h1 = bf16_round(p1);
-                    ph[e / 2] = pack_bf16x2(h0, h1);
-                    pl[e / 2] = pack_bf16x2(p0 - h0, p1 - h1);
-                }
-                tmem_st16(tS + lane_base + c4 * 16, ph);
-                tmem_st16(tS + lane_base + 64 + c4 * 16, pl);
-            }
-            l_run = l_run * corr + lsum;
-            // rescale the O accumulator; tcgen05.ld/st are warp-collective, so
-            // the whole warp takes the branch when any of its rows needs it
-            if (t > 0 && __any_sync(0xffffffffu, corr != 1.0f)) {
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t ov[32];
-                    tmem_ld32(tO + lane_base + c4 * 32, ov);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-                    tmem_st32(tO + lane_base + c4 * 32, ov);
-                }
-            }
-            m_run = m_new;
-            tmem_st_wait();
-            tc_fence_before();
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t v0 = smem_u32(sm + PfSmem::kStage + st * PfSmem::kStageBytes + 32768);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint64_t vd = umma_sdesc_sw128(v0 + k * 2048, 16384, 1024);
-                    umma_ts(tO, tS + k * 8, vd, kIdescPV, (t > 0 || k > 0) ? 1u : 0u);   // P_hi
-                    umma_ts(tO, tS + 64 + k * 8, vd, kIdescPV, 1u);                       // P_lo
-                }
-                umma_commit(bar_o);
-            }
-            if (!mbar_wait_bounded(bar_o, o_use & 1)) timed_out = true;
-            ++o_use;
-            tc_fence_after();
-        }
-        // ---- epilogue: this item's partial for every live row (the TMEM loads
-        // are warp-collective and run for every row; dead rows drop them)
-        const int qi = rowq[tid];
-        int64_t rec = -1;
-        if (qi >= 0) {
-            const int hh = local ? (tid % G) : ((mtile * kTile + tid) % G);
-            int slot = 0;
-            if (!local) {
-                const uint32_t *bm = a.bitmap + ((int64_t)qi * a.Hkv + g) * kPfWords;
-                for (int w = 0; w < (jblk >> 5); ++w) slot += __popc(bm[w]);
-                slot += __popc(bm[jblk >> 5] & ((1u << (jblk & 31)) - 1u)) + 1;
-            }
-            if (slot < kPfSlots) rec = (((int64_t)qi * a.Hkv + g) * kPfSlots + slot) * G + hh;
-        }
-        float *po = rec >= 0 ? a.part_o + rec * D : nullptr;
-        if (ntiles > 0) {
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t ov[32];
-                tmem_ld32(tO + lane_base + c4 * 32, ov);
+                const uint32_t tS = tmem + (t & 1) * 128;
+                uint32_t sv[2][32];
+                tmem_ld32(tS + lane_base + half * 64, sv[0]);
+                tmem_ld32(tS + lane_base + half * 64 + 32, sv[1]);
                 tmem_ld_wait();
-                if (po) {
+                const int key0 = it.kbeg + t * kTile + half * 64;
+                float mx = kPfNegInf;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4 *>(po + c4 * 32 + e) =
-                            make_float4(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1]),
-                                        __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
+                for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int kr = key0 + c2 * 32 + e;
+                        const bool ok = kr < it.kend && kr <= my_pos;
+                        const float v = ok ? __uint_as_float(sv[c2][e]) * a.scale_log2 : kPfNegInf;
+                        sv[c2][e] = __float_as_uint(v);
+                        mx = fmaxf(mx, v);
+                    }
+                // both halves of the row have read S(t) before either writes P
+                pairv[half * kTile + r] = mx;
+                pair_sync(q);
+                const float m_tile = fmaxf(pairv[r], pairv[kTile + r]);
+                pair_sync(q);
+                // lazy rescale: keep the reference maximum unless this tile
+                // exceeds it by more than 2^8
+                bool rescale = false;
+                float factor = 1.0f, m_ref = m_used;
+                if (m_tile != kPfNegInf) {
+                    if (m_used == kPfNegInf) {
+                        m_ref = m_tile;   // nothing accumulated yet for this row
+                    } else if (m_tile > m_used + kPfRescale) {
+                        rescale = true;
+                        factor = exp2f(m_used - m_tile);
+                        m_ref = m_tile;
+                    }
                 }
+                if (t > 0 && __any_sync(0xffffffffu, rescale)) {
+                    // O must hold P.V(t-1) before it is scaled
+                    if (!timed_out && !mbar_wait_bounded(&odone[(t - 1) & 1], par(obase[(t - 1) & 1], t - 1)))
+                        timed_out = true;
+                    tc_fence_after();
+#pragma unroll
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        uint32_t ov[32];
+                        tmem_ld32(tO + lane_base + half * 64 + c2 * 32, ov);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+                        tmem_st32(tO + lane_base + half * 64 + c2 * 32, ov);
+                    }
+                }
+                l_part *= factor;
+                m_used = m_ref;
+                // P = P_hi + P_lo (bf16) over this half's 64 keys: P_hi in the
+                // tile's S columns 32*half.., P_lo in 64 + 32*half..
+                float lsum = 0.0f;
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    uint32_t ph[16], pl[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float p0 = m_used == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[c2][e]) - m_used);
+                        const float p1 = m_used == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[c2][e + 1]) - m_used);
+                        lsum += p0 + p1;
+                        const float h0 = bf16_round(p0), h1 = bf16_round(p1);
+                        ph[e / 2] = pack_bf16x2(h0, h1);
+                        pl[e / 2] = pack_bf16x2(p0 - h0, p1 - h1);
+                    }
+                    tmem_st16(tS + lane_base + half * 32 + c2 * 16, ph);
+                    tmem_st16(tS + lane_base + 64 + half * 32 + c2 * 16, pl);
+                }
+                l_part += lsum;
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pfull[t & 1]);
             }
-        } else if (po) {
-            for (int d = 0; d < D; ++d) po[d] = 0.0f;
+            // ---- epilogue: wait for the last two P.V, then this item's partial
+            if (T >= 1 && !timed_out && !mbar_wait_bounded(&odone[(T - 1) & 1], par(obase[(T - 1) & 1], T - 1)))
+                timed_out = true;
+            if (T >= 2 && !timed_out && !mbar_wait_bounded(&odone[(T - 2) & 1], par(obase[(T - 2) & 1], T - 2)))
+                timed_out = true;
+            tc_fence_after();
+            pairv[half * kTile + r] = l_part;
+            pair_sync(q);
+            const float l_row = pairv[r] + pairv[kTile + r];
+            pair_sync(q);
+            const int qi = rowq[r];
+            int64_t rec = -1;
+            if (qi >= 0) {
+                int slot = 0;
+                if (!it.local) {
+                    const uint32_t *bm = a.bitmap + ((int64_t)qi * a.Hkv + g) * kPfWords;
+                    for (int w = 0; w < (it.jblk >> 5); ++w) slot += __popc(bm[w]);
+                    slot += __popc(bm[it.jblk >> 5] & ((1u << (it.jblk & 31)) - 1u)) + 1;
+                }
+                if (slot < kPfSlots)
+                    rec = (((int64_t)qi * a.Hkv + g) * kPfSlots + slot) * G + (r % G);
+            }
+            float *po = rec >= 0 ? a.part_o + rec * D + half * 64 : nullptr;
+            if (T > 0) {
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + lane_base + half * 64 + c2 * 32, ov);
+                    tmem_ld_wait();
+                    if (po) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4 *>(po + c2 * 32 + e) =
+                                make_float4(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1]),
+                                            __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
+                    }
+                }
+            } else if (po) {
+                for (int d = 0; d < 64; ++d) po[d] = 0.0f;
+            }
+            if (rec >= 0 && half == 0) a.part_ml[rec] = make_float2(m_used, l_row);
         }
-        if (rec >= 0) a.part_ml[rec] = make_float2(m_run, l_run);
+        // every role advances the per-barrier MMA counts by this item's tiles
+        sbase[0] += (uint32_t)((T + 1) >> 1);
+        sbase[1] += (uint32_t)(T >> 1);
+        obase[0] += (uint32_t)((T + 1) >> 1);
+        obase[1] += (uint32_t)(T >> 1);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
@@ -438,7 +533,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (timed_out) atomicOr(a.status, 8u);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
 }
 
 // ---------------------------------------------------------------- P4
@@ -547,7 +642,7 @@ bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
     // P3: persistent tensor-core attention over local and grouped tiles
     BSA_CUDA_TRY(cudaFuncSetAttribute(prefill_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       PfSmem::kBytes));
-    prefill_attend_kernel<<<num_sms(), kPfThreads, PfSmem::kBytes, st>>>(kp, vp, kl, vl, a);
+    prefill_attend_kernel<<<num_sms(), kPfAttThreads, PfSmem::kBytes, st>>>(kp, vp, kl, vl, a);
     BSA_LAUNCH_CHECK();
     // P4: merge of every query's slots
     BSA_CUDA_TRY(launch_pdl(prefill_merge_kernel, dim3((unsigned)Tq, (unsigned)d->Hkv), dim3(128), 0,

@@ -43,6 +43,7 @@ def _check_chunk(cfg, wl, sess, p, Tq, rows):
     out_h, lse_h = out.cpu().numpy(), lse.cpu().numpy()
     assert np.isfinite(out_h).all() and np.isfinite(lse_h).all()
     ws_u32 = ws.cpu().numpy().view(np.uint32)
+    assert ws_u32[0] == 0, f"device status bits {ws_u32[0]:#x} (timeout or selection overflow)"
     cb = 256 // 4   # status + counters area of the workspace, in words (B*Hkv <= 63)
     bitmap = ws_u32[cb:cb + Tq * cfg.Hkv * 8].reshape(Tq, cfg.Hkv, 8)
     sparse = p >= cfg.dense_below
