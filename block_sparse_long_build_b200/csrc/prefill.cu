@@ -75,24 +75,19 @@ __global__ void __launch_bounds__(256) prefill_select_kernel(PfArgs a) {
     float *cs = psm;                                   // [nb][D+1]
     float *qv = cs + nb * (D + 1);                     // [8 warps][G][D]
     int *visS = reinterpret_cast<int *>(qv + 8 * G * D);   // [nb]
-    __shared__ int min_vis_sh;
     const int g = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_wait();
     const float *cg = a.cent + (int64_t)g * nb * D;
     for (int e = tid; e < nb * D; e += blockDim.x) cs[(e / D) * (D + 1) + e % D] = cg[e];
     const int32_t *off = a.offsets + (int64_t)g * (nb + 1);
     const int32_t *pos = a.kv_pos + (int64_t)g * a.L_max;
-    if (tid == 0) min_vis_sh = 0x7fffffff;
-    __syncthreads();
     for (int j = tid; j < nb; j += blockDim.x) {
         const int r0 = min(max(off[j], 0), a.L_max), r1 = min(max(off[j + 1], r0), a.L_max);
         const int v = pf_visible(pos, r0, r1, a.pos_limit);
         visS[j] = v;
         if (blockIdx.x == 0) a.vis[g * nb + j] = v;
-        if (v > 0) atomicMin(&min_vis_sh, v);
     }
     __syncthreads();
-    const int min_vis = min_vis_sh;
     float *qw = qv + warp * G * D;
     for (int r = 0; r < kPfRowsPerCta / 8; ++r) {
         const int i = blockIdx.x * kPfRowsPerCta + warp * (kPfRowsPerCta / 8) + r;
@@ -100,30 +95,56 @@ __global__ void __launch_bounds__(256) prefill_select_kernel(PfArgs a) {
         const uint16_t *qi = a.Q + ((int64_t)i * a.Hq + (int64_t)g * G) * D;
         for (int e = lane; e < G * D; e += 32) qw[e] = bf16_to_f32(qi[e]);
         __syncwarp();
-        // lane owns blocks lane + 32 t; composite keys (orderable score, ~index)
+        // lane owns blocks lane + 32 t; composite keys (orderable score, ~index).
+        // The (block, head) fma chains are interleaved over d for ILP; each
+        // chain still runs d = 0..D-1 in order.
         unsigned long long key[kPfWords];
+        {
+            constexpr int kMaxGh = 4;   // heads accumulated together per pass
+            float tot[kPfWords];
+            for (int h0 = 0; h0 < G; h0 += kMaxGh) {
+                float acc[kPfWords][kMaxGh];
 #pragma unroll
-        for (int t = 0; t < kPfWords; ++t) {
-            key[t] = 0ull;
-            const int j = lane + 32 * t;
-            if (j < nb && visS[j] > 0) {
-                const float *c = cs + j * (D + 1);
-                float tot = 0.0f;
-                for (int h = 0; h < G; ++h) {
-                    const float *qh = qw + h * D;
-                    float acc = 0.0f;
-                    for (int d = 0; d < D; ++d) acc = __fmaf_rn(qh[d], c[d], acc);
-                    tot = h == 0 ? acc : __fadd_rn(tot, acc);
+                for (int t = 0; t < kPfWords; ++t)
+#pragma unroll
+                    for (int h = 0; h < kMaxGh; ++h) acc[t][h] = 0.0f;
+                for (int d = 0; d < D; ++d) {
+                    float qd[kMaxGh];
+#pragma unroll
+                    for (int h = 0; h < kMaxGh; ++h) qd[h] = h0 + h < G ? qw[(h0 + h) * D + d] : 0.0f;
+#pragma unroll
+                    for (int t = 0; t < kPfWords; ++t) {
+                        const int j = min(lane + 32 * t, nb - 1);
+                        const float c = cs[j * (D + 1) + d];
+#pragma unroll
+                        for (int h = 0; h < kMaxGh; ++h) acc[t][h] = __fmaf_rn(qd[h], c, acc[t][h]);
+                    }
                 }
-                uint32_t k32 = f32_order_key(__fadd_rn(tot, 0.0f));
-                if (k32 == 0) k32 = 1;
-                key[t] = ((unsigned long long)k32 << 32) | (0xffffffffu - (uint32_t)j);
+#pragma unroll
+                for (int t = 0; t < kPfWords; ++t)
+#pragma unroll
+                    for (int h = 0; h < kMaxGh; ++h)
+                        if (h0 + h < G) tot[t] = (h0 + h == 0) ? acc[t][h] : __fadd_rn(tot[t], acc[t][h]);
+            }
+#pragma unroll
+            for (int t = 0; t < kPfWords; ++t) {
+                key[t] = 0ull;
+                const int j = lane + 32 * t;
+                // only candidates that can ever fit the budget
+                if (j < nb && visS[j] > 0 && visS[j] <= a.budget) {
+                    uint32_t k32 = f32_order_key(__fadd_rn(tot[t], 0.0f));
+                    if (k32 == 0) k32 = 1;
+                    key[t] = ((unsigned long long)k32 << 32) | (0xffffffffu - (uint32_t)j);
+                }
             }
         }
-        // greedy walk in rank order: take a block when its visible rows fit
+        // greedy walk in rank order: take a block when its visible rows fit.
+        // What is left of the budget only shrinks, so a block that does not
+        // fit now never will: after each take such blocks are dropped, and the
+        // best remaining candidate always fits.
         uint32_t selbits = 0;   // bit t: block lane + 32 t selected
         int remaining = a.budget, nsel = 0;
-        while (remaining >= min_vis && nsel < kPfMaxSel) {
+        while (nsel < kPfMaxSel) {
             unsigned long long best = 0ull;
 #pragma unroll
             for (int t = 0; t < kPfWords; ++t) best = key[t] > best ? key[t] : best;
@@ -134,23 +155,17 @@ __global__ void __launch_bounds__(256) prefill_select_kernel(PfArgs a) {
             }
             if (best == 0ull) break;
             const int j = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
-            const int v = visS[j];
-            const bool take = v <= remaining;
-            if (lane == (j & 31)) {
-#pragma unroll
-                for (int t = 0; t < kPfWords; ++t)
-                    if (t == (j >> 5)) {
-                        key[t] = 0ull;
-                        if (take) selbits |= 1u << t;
-                    }
+            remaining -= visS[j];
+            ++nsel;
+            if (lane == (j & 31)) selbits |= 1u << (j >> 5);
+            if (lane == 0) {
+                const int p = atomicAdd(&a.qcount[g * nb + j], 1);
+                a.qlist[((int64_t)g * nb + j) * a.Tq + p] = i;
             }
-            if (take) {
-                remaining -= v;
-                ++nsel;
-                if (lane == 0) {
-                    const int p = atomicAdd(&a.qcount[g * nb + j], 1);
-                    a.qlist[((int64_t)g * nb + j) * a.Tq + p] = i;
-                }
+#pragma unroll
+            for (int t = 0; t < kPfWords; ++t) {
+                const int jj = lane + 32 * t;
+                if (key[t] && (jj == j || visS[jj] > remaining)) key[t] = 0ull;
             }
         }
         if (nsel >= kPfMaxSel && lane == 0) atomicOr(a.status, 4u);
@@ -544,24 +559,31 @@ __global__ void __launch_bounds__(128) prefill_merge_kernel(PfArgs a) {
     int nsel = 0;
     for (int w = 0; w < kPfWords; ++w) nsel += __popc(bm[w]);
     const int nslot = min(1 + nsel, kPfSlots);
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-        const int hh = e / D, d = e % D;
-        float m = kPfNegInf, l = 0.0f, o = 0.0f;
+    const int D4 = D / 4;
+    // one thread per (head, 4 dimensions); slots merged in slot order, with
+    // all of a pass's loads independent of one another
+    for (int e = threadIdx.x; e < G * D4; e += blockDim.x) {
+        const int hh = e / D4, d4 = e % D4;
+        const int64_t rec0 = ((int64_t)i * a.Hkv + g) * kPfSlots * G + hh;
+        float M = kPfNegInf;
+#pragma unroll 8
+        for (int s = 0; s < nslot; ++s) M = fmaxf(M, __ldcg(&a.part_ml[rec0 + (int64_t)s * G]).x);
+        float L = 0.0f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
         for (int s = 0; s < nslot; ++s) {
-            const int64_t rec = (((int64_t)i * a.Hkv + g) * kPfSlots + s) * G + hh;
+            const int64_t rec = rec0 + (int64_t)s * G;
             const float2 ml = __ldcg(&a.part_ml[rec]);
-            const float ov = __ldcg(&a.part_o[rec * D + d]);
-            if (ml.x != kPfNegInf) {
-                const float mn = fmaxf(m, ml.x);
-                const float c_old = exp2f(m - mn), c_new = exp2f(ml.x - mn);
-                l = l * c_old + ml.y * c_new;
-                o = o * c_old + ov * c_new;
-                m = mn;
-            }
+            const float4 ov = __ldcg(reinterpret_cast<const float4 *>(a.part_o + rec * D) + d4);
+            const float w = ml.x != kPfNegInf ? exp2f(ml.x - M) : 0.0f;
+            L += ml.y * w;
+            O.x += ov.x * w; O.y += ov.y * w; O.z += ov.z * w; O.w += ov.w * w;
         }
         const int64_t orow = (int64_t)i * a.Hq + (int64_t)g * G + hh;
-        a.out[orow * D + d] = l > 0.0f ? o / l : 0.0f;
-        if (d == 0 && a.lse) a.lse[orow] = l > 0.0f ? (m + log2f(l)) * kPfLn2 : kPfNegInf;
+        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+        reinterpret_cast<float4 *>(a.out + orow * D)[d4] =
+            make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+        if (d4 == 0 && a.lse) a.lse[orow] = L > 0.0f ? (M + log2f(L)) * kPfLn2 : kPfNegInf;
     }
 }
 
