@@ -32,8 +32,11 @@ constexpr int kPfMaxBlocks = 256;          // blocks per KV head (bitmap of 8 wo
 constexpr int kPfWords = kPfMaxBlocks / 32;
 constexpr int kPfMaxSel = 64;              // selected blocks kept per (query, KV head)
 constexpr int kPfSlots = kPfMaxSel + 1;    // slot 0 = local part
-constexpr int kPfRowsPerCta = 64;          // P1 query rows per CTA
+constexpr int kPfSelWarps = 16;            // P1 warps per CTA (8 when shared memory is short)
+constexpr int kPfRowsPerWarp = 8;          // P1 query rows per warp
+constexpr int kPfCentStride = 132;         // padded centre row (floats): 16-byte rows, conflict-free
 constexpr int kTile = 128;                 // rows per MMA tile, keys per key tile
+constexpr size_t kMaxSmemPerCta = 227 * 1024;   // opt-in dynamic shared memory per CTA
 constexpr int kPfThreads = 128;
 constexpr float kPfNegInf = -__builtin_huge_valf();
 constexpr float kPfLn2 = 0.69314718055994530942f;
@@ -69,16 +72,17 @@ __device__ __forceinline__ int pf_visible(const int32_t *pos, int r0, int r1, in
 }
 
 // ---------------------------------------------------------------- P1
-__global__ void __launch_bounds__(256) prefill_select_kernel(PfArgs a) {
+__global__ void __launch_bounds__(32 * kPfSelWarps) prefill_select_kernel(PfArgs a) {
     extern __shared__ float psm[];
     const int D = a.D, G = a.G, nb = a.nb;
-    float *cs = psm;                                   // [nb][D+1]
-    float *qv = cs + nb * (D + 1);                     // [8 warps][G][D]
-    int *visS = reinterpret_cast<int *>(qv + 8 * G * D);   // [nb]
+    const int nw = blockDim.x >> 5;
+    float *cs = psm;                                   // [nb][kPfCentStride]
+    float *qv = cs + nb * kPfCentStride;               // [nw][G][D]
+    int *visS = reinterpret_cast<int *>(qv + nw * G * D);   // [nb]
     const int g = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_wait();
     const float *cg = a.cent + (int64_t)g * nb * D;
-    for (int e = tid; e < nb * D; e += blockDim.x) cs[(e / D) * (D + 1) + e % D] = cg[e];
+    for (int e = tid; e < nb * D; e += blockDim.x) cs[(e / D) * kPfCentStride + e % D] = cg[e];
     const int32_t *off = a.offsets + (int64_t)g * (nb + 1);
     const int32_t *pos = a.kv_pos + (int64_t)g * a.L_max;
     for (int j = tid; j < nb; j += blockDim.x) {
@@ -89,8 +93,8 @@ __global__ void __launch_bounds__(256) prefill_select_kernel(PfArgs a) {
     }
     __syncthreads();
     float *qw = qv + warp * G * D;
-    for (int r = 0; r < kPfRowsPerCta / 8; ++r) {
-        const int i = blockIdx.x * kPfRowsPerCta + warp * (kPfRowsPerCta / 8) + r;
+    for (int r = 0; r < kPfRowsPerWarp; ++r) {
+        const int i = (blockIdx.x * nw + warp) * kPfRowsPerWarp + r;
         if (i >= a.Tq) break;
         const uint16_t *qi = a.Q + ((int64_t)i * a.Hq + (int64_t)g * G) * D;
         for (int e = lane; e < G * D; e += 32) qw[e] = bf16_to_f32(qi[e]);
@@ -108,16 +112,23 @@ __global__ void __launch_bounds__(256) prefill_select_kernel(PfArgs a) {
                 for (int t = 0; t < kPfWords; ++t)
 #pragma unroll
                     for (int h = 0; h < kMaxGh; ++h) acc[t][h] = 0.0f;
-                for (int d = 0; d < D; ++d) {
-                    float qd[kMaxGh];
+                for (int d = 0; d < D; d += 4) {
+                    float4 qd[kMaxGh];
 #pragma unroll
-                    for (int h = 0; h < kMaxGh; ++h) qd[h] = h0 + h < G ? qw[(h0 + h) * D + d] : 0.0f;
+                    for (int h = 0; h < kMaxGh; ++h)
+                        qd[h] = h0 + h < G ? *reinterpret_cast<const float4 *>(qw + (h0 + h) * D + d)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                     for (int t = 0; t < kPfWords; ++t) {
                         const int j = min(lane + 32 * t, nb - 1);
-                        const float c = cs[j * (D + 1) + d];
+                        const float4 c = *reinterpret_cast<const float4 *>(cs + j * kPfCentStride + d);
 #pragma unroll
-                        for (int h = 0; h < kMaxGh; ++h) acc[t][h] = __fmaf_rn(qd[h], c, acc[t][h]);
+                        for (int h = 0; h < kMaxGh; ++h) {
+                            acc[t][h] = __fmaf_rn(qd[h].x, c.x, acc[t][h]);
+                            acc[t][h] = __fmaf_rn(qd[h].y, c.y, acc[t][h]);
+                            acc[t][h] = __fmaf_rn(qd[h].z, c.z, acc[t][h]);
+                            acc[t][h] = __fmaf_rn(qd[h].w, c.w, acc[t][h]);
+                        }
                     }
                 }
 #pragma unroll
@@ -652,12 +663,16 @@ bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
     BSA_CUDA_TRY(cudaMemsetAsync(w + L.qcount, 0, (size_t)d->Hkv * p->n_blocks * 4, st));
     BSA_CUDA_TRY(cudaMemsetAsync(w + L.work, 0, 4, st));
     // P1: selection
-    const size_t smem1 = ((size_t)a.nb * (a.D + 1) + (size_t)8 * G * a.D + a.nb) * 4;
+    auto smem1_for = [&](int nw) {
+        return ((size_t)a.nb * kPfCentStride + (size_t)nw * G * a.D + a.nb) * 4;
+    };
+    const int nw1 = smem1_for(kPfSelWarps) <= kMaxSmemPerCta ? kPfSelWarps : kPfSelWarps / 2;
+    const size_t smem1 = smem1_for(nw1);
     BSA_CUDA_TRY(cudaFuncSetAttribute(prefill_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem1));
     BSA_CUDA_TRY(launch_pdl(prefill_select_kernel,
-                            dim3((unsigned)div_up(Tq, kPfRowsPerCta), (unsigned)d->Hkv), dim3(256),
-                            smem1, st, a));
+                            dim3((unsigned)div_up(Tq, nw1 * kPfRowsPerWarp), (unsigned)d->Hkv),
+                            dim3(32 * nw1), smem1, st, a));
     // P2: tile prefix over (KV head, block)
     prefill_tiles_kernel<<<1, 1024, 0, st>>>(a);
     BSA_LAUNCH_CHECK();
