@@ -3,7 +3,7 @@
 #include <algorithm>
 #include <mutex>
 
-#include "common.cuh"
+#include "summary_rows.cuh"
 
 namespace bsa {
 
@@ -17,7 +17,8 @@ bsa_status launch_select(const bsa_kv_desc *, const float *, const void *, int,
                          cudaStream_t);
 bsa_status launch_decode(const bsa_kv_desc *, const float *, const void *, const void *,
                          const int32_t *, const int32_t *, int, const int32_t *, int, float, float *,
-                         float *, uint32_t *, uint32_t *, void *, cudaStream_t);
+                         float *, uint32_t *, uint32_t *, void *, cudaStream_t, const DecAppend *);
+bool decode_can_fuse_append(const bsa_kv_desc *);
 int decode_nsplit(const bsa_kv_desc *, int, int);
 size_t decode_scratch_bytes(const bsa_kv_desc *, int);
 bsa_status launch_prefill(const bsa_kv_desc *, const void *, const void *, const bsa_sel_params *,
@@ -264,7 +265,51 @@ bsa_status bsa_decode(const bsa_kv_desc *d, const float *q, const void *K, const
     uint32_t *cnt = status + 1 + d->B * d->Hkv;
     void *scr = static_cast<char *>(ws) + counters_bytes(d);
     return launch_decode(d, q, K, V, ranges, n_ranges, max_r, cur_len, std::max(tokens_hint, 1),
-                         scale, out, lse, status, cnt, scr, (cudaStream_t)stream);
+                         scale, out, lse, status, cnt, scr, (cudaStream_t)stream, nullptr);
+}
+
+bsa_status bsa_decode_step(const bsa_kv_desc *d, const float *q, void *K, void *V,
+                           const void *k_new, const void *v_new, int32_t *cur_len,
+                           const bsa_sel_params *p, bsa_summary_kind kind, void *summaries,
+                           const int32_t *ranges, const int32_t *n_ranges, int32_t max_r,
+                           int32_t tokens_hint, float scale, float *out, float *lse, void *ws,
+                           size_t ws_bytes, bsa_stream_t stream) {
+    // the arguments of both halves, checked before anything is launched
+    if (!desc_ok(d) || !K || !V || !k_new || !v_new || !cur_len) return BSA_ERR_ARG;
+    if (p && !sel_ok(d, p)) return BSA_ERR_ARG;
+    if (summaries && (!p || kind < BSA_SUM_CENTROID || kind > BSA_SUM_MINMAX)) return BSA_ERR_ARG;
+    if (!q || !ranges || !n_ranges || !out) return BSA_ERR_ARG;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(q)) return BSA_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(ranges) % 8) return BSA_ERR_ARG;
+    if (max_r < 1 || max_r > 4096 || tokens_hint < 0) return BSA_ERR_ARG;
+    if (d->Hq / d->Hkv > kMaxG) return BSA_ERR_UNSUPPORTED;
+    if (!(scale > 0.0f) || scale != scale) return BSA_ERR_ARG;
+    const int nsplit = decode_nsplit(d, std::max(tokens_hint, 1), max_r);
+    const size_t need = counters_bytes(d) + decode_scratch_bytes(d, nsplit);
+    if (!ws_ok(ws, ws_bytes, need)) return BSA_ERR_WORKSPACE;
+    const bool fixed_summ = summaries && p && p->block_size > 0;
+    const bool fuse = decode_can_fuse_append(d) && aligned16(k_new) && aligned16(v_new) &&
+                      (!fixed_summ || kind != BSA_SUM_CENTROID_NORM);
+    if (!fuse) {   // the same two steps as separate launches
+        const bsa_status r = bsa_append_kv(d, K, V, k_new, v_new, cur_len, p, kind, summaries, stream);
+        if (r != BSA_OK) return r;
+        return bsa_decode(d, q, K, V, ranges, n_ranges, max_r, cur_len, tokens_hint, scale, out, lse,
+                          ws, ws_bytes, stream);
+    }
+    DecAppend app;
+    app.k_new = k_new;
+    app.v_new = v_new;
+    app.cur_len = cur_len;
+    app.summ = fixed_summ ? summaries : nullptr;
+    app.S = p ? p->block_size : 0;
+    app.nb_total = p ? nb_total(d, p) : 0;
+    app.kind = kind;
+    app.row_bytes = (int)summary_row_bytes(kind, d->D, d->kv_dtype);
+    uint32_t *status = static_cast<uint32_t *>(ws);
+    uint32_t *cnt = status + 1 + d->B * d->Hkv;
+    void *scr = static_cast<char *>(ws) + counters_bytes(d);
+    return launch_decode(d, q, K, V, ranges, n_ranges, max_r, cur_len, std::max(tokens_hint, 1),
+                         scale, out, lse, status, cnt, scr, (cudaStream_t)stream, &app);
 }
 
 bsa_status bsa_append_kv(const bsa_kv_desc *d, void *K, void *V, const void *k_new,

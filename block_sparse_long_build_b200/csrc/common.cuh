@@ -371,4 +371,13 @@ struct WsLayout {
     size_t total = 0;
 };
 
+// Fused append of the step's new row (k_new == nullptr: none): the same
+// bookkeeping as the append kernel, done inside the decode grid.
+struct DecAppend {
+    const void *k_new, *v_new;   // [B][Hkv][D] bf16
+    int32_t *cur_len;            // incremented by the last CTA of each sequence
+    void *summ;                  // fixed-block summaries (CENTROID or MINMAX), or nullptr
+    int S, nb_total, kind, row_bytes;
+};
+
 }  // namespace bsa

@@ -25,7 +25,7 @@
 #include <utility>
 #include <vector>
 
-#include "common.cuh"
+#include "summary_rows.cuh"
 
 namespace bsa {
 
@@ -33,8 +33,8 @@ constexpr int kPiece = 16;
 constexpr int kDecWarps = 4;
 constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kBoxBytes = kPiece * 128;            // 16 rows x 64 bf16
-constexpr int kHalfBytes = kDecWarps * kBoxBytes;  // one 64-column half of a tile
-constexpr int kPieceCap = 512;                     // CTA piece table held in shared memory
+constexpr int kWarpCap = 128;                      // per-warp piece table (refilled when exceeded)
+constexpr int kRegRanges = 12;                     // range slots per lane loaded in one batch
 constexpr int kMaxClusterSplits = 16;              // splits merged inside one cluster
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kNegInf = -__builtin_huge_valf();
@@ -51,8 +51,9 @@ struct DecArgs {
     float scale_log2;
     float *part_o;        // [nseg][nsplit][G][D]
     float2 *part_ml;      // [nseg][nsplit][G]
-    uint32_t *counters;   // [nseg]
+    uint32_t *counters;   // [nseg]; entry b * Hkv counts the CTAs of sequence b (fused append)
     uint32_t *status;     // sticky error bits
+    DecAppend app;
 };
 
 // Exclusive scan over the CTA (blockDim.x a multiple of 32, <= 1024).
@@ -122,6 +123,107 @@ __device__ int load_ranges(const DecArgs &a, int s, int b, int *rs, int *re, int
     return carry;
 }
 
+// A range slot of segment s, clamped to [0, L_max); the last range is
+// extended to the sequence length cl.
+__device__ __forceinline__ int2 clamp_range(const DecArgs &a, int2 v, bool last, int cl) {
+    const int lo = min(max(v.x, 0), a.L_max);
+    int hi = min(max(v.y, lo), a.L_max);
+    if (last && cl > hi) hi = cl;
+    return make_int2(lo, hi);
+}
+
+// Warp-local view of a segment's range table (no CTA-wide barrier): lane l
+// owns the slots [r0, r1) = [l k, l k + k), k = ceil(max_ranges / 32), and
+// pbase is the number of 16-row pieces in the slots before r0.  The CTA's
+// pieces are [first, last); this warp streams first + warp + 4 i.
+struct WarpRanges {
+    const int32_t *R;
+    int nr, cl, r0, r1, pbase, P, first, last;
+    int app;   // row the fused append writes (then cl = app + 1), or -1
+};
+
+// Writes the table entries of range x (first piece pp) for warp-local
+// indices i in [i0, i0 + kWarpCap).
+__device__ __forceinline__ void fill_range(const WarpRanges &w, int2 x, int pp, int warp, int i0,
+                                           int2 *tab) {
+    const int cnt = (x.y - x.x + kPiece - 1) / kPiece;
+    const int lo_p = pp - w.first - warp;                       // i >= ceil(lo_p / 4)
+    const int hi_p = min(pp + cnt, w.last) - w.first - warp;    // i <  ceil(hi_p / 4)
+    const int ia = max(lo_p > 0 ? (lo_p + kDecWarps - 1) / kDecWarps : 0, i0);
+    const int ib = min(hi_p > 0 ? (hi_p + kDecWarps - 1) / kDecWarps : 0, i0 + kWarpCap);
+    for (int i = ia; i < ib; ++i) {
+        const int row = x.x + (w.first + warp + kDecWarps * i - pp) * kPiece;
+        tab[i - i0] = make_int2(row, min(kPiece, x.y - row));
+    }
+}
+
+// Scans the range table and fills the first window of this warp's piece
+// table (the caller syncs the warp before reading it).
+__device__ __forceinline__ WarpRanges warp_ranges(const DecArgs &a, int s, int b, int c, int warp,
+                                                  int lane, int2 *tab) {
+    WarpRanges w;
+    w.R = a.ranges + (int64_t)s * a.max_ranges * 2;
+    const int k = (a.max_ranges + 31) >> 5;
+    w.r0 = min(lane * k, a.max_ranges);
+    w.r1 = min(w.r0 + k, a.max_ranges);
+    const int2 *R2 = reinterpret_cast<const int2 *>(w.R);
+    // one round trip: the count, the length and this lane's slots together
+    int2 rv[kRegRanges];
+#pragma unroll
+    for (int j = 0; j < kRegRanges; ++j) rv[j] = w.r0 + j < w.r1 ? __ldg(R2 + w.r0 + j) : make_int2(0, 0);
+    w.nr = min(max(a.n_ranges[s], 0), a.max_ranges);
+    const int len = a.cur_len[b];
+    w.app = a.app.k_new && len >= 0 && len < a.L_max ? len : -1;
+    w.cl = w.app >= 0 ? len + 1 : min(max(len, 0), a.L_max);
+    const int end = min(w.r1, w.nr);
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < kRegRanges; ++j) {
+        rv[j] = clamp_range(a, rv[j], w.r0 + j == w.nr - 1, w.cl);
+        if (w.r0 + j < end) cnt += (rv[j].y - rv[j].x + kPiece - 1) / kPiece;
+    }
+    for (int r = w.r0 + kRegRanges; r < end; ++r) {
+        const int2 x = clamp_range(a, __ldg(R2 + r), r == w.nr - 1, w.cl);
+        cnt += (x.y - x.x + kPiece - 1) / kPiece;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+    }
+    w.pbase = incl - cnt;
+    w.P = __shfl_sync(0xffffffffu, incl, 31);
+    int per = (w.P + a.nsplit - 1) / a.nsplit;
+    per = (per + kDecWarps - 1) / kDecWarps * kDecWarps;
+    w.first = min(c * per, w.P);
+    w.last = min(w.P, w.first + per);
+    int pp = w.pbase;
+#pragma unroll
+    for (int j = 0; j < kRegRanges; ++j)
+        if (w.r0 + j < end && pp < w.last) {
+            fill_range(w, rv[j], pp, warp, 0, tab);
+            pp += (rv[j].y - rv[j].x + kPiece - 1) / kPiece;
+        }
+    for (int r = w.r0 + kRegRanges; r < end && pp < w.last; ++r) {
+        const int2 x = clamp_range(a, __ldg(R2 + r), r == w.nr - 1, w.cl);
+        fill_range(w, x, pp, warp, 0, tab);
+        pp += (x.y - x.x + kPiece - 1) / kPiece;
+    }
+    return w;
+}
+
+// Refills the table with the window i in [i0, i0 + kWarpCap).
+__device__ __forceinline__ void warp_refill(const DecArgs &a, const WarpRanges &w, int warp, int i0, int2 *tab) {
+    int pp = w.pbase;
+    const int end = min(w.r1, w.nr);
+    for (int r = w.r0; r < end && pp < w.last; ++r) {
+        const int2 x = clamp_range(a, __ldg(reinterpret_cast<const int2 *>(w.R) + r), r == w.nr - 1, w.cl);
+        fill_range(w, x, pp, warp, i0, tab);
+        pp += (x.y - x.x + kPiece - 1) / kPiece;
+    }
+}
+
 // Piece p -> (first row, valid rows).
 __device__ __forceinline__ int2 piece_rows(int p, const int *rs, const int *re, const int *ps,
                                            int nr) {
@@ -183,13 +285,20 @@ __device__ __forceinline__ void cluster_sync_all() {
                  ::: "memory");
 }
 
-// Reads a float from the shared memory of CTA `rank` of this cluster at the
-// address `local` has in this CTA.
+// Reads from the shared memory of CTA `rank` of this cluster at the address
+// `local` has in this CTA.
 __device__ __forceinline__ float ld_peer(uint32_t local, uint32_t rank) {
     uint32_t remote;
     float v;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+__device__ __forceinline__ float2 ld_peer2(uint32_t local, uint32_t rank) {
+    uint32_t remote;
+    float2 v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(remote) : "memory");
     return v;
 }
 
@@ -231,23 +340,31 @@ __device__ void cluster_finish(const DecArgs &a, int b, int g, const float *wm, 
     const int64_t qrow = (int64_t)b * a.Hq + (int64_t)g * G;
     for (int e = rank * blockDim.x + threadIdx.x; e < G * D; e += n * blockDim.x) {
         const int h = e / D, d = e % D;
+        // all of the peers' values are requested before any is used
+        float2 mlk[kMaxClusterSplits];
+        float ok[kMaxClusterSplits];
+#pragma unroll
+        for (uint32_t k = 0; k < (uint32_t)kMaxClusterSplits; ++k)
+            if (k < n) {
+                mlk[k] = ld_peer2(sml_a + 8 * h, k);
+                ok[k] = ld_peer(part_a + 4 * e, k);
+            }
         float m = kNegInf, l = 0.0f, o = 0.0f;
-        for (uint32_t k = 0; k < n; ++k) {
-            const float mk = ld_peer(sml_a + 8 * h, k);
-            const float lk = ld_peer(sml_a + 8 * h + 4, k);
-            const float ok = ld_peer(part_a + 4 * e, k);
-            if (mk != kNegInf) {
-                const float mn = fmaxf(m, mk);
-                const float c_old = exp2f(m - mn), c_new = exp2f(mk - mn);
-                l = l * c_old + lk * c_new;
-                o = o * c_old + ok * c_new;
+#pragma unroll
+        for (uint32_t k = 0; k < (uint32_t)kMaxClusterSplits; ++k)
+            if (k < n && mlk[k].x != kNegInf) {
+                const float mn = fmaxf(m, mlk[k].x);
+                const float c_old = exp2f(m - mn), c_new = exp2f(mlk[k].x - mn);
+                l = l * c_old + mlk[k].y * c_new;
+                o = o * c_old + ok[k] * c_new;
                 m = mn;
             }
-        }
         a.out[(qrow + h) * D + d] = l > 0.0f ? o / l : 0.0f;
         if (d == 0 && a.lse) a.lse[qrow + h] = l > 0.0f ? (m + log2f(l)) * kLn2 : kNegInf;
     }
-    cluster_sync_all();
+    // the partials stay alive until every peer has read them; the values read
+    // were consumed above, so this barrier orders no memory
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
 // Log-sum-exp merge of the split partials (A5), one CTA per (segment, query
@@ -283,6 +400,34 @@ __global__ void __launch_bounds__(128) lse_merge_kernel(DecArgs a) {
     }
 }
 
+// End of a fused step for one CTA of segment (b, g): the CTA that wrote row n
+// builds the summary of the fixed block that row completes; the last CTA of
+// sequence b to get here (every CTA of it has read cur_len by then) sets
+// cur_len[b] = n + 1 and resets the counter.
+__device__ __forceinline__ void finish_append(const DecArgs &a, int b, int g, int n, bool owner) {
+    if (n < 0) return;
+    const DecAppend &p = a.app;
+    if (owner && p.summ && p.S > 0 && (n + 1) % p.S == 0) {
+        const int j = (n + 1) / p.S - 1;
+        const uint16_t *Kseg = static_cast<const uint16_t *>(a.K) + b * a.stride_b + g * a.stride_h;
+        char *out = static_cast<char *>(p.summ) + ((int64_t)(b * a.Hkv + g) * p.nb_total + j) * p.row_bytes;
+        if (p.kind == BSA_SUM_MINMAX)
+            summarize_minmax<uint16_t>(Kseg, a.stride_t, a.D, (int64_t)j * p.S, (int64_t)(j + 1) * p.S,
+                                       reinterpret_cast<uint16_t *>(out));
+        else
+            summarize_centroid<uint16_t>(Kseg, a.stride_t, a.D, (int64_t)j * p.S,
+                                         (int64_t)(j + 1) * p.S, reinterpret_cast<float *>(out));
+    }
+    if (threadIdx.x == 0) {
+        __threadfence();
+        uint32_t *ctr = a.counters + b * a.Hkv;
+        if (atomicAdd(ctr, 1u) == (uint32_t)(a.Hkv * gridDim.x) - 1u) {
+            p.cur_len[b] = n + 1;
+            *ctr = 0u;
+        }
+    }
+}
+
 // ======================================================================
 // Tensor-core path
 // ======================================================================
@@ -295,9 +440,8 @@ struct TcSmem {
     static constexpr int kInfo = kRing;                               // int2 [warps][NST]
     static constexpr int kBars = kInfo + kDecWarps * NST * 8;         // u64  [warps][NST]
     static constexpr int kMisc = kBars + kDecWarps * NST * 8;         // float sml[2*kMaxG], int tmp[36]
-    static constexpr int kPtab = kMisc + 2 * kMaxG * 4 + 36 * 4;      // int2 [kPieceCap]
-    static constexpr int kRanges = kPtab + kPieceCap * 8;
-    static constexpr int bytes(int max_ranges) { return kRanges + (3 * max_ranges + 1) * 4 + 1024; }
+    static constexpr int kPtab = kMisc + 2 * kMaxG * 4 + 36 * 4;      // int2 [warps][kWarpCap]
+    static constexpr int kBytes = kPtab + kDecWarps * kWarpCap * 8 + 1024;
     static_assert(kRing >= kDecWarps * kMaxG * (2 + 64 * NH) * 4,
                   "per-warp partials must fit in the ring");
 };
@@ -315,42 +459,45 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     int2 *info = reinterpret_cast<int2 *>(dsm + L::kInfo);
     uint64_t *full = reinterpret_cast<uint64_t *>(dsm + L::kBars);
     float *sml = reinterpret_cast<float *>(dsm + L::kMisc);
-    int *tmp = reinterpret_cast<int *>(dsm + L::kMisc + 2 * kMaxG * 4);
     int2 *ptab = reinterpret_cast<int2 *>(dsm + L::kPtab);
-    int *rs = reinterpret_cast<int *>(dsm + L::kRanges);
-    int *re = rs + a.max_ranges;
-    int *ps = re + a.max_ranges;
 
     const int c = blockIdx.x, s = blockIdx.y;
     const int b = s / a.Hkv, g = s % a.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, tig = lane & 3;
 
-    if (tid == 0) {
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
-        for (int i = 0; i < kDecWarps * NST; ++i) mbar_init(&full[i], 1);
-        fence_mbar_init();
-    }
-    pdl_wait();   // ranges, lengths and the cache come from earlier kernels
-    int nr;
-    const int P = load_ranges(a, s, b, rs, re, ps, tmp, &nr);
-    int per = (P + a.nsplit - 1) / a.nsplit;
-    per = (per + kDecWarps - 1) / kDecWarps * kDecWarps;
-    const int first = c * per, last = min(P, first + per);
-    const int n_my = max(0, last - first);
-    for (int i = tid; i < min(n_my, kPieceCap); i += kDecThreads)
-        ptab[i] = piece_rows(first + i, rs, re, ps, nr);
-    __syncthreads();
-
-    // this warp's pieces: local indices warp, warp + 4, warp + 8, ...
-    const int my_count = n_my > warp ? (n_my - warp + kDecWarps - 1) / kDecWarps : 0;
+    // Every warp works out its own pieces: no CTA-wide barrier before the
+    // first load.
     unsigned char *ring = dsm + warp * NST * L::kPieceBytes;
     uint64_t *wfull = full + warp * NST;
     int2 *winfo = info + warp * NST;
+    int2 *wtab = ptab + warp * kWarpCap;
+    if (tid == 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    if (lane == 0) {
+        for (int i = 0; i < NST; ++i) mbar_init(&wfull[i], 1);
+        fence_mbar_init();
+    }
+    pdl_wait();   // ranges, lengths and the cache come from earlier kernels
+    // fused append: lanes 0.. hold 16-byte chunks of the new key, lanes 16..
+    // of the new value
+    constexpr int kChunks = D / 8;
+    uint4 nkv = make_uint4(0u, 0u, 0u, 0u);
+    if (a.app.k_new) {
+        if (lane < kChunks)
+            nkv = __ldg(static_cast<const uint4 *>(a.app.k_new) + (int64_t)s * kChunks + lane);
+        else if (lane >= 16 && lane - 16 < kChunks)
+            nkv = __ldg(static_cast<const uint4 *>(a.app.v_new) + (int64_t)s * kChunks + lane - 16);
+    }
+    const WarpRanges wr = warp_ranges(a, s, b, c, warp, lane, wtab);
+    const int n_my = wr.last - wr.first;
+    // this warp's pieces: CTA-local indices warp, warp + 4, warp + 8, ...
+    const int my_count = n_my > warp ? (n_my - warp + kDecWarps - 1) / kDecWarps : 0;
+    __syncwarp();
     auto issue = [&](int idx, int st) {   // lane 0 only
-        const int i = warp + idx * kDecWarps;
-        const int2 pr = i < kPieceCap ? ptab[i] : piece_rows(first + i, rs, re, ps, nr);
+        const int2 pr = wtab[idx % kWarpCap];
         winfo[st] = pr;
         mbar_arrive_expect_tx(&wfull[st], (uint32_t)(2 * NH * kBoxBytes));
         unsigned char *dst = ring + st * L::kPieceBytes;
@@ -360,8 +507,27 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             tma_load_4d(dst + (NH + h) * kBoxBytes, &tmV, &wfull[st], h * 64, pr.x, g, b);
         }
     };
-    if (lane == 0)
-        for (int j = 0; j < NST && j < my_count; ++j) issue(j, j);
+    // Warp-collective, before piece idx is issued: if the piece holds the
+    // appended row, write the row (its TMA load then sees it).
+    bool wrote = false;
+    auto maybe_append = [&](int idx) {
+        if (wr.app < 0) return;
+        const int2 pr = wtab[idx % kWarpCap];
+        if (pr.x <= wr.app && wr.app < pr.x + pr.y) {
+            const int64_t off = b * a.stride_b + g * a.stride_h + (int64_t)wr.app * a.stride_t;
+            if (lane < kChunks)
+                reinterpret_cast<uint4 *>(static_cast<uint16_t *>(const_cast<void *>(a.K)) + off)[lane] = nkv;
+            else if (lane >= 16 && lane - 16 < kChunks)
+                reinterpret_cast<uint4 *>(static_cast<uint16_t *>(const_cast<void *>(a.V)) + off)[lane - 16] = nkv;
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __syncwarp();
+            wrote = true;
+        }
+    };
+    for (int j = 0; j < NST && j < my_count; ++j) {
+        maybe_append(j);
+        if (lane == 0) issue(j, j);
+    }
 
     // q fragments: rows 0-7 q_hi of head gid, rows 8-15 q_lo; zero past G
     uint32_t qa[D / 16][4];
@@ -484,7 +650,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             mma_bf16_16816(o[2 * cp + 1], pa, r2, r3);
         }
         __syncwarp();
-        if (lane == 0 && idx + NST < my_count) issue(idx + NST, st);
+        if (idx + NST < my_count) {
+            if ((idx + NST) % kWarpCap == 0) {   // next window of this warp's pieces
+                warp_refill(a, wr, warp, idx + NST, wtab);
+                __syncwarp();
+            }
+            maybe_append(idx + NST);
+            if (lane == 0) issue(idx + NST, st);
+        }
     }
     if (timed_out) atomicOr(a.status, 1u);
     // the merge kernel may be scheduled now; it waits for this grid to finish
@@ -496,7 +669,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     float *wm = reinterpret_cast<float *>(dsm);
     float *wl = wm + kDecWarps * kMaxG;
     float *wo = wl + kDecWarps * kMaxG;
-    __syncthreads();
+    const bool cta_wrote = __syncthreads_or(wrote);
     if (tig == 0) {
         wm[warp * kMaxG + gid] = m_run;
         wl[warp * kMaxG + gid] = l_run;
@@ -512,6 +685,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         cluster_finish(a, b, g, wm, wl, wo, sml, reinterpret_cast<float *>(dsm + 32768));
     else
         finish(a, s, b, g, c, wm, wl, wo, sml);
+    if (a.app.k_new) finish_append(a, b, g, wr.app, cta_wrote);
 }
 
 // ======================================================================
@@ -608,6 +782,8 @@ static bool use_tc(const bsa_kv_desc *d) {
            d->stride_t == d->D;
 }
 
+bool decode_can_fuse_append(const bsa_kv_desc *d) { return use_tc(d); }
+
 int decode_nsplit(const bsa_kv_desc *d, int tokens_hint, int max_ranges) {
     const int nseg = d->B * d->Hkv;
     const int64_t pieces = div_up(tokens_hint > 0 ? tokens_hint : 1, kPiece) + max_ranges;
@@ -658,8 +834,10 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
                          const int32_t *ranges, const int32_t *n_ranges, int max_ranges,
                          const int32_t *cur_len, int tokens_hint, float scale, float *out,
                          float *lse, uint32_t *status, uint32_t *counters, void *scratch,
-                         cudaStream_t st) {
+                         cudaStream_t st, const DecAppend *app) {
+    if (app && !use_tc(d)) return BSA_ERR_UNSUPPORTED;
     DecArgs a;
+    a.app = app ? *app : DecAppend{};
     a.q = q; a.out = out; a.lse = lse; a.ranges = ranges; a.n_ranges = n_ranges;
     a.max_ranges = max_ranges; a.cur_len = cur_len; a.K = K; a.V = V;
     a.stride_b = d->stride_b; a.stride_h = d->stride_h; a.stride_t = d->stride_t;
@@ -714,10 +892,10 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
         bsa_status r;
         if (d->D == 128)
             r = go_tc(decode_tc_kernel<2, kTcStages, false>, decode_tc_kernel<2, kTcStages, true>,
-                      TcSmem<2, kTcStages>::bytes(max_ranges));
+                      TcSmem<2, kTcStages>::kBytes);
         else   // D = 64
             r = go_tc(decode_tc_kernel<1, 2 * kTcStages, false>, decode_tc_kernel<1, 2 * kTcStages, true>,
-                      TcSmem<1, 2 * kTcStages>::bytes(max_ranges));
+                      TcSmem<1, 2 * kTcStages>::kBytes);
         if (r != BSA_OK) return r;
         BSA_LAUNCH_CHECK();
         if (clustered) return BSA_OK;

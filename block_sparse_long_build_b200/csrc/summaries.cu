@@ -4,109 +4,11 @@
 // Summaries ("Module 14: Sparse attention and long context", §14.3 MoBA,
 // mean-pooled here; "Semantic blocks for sparse attention", normalised block
 // centres; "Sparse attention in hybrid LLMs", Quest min/max page bounds).
-// The arithmetic order is fixed so that the scores computed from these
-// summaries, and hence the selected blocks, are reproducible bit for bit:
-//   centroid       c[i] = (((0 + k_r0[i]) + k_r1[i]) + ...) / n   (rows in order)
-//   centroid_norm  u_r = k_r / ||k_r|| (||.|| = sqrt of an fma chain over i),
-//                  m = mean of u_r as above, c = m / ||m||
-//   minmax         running min / max over rows in order (first wins on ties)
-#include "common.cuh"
+// The arithmetic (fixed order, reproducible bit for bit) is in
+// summary_rows.cuh.
+#include "summary_rows.cuh"
 
 namespace bsa {
-
-constexpr int kNormChunk = 64;   // rows staged at once for the per-row norms
-
-// fp32 norm of a row held in shared memory: fma chain over i, then sqrt.
-__device__ __forceinline__ float row_norm_f32(const float *x, int D) {
-    float acc = 0.0f;
-    for (int i = 0; i < D; ++i) acc = __fmaf_rn(x[i], x[i], acc);
-    return __fsqrt_rn(acc);
-}
-
-// Summary of rows [r0, r1) of one segment, computed by the whole CTA
-// (blockDim.x >= D).  `out` points at this block's summary: D floats for the
-// centroid kinds, 2*D cache elements (min row, then max row) for MINMAX.
-// `sm` must hold kNormChunk*(D+1) + D + 1 floats.
-template <typename T>
-__device__ void summarize_rows(const T *Kseg, int64_t st, int D, int64_t r0, int64_t r1,
-                               int kind, void *out, float *sm) {
-    const int i = threadIdx.x;
-    const int64_t n = r1 - r0;
-    if (kind == BSA_SUM_CENTROID) {
-        if (i < D) {
-            float acc = 0.0f;
-            int64_t r = r0;
-            for (; r + 4 <= r1; r += 4) {   // loads batched, adds stay in order
-                float v0 = load_elem(Kseg, r * st + i), v1 = load_elem(Kseg, (r + 1) * st + i);
-                float v2 = load_elem(Kseg, (r + 2) * st + i), v3 = load_elem(Kseg, (r + 3) * st + i);
-                acc = __fadd_rn(acc, v0);
-                acc = __fadd_rn(acc, v1);
-                acc = __fadd_rn(acc, v2);
-                acc = __fadd_rn(acc, v3);
-            }
-            for (; r < r1; ++r) acc = __fadd_rn(acc, load_elem(Kseg, r * st + i));
-            static_cast<float *>(out)[i] = n > 0 ? __fdiv_rn(acc, (float)n) : 0.0f;
-        }
-        return;
-    }
-    if (kind == BSA_SUM_MINMAX) {
-        if (i < D) {
-            float lo = __int_as_float(0x7f800000), hi = __int_as_float(0xff800000);  // +inf, -inf
-            for (int64_t r = r0; r < r1; ++r) {
-                float v = load_elem(Kseg, r * st + i);
-                if (v < lo) lo = v;
-                if (v > hi) hi = v;
-            }
-            if (n <= 0) lo = hi = 0.0f;
-            T *o = static_cast<T *>(out);
-            if constexpr (sizeof(T) == 2) {
-                o[i] = static_cast<uint16_t>(__float_as_uint(lo) >> 16);
-                o[D + i] = static_cast<uint16_t>(__float_as_uint(hi) >> 16);
-            } else {
-                o[i] = lo;
-                o[D + i] = hi;
-            }
-        }
-        return;
-    }
-    // BSA_SUM_CENTROID_NORM
-    float *rows = sm;                              // [kNormChunk][D+1]
-    float *nrm = sm + kNormChunk * (D + 1);        // [kNormChunk] (aliases the tail)
-    float acc = 0.0f;
-    for (int64_t c0 = r0; c0 < r1; c0 += kNormChunk) {
-        const int cn = (int)((r1 - c0) < kNormChunk ? (r1 - c0) : kNormChunk);
-        __syncthreads();
-        for (int e = threadIdx.x; e < cn * D; e += blockDim.x) {
-            int rr = e / D, ii = e % D;
-            rows[rr * (D + 1) + ii] = load_elem(Kseg, (c0 + rr) * st + ii);
-        }
-        __syncthreads();
-        if (threadIdx.x < cn) nrm[threadIdx.x] = row_norm_f32(rows + threadIdx.x * (D + 1), D);
-        __syncthreads();
-        if (i < D) {
-            for (int rr = 0; rr < cn; ++rr) {
-                float nr = nrm[rr];
-                acc = __fadd_rn(acc, nr > 0.0f ? __fdiv_rn(rows[rr * (D + 1) + i], nr) : 0.0f);
-            }
-        }
-    }
-    __syncthreads();
-    float *mean = sm;   // reuse
-    if (i < D) mean[i] = n > 0 ? __fdiv_rn(acc, (float)n) : 0.0f;
-    __syncthreads();
-    if (threadIdx.x == 0) mean[D] = row_norm_f32(mean, D);
-    __syncthreads();
-    if (i < D) {
-        float nc = mean[D];
-        static_cast<float *>(out)[i] = nc > 0.0f ? __fdiv_rn(mean[i], nc) : 0.0f;
-    }
-    __syncthreads();
-}
-
-__host__ __device__ inline size_t summary_row_bytes(int kind, int D, int kv_dtype) {
-    return kind == BSA_SUM_MINMAX ? (size_t)2 * D * (kv_dtype == BSA_BF16 ? 2 : 4)
-                                  : (size_t)D * 4;
-}
 
 struct SumArgs {
     const void *K;

@@ -23,7 +23,7 @@ BSA_OP_SELECT, BSA_OP_DECODE, BSA_OP_PREFILL, BSA_OP_APPEND = 0, 1, 2, 3
 
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_summary_blocks", "bsa_summary_bytes",
             "bsa_max_selected", "bsa_max_ranges", "bsa_workspace_size", "bsa_build_summaries",
-            "bsa_select", "bsa_decode", "bsa_decode_noalloc", "bsa_append_kv",
+            "bsa_select", "bsa_decode", "bsa_decode_noalloc", "bsa_append_kv", "bsa_decode_step",
             "bsa_prefill_grouped")
 
 
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "bsa_decode": (ctypes.c_int, [pd, P, P, P, P, P, I32, P, I32, F, P, P, P, SZ, P]),
             "bsa_decode_noalloc": (ctypes.c_int, [pd, P, P, P, P, P, I32, P, I32, F, P, P, P]),
             "bsa_append_kv": (ctypes.c_int, [pd, P, P, P, P, P, pp, ctypes.c_int, P, P]),
+            "bsa_decode_step": (ctypes.c_int, [pd, P, P, P, P, P, P, pp, ctypes.c_int, P, P, P, I32,
+                                               I32, F, P, P, P, SZ, P]),
             "bsa_prefill_grouped": (ctypes.c_int, [pd, P, P, pp, P, pd, P, P, P, I32, I32, F, P, P,
                                                    P, SZ, P]),
         }
@@ -188,6 +190,18 @@ def bsa_append_kv(desc, K, V, k_new, v_new, cur_len, sel, kind, summaries, strea
            lib().bsa_append_kv(ctypes.byref(desc), _p(K), _p(V), _p(k_new), _p(v_new),
                                _p(cur_len), ctypes.byref(sel) if sel is not None else None, kind,
                                _p(summaries), _stream(stream)))
+
+
+def bsa_decode_step(desc, q, K, V, k_new, v_new, cur_len, sel, kind, summaries, ranges, n_ranges,
+                    max_ranges, tokens_hint, scale, out, lse, ws, stream=None):
+    """bsa_append_kv then bsa_decode, in one launch where the tensor-core
+    path applies."""
+    _check("bsa_decode_step",
+           lib().bsa_decode_step(ctypes.byref(desc), _p(q), _p(K), _p(V), _p(k_new), _p(v_new),
+                                 _p(cur_len), ctypes.byref(sel) if sel is not None else None,
+                                 kind, _p(summaries), _p(ranges), _p(n_ranges), max_ranges,
+                                 tokens_hint, scale, _p(out), _p(lse), _p(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def bsa_prefill_grouped(desc, K, V, sel, summaries, pos_desc, K_pos, V_pos, Q, q_pos0, Tq, scale,

@@ -8,6 +8,10 @@ order:
     select (score + top-k/budget + ranges), every `refresh` steps -- bsa_select
     decode (split-K attention over the ranges + LSE merge)   -- bsa_decode
 
+Steps that do not refresh the selection run append and decode as one call
+(bsa_decode_step: one launch on the tensor-core path) unless `fused` is
+False.
+
 Everything here is allocation and sequencing; the arithmetic runs in
 libbsa's kernels.
 """
@@ -22,8 +26,9 @@ from .workloads import Config, Workload
 
 
 class DecodeSession:
-    def __init__(self, wl: Workload, stream: torch.cuda.Stream | None = None):
+    def __init__(self, wl: Workload, stream: torch.cuda.Stream | None = None, fused: bool = True):
         self.wl = wl
+        self.fused = fused
         c = self.cfg = wl.cfg
         dev = wl.device
         self.stream = stream
@@ -94,12 +99,24 @@ class DecodeSession:
                      self.out if out is None else out, self.lse if lse is None else lse,
                      self.ws, self.stream)
 
+    def decode_step(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor):
+        """Append the new row and attend (no selection refresh)."""
+        N.bsa_decode_step(self.desc, q, self.wl.K, self.wl.V, k_new, v_new, self.wl.cur_len,
+                          self.sel, self.kind,
+                          self.summaries if self.cfg.block_size > 0 else None, self.ranges,
+                          self.n_ranges, self.max_ranges, self.tokens_hint, self.scale, self.out,
+                          self.lse, self.ws, self.stream)
+
     def step(self, t: int, q: torch.Tensor, k_new: torch.Tensor | None, v_new: torch.Tensor | None):
         """Decode step t: append (when new K/V are given), select on refresh
         steps, attend."""
+        refresh = t % self.cfg.refresh == 0
+        if k_new is not None and self.fused and not refresh:
+            self.decode_step(q, k_new, v_new)
+            return
         if k_new is not None:
             self.append(k_new, v_new)
-        if t % self.cfg.refresh == 0:
+        if refresh:
             self.select(q)
         self.decode(q)
 
@@ -141,8 +158,11 @@ class DecodeSession:
             self.select(self.q_in)
             self.decode(self.q_in)
         with torch.cuda.graph(self.g_plain):
-            self.append(self.k_in, self.v_in)
-            self.decode(self.q_in)
+            if self.fused:
+                self.decode_step(self.q_in, self.k_in, self.v_in)
+            else:
+                self.append(self.k_in, self.v_in)
+                self.decode(self.q_in)
 
     def replay(self, t: int):
         """Decode step t from the captured graphs (inputs already in q_in,
@@ -150,4 +170,14 @@ class DecodeSession:
         (self.g_refresh if t % self.cfg.refresh == 0 else self.g_plain).replay()
 
     def launches_per_step(self, t: int) -> int:
-        return 3 if t % self.cfg.refresh == 0 else 2
+        """Library calls one step makes: append, select on refresh steps, and
+        decode; a fused step is one."""
+        if t % self.cfg.refresh == 0:
+            return 3
+        return 1 if self.fused and self.fuses() else 2
+
+    def fuses(self) -> bool:
+        """Whether bsa_decode_step runs as one launch for this workload."""
+        c = self.cfg
+        return (c.kv_dtype == torch.bfloat16 and c.D in (64, 128) and c.G <= 8
+                and not (c.block_size > 0 and self.kind == N.BSA_SUM_CENTROID_NORM))

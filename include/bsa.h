@@ -232,6 +232,29 @@ BSA_API bsa_status bsa_append_kv(const bsa_kv_desc *desc, void *K, void *V, cons
                          const void *v_new, int32_t *cur_len, const bsa_sel_params *sel,
                          bsa_summary_kind kind, void *summaries, bsa_stream_t stream);
 
+/* One whole decode step after the selection: exactly bsa_append_kv(desc, K,
+ * V, k_new, v_new, cur_len, sel, kind, summaries) followed by bsa_decode(desc,
+ * q, K, V, ranges, n_ranges, max_ranges, cur_len, tokens_hint, scale, out,
+ * lse, ws, ws_bytes), with the arguments and the results of those two calls
+ * ("Sparse attention in hybrid LLMs": between selection refreshes a step
+ * appends its token and attends over the kept pages plus the grown window).
+ * On the tensor-core path (bf16 cache, D in {64, 128}, Hq/Hkv <= 8, rows
+ * contiguous, k_new and v_new 16-byte aligned) both run in one launch: the
+ * CTA whose tile holds row cur_len[b] writes that row before loading the
+ * tile, builds the summary of a fixed block the row completes (CENTROID or
+ * MINMAX summaries), and the last CTA of each sequence increments cur_len.
+ * Elsewhere (and for CENTROID_NORM summaries of fixed blocks) it issues the
+ * two launches.  A step that refreshes the selection must append before
+ * selecting: use bsa_append_kv, bsa_select, bsa_decode there.  Workspace:
+ * bsa_workspace_size(BSA_OP_DECODE). */
+BSA_API bsa_status bsa_decode_step(const bsa_kv_desc *desc, const float *q, void *K, void *V,
+                                   const void *k_new, const void *v_new, int32_t *cur_len,
+                                   const bsa_sel_params *sel, bsa_summary_kind kind,
+                                   void *summaries, const int32_t *ranges,
+                                   const int32_t *n_ranges, int32_t max_ranges,
+                                   int32_t tokens_hint, float scale, float *out, float *lse,
+                                   void *ws, size_t ws_bytes, bsa_stream_t stream);
+
 /* Block-grouped prefill for variable (semantic) blocks, batch 1.
  * Query row i sits at position q_pos0 + i and reads
  *   (a) the positions [pos_limit, q_pos0 + i] densely and causally from the

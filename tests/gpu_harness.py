@@ -46,10 +46,10 @@ def gpu_summaries(sess: DecodeSession, s: int, nb: int):
 class FixedDecodeCheck:
     """Runs fixed-block decode steps on both sides and compares."""
 
-    def __init__(self, cfg, device="cuda"):
+    def __init__(self, cfg, device="cuda", fused=True):
         self.cfg = cfg
         self.wl = Workload(cfg, device)
-        self.sess = DecodeSession(self.wl)
+        self.sess = DecodeSession(self.wl, fused=fused)
         self.K = host(self.wl.K)     # the oracle's own copy of the cache
         self.V = host(self.wl.V)
         self.n = [int(x) for x in self.wl.cur_len.cpu()]

@@ -49,6 +49,35 @@ def test_decode_matches_oracle(name):
     assert worst <= 2e-3
 
 
+# Steps between refreshes run append + decode as one launch (bsa_decode_step).
+# These cases make a fixed block complete during such a step, so the summary
+# built inside the decode grid is compared at the next refresh.
+FUSED = {
+    # pages of 16 (min/max): row 16k+15 is appended at step 2, refresh at 8
+    "quest_page_completes": _cfg(W.quest(0), B=2, Hkv=2, Hq=8, L=16 * 300 + 13, budget_tokens=512,
+                                 sink=32, window=128, refresh=8, steps=10),
+    # blocks of 128 (centroid, current block): row 128k+127 appended at step 1
+    "moba_block_completes": _cfg(W.moba(0), Hkv=2, Hq=16, L=128 * 30 + 126, block_size=128,
+                                 topk=6, n_needles=4, refresh=4, steps=6),
+    # D 64, G 4
+    "quest_d64_fused": _cfg(W.quest(0), B=3, Hkv=1, Hq=4, D=64, L=2048 + 14, budget_tokens=256,
+                            sink=16, window=64, refresh=5, steps=7),
+}
+
+
+@pytest.mark.parametrize("name", list(FUSED))
+def test_fused_step_matches_oracle(name):
+    chk = FixedDecodeCheck(FUSED[name])
+    assert chk.sess.fuses()
+    chk.run(FUSED[name].steps)
+
+
+def test_unfused_steps_match_oracle():
+    """The same step sequence with separate append and decode launches."""
+    chk = FixedDecodeCheck(CASES["quest_small"], fused=False)
+    chk.run(CASES["quest_small"].steps)
+
+
 EDGE = {
     # budget 0: sink + window only
     "budget_zero": _cfg(W.quest(0), B=1, Hkv=2, Hq=8, L=3000, budget_tokens=0, sink=16, window=100,
