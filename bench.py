@@ -161,6 +161,22 @@ def _step_bytes(sess, t: int) -> tuple[int, int]:
     return tot, dec
 
 
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The slowest rank's time: every rank runs its own replica and the job
+    takes as long as the slowest (all ranks must call this, in the same
+    order)."""
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, batch: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank decodes `batch` sequences for
+    `steps` steps (weak scaling), over the slowest rank's time."""
+    return world * batch * steps / (total_ms / 1e3)
+
+
 def run_ours(args, rank: int, world: int, device):
     from block_sparse_long_build_b200 import build as Bld
     from block_sparse_long_build_b200 import workloads as W
@@ -232,12 +248,8 @@ def run_ours(args, rank: int, world: int, device):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = float(sum(step_ms))
     assert torch.allclose(sess.out, out_census, atol=0, rtol=0) or True
-    t_max = torch.tensor([total_ms], device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t_max.item())
-    tokens = world * cfg.B * K_steps
-    value = tokens / (total_ms / 1e3)
+    total_ms = max_over_ranks(total_ms, device, world)
+    value = job_tokens_per_s(world, cfg.B, K_steps, total_ms)
     eff_gbs = world * sum(step_bytes) / (total_ms / 1e3) / 1e9
 
     # ---- dominant kernel alone: the split-K decode, L2 flushed before each
@@ -281,10 +293,7 @@ def run_ours(args, rank: int, world: int, device):
         eev[t][1].record(stream)
         eev[t][1].synchronize()
     e2e_ms = float(sum(a.elapsed_time(b) for a, b in eev))
-    e_max = torch.tensor([e2e_ms], device=device)
-    if world > 1:
-        torch.distributed.all_reduce(e_max, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(e_max.item())
+    e2e_ms = max_over_ranks(e2e_ms, device, world)
     h2d = sum(x.numel() * x.element_size() for x in pin_in[0])
     d2h = out_h.numel() * 4 + lse_h.numel() * 4
 
