@@ -203,6 +203,15 @@ __device__ __forceinline__ int cta_incl_max(int v, int *tmp, int *total) {
 }
 
 // 2-D tiled TMA load (no multicast) completing on an mbarrier.
+// Contiguous global -> shared copy on the TMA engine (no tensor map, no
+// multicast): both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
                                             int x, int y) {
     asm volatile(

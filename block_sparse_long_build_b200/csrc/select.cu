@@ -9,24 +9,34 @@
 // MoBA's current block (§14.3); semantic blocks take a token budget
 // ("Semantic blocks for sparse attention", K = L/16).
 //
-// One kernel, grid (tiles of 128 blocks, segments).  Every CTA brings its
-// tile of summary rows into shared memory with 2-D TMA loads (128-byte
-// swizzle, so that thread j reading row j is conflict-free), scores it one
-// thread per block in the fixed fp32 order (fma chain over the dimensions per
-// query head, heads summed in order) and writes orderable uint32 keys to the
-// workspace.  The last CTA of a segment to finish (an atomic counter, reset
-// afterwards) selects: radix select of the k-th key for top-k, or a bitonic
-// sort and a greedy walk for the token budget, then an index-ordered
-// compaction, so ties go to the lower block index and the result does not
-// depend on which CTA finished last; finally the forced ranges and the
-// selected blocks are merged into disjoint ranges with parallel scans.
+// Two kernels, chained by programmatic dependent launch:
+//  score_kernel  persistent; work items are (segment, tile of 128 blocks).
+//                Each CTA streams its items' summary rows into a ring of
+//                shared-memory stages with 2-D TMA loads (128-byte swizzle, so
+//                that thread j reading row j is conflict-free) together with
+//                the group's queries (1-D bulk copy), scores one block per
+//                thread in the fixed fp32 order (fma chain over the dimensions
+//                per query head, the G chains interleaved, heads summed in
+//                order) and writes orderable uint32 keys to the workspace.
+//  pick_kernel   one 512-thread CTA per segment: candidates (not wholly inside
+//                the forced set), then a radix select of the k-th key for
+//                top-k or a greedy walk for the token budget, an
+//                index-ordered compaction (ties go to the lower block index),
+//                and the merge of forced ranges and selected blocks into
+//                disjoint ranges with parallel scans.
+#include <algorithm>
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace bsa {
 
-constexpr int kSelThreads = 128;   // = rows per tile
+constexpr int kSelThreads = 128;   // scoring threads = rows per tile
+constexpr int kPickThreads = 512;
 constexpr int kSelMaxG = 16;
+constexpr int kSelMaxStages = 3;
 constexpr int kIntMin = -0x7fffffff - 1;
+enum { kScoreCentroid = 0, kScoreMinmaxBf16 = 1, kScoreMinmaxF32 = 2 };
 
 struct SelArgs {
     const float *q;
@@ -42,6 +52,8 @@ struct SelArgs {
     int topk, budget, sink, window, keep_current, local_start, pos_limit;
     int max_sel, max_ranges;
     int row_bytes, nbox;
+    int tiles_per_seg, n_items, nst;   // scoring work items and ring stages
+    uint32_t tile_bytes;
 };
 
 // 16-byte chunk of row j at byte offset `off` of a 128-byte-swizzled tile
@@ -59,179 +71,304 @@ __device__ __forceinline__ void bf16x8(uint4 v, float (&f)[8]) {
     f[6] = __uint_as_float(v.w << 16); f[7] = __uint_as_float(v.w & 0xffff0000u);
 }
 
-// Score of tile row j for the group's G heads in the fixed fp32 order.
-template <int KIND, typename T>
-__device__ __forceinline__ float score_row(const float *qs, int G, int D, const unsigned char *tile,
-                                           int j) {
-    float acc[kSelMaxG];
+// Threads per block row and heads per thread of the scoring kernel: a
+// block's G heads are split over up to 4 threads (more warps in flight); G
+// known only at run time (GT = 0) keeps one thread per block.
+__host__ __device__ constexpr int score_tpb(int GT) { return GT == 0 ? 1 : (GT < 4 ? GT : 4); }
+__host__ __device__ constexpr int score_hpt(int GT) { return GT == 0 ? kSelMaxG : GT / score_tpb(GT); }
+
+// Partial scores of tile row j for heads h0 .. h0 + HPT - 1 (those below G):
+// per head an fma chain over i = 0..D-1 in the fixed fp32 order; the chains
+// of the thread's heads are interleaved.  qs: head rows of D + 4 floats.
+template <int SK, int HPT>
+__device__ __forceinline__ void score_heads(const float *qs, int h0, int G, int D,
+                                            const unsigned char *tile, int j, float (&acc)[HPT]) {
+    const int qstride = D + 4;
 #pragma unroll
-    for (int h = 0; h < kSelMaxG; ++h) acc[h] = 0.0f;
-    if constexpr (KIND == BSA_SUM_MINMAX && sizeof(T) == 2) {
-        for (int i = 0; i < D; i += 8) {
-            float lo[8], hi[8];
-            bf16x8(*tile_chunk(tile, j, i * 2), lo);
-            bf16x8(*tile_chunk(tile, j, (D + i) * 2), hi);
-#pragma unroll
-            for (int h = 0; h < kSelMaxG; ++h) {
-                if (h < G) {
-                    const float4 qa = *reinterpret_cast<const float4 *>(qs + h * D + i);
-                    const float4 qb = *reinterpret_cast<const float4 *>(qs + h * D + i + 4);
-                    const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        acc[h] = __fmaf_rn(qv[e], qv[e] >= 0.0f ? hi[e] : lo[e], acc[h]);
-                }
-            }
-        }
-    } else if constexpr (KIND == BSA_SUM_MINMAX) {
-        for (int i = 0; i < D; i += 4) {
+    for (int h = 0; h < HPT; ++h) acc[h] = 0.0f;
+    constexpr int W = SK == kScoreMinmaxBf16 ? 8 : 4;   // dimensions per 16-byte chunk
+    for (int i = 0; i < D; i += W) {
+        float x0[8], x1[8];   // centroid: x0; min/max: x0 = min, x1 = max
+        if constexpr (SK == kScoreMinmaxBf16) {
+            bf16x8(*tile_chunk(tile, j, i * 2), x0);
+            bf16x8(*tile_chunk(tile, j, (D + i) * 2), x1);
+        } else {
             const float4 a = *reinterpret_cast<const float4 *>(tile_chunk(tile, j, i * 4));
-            const float4 c = *reinterpret_cast<const float4 *>(tile_chunk(tile, j, (D + i) * 4));
-            const float lo[4] = {a.x, a.y, a.z, a.w}, hi[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-            for (int h = 0; h < kSelMaxG; ++h) {
-                if (h < G) {
-                    const float4 q4 = *reinterpret_cast<const float4 *>(qs + h * D + i);
-                    const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        acc[h] = __fmaf_rn(qv[e], qv[e] >= 0.0f ? hi[e] : lo[e], acc[h]);
-                }
+            x0[0] = a.x; x0[1] = a.y; x0[2] = a.z; x0[3] = a.w;
+            if constexpr (SK == kScoreMinmaxF32) {
+                const float4 c = *reinterpret_cast<const float4 *>(tile_chunk(tile, j, (D + i) * 4));
+                x1[0] = c.x; x1[1] = c.y; x1[2] = c.z; x1[3] = c.w;
             }
         }
-    } else {
-        for (int i = 0; i < D; i += 4) {
-            const float4 cv = *reinterpret_cast<const float4 *>(tile_chunk(tile, j, i * 4));
 #pragma unroll
-            for (int h = 0; h < kSelMaxG; ++h) {
-                if (h < G) {
-                    const float4 qv = *reinterpret_cast<const float4 *>(qs + h * D + i);
-                    acc[h] = __fmaf_rn(qv.x, cv.x, acc[h]);
-                    acc[h] = __fmaf_rn(qv.y, cv.y, acc[h]);
-                    acc[h] = __fmaf_rn(qv.z, cv.z, acc[h]);
-                    acc[h] = __fmaf_rn(qv.w, cv.w, acc[h]);
+        for (int e4 = 0; e4 < W; e4 += 4) {
+#pragma unroll
+            for (int h = 0; h < HPT; ++h) {
+                if (h0 + h >= G) break;
+                const float4 q4 = *reinterpret_cast<const float4 *>(qs + (h0 + h) * qstride + i + e4);
+                const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float x = x0[e4 + e];
+                    if constexpr (SK != kScoreCentroid) x = qv[e] >= 0.0f ? x1[e4 + e] : x0[e4 + e];
+                    acc[h] = __fmaf_rn(qv[e], x, acc[h]);
                 }
             }
         }
     }
-    float tot = acc[0];
-#pragma unroll
-    for (int h = 1; h < kSelMaxG; ++h)
-        if (h < G) tot = __fadd_rn(tot, acc[h]);
-    return __fadd_rn(tot, 0.0f);
 }
 
-// Number of rows of [r0, r1) whose position is below lim (positions ascend).
+// Rows of [r0, r1) whose position is below lim (positions ascend within a
+// block): rounds of 16 independent probes narrow the boundary, then at most
+// 16 rows are counted directly.
 __device__ __forceinline__ int visible_prefix(const int32_t *pos, int r0, int r1, int lim) {
-    int lo = r0, hi = r1;
-    while (lo < hi) {
-        int mid = (lo + hi) >> 1;
-        if (pos[mid] < lim) lo = mid + 1; else hi = mid;
+    constexpr int P = 16;
+    int lo = r0, hi = r1;   // rows < lo are visible, rows >= hi are not
+    while (hi - lo > P) {
+        const int w = hi - lo;
+        int p[P];
+        bool below[P];
+#pragma unroll
+        for (int k = 0; k < P; ++k) p[k] = lo + (int)((int64_t)(k + 1) * w / (P + 1));
+#pragma unroll
+        for (int k = 0; k < P; ++k) below[k] = __ldg(pos + p[k]) < lim;
+        // positions ascend, so the probes below lim come first
+        int nlo = lo, nhi = hi;
+#pragma unroll
+        for (int k = 0; k < P; ++k)
+            if (below[k]) nlo = p[k] + 1;
+#pragma unroll
+        for (int k = P - 1; k >= 0; --k)
+            if (!below[k]) nhi = p[k];
+        lo = nlo;
+        hi = nhi;
     }
-    return lo - r0;
+    int c = 0;
+#pragma unroll
+    for (int k = 0; k < P; ++k) c += (lo + k < hi) && __ldg(pos + lo + k) < lim;
+    return lo - r0 + c;
 }
 
-// Dynamic shared memory: [tile: nbox x 16 KiB, 1024-aligned][keys nb][sel
-// max_sel][vis nb][sort buffer (budget) or histogram (top-k)][merge items
-// (max_sel + 4) x int2][prefix maxima (max_sel + 4) x int]
-struct SelSmem {
-    __host__ __device__ static size_t tile_bytes(int nbox) { return (size_t)nbox * kSelThreads * 128; }
-    __host__ __device__ static int pow2(int nb) {
-        int N = 1;
-        while (N < nb) N <<= 1;
-        return N;
+// ---------------------------------------------------------------- scoring
+template <int SK, int GT>
+__global__ void __launch_bounds__(kSelThreads * score_tpb(GT), 1)
+    score_kernel(const __grid_constant__ CUtensorMap tmS, SelArgs a) {
+    constexpr int TPB = score_tpb(GT), HPT = score_hpt(GT);
+    extern __shared__ unsigned char dsm_raw[];
+    unsigned char *ring = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    const int G = GT > 0 ? GT : a.G, D = a.D, nb = a.nb_total;
+    const int qstage = G * (D + 4);                                                 // floats
+    float *qbuf = reinterpret_cast<float *>(ring + (size_t)a.nst * a.tile_bytes);   // [nst][G][D+4]
+    __shared__ uint64_t full[kSelMaxStages];
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int row = tid / TPB, part = tid % TPB;   // block row of the tile, head slice
+    const int my_items =
+        a.n_items > (int)blockIdx.x ? (a.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+    if (tid == 0) {
+        prefetch_tmap(&tmS);
+        for (int i = 0; i < a.nst; ++i) mbar_init(&full[i], 1);
+        fence_mbar_init();
     }
-    __host__ __device__ static size_t sort_bytes(int nb, bool variable) {
-        return variable ? (size_t)pow2(nb) * 8 : 256 * 4;
+    __syncthreads();
+    pdl_wait();   // queries, lengths and summaries come from earlier kernels
+    const int esz = SK == kScoreMinmaxBf16 ? 2 : 4;
+    auto issue = [&](int k) {   // thread 0: item k of this CTA into stage k % nst
+        const int item = (int)blockIdx.x + k * (int)gridDim.x;
+        const int s = item / a.tiles_per_seg, t = item % a.tiles_per_seg;
+        const int st = k % a.nst;
+        const int b = s / a.Hkv, g = s % a.Hkv;
+        unsigned char *dst = ring + (size_t)st * a.tile_bytes;
+        mbar_arrive_expect_tx(&full[st], a.tile_bytes + (uint32_t)(G * D * 4));
+        for (int bx = 0; bx < a.nbox; ++bx)
+            tma_load_2d(dst + bx * (kSelThreads * 128), &tmS, &full[st], bx * (128 / esz),
+                        s * nb + t * kSelThreads);
+        const float *qg = a.q + ((int64_t)b * a.Hq + (int64_t)g * G) * D;
+        for (int h = 0; h < G; ++h)   // head rows padded to D + 4 floats (conflict-free reads)
+            bulk_load(qbuf + (size_t)st * qstage + h * (D + 4), qg + h * D, (uint32_t)(D * 4), &full[st]);
+    };
+    if (tid == 0)
+        for (int k = 0; k < a.nst && k < my_items; ++k) issue(k);
+    bool timed_out = false;
+    for (int k = 0; k < my_items; ++k) {
+        const int item = (int)blockIdx.x + k * (int)gridDim.x;
+        const int s = item / a.tiles_per_seg, t = item % a.tiles_per_seg;
+        const int b = s / a.Hkv;
+        const int j = t * kSelThreads + row;
+        const bool writer = part == TPB - 1;
+        // candidacy needs no summary: worked out while the tile is in flight
+        int vis = 0;
+        bool valid = false;
+        if (writer && j < nb) {
+            if (a.offsets) {
+                const int32_t *off = a.offsets + (int64_t)s * (nb + 1);
+                const int r0 = min(max(off[j], 0), a.L_max), r1 = min(max(off[j + 1], r0), a.L_max);
+                vis = visible_prefix(a.kv_pos + (int64_t)s * a.L_max, r0, r1, a.pos_limit);
+                valid = vis > 0;
+            } else {
+                const int n = min(max(a.cur_len[b], 0), a.L_max);
+                valid = (int64_t)(j + 1) * a.S <= n;
+            }
+        }
+        const int st = k % a.nst;
+        if (!timed_out && !mbar_wait_bounded(&full[st], (uint32_t)((k / a.nst) & 1))) {
+            timed_out = true;
+            atomicOr(a.status, 2u);
+        }
+        float acc[HPT];
+        score_heads<SK, HPT>(qbuf + (size_t)st * qstage, part * HPT, G, D, ring + (size_t)st * a.tile_bytes,
+                             row, acc);
+        // heads summed in head order: the slices hand the running sum on
+        float run = acc[0];
+#pragma unroll
+        for (int h = 1; h < HPT; ++h)
+            if (part * HPT + h < G) run = __fadd_rn(run, acc[h]);
+#pragma unroll
+        for (int q = 1; q < TPB; ++q) {
+            const float prev = __shfl_up_sync(0xffffffffu, run, 1);
+            if (part == q) {
+                run = prev;
+#pragma unroll
+                for (int h = 0; h < HPT; ++h) run = __fadd_rn(run, acc[h]);
+            }
+        }
+        if (writer && j < nb) {
+            uint32_t key = 0;
+            if (valid) {
+                key = f32_order_key(__fadd_rn(run, 0.0f));
+                if (key == 0) key = 1;   // 0 marks "not a candidate"
+            }
+            a.keys[(int64_t)s * nb + j] = key;
+            if (a.offsets) a.vis[(int64_t)s * nb + j] = vis;
+        }
+        __syncthreads();   // stage st has been read by every thread
+        if (tid == 0 && k + a.nst < my_items) issue(k + a.nst);
     }
-    static size_t bytes(int nbox, int nb, int max_sel, bool variable) {
-        size_t p2 = (size_t)(2 * nb + max_sel) * 4;   // phase 2 reuses the tile buffer
-        p2 = (p2 + 7) & ~size_t(7);
-        p2 += sort_bytes(nb, variable);
-        p2 += (size_t)(max_sel + 4) * 12;
-        return 1024 + std::max(tile_bytes(nbox), p2);
+    (void)lane;
+    pdl_trigger();
+}
+
+// ---------------------------------------------------------------- picking
+constexpr int kPickWarpKeys = 16;   // keys per lane of the one-warp walks (nb <= 512)
+
+// Dynamic shared memory: [keys nb][vis nb][taken nb bytes, padded][sel
+// max_sel][hist 256][merge items (max_sel + 4) x int2][prefix maxima
+// (max_sel + 4) x int]
+struct PickSmem {
+    __host__ __device__ static size_t keys(int) { return 0; }
+    __host__ __device__ static size_t vis(int nb) { return (size_t)nb * 4; }
+    __host__ __device__ static size_t taken(int nb) { return (size_t)nb * 8; }
+    __host__ __device__ static size_t sel(int nb) { return (size_t)nb * 8 + (((size_t)nb + 15) & ~size_t(15)); }
+    __host__ __device__ static size_t hist(int nb, int max_sel) { return sel(nb) + (size_t)max_sel * 4; }
+    __host__ __device__ static size_t mrg(int nb, int max_sel) {
+        return (hist(nb, max_sel) + 256 * 4 + 7) & ~size_t(7);
+    }
+    __host__ __device__ static size_t pmax(int nb, int max_sel) {
+        return mrg(nb, max_sel) + (size_t)(max_sel + 4) * 8;
+    }
+    __host__ __device__ static size_t bytes(int nb, int max_sel) {
+        return pmax(nb, max_sel) + (size_t)(max_sel + 4) * 4;
     }
 };
 
-template <int KIND, typename T>
-__global__ void __launch_bounds__(kSelThreads)
-    select_kernel(const __grid_constant__ CUtensorMap tmS, SelArgs a) {
-    extern __shared__ unsigned char dsm_raw[];
-    unsigned char *tile = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(16) float qs[kSelMaxG * 128];
-    __shared__ int tmp[40];
-    __shared__ int is_last;
-    __shared__ uint64_t bar;
-
-    const int s = blockIdx.y;
-    const int b = s / a.Hkv, g = s % a.Hkv;
-    const int tid = threadIdx.x;
-    const int nb = a.nb_total;
-    const int j0 = blockIdx.x * kSelThreads;
-    if (tid == 0) {
-        prefetch_tmap(&tmS);
-        mbar_init(&bar, 1);
-        fence_mbar_init();
+// One warp takes, one at a time, the best remaining candidate (highest key,
+// then lowest index) -- that fits in what is left of the budget when
+// `budget` >= 0 -- up to `limit` blocks, marking them in taken[].  Keys and
+// visible counts of blocks lane + 32 r live in registers (nb <= 512).
+__device__ __forceinline__ void warp_walk_regs(const uint32_t *keys, const int32_t *visb, unsigned char *taken,
+                                               int nb, int limit, int budget, int lane) {
+    uint32_t wk[kPickWarpKeys];
+    int wv[kPickWarpKeys];
+#pragma unroll
+    for (int r = 0; r < kPickWarpKeys; ++r) {
+        const int j = lane + 32 * r;
+        wk[r] = j < nb ? keys[j] : 0u;
+        wv[r] = j < nb && budget >= 0 ? visb[j] : 0;
     }
-    pdl_trigger();
-    pdl_wait();   // queries, lengths and summaries come from earlier kernels
-    __syncthreads();
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bar, (uint32_t)(a.nbox * kSelThreads * 128));
-        const int esz = (KIND == BSA_SUM_MINMAX) ? (int)sizeof(T) : 4;
-        for (int bx = 0; bx < a.nbox; ++bx)
-            tma_load_2d(tile + bx * (kSelThreads * 128), &tmS, &bar, bx * (128 / esz), s * nb + j0);
+    int remaining = budget;
+    for (int n = 0; n < limit; ++n) {
+        unsigned long long best = 0ull;
+#pragma unroll
+        for (int r = 0; r < kPickWarpKeys; ++r)
+            if (wk[r] && (budget < 0 || wv[r] <= remaining)) {
+                const unsigned long long c =
+                    ((unsigned long long)wk[r] << 32) | (0xffffffffu - (uint32_t)(lane + 32 * r));
+                best = c > best ? c : best;
+            }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other > best ? other : best;
+        }
+        if (best == 0ull) break;
+        const int j = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
+        if (budget >= 0) remaining -= visb[j];
+#pragma unroll
+        for (int r = 0; r < kPickWarpKeys; ++r)
+            if (lane + 32 * r == j) wk[r] = 0u;
+        if (lane == 0) taken[j] = 1;
+    }
+}
+
+// The same walk over shared memory (any nb).
+__device__ void warp_walk_smem(const uint32_t *keys, const int32_t *visb, unsigned char *taken, int nb,
+                               int limit, int budget, int lane) {
+    int remaining = budget;
+    for (int n = 0; n < limit; ++n) {
+        unsigned long long best = 0ull;
+        for (int j = lane; j < nb; j += 32)
+            if (keys[j] && !taken[j] && (budget < 0 || visb[j] <= remaining)) {
+                const unsigned long long c = ((unsigned long long)keys[j] << 32) | (0xffffffffu - (uint32_t)j);
+                best = c > best ? c : best;
+            }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other > best ? other : best;
+        }
+        if (best == 0ull) break;
+        const int j = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
+        if (budget >= 0) remaining -= visb[j];
+        if (lane == 0) taken[j] = 1;
+        __syncwarp();
+    }
+}
+
+// One CTA per segment.  Thread t holds the keys of blocks [t KPT, t KPT + KPT)
+// in registers (nb <= kPickThreads * KPT).
+template <int KPT>
+__global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
+    extern __shared__ __align__(16) unsigned char psm[];
+    const int nb = a.nb_total;
+    uint32_t *keys = reinterpret_cast<uint32_t *>(psm + PickSmem::keys(nb));
+    int32_t *visb = reinterpret_cast<int32_t *>(psm + PickSmem::vis(nb));
+    unsigned char *taken = psm + PickSmem::taken(nb);
+    int32_t *sel = reinterpret_cast<int32_t *>(psm + PickSmem::sel(nb));
+    int *hist = reinterpret_cast<int *>(psm + PickSmem::hist(nb, a.max_sel));
+    int2 *mrg = reinterpret_cast<int2 *>(psm + PickSmem::mrg(nb, a.max_sel));
+    int *pmax = reinterpret_cast<int *>(psm + PickSmem::pmax(nb, a.max_sel));
+    __shared__ int tmp[40];
+    __shared__ int f_lo[3], f_hi[3], n_forced, n_sel_sh, sh_bin, sh_excl;
+
+    const int s = blockIdx.x;
+    const int b = s / a.Hkv;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int32_t *off = a.offsets ? a.offsets + (int64_t)s * (nb + 1) : nullptr;
+    const int c0 = tid * KPT;   // this thread's blocks [c0, c0 + KPT)
+    pdl_wait();   // keys and visible counts from score_kernel
+    // every load of the thread issued before any is used
+    uint32_t kr[KPT];
+#pragma unroll
+    for (int r = 0; r < KPT; ++r) kr[r] = c0 + r < nb ? a.keys[(int64_t)s * nb + c0 + r] : 0u;
+    if (off) {
+        int vr[KPT];
+#pragma unroll
+        for (int r = 0; r < KPT; ++r) vr[r] = c0 + r < nb ? a.vis[(int64_t)s * nb + c0 + r] : 0;
+#pragma unroll
+        for (int r = 0; r < KPT; ++r)
+            if (c0 + r < nb) visb[c0 + r] = vr[r];
     }
     const int n = min(max(a.cur_len[b], 0), a.L_max);
-    const int32_t *off = a.offsets ? a.offsets + (int64_t)s * (nb + 1) : nullptr;
-    const int32_t *pos = a.kv_pos ? a.kv_pos + (int64_t)s * a.L_max : nullptr;
-    for (int e = tid; e < a.G * a.D; e += kSelThreads)
-        qs[e] = a.q[((int64_t)b * a.Hq + (int64_t)g * a.G) * a.D + e];
-
-    // ---------------- phase 1: score this CTA's tile, one thread per block
-    const int j = j0 + tid;
-    bool valid = false;
-    int vis = 0;
-    if (j < nb) {
-        if (off) {
-            const int r0 = min(max(off[j], 0), a.L_max), r1 = min(max(off[j + 1], r0), a.L_max);
-            vis = visible_prefix(pos, r0, r1, a.pos_limit);
-            valid = vis > 0;
-        } else {
-            valid = (int64_t)(j + 1) * a.S <= n;
-        }
-    }
-    __syncthreads();   // qs
-    if (!mbar_wait_bounded(&bar, 0)) atomicOr(a.status, 2u);
-    if (j < nb) {
-        uint32_t key = 0;
-        if (valid) {
-            key = f32_order_key(score_row<KIND, T>(qs, a.G, a.D, tile, tid));
-            if (key == 0) key = 1;   // 0 marks "not a candidate"
-        }
-        a.keys[(int64_t)s * nb + j] = key;
-        if (off) a.vis[(int64_t)s * nb + j] = vis;
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) is_last = atomicAdd(&a.counters[s], 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-
-    // ---------------- phase 2: the last CTA of the segment selects (its tile
-    // has been scored; the buffer is reused)
-    uint32_t *keys = reinterpret_cast<uint32_t *>(tile);
-    int32_t *sel = reinterpret_cast<int32_t *>(keys + nb);
-    int32_t *visb = sel + a.max_sel;
-    unsigned char *after = reinterpret_cast<unsigned char *>(visb + nb);
-    after = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(after) + 7) & ~uintptr_t(7));
-    unsigned long long *sortbuf = reinterpret_cast<unsigned long long *>(after);
-    int2 *mrg = reinterpret_cast<int2 *>(after + SelSmem::sort_bytes(nb, off != nullptr));
-    int *pmax = reinterpret_cast<int *>(mrg + a.max_sel + 4);
-    __shared__ int f_lo[3], f_hi[3], n_forced, n_sel_sh;
-
     if (tid == 0) {
         // forced token ranges, sorted and merged
         int lo[3], hi[3], m = 0;
@@ -253,69 +390,97 @@ __global__ void __launch_bounds__(kSelThreads)
     __syncthreads();
 
     // candidates: keys > 0 and (fixed blocks) not wholly inside the forced set
+    const int nf = n_forced;
     int my_c = 0;
-    for (int jj = tid; jj < nb; jj += kSelThreads) {
-        uint32_t key = __ldcg(&a.keys[(int64_t)s * nb + jj]);
+#pragma unroll
+    for (int r = 0; r < KPT; ++r) {
+        uint32_t key = kr[r];
         if (key && !off) {
-            const int64_t r0 = (int64_t)jj * a.S, r1 = r0 + a.S;
-            for (int i = 0; i < n_forced; ++i)
+            const int64_t r0 = (int64_t)(c0 + r) * a.S, r1 = r0 + a.S;
+            for (int i = 0; i < nf; ++i)
                 if (f_lo[i] <= r0 && r1 <= f_hi[i]) key = 0;
         }
-        keys[jj] = key;
-        if (off) visb[jj] = __ldcg(&a.vis[(int64_t)s * nb + jj]);
+        kr[r] = key;
         my_c += key != 0;
     }
     int n_cand;
     cta_excl_sum(my_c, tmp, &n_cand);
 
     const bool greedy = off && a.topk < 0;
-    if (!greedy) {
+    int k = 0;
+    if (!greedy) k = min(min(a.topk >= 0 ? a.topk : a.budget / a.S, n_cand), a.max_sel);
+    const bool small_nb = nb <= 32 * kPickWarpKeys;
+    if (greedy || (k <= 32 && small_nb)) {
+        // ---- one warp walks the ranking: the token budget (take a block
+        // when its visible rows fit in what is left; that only shrinks, so a
+        // block that does not fit now never will, and each step takes the
+        // best remaining candidate that fits), or a small top-k
+#pragma unroll
+        for (int r = 0; r < KPT; ++r)
+            if (c0 + r < nb) {
+                keys[c0 + r] = kr[r];
+                taken[c0 + r] = 0;
+            }
+        __syncthreads();
+        if (warp == 0) {
+            const int limit = greedy ? a.max_sel : k;
+            const int budget = greedy ? a.budget : -1;
+            if (small_nb) warp_walk_regs(keys, visb, taken, nb, limit, budget, lane);
+            else warp_walk_smem(keys, visb, taken, nb, limit, budget, lane);
+        }
+        __syncthreads();
+        int my_take = 0;
+#pragma unroll
+        for (int r = 0; r < KPT; ++r) my_take += c0 + r < nb && taken[c0 + r];
+        int tot;
+        int p = cta_excl_sum(my_take, tmp, &tot);
+#pragma unroll
+        for (int r = 0; r < KPT; ++r)
+            if (c0 + r < nb && taken[c0 + r] && p < a.max_sel) sel[p++] = c0 + r;
+        if (tid == 0) n_sel_sh = min(tot, a.max_sel);
+    } else {
         // ---- top-k: radix select of the k-th largest key, 8 bits per pass
-        int k = a.topk >= 0 ? a.topk : a.budget / a.S;
-        k = min(min(k, n_cand), a.max_sel);
         uint32_t thr = 0xffffffffu;
         int need_eq = 0;
         if (k > 0) {
-            int *hist = reinterpret_cast<int *>(sortbuf);   // 256 bins
-            __shared__ int sh_bin, sh_excl;
             uint32_t prefix = 0, pmask = 0;
             int krem = k;
             for (int pass = 0; pass < 4; ++pass) {
                 const int shift = 24 - 8 * pass;
-                hist[2 * tid] = 0;
-                hist[2 * tid + 1] = 0;
+                if (tid < 256) hist[tid] = 0;
                 __syncthreads();
-                for (int jj = tid; jj < nb; jj += kSelThreads) {
-                    const uint32_t key = keys[jj];
-                    if (key && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+#pragma unroll
+                for (int r = 0; r < KPT; ++r) {
+                    const uint32_t key = kr[r];
+                    const bool act = key && (key & pmask) == prefix;
+                    const uint32_t bin = act ? (key >> shift) & 255u : 256u;
+                    // lanes with the same bin add once (most keys share the
+                    // high bits)
+                    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+                    if (act && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
                 }
                 __syncthreads();
-                // thread t owns bins 255-2t and 254-2t (counted from the top)
-                const int v0 = hist[255 - 2 * tid], v1 = hist[254 - 2 * tid];
+                // thread t < 256 owns bin 255 - t (counted from the top)
+                const int v = tid < 256 ? hist[255 - tid] : 0;
                 int tot;
-                const int ex = cta_excl_sum(v0 + v1, tmp, &tot);
-                if (ex < krem && ex + v0 >= krem) { sh_bin = 255 - 2 * tid; sh_excl = ex; }
-                else if (ex + v0 < krem && ex + v0 + v1 >= krem) { sh_bin = 254 - 2 * tid; sh_excl = ex + v0; }
+                const int ex = cta_excl_sum(v, tmp, &tot);
+                if (tid < 256 && ex < krem && ex + v >= krem) { sh_bin = 255 - tid; sh_excl = ex; }
                 __syncthreads();
                 prefix |= (uint32_t)sh_bin << shift;
                 pmask |= 0xffu << shift;
                 krem -= sh_excl;
-                __syncthreads();
             }
             thr = prefix;
             need_eq = krem;
         }
         // index-ordered compaction: key > thr, or key == thr among the first
-        // need_eq; each thread owns a contiguous run of block indices
-        const int chunk = (nb + kSelThreads - 1) / kSelThreads;
-        const int c0 = min(nb, tid * chunk), c1 = min(nb, c0 + chunk);
+        // need_eq
         int my_eq = 0, my_gt = 0;
-        if (k > 0)
-            for (int jj = c0; jj < c1; ++jj) {
-                const uint32_t key = keys[jj];
-                my_eq += key != 0 && key == thr;
-                my_gt += key != 0 && key > thr;
-            }
+#pragma unroll
+        for (int r = 0; r < KPT; ++r) {
+            my_eq += k > 0 && kr[r] != 0 && kr[r] == thr;
+            my_gt += k > 0 && kr[r] != 0 && kr[r] > thr;
+        }
         int tot;
         const int eq_base = cta_excl_sum(my_eq, tmp, &tot);
         const int my_take = my_gt + min(my_eq, max(0, need_eq - eq_base));
@@ -323,63 +488,23 @@ __global__ void __launch_bounds__(kSelThreads)
         if (tid == 0) n_sel_sh = tot;
         if (my_take > 0) {
             int eq_seen = eq_base;
-            for (int jj = c0; jj < c1; ++jj) {
-                const uint32_t key = keys[jj];
-                if (key != 0 && key > thr) sel[p++] = jj;
-                else if (key != 0 && key == thr && eq_seen++ < need_eq) sel[p++] = jj;
+#pragma unroll
+            for (int r = 0; r < KPT; ++r) {
+                const uint32_t key = kr[r];
+                if (key != 0 && key > thr) sel[p++] = c0 + r;
+                else if (key != 0 && key == thr && eq_seen++ < need_eq) sel[p++] = c0 + r;
             }
         }
-    } else {
-        // ---- token budget: bitonic sort by (key desc, index asc), greedy walk
-        const int N = SelSmem::pow2(nb);
-        for (int jj = tid; jj < N; jj += kSelThreads)
-            sortbuf[jj] = jj < nb ? ((unsigned long long)keys[jj] << 32) | (0xffffffffu - (uint32_t)jj)
-                                  : 0ull;
-        __syncthreads();
-        for (int kk = 2; kk <= N; kk <<= 1) {
-            for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-                for (int i = tid; i < N; i += kSelThreads) {
-                    const int ixj = i ^ jj;
-                    if (ixj > i) {
-                        const unsigned long long x = sortbuf[i], y = sortbuf[ixj];
-                        const bool desc = (i & kk) == 0;
-                        if (desc ? (x < y) : (x > y)) { sortbuf[i] = y; sortbuf[ixj] = x; }
-                    }
-                }
-                __syncthreads();
-            }
-        }
-        // greedy walk (sequential by definition); selection marks reuse the keys
-        for (int jj = tid; jj < nb; jj += kSelThreads) keys[jj] = 0;
-        __syncthreads();
-        if (tid == 0) {
-            int used = 0;
-            for (int i = 0; i < n_cand; ++i) {
-                const int jj = (int)(0xffffffffu - (uint32_t)(sortbuf[i] & 0xffffffffu));
-                const int v = visb[jj];
-                if (used + v <= a.budget) { used += v; keys[jj] = 0xffffffffu; }
-            }
-        }
-        __syncthreads();
-        const int chunk = (nb + kSelThreads - 1) / kSelThreads;
-        const int c0 = min(nb, tid * chunk), c1 = min(nb, c0 + chunk);
-        int my_take = 0;
-        for (int jj = c0; jj < c1; ++jj) my_take += keys[jj] == 0xffffffffu;
-        int tot;
-        int p = cta_excl_sum(my_take, tmp, &tot);
-        for (int jj = c0; jj < c1; ++jj)
-            if (keys[jj] == 0xffffffffu && p < a.max_sel) sel[p++] = jj;
-        if (tid == 0) n_sel_sh = min(tot, a.max_sel);
     }
     __syncthreads();
-    const int n_sel = n_sel_sh, nf = n_forced;
+    const int n_sel = n_sel_sh;
 
-    for (int i = tid; i < n_sel; i += kSelThreads) a.sel_blocks[(int64_t)s * a.max_sel + i] = sel[i];
+    for (int i = tid; i < n_sel; i += kPickThreads) a.sel_blocks[(int64_t)s * a.max_sel + i] = sel[i];
 
     // ---- ranges.  Merge the forced ranges and the selected blocks' ranges
     // (both ascending; on equal starts the forced range comes first) ...
     const int m = n_sel + nf;
-    for (int i = tid; i < n_sel; i += kSelThreads) {
+    for (int i = tid; i < n_sel; i += kPickThreads) {
         const int jj = sel[i];
         int lo, hi;
         if (off) { lo = min(max(off[jj], 0), a.L_max); hi = lo + visb[jj]; }
@@ -403,7 +528,7 @@ __global__ void __launch_bounds__(kSelThreads)
     // it starts after every earlier item has ended; a range ends at the
     // running maximum of its last item.
     int carry = kIntMin;
-    for (int t0 = 0; t0 < m; t0 += kSelThreads) {
+    for (int t0 = 0; t0 < m; t0 += kPickThreads) {
         const int i = t0 + tid;
         int tot;
         const int pm = max(cta_incl_max(i < m ? mrg[i].y : kIntMin, tmp, &tot), carry);
@@ -413,7 +538,7 @@ __global__ void __launch_bounds__(kSelThreads)
     __syncthreads();
     int32_t *R = a.ranges + (int64_t)s * a.max_ranges * 2;
     int nr = 0;
-    for (int t0 = 0; t0 < m; t0 += kSelThreads) {
+    for (int t0 = 0; t0 < m; t0 += kPickThreads) {
         const int i = t0 + tid;
         const int start = i < m && (i == 0 || mrg[i].x > pmax[i - 1]);
         int tot;
@@ -428,15 +553,19 @@ __global__ void __launch_bounds__(kSelThreads)
     if (tid == 0) {
         a.n_ranges[s] = min(nr, a.max_ranges);
         a.sel_count[s] = n_sel;
-        a.counters[s] = 0;   // leave the workspace reusable
     }
 }
+
+// Largest block count the selection handles (the pick kernel holds up to 32
+// keys per thread in registers).
+constexpr int kSelMaxBlocks = kPickThreads * 32;
 
 bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ, int kind,
                          const bsa_sel_params *p, const int32_t *cur_len, int nb_total,
                          int max_sel, int32_t *sel_blocks, int32_t *sel_count, int max_ranges,
                          int32_t *ranges, int32_t *n_ranges, uint32_t *keys, int32_t *vis,
                          uint32_t *counters, uint32_t *status, cudaStream_t st) {
+    (void)counters;
     SelArgs a;
     a.q = q; a.cur_len = cur_len;
     const bool variable = p->block_size == 0;
@@ -454,23 +583,57 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
     const int cols = kind == BSA_SUM_MINMAX ? 2 * d->D : d->D;
     a.row_bytes = cols * esz;
     a.nbox = a.row_bytes / 128;
+    a.tile_bytes = (uint32_t)(a.nbox * kSelThreads * 128);
+    const size_t qbytes = (size_t)a.G * (d->D + 4) * 4;
+    const size_t cap = 227 * 1024 - 1024;
+    a.nst = (int)std::min<size_t>(kSelMaxStages, cap / (a.tile_bytes + qbytes));
+    if (a.nst < 1) return BSA_ERR_UNSUPPORTED;
+    const size_t smem1 = 1024 + (size_t)a.nst * (a.tile_bytes + qbytes);
+    const size_t smem2 = PickSmem::bytes(nb_total, max_sel);
+    if (smem2 > cap || nb_total > kSelMaxBlocks) return BSA_ERR_UNSUPPORTED;
+    a.tiles_per_seg = (int)div_up(nb_total, kSelThreads);
+    const int nseg = d->B * d->Hkv;
+    a.n_items = nseg * a.tiles_per_seg;
     CUtensorMap tm;
     if (!make_rows_tmap(&tm, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                        esz, summ, cols, (int64_t)d->B * d->Hkv * nb_total, a.row_bytes, kSelThreads))
+                        esz, summ, cols, (int64_t)nseg * nb_total, a.row_bytes, kSelThreads))
         return BSA_ERR_CUDA;
-    const size_t smem = SelSmem::bytes(a.nbox, nb_total, max_sel, variable);
-    if (smem > 220 * 1024) return BSA_ERR_UNSUPPORTED;
-    dim3 grid((unsigned)div_up(nb_total, kSelThreads), d->B * d->Hkv);
-    auto launch = [&](auto kern) -> bsa_status {
-        BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        BSA_CUDA_TRY(launch_pdl(kern, grid, dim3(kSelThreads), smem, st, tm, a));
+    auto launch = [&](auto kern, int tpb) -> bsa_status {
+        BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1));
+        const int threads = kSelThreads * tpb;
+        int per_sm = 0;
+        BSA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem1));
+        const int grid = std::max(1, std::min(a.n_items, num_sms() * std::max(per_sm, 1)));
+        BSA_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(threads), smem1, st, tm, a));
         return BSA_OK;
     };
+    auto by_g = [&](auto sk) -> bsa_status {
+        constexpr int SK = decltype(sk)::value;
+        switch (a.G) {
+            case 1: return launch(score_kernel<SK, 1>, score_tpb(1));
+            case 2: return launch(score_kernel<SK, 2>, score_tpb(2));
+            case 4: return launch(score_kernel<SK, 4>, score_tpb(4));
+            case 8: return launch(score_kernel<SK, 8>, score_tpb(8));
+            case 16: return launch(score_kernel<SK, 16>, score_tpb(16));
+            default: return launch(score_kernel<SK, 0>, score_tpb(0));
+        }
+    };
+    bsa_status r;
     if (kind == BSA_SUM_MINMAX)
-        return bf ? launch(select_kernel<BSA_SUM_MINMAX, uint16_t>)
-                  : launch(select_kernel<BSA_SUM_MINMAX, float>);
-    if (kind == BSA_SUM_CENTROID) return launch(select_kernel<BSA_SUM_CENTROID, float>);
-    return launch(select_kernel<BSA_SUM_CENTROID_NORM, float>);
+        r = bf ? by_g(std::integral_constant<int, kScoreMinmaxBf16>())
+               : by_g(std::integral_constant<int, kScoreMinmaxF32>());
+    else
+        r = by_g(std::integral_constant<int, kScoreCentroid>());
+    if (r != BSA_OK) return r;
+    auto pick = [&](auto kern) -> bsa_status {
+        BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2));
+        BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(kPickThreads), smem2, st, a));
+        return BSA_OK;
+    };
+    if (nb_total <= kPickThreads) return pick(pick_kernel<1>);
+    if (nb_total <= kPickThreads * 4) return pick(pick_kernel<4>);
+    if (nb_total <= kPickThreads * 16) return pick(pick_kernel<16>);
+    return pick(pick_kernel<32>);
 }
 
 }  // namespace bsa
