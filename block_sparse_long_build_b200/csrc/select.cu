@@ -35,6 +35,7 @@ constexpr int kSelThreads = 128;   // scoring threads = rows per tile
 constexpr int kPickThreads = 512;
 constexpr int kSelMaxG = 16;
 constexpr int kSelMaxStages = 3;
+constexpr int kScoreStages = 1;    // tile stages per CTA: several CTAs per SM overlap instead
 constexpr int kIntMin = -0x7fffffff - 1;
 enum { kScoreCentroid = 0, kScoreMinmaxBf16 = 1, kScoreMinmaxF32 = 2 };
 
@@ -64,57 +65,90 @@ __device__ __forceinline__ const uint4 *tile_chunk(const unsigned char *tile, in
                                            ((c ^ (j & 7)) << 4));
 }
 
-__device__ __forceinline__ void bf16x8(uint4 v, float (&f)[8]) {
-    f[0] = __uint_as_float(v.x << 16); f[1] = __uint_as_float(v.x & 0xffff0000u);
-    f[2] = __uint_as_float(v.y << 16); f[3] = __uint_as_float(v.y & 0xffff0000u);
-    f[4] = __uint_as_float(v.z << 16); f[5] = __uint_as_float(v.z & 0xffff0000u);
-    f[6] = __uint_as_float(v.w << 16); f[7] = __uint_as_float(v.w & 0xffff0000u);
-}
+// Threads per block row and heads per thread of the scoring kernel: one
+// thread per block row holds all G head chains, so each summary row is read
+// from shared memory once and the query values are warp-wide broadcasts.
+__host__ __device__ constexpr int score_tpb(int) { return 1; }
+__host__ __device__ constexpr int score_hpt(int GT) { return GT == 0 ? kSelMaxG : GT; }
 
-// Threads per block row and heads per thread of the scoring kernel: a
-// block's G heads are split over up to 4 threads (more warps in flight); G
-// known only at run time (GT = 0) keeps one thread per block.
-__host__ __device__ constexpr int score_tpb(int GT) { return GT == 0 ? 1 : (GT < 4 ? GT : 4); }
-__host__ __device__ constexpr int score_hpt(int GT) { return GT == 0 ? kSelMaxG : GT / score_tpb(GT); }
+// Byte-permute selectors that widen the min (bytes 0-1) or the max (bytes
+// 2-3) of a packed (min, max) bf16 pair into fp32 bits (zeros from the second
+// operand below): x = max where q >= 0, else min.
+constexpr uint32_t kPickMin = 0x1044u, kPickMax = 0x3244u;
+
+__device__ __forceinline__ float widen_bf16(uint32_t pair, uint32_t sel) {
+    uint32_t x;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(x) : "r"(pair), "r"(sel));
+    return __uint_as_float(x);
+}
 
 // Partial scores of tile row j for heads h0 .. h0 + HPT - 1 (those below G):
 // per head an fma chain over i = 0..D-1 in the fixed fp32 order; the chains
-// of the thread's heads are interleaved.  qs: head rows of D + 4 floats.
-template <int SK, int HPT>
-__device__ __forceinline__ void score_heads(const float *qs, int h0, int G, int D,
+// of the thread's heads are interleaved.  qs: head rows of D + 4 floats; sl:
+// the same layout of min/max selectors (bf16 min/max only).  DT: D when
+// known at compile time (the dimension loop unrolls and the row's swizzled
+// chunk offsets are computed once), 0 otherwise.
+template <int SK, int HPT, int DT>
+__device__ __forceinline__ void score_heads(const float *qs, const uint32_t *sl, int h0, int G, int Drt,
                                             const unsigned char *tile, int j, float (&acc)[HPT]) {
+    const int D = DT > 0 ? DT : Drt;
     const int qstride = D + 4;
 #pragma unroll
     for (int h = 0; h < HPT; ++h) acc[h] = 0.0f;
-    constexpr int W = SK == kScoreMinmaxBf16 ? 8 : 4;   // dimensions per 16-byte chunk
-    for (int i = 0; i < D; i += W) {
-        float x0[8], x1[8];   // centroid: x0; min/max: x0 = min, x1 = max
-        if constexpr (SK == kScoreMinmaxBf16) {
-            bf16x8(*tile_chunk(tile, j, i * 2), x0);
-            bf16x8(*tile_chunk(tile, j, (D + i) * 2), x1);
-        } else {
-            const float4 a = *reinterpret_cast<const float4 *>(tile_chunk(tile, j, i * 4));
-            x0[0] = a.x; x0[1] = a.y; x0[2] = a.z; x0[3] = a.w;
-            if constexpr (SK == kScoreMinmaxF32) {
-                const float4 c = *reinterpret_cast<const float4 *>(tile_chunk(tile, j, (D + i) * 4));
-                x1[0] = c.x; x1[1] = c.y; x1[2] = c.z; x1[3] = c.w;
-            }
-        }
+    const unsigned char *row = tile + j * 128;
+    uint32_t sw[8];   // swizzled offset of 16-byte chunk c within the row's 128 bytes
 #pragma unroll
-        for (int e4 = 0; e4 < W; e4 += 4) {
+    for (int c = 0; c < 8; ++c) sw[c] = (uint32_t)((c ^ (j & 7)) << 4);
+    auto chunk = [&](int off) -> uint4 {
+        if constexpr (DT > 0)
+            return *reinterpret_cast<const uint4 *>(row + (off >> 7) * (kSelThreads * 128) + sw[(off >> 4) & 7]);
+        else
+            return *tile_chunk(tile, j, off);
+    };
+    auto step = [&](int i) {
+        if constexpr (SK == kScoreMinmaxBf16) {   // dimensions i .. i+3, one (min, max) pair each
+            const uint4 w = chunk(i * 4);
 #pragma unroll
             for (int h = 0; h < HPT; ++h) {
                 if (h0 + h >= G) break;
-                const float4 q4 = *reinterpret_cast<const float4 *>(qs + (h0 + h) * qstride + i + e4);
+                const float4 q4 = *reinterpret_cast<const float4 *>(qs + (h0 + h) * qstride + i);
+                const uint4 s4 = *reinterpret_cast<const uint4 *>(sl + (h0 + h) * qstride + i);
+                acc[h] = __fmaf_rn(q4.x, widen_bf16(w.x, s4.x), acc[h]);
+                acc[h] = __fmaf_rn(q4.y, widen_bf16(w.y, s4.y), acc[h]);
+                acc[h] = __fmaf_rn(q4.z, widen_bf16(w.z, s4.z), acc[h]);
+                acc[h] = __fmaf_rn(q4.w, widen_bf16(w.w, s4.w), acc[h]);
+            }
+        } else if constexpr (SK == kScoreMinmaxF32) {   // dimensions i, i+1: (min, max) pairs
+            const uint4 w = chunk(i * 8);
+#pragma unroll
+            for (int h = 0; h < HPT; ++h) {
+                if (h0 + h >= G) break;
+                const float2 q2 = *reinterpret_cast<const float2 *>(qs + (h0 + h) * qstride + i);
+                const float x0 = q2.x >= 0.0f ? __uint_as_float(w.y) : __uint_as_float(w.x);
+                const float x1 = q2.y >= 0.0f ? __uint_as_float(w.w) : __uint_as_float(w.z);
+                acc[h] = __fmaf_rn(q2.x, x0, acc[h]);
+                acc[h] = __fmaf_rn(q2.y, x1, acc[h]);
+            }
+        } else {   // centroid: dimensions i .. i+3
+            const uint4 a = chunk(i * 4);
+            const float x[4] = {__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z),
+                                __uint_as_float(a.w)};
+#pragma unroll
+            for (int h = 0; h < HPT; ++h) {
+                if (h0 + h >= G) break;
+                const float4 q4 = *reinterpret_cast<const float4 *>(qs + (h0 + h) * qstride + i);
                 const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float x = x0[e4 + e];
-                    if constexpr (SK != kScoreCentroid) x = qv[e] >= 0.0f ? x1[e4 + e] : x0[e4 + e];
-                    acc[h] = __fmaf_rn(qv[e], x, acc[h]);
-                }
+                for (int e = 0; e < 4; ++e) acc[h] = __fmaf_rn(qv[e], x[e], acc[h]);
             }
         }
+    };
+    constexpr int W = SK == kScoreMinmaxF32 ? 2 : 4;   // dimensions per 16-byte chunk
+    if constexpr (DT > 0) {
+#pragma unroll
+        for (int i = 0; i < DT; i += W) step(i);
+    } else {
+        for (int i = 0; i < D; i += W) step(i);
     }
 }
 
@@ -150,8 +184,8 @@ __device__ __forceinline__ int visible_prefix(const int32_t *pos, int r0, int r1
 }
 
 // ---------------------------------------------------------------- scoring
-template <int SK, int GT>
-__global__ void __launch_bounds__(kSelThreads * score_tpb(GT), 1)
+template <int SK, int GT, int DT>
+__global__ void __launch_bounds__(kSelThreads * score_tpb(GT), 3)
     score_kernel(const __grid_constant__ CUtensorMap tmS, SelArgs a) {
     constexpr int TPB = score_tpb(GT), HPT = score_hpt(GT);
     extern __shared__ unsigned char dsm_raw[];
@@ -160,6 +194,7 @@ __global__ void __launch_bounds__(kSelThreads * score_tpb(GT), 1)
     const int G = GT > 0 ? GT : a.G, D = a.D, nb = a.nb_total;
     const int qstage = G * (D + 4);                                                 // floats
     float *qbuf = reinterpret_cast<float *>(ring + (size_t)a.nst * a.tile_bytes);   // [nst][G][D+4]
+    uint32_t *selb = reinterpret_cast<uint32_t *>(qbuf + (size_t)a.nst * qstage);   // [G][D+4]
     __shared__ uint64_t full[kSelMaxStages];
     const int tid = threadIdx.x, lane = tid & 31;
     const int row = tid / TPB, part = tid % TPB;   // block row of the tile, head slice
@@ -215,9 +250,17 @@ __global__ void __launch_bounds__(kSelThreads * score_tpb(GT), 1)
             timed_out = true;
             atomicOr(a.status, 2u);
         }
+        const float *qs = qbuf + (size_t)st * qstage;
+        if constexpr (SK == kScoreMinmaxBf16) {
+            // per (head, dimension): which bound the query's sign picks
+            for (int e = tid; e < G * D; e += blockDim.x) {
+                const int h = e / D, i = e % D;
+                selb[h * (D + 4) + i] = qs[h * (D + 4) + i] < 0.0f ? kPickMin : kPickMax;
+            }
+            __syncthreads();
+        }
         float acc[HPT];
-        score_heads<SK, HPT>(qbuf + (size_t)st * qstage, part * HPT, G, D, ring + (size_t)st * a.tile_bytes,
-                             row, acc);
+        score_heads<SK, HPT, DT>(qs, selb, part * HPT, G, D, ring + (size_t)st * a.tile_bytes, row, acc);
         // heads summed in head order: the slices hand the running sum on
         float run = acc[0];
 #pragma unroll
@@ -334,9 +377,10 @@ __device__ void warp_walk_smem(const uint32_t *keys, const int32_t *visb, unsign
     }
 }
 
-// One CTA per segment.  Thread t holds the keys of blocks [t KPT, t KPT + KPT)
-// in registers (nb <= kPickThreads * KPT).
-template <int KPT>
+// One CTA per segment.  The candidate keys live in shared memory; thread t
+// owns the contiguous blocks [t kpt, t kpt + kpt) for the index-ordered
+// compactions.  Loops stay rolled (short unrolls batch the loads): the
+// kernel runs once per selection, so compact code beats straight-line code.
 __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
     extern __shared__ __align__(16) unsigned char psm[];
     const int nb = a.nb_total;
@@ -354,23 +398,12 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
     const int b = s / a.Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int32_t *off = a.offsets ? a.offsets + (int64_t)s * (nb + 1) : nullptr;
-    const int c0 = tid * KPT;   // this thread's blocks [c0, c0 + KPT)
+    const int kpt = (nb + kPickThreads - 1) / kPickThreads;
+    const int c0 = tid * kpt;   // this thread's blocks [c0, c0 + kpt)
     pdl_wait();   // keys and visible counts from score_kernel
-    // every load of the thread issued before any is used
-    uint32_t kr[KPT];
-#pragma unroll
-    for (int r = 0; r < KPT; ++r) kr[r] = c0 + r < nb ? a.keys[(int64_t)s * nb + c0 + r] : 0u;
-    if (off) {
-        int vr[KPT];
-#pragma unroll
-        for (int r = 0; r < KPT; ++r) vr[r] = c0 + r < nb ? a.vis[(int64_t)s * nb + c0 + r] : 0;
-#pragma unroll
-        for (int r = 0; r < KPT; ++r)
-            if (c0 + r < nb) visb[c0 + r] = vr[r];
-    }
-    const int n = min(max(a.cur_len[b], 0), a.L_max);
     if (tid == 0) {
         // forced token ranges, sorted and merged
+        const int n = min(max(a.cur_len[b], 0), a.L_max);
         int lo[3], hi[3], m = 0;
         if (off) {
             if (n > a.local_start) { lo[m] = max(a.local_start, 0); hi[m] = n; ++m; }
@@ -388,23 +421,26 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
         n_forced = m;
     }
     __syncthreads();
-
-    // candidates: keys > 0 and (fixed blocks) not wholly inside the forced set
     const int nf = n_forced;
+
+    // candidates: keys > 0 and (fixed blocks) not wholly inside the forced
+    // set; coalesced loads, eight in flight per thread
     int my_c = 0;
-#pragma unroll
-    for (int r = 0; r < KPT; ++r) {
-        uint32_t key = kr[r];
+#pragma unroll 8
+    for (int jj = tid; jj < nb; jj += kPickThreads) {
+        uint32_t key = a.keys[(int64_t)s * nb + jj];
         if (key && !off) {
-            const int64_t r0 = (int64_t)(c0 + r) * a.S, r1 = r0 + a.S;
+            const int64_t r0 = (int64_t)jj * a.S, r1 = r0 + a.S;
             for (int i = 0; i < nf; ++i)
                 if (f_lo[i] <= r0 && r1 <= f_hi[i]) key = 0;
         }
-        kr[r] = key;
+        keys[jj] = key;
+        taken[jj] = 0;
+        if (off) visb[jj] = a.vis[(int64_t)s * nb + jj];
         my_c += key != 0;
     }
     int n_cand;
-    cta_excl_sum(my_c, tmp, &n_cand);
+    cta_excl_sum(my_c, tmp, &n_cand);   // also publishes keys[] to the CTA
 
     const bool greedy = off && a.topk < 0;
     int k = 0;
@@ -415,13 +451,6 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
         // when its visible rows fit in what is left; that only shrinks, so a
         // block that does not fit now never will, and each step takes the
         // best remaining candidate that fits), or a small top-k
-#pragma unroll
-        for (int r = 0; r < KPT; ++r)
-            if (c0 + r < nb) {
-                keys[c0 + r] = kr[r];
-                taken[c0 + r] = 0;
-            }
-        __syncthreads();
         if (warp == 0) {
             const int limit = greedy ? a.max_sel : k;
             const int budget = greedy ? a.budget : -1;
@@ -430,12 +459,10 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
         }
         __syncthreads();
         int my_take = 0;
-#pragma unroll
-        for (int r = 0; r < KPT; ++r) my_take += c0 + r < nb && taken[c0 + r];
+        for (int r = 0; r < kpt; ++r) my_take += c0 + r < nb && taken[c0 + r];
         int tot;
         int p = cta_excl_sum(my_take, tmp, &tot);
-#pragma unroll
-        for (int r = 0; r < KPT; ++r)
+        for (int r = 0; r < kpt; ++r)
             if (c0 + r < nb && taken[c0 + r] && p < a.max_sel) sel[p++] = c0 + r;
         if (tid == 0) n_sel_sh = min(tot, a.max_sel);
     } else {
@@ -449,9 +476,9 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
                 const int shift = 24 - 8 * pass;
                 if (tid < 256) hist[tid] = 0;
                 __syncthreads();
-#pragma unroll
-                for (int r = 0; r < KPT; ++r) {
-                    const uint32_t key = kr[r];
+#pragma unroll 4
+                for (int r = 0; r < kpt; ++r) {
+                    const uint32_t key = c0 + r < nb ? keys[c0 + r] : 0u;
                     const bool act = key && (key & pmask) == prefix;
                     const uint32_t bin = act ? (key >> shift) & 255u : 256u;
                     // lanes with the same bin add once (most keys share the
@@ -476,11 +503,12 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
         // index-ordered compaction: key > thr, or key == thr among the first
         // need_eq
         int my_eq = 0, my_gt = 0;
-#pragma unroll
-        for (int r = 0; r < KPT; ++r) {
-            my_eq += k > 0 && kr[r] != 0 && kr[r] == thr;
-            my_gt += k > 0 && kr[r] != 0 && kr[r] > thr;
-        }
+        if (k > 0)
+            for (int r = 0; r < kpt; ++r) {
+                const uint32_t key = c0 + r < nb ? keys[c0 + r] : 0u;
+                my_eq += key != 0 && key == thr;
+                my_gt += key != 0 && key > thr;
+            }
         int tot;
         const int eq_base = cta_excl_sum(my_eq, tmp, &tot);
         const int my_take = my_gt + min(my_eq, max(0, need_eq - eq_base));
@@ -488,9 +516,8 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
         if (tid == 0) n_sel_sh = tot;
         if (my_take > 0) {
             int eq_seen = eq_base;
-#pragma unroll
-            for (int r = 0; r < KPT; ++r) {
-                const uint32_t key = kr[r];
+            for (int r = 0; r < kpt && c0 + r < nb; ++r) {
+                const uint32_t key = keys[c0 + r];
                 if (key != 0 && key > thr) sel[p++] = c0 + r;
                 else if (key != 0 && key == thr && eq_seen++ < need_eq) sel[p++] = c0 + r;
             }
@@ -556,9 +583,6 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
     }
 }
 
-// Largest block count the selection handles (the pick kernel holds up to 32
-// keys per thread in registers).
-constexpr int kSelMaxBlocks = kPickThreads * 32;
 
 bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ, int kind,
                          const bsa_sel_params *p, const int32_t *cur_len, int nb_total,
@@ -586,11 +610,11 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
     a.tile_bytes = (uint32_t)(a.nbox * kSelThreads * 128);
     const size_t qbytes = (size_t)a.G * (d->D + 4) * 4;
     const size_t cap = 227 * 1024 - 1024;
-    a.nst = (int)std::min<size_t>(kSelMaxStages, cap / (a.tile_bytes + qbytes));
+    a.nst = (int)std::min<size_t>(kScoreStages, (cap - qbytes) / (a.tile_bytes + qbytes));
     if (a.nst < 1) return BSA_ERR_UNSUPPORTED;
-    const size_t smem1 = 1024 + (size_t)a.nst * (a.tile_bytes + qbytes);
+    const size_t smem1 = 1024 + (size_t)a.nst * (a.tile_bytes + qbytes) + qbytes;   // + selectors
     const size_t smem2 = PickSmem::bytes(nb_total, max_sel);
-    if (smem2 > cap || nb_total > kSelMaxBlocks) return BSA_ERR_UNSUPPORTED;
+    if (smem2 > cap) return BSA_ERR_UNSUPPORTED;
     a.tiles_per_seg = (int)div_up(nb_total, kSelThreads);
     const int nseg = d->B * d->Hkv;
     a.n_items = nseg * a.tiles_per_seg;
@@ -607,16 +631,21 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
         BSA_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(threads), smem1, st, tm, a));
         return BSA_OK;
     };
-    auto by_g = [&](auto sk) -> bsa_status {
-        constexpr int SK = decltype(sk)::value;
+    auto by_gd = [&](auto sk, auto dt) -> bsa_status {
+        constexpr int SK = decltype(sk)::value, DT = decltype(dt)::value;
         switch (a.G) {
-            case 1: return launch(score_kernel<SK, 1>, score_tpb(1));
-            case 2: return launch(score_kernel<SK, 2>, score_tpb(2));
-            case 4: return launch(score_kernel<SK, 4>, score_tpb(4));
-            case 8: return launch(score_kernel<SK, 8>, score_tpb(8));
-            case 16: return launch(score_kernel<SK, 16>, score_tpb(16));
-            default: return launch(score_kernel<SK, 0>, score_tpb(0));
+            case 1: return launch(score_kernel<SK, 1, DT>, score_tpb(1));
+            case 2: return launch(score_kernel<SK, 2, DT>, score_tpb(2));
+            case 4: return launch(score_kernel<SK, 4, DT>, score_tpb(4));
+            case 8: return launch(score_kernel<SK, 8, DT>, score_tpb(8));
+            case 16: return launch(score_kernel<SK, 16, DT>, score_tpb(16));
+            default: return launch(score_kernel<SK, 0, 0>, score_tpb(0));
         }
+    };
+    auto by_g = [&](auto sk) -> bsa_status {
+        if (d->D == 128) return by_gd(sk, std::integral_constant<int, 128>());
+        if (d->D == 64) return by_gd(sk, std::integral_constant<int, 64>());
+        return by_gd(sk, std::integral_constant<int, 0>());
     };
     bsa_status r;
     if (kind == BSA_SUM_MINMAX)
@@ -630,10 +659,7 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
         BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(kPickThreads), smem2, st, a));
         return BSA_OK;
     };
-    if (nb_total <= kPickThreads) return pick(pick_kernel<1>);
-    if (nb_total <= kPickThreads * 4) return pick(pick_kernel<4>);
-    if (nb_total <= kPickThreads * 16) return pick(pick_kernel<16>);
-    return pick(pick_kernel<32>);
+    return pick(pick_kernel);
 }
 
 }  // namespace bsa

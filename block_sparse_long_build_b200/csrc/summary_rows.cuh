@@ -43,8 +43,8 @@ __device__ __forceinline__ void summarize_centroid(const T *Kseg, int64_t st, in
     }
 }
 
-// Min/max rows of rows [r0, r1) in the cache dtype: thread i < D scans
-// dimension i in row order.
+// Min/max of rows [r0, r1) in the cache dtype, stored as (min, max) pairs
+// per dimension: thread i < D scans dimension i in row order.
 template <typename T>
 __device__ __forceinline__ void summarize_minmax(const T *Kseg, int64_t st, int D, int64_t r0,
                                                  int64_t r1, T *o) {
@@ -59,18 +59,18 @@ __device__ __forceinline__ void summarize_minmax(const T *Kseg, int64_t st, int 
         }
         if (n <= 0) lo = hi = 0.0f;
         if constexpr (sizeof(T) == 2) {
-            o[i] = static_cast<uint16_t>(__float_as_uint(lo) >> 16);
-            o[D + i] = static_cast<uint16_t>(__float_as_uint(hi) >> 16);
+            o[2 * i] = static_cast<uint16_t>(__float_as_uint(lo) >> 16);
+            o[2 * i + 1] = static_cast<uint16_t>(__float_as_uint(hi) >> 16);
         } else {
-            o[i] = lo;
-            o[D + i] = hi;
+            o[2 * i] = lo;
+            o[2 * i + 1] = hi;
         }
     }
 }
 
 // Summary of rows [r0, r1) of one segment, computed by the whole CTA
 // (blockDim.x >= D).  `out` points at this block's summary: D floats for the
-// centroid kinds, 2*D cache elements (min row, then max row) for MINMAX.
+// centroid kinds, D (min, max) pairs of cache elements for MINMAX.
 // `sm` must hold kNormChunk*(D+1) + D + 1 floats.
 template <typename T>
 __device__ void summarize_rows(const T *Kseg, int64_t st, int D, int64_t r0, int64_t r1,

@@ -75,7 +75,7 @@ typedef enum {
 typedef enum {
     BSA_SUM_CENTROID = 0,       /* fp32 mean of the block's keys                  */
     BSA_SUM_CENTROID_NORM = 1,  /* fp32 normalised mean of normalised keys        */
-    BSA_SUM_MINMAX = 2          /* elementwise min then max, in the cache dtype   */
+    BSA_SUM_MINMAX = 2          /* elementwise (min, max) pairs, cache dtype      */
 } bsa_summary_kind;
 
 typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype;
@@ -128,7 +128,9 @@ typedef struct {
 BSA_API int32_t bsa_summary_blocks(const bsa_kv_desc *desc, const bsa_sel_params *sel);
 
 /* Bytes of the summaries buffer: segments x blocks x (D fp32 for the centroid
- * kinds | 2 x D cache elements, min row then max row, for MINMAX). */
+ * kinds | D (min, max) pairs of cache elements for MINMAX: element 2i is the
+ * block's minimum of dimension i, element 2i + 1 its maximum, so that one
+ * byte permute picks and widens the bound a query's sign selects). */
 BSA_API size_t bsa_summary_bytes(const bsa_kv_desc *desc, const bsa_sel_params *sel,
                          bsa_summary_kind kind);
 

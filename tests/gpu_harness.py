@@ -34,11 +34,12 @@ def gpu_summaries(sess: DecodeSession, s: int, nb: int):
         esz = 2 if c.kv_dtype == torch.bfloat16 else 4
         row = 2 * c.D * esz
         seg = raw[s * sess.nb * row:(s * sess.nb + nb) * row]
+        # (min, max) pairs per dimension
         if esz == 2:
-            x = oracle.bf16_bits_to_f32(seg.view(np.uint16)).reshape(nb, 2, c.D)
+            x = oracle.bf16_bits_to_f32(seg.view(np.uint16)).reshape(nb, c.D, 2)
         else:
-            x = seg.view(np.float32).reshape(nb, 2, c.D)
-        return x[:, 0], x[:, 1]
+            x = seg.view(np.float32).reshape(nb, c.D, 2)
+        return x[:, :, 0], x[:, :, 1]
     row = c.D * 4
     return raw[s * sess.nb * row:(s * sess.nb + nb) * row].view(np.float32).reshape(nb, c.D)
 
