@@ -32,12 +32,12 @@ constexpr int kPfMaxBlocks = 256;          // blocks per KV head (bitmap of 8 wo
 constexpr int kPfWords = kPfMaxBlocks / 32;
 constexpr int kPfMaxSel = 64;              // selected blocks kept per (query, KV head)
 constexpr int kPfSlots = kPfMaxSel + 1;    // slot 0 = local part
+constexpr int kPfSlotShift = 24;           // qlist entry: query | slot << 24
 constexpr int kPfSelWarps = 16;            // P1 warps per CTA (8 when shared memory is short)
 constexpr int kPfRowsPerWarp = 8;          // P1 query rows per warp
 constexpr int kPfCentStride = 132;         // padded centre row (floats): 16-byte rows, conflict-free
 constexpr int kTile = 128;                 // rows per MMA tile, keys per key tile
 constexpr size_t kMaxSmemPerCta = 227 * 1024;   // opt-in dynamic shared memory per CTA
-constexpr int kPfThreads = 128;
 constexpr float kPfNegInf = -__builtin_huge_valf();
 constexpr float kPfLn2 = 0.69314718055994530942f;
 
@@ -52,9 +52,8 @@ struct PfArgs {
     uint32_t *bitmap;          // [Tq][Hkv][kPfWords]
     int32_t *vis;              // [Hkv][nb]
     int32_t *qcount;           // [Hkv][nb]          (zeroed per call)
-    int32_t *qlist;            // [Hkv][nb][Tq]
+    int32_t *qlist;            // [Hkv][nb][Tq]       query | slot << kPfSlotShift
     int32_t *tile_prefix;      // [Hkv * nb + 1]
-    int32_t *work;             // [1]                (zeroed per call)
     float *part_o;             // [Tq][Hkv][kPfSlots][G][D]
     float2 *part_ml;           // [Tq][Hkv][kPfSlots][G]
     uint32_t *status;
@@ -169,10 +168,6 @@ __global__ void __launch_bounds__(32 * kPfSelWarps) prefill_select_kernel(PfArgs
             remaining -= visS[j];
             ++nsel;
             if (lane == (j & 31)) selbits |= 1u << (j >> 5);
-            if (lane == 0) {
-                const int p = atomicAdd(&a.qcount[g * nb + j], 1);
-                a.qlist[((int64_t)g * nb + j) * a.Tq + p] = i;
-            }
 #pragma unroll
             for (int t = 0; t < kPfWords; ++t) {
                 const int jj = lane + 32 * t;
@@ -181,10 +176,24 @@ __global__ void __launch_bounds__(32 * kPfSelWarps) prefill_select_kernel(PfArgs
         }
         if (nsel >= kPfMaxSel && lane == 0) atomicOr(a.status, 4u);
         uint32_t *bm = a.bitmap + ((int64_t)i * a.Hkv + g) * kPfWords;
+        uint32_t words[kPfWords];
 #pragma unroll
         for (int t = 0; t < kPfWords; ++t) {
-            const uint32_t word = __ballot_sync(0xffffffffu, (selbits >> t) & 1u);
-            if (lane == 0) bm[t] = word;
+            words[t] = __ballot_sync(0xffffffffu, (selbits >> t) & 1u);
+            if (lane == 0) bm[t] = words[t];
+        }
+        // the query joins each selected block's list with its partial slot:
+        // 1 + the block's rank among the selected blocks in index order
+        int below = 0;
+#pragma unroll
+        for (int t = 0; t < kPfWords; ++t) {
+            if ((selbits >> t) & 1u) {
+                const int j = lane + 32 * t;
+                const int slot = 1 + below + __popc(words[t] & ((1u << lane) - 1u));
+                const int p = atomicAdd(&a.qcount[g * nb + j], 1);
+                a.qlist[((int64_t)g * nb + j) * a.Tq + p] = i | (slot << kPfSlotShift);
+            }
+            below += __popc(words[t]);
         }
         __syncwarp();
     }
@@ -207,36 +216,52 @@ __global__ void __launch_bounds__(1024) prefill_tiles_kernel(PfArgs a) {
 }
 
 // ---------------------------------------------------------------- P3
-// Warp-specialised: warps 0..7 run the softmax, two threads per row (warp w
-// owns TMEM lanes 32*(w%4).. and the column half w/4); lane 0 of warp 8
-// issues every TMA load and every tcgen05.mma.  S is double-buffered in TMEM
-// so that S(t+1) = Q K(t+1)^T runs on the tensor cores while the softmax of
-// tile t runs; P.V of tile t follows the softmax.  O is rescaled only when a
-// row's running maximum grows by more than 2^8 (the exponentials then stay
-// below 256), so P.V rarely sits on the softmax's critical path.
-constexpr int kPfSoftWarps = 8;
-constexpr int kPfAttThreads = 32 * (kPfSoftWarps + 1);
+// Warp-specialised and pipelined across work items:
+//   warps 0-15  softmax + epilogue, four threads per row (warp w owns TMEM
+//               lanes 32 (w % 4).. and the column quarter w / 4)
+//   warp 16     lane 0 issues every tcgen05.mma
+//   warp 17     lane 0 streams the K tiles, lane 1 the V tiles by TMA (no
+//               multicast); the two lanes wait on different barriers
+//   warps 18-19 describe work items, gather their Q rows into one of two Q
+//               buffers and publish the item (rows, positions, records)
+// S is double-buffered in TMEM by a running tile counter u that crosses
+// items, O and the Q buffer by item parity, the item descriptions four deep.
+// A Q buffer is refilled as soon as its item's last S = QK^T is done, an O
+// buffer once its item's epilogue has read it, so the producers run up to
+// two items ahead and each epilogue overlaps the next item.  O is rescaled only
+// when a row's running maximum grows by more than 2^8 (the exponentials then
+// stay below 256).
+//
+// Barriers and their phases (every waiter derives the parity from an index):
+//   qready[m] item n (m = n & 3) described, Q gathered (32) parity (n >> 2) & 1
+//   qfree[b]  item n's last S complete (b = n & 1)          parity (n >> 1) & 1
+//   efree[b]  item n's epilogue done, 16 softmax warps      parity (n >> 1) & 1
+//   kfull/vfull[s] tile u (s = u & 1), TMA bytes           parity (u >> 1) & 1
+//   kfree/vfree[s] S(u) / P.V(u) complete (tcgen05.commit) parity (u >> 1) & 1
+//   sfull[s]  S(u) complete; pfull[s] P(u) in TMEM (16 warps); odone[s] P.V(u)
+constexpr int kPfSoftWarps = 16;
+constexpr int kPfMmaWarp = 16, kPfLoadWarp = 17, kPfProdWarp = 18;
+constexpr int kPfAttThreads = 32 * 20;
 constexpr float kPfRescale = 8.0f;   // log2 of the largest exponential kept without rescaling
+constexpr int kPfPrefixCap = 4097;   // tile prefix entries staged in shared memory
 
 struct PfSmem {
-    static constexpr int kQ = 0;                          // 2 boxes x 16 KiB
-    static constexpr int kK = 32768;                      // 2 stages x 32 KiB
-    static constexpr int kV = kK + 2 * 32768;             // 2 stages x 32 KiB
-    static constexpr int kRowQ = kV + 2 * 32768;          // int [128] query index
-    static constexpr int kRowPos = kRowQ + kTile * 4;     // int [128] query position
-    static constexpr int kPair = kRowPos + kTile * 4;     // float [2][128] half-row maxima / sums
-    static constexpr int kBars = kPair + 2 * kTile * 4;   // u64: kfull[2] vfull[2] sfull[2] pfull[2] odone[2]
-    static constexpr int kMisc = kBars + 10 * 8;          // int item, tmem base
-    static constexpr int kBytes = kMisc + 16 + 1024;
+    static constexpr int kQ = 0;                          // 2 items x 2 boxes x 16 KiB
+    static constexpr int kK = 65536;                      // 2 stages x 32 KiB
+    static constexpr int kV = kK + 65536;                 // 2 stages x 32 KiB
+    static constexpr int kRowPos = kV + 65536;            // int [4][128] query position
+    static constexpr int kRowQ = kRowPos + 4 * kTile * 4; // int [4][128] row of Q (-1: none)
+    static constexpr int kRowRec = kRowQ + 4 * kTile * 4; // int [4][128] partial record (-1: none)
+    static constexpr int kDesc = kRowRec + 4 * kTile * 4; // int [4][8]: g, kbeg, kend, T, local, end
+    static constexpr int kPair = kDesc + 4 * 8 * 4;       // float [4][128] quarter-row maxima / sums
+    static constexpr int kBars = kPair + 4 * kTile * 4;   // u64 [23]
+    static constexpr int kMisc = kBars + 23 * 8;          // tmem base
+    static constexpr int kPrefix = kMisc + 32;            // int [kPfPrefixCap]
+    static constexpr int kBytes = kPrefix + kPfPrefixCap * 4 + 1024;
 };
 
-struct PfItem {
-    int g, kbeg, kend, jblk, mtile, ntiles;
-    bool local;
-};
-
-__device__ __forceinline__ void pair_sync(int q) {   // the two warps holding rows 32q..32q+31
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+__device__ __forceinline__ void quad_sync(int q) {   // the four warps holding rows 32q..32q+31
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + q) : "memory");
 }
 
 __global__ void __launch_bounds__(kPfAttThreads, 1)
@@ -246,14 +271,17 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
     extern __shared__ unsigned char praw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(praw) + 1023) & ~uintptr_t(1023));
-    unsigned char *Qs = sm + PfSmem::kQ;
-    int *rowq = reinterpret_cast<int *>(sm + PfSmem::kRowQ);
-    int *rowpos = reinterpret_cast<int *>(sm + PfSmem::kRowPos);
+    int *rowpos_s = reinterpret_cast<int *>(sm + PfSmem::kRowPos);
+    int *rowq_s = reinterpret_cast<int *>(sm + PfSmem::kRowQ);
+    int *rowrec_s = reinterpret_cast<int *>(sm + PfSmem::kRowRec);
+    int *desc_s = reinterpret_cast<int *>(sm + PfSmem::kDesc);
     float *pairv = reinterpret_cast<float *>(sm + PfSmem::kPair);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PfSmem::kBars);
-    uint64_t *kfull = bars, *vfull = bars + 2, *sfull = bars + 4, *pfull = bars + 6, *odone = bars + 8;   // odone[2]
-    int *item_sh = reinterpret_cast<int *>(sm + PfSmem::kMisc);
-    uint32_t *tmem_sh = reinterpret_cast<uint32_t *>(sm + PfSmem::kMisc + 4);
+    uint64_t *qready = bars, *qfree = bars + 4, *efree = bars + 6, *kfull = bars + 8, *vfull = bars + 10,
+             *kfree = bars + 12, *vfree = bars + 14, *sfull = bars + 16, *pfull = bars + 18, *odone = bars + 20,
+             *drain = bars + 22;
+    uint32_t *tmem_sh = reinterpret_cast<uint32_t *>(sm + PfSmem::kMisc);
+    int *prefix_s = reinterpret_cast<int *>(sm + PfSmem::kPrefix);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = a.G, D = a.D;
@@ -264,192 +292,325 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
     }
     if (tid == 0) {
         prefetch_tmap(&tmKp); prefetch_tmap(&tmVp); prefetch_tmap(&tmKl); prefetch_tmap(&tmVl);
-        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
-        mbar_init(&pfull[0], kPfSoftWarps);
-        mbar_init(&pfull[1], kPfSoftWarps);
-        mbar_init(&odone[0], 1);
-        mbar_init(&odone[1], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&qready[i], 32);   // one producer warp per item
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&qfree[i], 1);
+            mbar_init(&efree[i], kPfSoftWarps);
+            mbar_init(&kfull[i], 1);
+            mbar_init(&vfull[i], 1);
+            mbar_init(&kfree[i], 1);
+            mbar_init(&vfree[i], 1);
+            mbar_init(&sfull[i], 1);
+            mbar_init(&pfull[i], kPfSoftWarps);
+            mbar_init(&odone[i], 1);
+        }
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     pdl_wait();
+    const int n_pref = a.Hkv * a.nb + 1;
+    const bool prefix_in_smem = n_pref <= kPfPrefixCap;
+    if (prefix_in_smem)
+        for (int e = tid; e < n_pref; e += kPfAttThreads) prefix_s[e] = a.tile_prefix[e];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_sh;
-    const uint32_t tO = tmem + 256;                 // S0 = cols 0..127, S1 = 128..255, O = 256..383
-    const int n_group = a.tile_prefix[a.Hkv * a.nb];
+    const uint32_t tmem = *tmem_sh;   // S0 = cols 0..127, S1 = 128..255, O0 = 256.., O1 = 384..
+    const int *prefix = prefix_in_smem ? prefix_s : a.tile_prefix;
+    const int n_group = prefix[a.Hkv * a.nb];
     const int n_items = a.n_local + n_group;
     const int qpt = kTile / G;
     const int tiles_per_head = (a.Tq + qpt - 1) / qpt;
-    constexpr uint32_t kIdescQK = umma_idesc_bf16(128, 128, 0, 0);
-    constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 128, 0, 1);
-    // phase counters (every role tracks the barriers it waits on)
-    uint32_t kuse[2] = {0, 0}, vuse[2] = {0, 0}, puse[2] = {0, 0};   // issuing lane only
-    uint32_t sbase[2] = {0, 0}, obase[2] = {0, 0};                       // every thread
     bool timed_out = false;
+    auto wait = [&](uint64_t *bar, uint32_t parity) {
+        if (!timed_out && !mbar_wait_bounded(bar, parity)) timed_out = true;
+    };
 
-    for (;;) {
-        if (tid == 0) *item_sh = atomicAdd(a.work, 1);
-        __syncthreads();
-        const int item = *item_sh;
-        if (item >= n_items) break;
-        // ---- decode the work item (every thread, same result)
-        PfItem it;
-        it.local = item < a.n_local;
-        it.jblk = -1;
-        if (it.local) {
-            it.g = item / tiles_per_head;
-            const int i0 = (item % tiles_per_head) * qpt;
-            it.mtile = i0;
-            it.kbeg = a.pos_limit;
-            it.kend = a.q_pos0 + min(a.Tq, i0 + qpt);
-        } else {
-            const int u = item - a.n_local;
-            int lo = 0, hi = a.Hkv * a.nb - 1;   // largest e with prefix[e] <= u
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (a.tile_prefix[mid] <= u) lo = mid; else hi = mid - 1;
+    if (warp >= kPfProdWarp) {
+        // ================= producers.  The CTA's n-th item is blockIdx.x +
+        // n gridDim.x; warp kPfProdWarp + p takes the items with n = p (mod 2),
+        // i.e. Q buffer p.  A warp describes its next item (rows, positions,
+        // records: two rounds of dependent loads) as soon as it has published
+        // the current one, so only the Q copies sit between a free buffer and
+        // the next item.
+        const int pt = lane;
+        // item n's description into slot n & 3; false for the end marker
+        auto describe = [&](int n) -> bool {
+            const int m = n & 3;
+            const int item = (int)blockIdx.x + n * (int)gridDim.x;
+            int *desc = desc_s + m * 8;
+            if (item >= n_items) {
+                if (pt == 0) desc[5] = 1;
+                __syncwarp();
+                return false;
             }
-            it.g = lo / a.nb;
-            it.jblk = lo % a.nb;
-            it.mtile = u - a.tile_prefix[lo];
-            it.kbeg = min(max(a.offsets[(int64_t)it.g * (a.nb + 1) + it.jblk], 0), a.L_max);
-            it.kend = it.kbeg + a.vis[it.g * a.nb + it.jblk];
-        }
-        it.ntiles = max(0, (it.kend - it.kbeg + kTile - 1) / kTile);
-        const int g = it.g;
-        if (tid < kTile) {
-            const int r = tid;
-            if (it.local) {
-                const int i = it.mtile + r / G;
-                rowq[r] = i < a.Tq ? i : -1;
-                rowpos[r] = a.q_pos0 + i;
+            int g, kbeg, kend, mtile, jblk = -1;
+            const bool local = item < a.n_local;
+            if (local) {
+                g = item / tiles_per_head;
+                mtile = (item % tiles_per_head) * qpt;   // first query
+                kbeg = a.pos_limit;
+                kend = a.q_pos0 + min(a.Tq, mtile + qpt);
             } else {
-                const int cnt = a.qcount[g * a.nb + it.jblk];
-                const int idx = it.mtile * kTile + r, qi = idx / G;
-                rowq[r] = qi < cnt ? a.qlist[((int64_t)g * a.nb + it.jblk) * a.Tq + qi] : -1;
-                rowpos[r] = 0x7fffffff;   // every key of a visible prefix is earlier
+                const int u = item - a.n_local;
+                int lo = 0, hi = a.Hkv * a.nb - 1;   // largest e with prefix[e] <= u
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (prefix[mid] <= u) lo = mid; else hi = mid - 1;
+                }
+                g = lo / a.nb;
+                jblk = lo % a.nb;
+                mtile = u - prefix[lo];
+                kbeg = min(max(a.offsets[(int64_t)g * (a.nb + 1) + jblk], 0), a.L_max);
+                kend = kbeg + a.vis[g * a.nb + jblk];
             }
-        }
-        __syncthreads();
-        // ---- gather Q rows (bf16) into the swizzled K-major layout
-        for (int c = tid; c < kTile * 16; c += kPfAttThreads) {
-            const int r = c >> 4, ch = c & 15, half = ch >> 3, cc = ch & 7;
-            const int qi = rowq[r];
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (qi >= 0) {
-                const int hh = r % G;
-                v = *reinterpret_cast<const uint4 *>(
-                    a.Q + ((int64_t)qi * a.Hq + (int64_t)g * G + hh) * D + ch * 8);
+            if (pt == 0) {
+                // every item has at least one key tile (a wholly masked one
+                // gives o = 0, l = 0), so each role sees the same tiles and
+                // the barrier phases stay in step
+                kend = max(kend, kbeg);
+                desc[0] = g; desc[1] = kbeg; desc[2] = kend;
+                desc[3] = max(1, (kend - kbeg + kTile - 1) / kTile);
+                desc[4] = local; desc[5] = 0;
             }
-            *reinterpret_cast<uint4 *>(Qs + half * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+            const int cnt = local ? 0 : a.qcount[g * a.nb + jblk];
+            for (int r = pt; r < kTile; r += 32) {
+                int qi = -1, rec = -1, pos;
+                if (local) {
+                    const int i = mtile + r / G;
+                    pos = a.q_pos0 + i;
+                    if (i < a.Tq) { qi = i; rec = ((i * a.Hkv + g) * kPfSlots) * G + (r % G); }
+                } else {
+                    pos = 0x7fffffff;   // every key of a visible prefix is earlier
+                    const int idx = (mtile * kTile + r) / G;
+                    if (idx < cnt) {
+                        const int e = a.qlist[((int64_t)g * a.nb + jblk) * a.Tq + idx];
+                        qi = e & ((1 << kPfSlotShift) - 1);
+                        const int slot = e >> kPfSlotShift;
+                        rec = ((qi * a.Hkv + g) * kPfSlots + slot) * G + (r % G);
+                    }
+                }
+                rowpos_s[m * kTile + r] = pos;
+                rowq_s[m * kTile + r] = qi >= 0 ? qi * a.Hq + g * G + (r % G) : -1;   // row of Q
+                rowrec_s[m * kTile + r] = rec;
+            }
+            __syncwarp();
+            return true;
+        };
+        // item n's Q rows (bf16) into buffer n & 1, swizzled K-major, with
+        // asynchronous 16-byte copies (a row with no query is zero-filled)
+        auto gather = [&](int n) {
+            const int m = n & 3;
+            unsigned char *Qs = sm + PfSmem::kQ + (n & 1) * 32768;
+#pragma unroll 4
+            for (int c = pt; c < kTile * 16; c += 32) {
+                const int r = c >> 4, ch = c & 15, half = ch >> 3, cc = ch & 7;
+                const int row = rowq_s[m * kTile + r];
+                const uint16_t *src = row >= 0 ? a.Q + (int64_t)row * D + ch * 8 : a.Q;
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                                 smem_u32(Qs + half * 16384 + r * 128 + ((cc ^ (r & 7)) << 4))),
+                             "l"(src), "r"(row >= 0 ? 16 : 0)
+                             : "memory");
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+        int n = warp - kPfProdWarp;
+        bool valid = describe(n);
+        for (;;) {
+            const int b = n & 1, m = n & 3;
+            if (!valid) {   // end marker: nothing to gather
+                mbar_arrive(&qready[m]);
+                break;
+            }
+            if (n >= 2) wait(&qfree[b], ((n - 2) >> 1) & 1);   // item n-2's Q buffer is free
+            if (timed_out) break;
+            gather(n);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            fence_proxy_async_smem();
+            __syncwarp();
+            mbar_arrive(&qready[m]);
+            // the next item's rows go to slot (n + 2) & 3 once item n-2's
+            // epilogue has read them; its dependent loads then overlap the
+            // consumption of items n-1 and n
+            if (n >= 2) wait(&efree[b], ((n - 2) >> 1) & 1);
+            valid = describe(n + 2);
+            n += 2;
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        const int T = it.ntiles;
-
-        // Barrier protocol.  kfull/vfull/pfull are waited by the issuing lane
-        // for every phase (plain counters).  S(t) completes on sfull[t&1] and
-        // P.V(t) on odone[t&1]; a wait for one of them is for a specific MMA
-        // whose predecessor on the same barrier is already known complete, so
-        // the parity follows from the MMA's index: base[b] (MMAs on barrier b
-        // in earlier items) + t/2.
-        auto par = [](uint32_t base, int t) { return (base + (uint32_t)(t >> 1)) & 1u; };
-        if (warp == kPfSoftWarps) {
-            // ================= TMA + MMA issue (one lane)
-            if (lane == 0) {
-                const CUtensorMap *mk = it.local ? &tmKl : &tmKp;
-                const CUtensorMap *mv = it.local ? &tmVl : &tmVp;
-                auto load_k = [&](int t) {
-                    unsigned char *dst = sm + PfSmem::kK + (t & 1) * 32768;
-                    mbar_arrive_expect_tx(&kfull[t & 1], 32768);
-                    tma_load_4d(dst, mk, &kfull[t & 1], 0, it.kbeg + t * kTile, g, 0);
-                    tma_load_4d(dst + 16384, mk, &kfull[t & 1], 64, it.kbeg + t * kTile, g, 0);
-                };
-                auto load_v = [&](int t) {
-                    unsigned char *dst = sm + PfSmem::kV + (t & 1) * 32768;
-                    mbar_arrive_expect_tx(&vfull[t & 1], 32768);
-                    tma_load_4d(dst, mv, &vfull[t & 1], 0, it.kbeg + t * kTile, g, 0);
-                    tma_load_4d(dst + 16384, mv, &vfull[t & 1], 64, it.kbeg + t * kTile, g, 0);
-                };
-                auto pv = [&](int t) {   // O (+)= P(t) V(t), P read from S(t & 1)
-                    if (!timed_out && !mbar_wait_bounded(&pfull[t & 1], puse[t & 1] & 1)) timed_out = true;
-                    ++puse[t & 1];
-                    if (!timed_out && !mbar_wait_bounded(&vfull[t & 1], vuse[t & 1] & 1)) timed_out = true;
-                    ++vuse[t & 1];
-                    tc_fence_after();
-                    const uint32_t v0 = smem_u32(sm + PfSmem::kV + (t & 1) * 32768);
-                    const uint32_t tP = tmem + (t & 1) * 128;
+        asm volatile("cp.async.wait_all;" ::: "memory");   // nothing in flight at exit
+    } else if (warp == kPfLoadWarp) {
+        // ================= K loader (lane 0) and V loader (lane 1)
+        if (lane < 2) {
+            const bool isk = lane == 0;
+            uint64_t *full = isk ? kfull : vfull, *freeb = isk ? kfree : vfree;
+            unsigned char *base = sm + (isk ? PfSmem::kK : PfSmem::kV);
+            int u = 0;
+            for (int n = 0;; ++n) {
+                const int m = n & 3;
+                wait(&qready[m], (n >> 2) & 1);
+                const int *desc = desc_s + m * 8;
+                if (timed_out || desc[5]) break;
+                const int g = desc[0], kbeg = desc[1], T = desc[3];
+                const CUtensorMap *map = desc[4] ? (isk ? &tmKl : &tmVl) : (isk ? &tmKp : &tmVp);
+                for (int t = 0; t < T; ++t, ++u) {
+                    const int st = u & 1;
+                    if (u >= 2) wait(&freeb[st], ((u - 2) >> 1) & 1);
+                    unsigned char *dst = base + st * 32768;
+                    mbar_arrive_expect_tx(&full[st], 32768);
+                    tma_load_4d(dst, map, &full[st], 0, kbeg + t * kTile, g, 0);
+                    tma_load_4d(dst + 16384, map, &full[st], 64, kbeg + t * kTile, g, 0);
+                }
+            }
+            // the last loads of each stage have landed before the CTA can exit
+            const bool to = timed_out;
+            timed_out = false;
+            for (int v = max(0, u - 2); v < u; ++v) wait(&full[v & 1], (v >> 1) & 1);
+            timed_out = timed_out || to;
+        }
+        __syncwarp();
+    } else if (warp == kPfMmaWarp) {
+        // ================= tcgen05.mma issue (one lane)
+        if (lane == 0) {
+            constexpr uint32_t kIdescQK = umma_idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 128, 0, 1);
+            int pend_u = -1, pend_n = 0;
+            bool pend_first = false;
+            auto pv = [&](int v, int pn, bool first) {   // O[pn & 1] (+)= P(v) V(v)
+                const int st = v & 1, b = pn & 1;
+                if (first && pn >= 2) wait(&efree[b], ((pn - 2) >> 1) & 1);   // O[b] read out
+                wait(&pfull[st], (v >> 1) & 1);
+                wait(&vfull[st], (v >> 1) & 1);
+                tc_fence_after();
+                const uint32_t v0 = smem_u32(sm + PfSmem::kV + st * 32768);
+                const uint32_t tP = tmem + st * 128, tO = tmem + 256 + b * 128;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint64_t vd = umma_sdesc_sw128(v0 + k * 2048, 16384, 1024);
-                        umma_ts(tO, tP + k * 8, vd, kIdescPV, (t > 0 || k > 0) ? 1u : 0u);
-                        umma_ts(tO, tP + 64 + k * 8, vd, kIdescPV, 1u);
-                    }
-                    umma_commit(&odone[t & 1]);
-                };
-                for (int t = 0; t < 2 && t < T; ++t) { load_k(t); load_v(t); }
-                for (int t = 0; t < T; ++t) {
-                    if (!timed_out && !mbar_wait_bounded(&kfull[t & 1], kuse[t & 1] & 1)) timed_out = true;
-                    ++kuse[t & 1];
-                    if (t >= 2) {   // S(t&1) and V stage t&1 are free once P.V(t-2) is done
-                        if (!timed_out && !mbar_wait_bounded(&odone[t & 1], par(obase[t & 1], t - 2))) timed_out = true;
-                        load_v(t);
-                    }
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t vd = umma_sdesc_sw128(v0 + k * 2048, 16384, 1024);
+                    umma_ts(tO, tP + k * 8, vd, kIdescPV, (!first || k > 0) ? 1u : 0u);
+                    umma_ts(tO, tP + 64 + k * 8, vd, kIdescPV, 1u);
+                }
+                umma_commit(&odone[st]);
+                umma_commit(&vfree[st]);
+            };
+            int u = 0;
+            for (int n = 0;; ++n) {
+                const int b = n & 1, m = n & 3;
+                wait(&qready[m], (n >> 2) & 1);
+                const int *desc = desc_s + m * 8;
+                if (timed_out || desc[5]) break;
+                const int T = desc[3];
+                const uint32_t q0 = smem_u32(sm + PfSmem::kQ + b * 32768);
+                for (int t = 0; t < T; ++t, ++u) {
+                    const int st = u & 1;
+                    wait(&kfull[st], (u >> 1) & 1);
+                    if (u >= 2) wait(&odone[st], ((u - 2) >> 1) & 1);   // P(u-2) consumed: S[st] free
                     tc_fence_after();
-                    const uint32_t q0 = smem_u32(Qs);
-                    const uint32_t k0 = smem_u32(sm + PfSmem::kK + (t & 1) * 32768);
-                    const uint32_t tS = tmem + (t & 1) * 128;
+                    const uint32_t k0 = smem_u32(sm + PfSmem::kK + st * 32768);
+                    const uint32_t tS = tmem + st * 128;
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                        umma_ss(tS, umma_sdesc_sw128(q0 + off, 16, 1024),
-                                umma_sdesc_sw128(k0 + off, 16, 1024), kIdescQK, k > 0);
+                        umma_ss(tS, umma_sdesc_sw128(q0 + off, 16, 1024), umma_sdesc_sw128(k0 + off, 16, 1024),
+                                kIdescQK, k > 0);
                     }
-                    umma_commit(&sfull[t & 1]);
-                    if (t + 2 < T) {   // K stage t&1 is free once S(t) is done
-                        if (!timed_out && !mbar_wait_bounded(&sfull[t & 1], par(sbase[t & 1], t))) timed_out = true;
-                        load_k(t + 2);
-                    }
-                    if (t >= 1) pv(t - 1);
+                    umma_commit(&sfull[st]);
+                    umma_commit(&kfree[st]);
+                    if (t == T - 1) umma_commit(&qfree[b]);   // the item's Q buffer is read
+                    if (pend_u >= 0) pv(pend_u, pend_n, pend_first);
+                    pend_u = u;
+                    pend_n = n;
+                    pend_first = t == 0;
                 }
-                if (T >= 1) pv(T - 1);
             }
-            __syncwarp();
-        } else {
-            // ================= softmax warps
-            const int q = warp & 3, half = warp >> 2;
-            const int r = q * 32 + lane;                 // this thread's row
-            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-            const int my_pos = rowpos[r];
-            float m_used = kPfNegInf, l_part = 0.0f;
-            for (int t = 0; t < T; ++t) {
-                if (!timed_out && !mbar_wait_bounded(&sfull[t & 1], par(sbase[t & 1], t))) timed_out = true;
-                tc_fence_after();
-                const uint32_t tS = tmem + (t & 1) * 128;
-                uint32_t sv[2][32];
-                tmem_ld32(tS + lane_base + half * 64, sv[0]);
-                tmem_ld32(tS + lane_base + half * 64 + 32, sv[1]);
-                tmem_ld_wait();
-                const int key0 = it.kbeg + t * kTile + half * 64;
-                float mx = kPfNegInf;
+            if (pend_u >= 0) pv(pend_u, pend_n, pend_first);
+            // every issued MMA has completed before the CTA frees its TMEM
+            const bool to = timed_out;
+            umma_commit(drain);
+            timed_out = false;
+            wait(drain, 0);
+            timed_out = timed_out || to;
+        }
+        __syncwarp();
+    } else {
+        // ================= softmax warps
+        const int q = warp & 3, cq = warp >> 2;      // row quarter (TMEM lanes), key quarter
+        const int r = q * 32 + lane;                 // this thread's row
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        // An item's epilogue (its last P.V, then its partial) runs after the
+        // softmax of the next item's first tile, so that the tensor cores
+        // work on that tile meanwhile.
+        bool pend = false;
+        int pend_n = 0, pend_u = 0;
+        float pend_m = 0.0f, pend_l = 0.0f;
+        auto epilogue = [&]() {
+            const int pend_b = pend_n & 1, pend_m4 = pend_n & 3;
+            wait(&odone[pend_u & 1], (pend_u >> 1) & 1);
+            tc_fence_after();
+            pairv[cq * kTile + r] = pend_l;
+            quad_sync(q);
+            const float l_row = (pairv[r] + pairv[kTile + r]) + (pairv[2 * kTile + r] + pairv[3 * kTile + r]);
+            quad_sync(q);
+            const int rec = rowrec_s[pend_m4 * kTile + r];
+            float *po = rec >= 0 ? a.part_o + (int64_t)rec * D + cq * 32 : nullptr;
+            uint32_t ov[32];
+            tmem_ld32(tmem + 256 + pend_b * 128 + lane_base + cq * 32, ov);
+            tmem_ld_wait();
+            if (po) {
 #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2)
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(po + e) =
+                        make_float4(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1]),
+                                    __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
+            }
+            if (rec >= 0 && cq == 0) a.part_ml[rec] = make_float2(pend_m, l_row);
+            // O[pend_b] and the item's shared-memory rows may be reused
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&efree[pend_b]);
+            pend = false;
+        };
+        int u = 0;
+        for (int n = 0;; ++n) {
+            const int b = n & 1, m = n & 3;
+            wait(&qready[m], (n >> 2) & 1);
+            const int *desc = desc_s + m * 8;
+            if (timed_out || desc[5]) break;
+            const int kbeg = desc[1], kend = desc[2], T = desc[3];
+            const int my_pos = rowpos_s[m * kTile + r];
+            const uint32_t tO = tmem + 256 + b * 128;
+            float m_used = kPfNegInf, l_part = 0.0f;
+            for (int t = 0; t < T; ++t, ++u) {
+                const int st = u & 1;
+                wait(&sfull[st], (u >> 1) & 1);
+                tc_fence_after();
+                const uint32_t tS = tmem + st * 128;
+                uint32_t sv[32];
+                tmem_ld32(tS + lane_base + cq * 32, sv);
+                tmem_ld_wait();
+                const int key0 = kbeg + t * kTile + cq * 32;
+                float mx = kPfNegInf;
+                if (key0 + 31 < kend && key0 + 31 <= my_pos) {   // every key of the quarter visible
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const int kr = key0 + c2 * 32 + e;
-                        const bool ok = kr < it.kend && kr <= my_pos;
-                        const float v = ok ? __uint_as_float(sv[c2][e]) * a.scale_log2 : kPfNegInf;
-                        sv[c2][e] = __float_as_uint(v);
+                        const float v = __uint_as_float(sv[e]) * a.scale_log2;
+                        sv[e] = __float_as_uint(v);
                         mx = fmaxf(mx, v);
                     }
-                // both halves of the row have read S(t) before either writes P
-                pairv[half * kTile + r] = mx;
-                pair_sync(q);
-                const float m_tile = fmaxf(pairv[r], pairv[kTile + r]);
-                pair_sync(q);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int kr = key0 + e;
+                        const bool ok = kr < kend && kr <= my_pos;
+                        const float v = ok ? __uint_as_float(sv[e]) * a.scale_log2 : kPfNegInf;
+                        sv[e] = __float_as_uint(v);
+                        mx = fmaxf(mx, v);
+                    }
+                }
+                // all quarters of the row have read S(u) before any writes P
+                pairv[cq * kTile + r] = mx;
+                quad_sync(q);
+                const float m_tile = fmaxf(fmaxf(pairv[r], pairv[kTile + r]),
+                                           fmaxf(pairv[2 * kTile + r], pairv[3 * kTile + r]));
+                quad_sync(q);
                 // lazy rescale: keep the reference maximum unless this tile
                 // exceeds it by more than 2^8
                 bool rescale = false;
@@ -464,97 +625,52 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                     }
                 }
                 if (t > 0 && __any_sync(0xffffffffu, rescale)) {
-                    // O must hold P.V(t-1) before it is scaled
-                    if (!timed_out && !mbar_wait_bounded(&odone[(t - 1) & 1], par(obase[(t - 1) & 1], t - 1)))
-                        timed_out = true;
+                    // O must hold P.V(u-1) before it is scaled
+                    wait(&odone[(u - 1) & 1], ((u - 1) >> 1) & 1);
                     tc_fence_after();
+                    uint32_t ov[32];
+                    tmem_ld32(tO + lane_base + cq * 32, ov);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int c2 = 0; c2 < 2; ++c2) {
-                        uint32_t ov[32];
-                        tmem_ld32(tO + lane_base + half * 64 + c2 * 32, ov);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
-                        tmem_st32(tO + lane_base + half * 64 + c2 * 32, ov);
-                    }
+                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+                    tmem_st32(tO + lane_base + cq * 32, ov);
                 }
                 l_part *= factor;
                 m_used = m_ref;
-                // P = P_hi + P_lo (bf16) over this half's 64 keys: P_hi in the
-                // tile's S columns 32*half.., P_lo in 64 + 32*half..
+                // P = P_hi + P_lo over this quarter's 32 keys: P_hi in the
+                // tile's S columns 16 cq.., P_lo in 64 + 16 cq..  P_hi is p cut
+                // to bf16 (its top 16 bits), P_lo = p - P_hi (exact in fp32) cut
+                // the same way, so P_hi + P_lo matches p to 2^-15 relative;
+                // the pairs are packed with byte permutes.
                 float lsum = 0.0f;
+                uint32_t ph[16], pl[16];
 #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    uint32_t ph[16], pl[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float p0 = m_used == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[c2][e]) - m_used);
-                        const float p1 = m_used == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[c2][e + 1]) - m_used);
-                        lsum += p0 + p1;
-                        const float h0 = bf16_round(p0), h1 = bf16_round(p1);
-                        ph[e / 2] = pack_bf16x2(h0, h1);
-                        pl[e / 2] = pack_bf16x2(p0 - h0, p1 - h1);
-                    }
-                    tmem_st16(tS + lane_base + half * 32 + c2 * 16, ph);
-                    tmem_st16(tS + lane_base + 64 + half * 32 + c2 * 16, pl);
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = m_used == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[e]) - m_used);
+                    const float p1 = m_used == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[e + 1]) - m_used);
+                    lsum += p0 + p1;
+                    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                    const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);
+                    const float r1 = p1 - __uint_as_float(b1 & 0xffff0000u);
+                    ph[e / 2] = __byte_perm(b0, b1, 0x7632);
+                    pl[e / 2] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
                 }
+                tmem_st16(tS + lane_base + cq * 16, ph);
+                tmem_st16(tS + lane_base + 64 + cq * 16, pl);
                 l_part += lsum;
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&pfull[t & 1]);
+                if (lane == 0) mbar_arrive(&pfull[st]);
+                if (t == 0 && pend) epilogue();   // the previous item's
             }
-            // ---- epilogue: wait for the last two P.V, then this item's partial
-            if (T >= 1 && !timed_out && !mbar_wait_bounded(&odone[(T - 1) & 1], par(obase[(T - 1) & 1], T - 1)))
-                timed_out = true;
-            if (T >= 2 && !timed_out && !mbar_wait_bounded(&odone[(T - 2) & 1], par(obase[(T - 2) & 1], T - 2)))
-                timed_out = true;
-            tc_fence_after();
-            pairv[half * kTile + r] = l_part;
-            pair_sync(q);
-            const float l_row = pairv[r] + pairv[kTile + r];
-            pair_sync(q);
-            const int qi = rowq[r];
-            int64_t rec = -1;
-            if (qi >= 0) {
-                int slot = 0;
-                if (!it.local) {
-                    const uint32_t *bm = a.bitmap + ((int64_t)qi * a.Hkv + g) * kPfWords;
-                    for (int w = 0; w < (it.jblk >> 5); ++w) slot += __popc(bm[w]);
-                    slot += __popc(bm[it.jblk >> 5] & ((1u << (it.jblk & 31)) - 1u)) + 1;
-                }
-                if (slot < kPfSlots)
-                    rec = (((int64_t)qi * a.Hkv + g) * kPfSlots + slot) * G + (r % G);
-            }
-            float *po = rec >= 0 ? a.part_o + rec * D + half * 64 : nullptr;
-            if (T > 0) {
-#pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    uint32_t ov[32];
-                    tmem_ld32(tO + lane_base + half * 64 + c2 * 32, ov);
-                    tmem_ld_wait();
-                    if (po) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            *reinterpret_cast<float4 *>(po + c2 * 32 + e) =
-                                make_float4(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1]),
-                                            __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
-                    }
-                }
-            } else if (po) {
-                for (int d = 0; d < 64; ++d) po[d] = 0.0f;
-            }
-            if (rec >= 0 && half == 0) a.part_ml[rec] = make_float2(m_used, l_row);
+            pend = true;   // T >= 1: the item's last tile is u - 1
+            pend_n = n;
+            pend_u = u - 1;
+            pend_m = m_used;
+            pend_l = l_part;
         }
-        // every role advances the per-barrier MMA counts by this item's tiles
-        sbase[0] += (uint32_t)((T + 1) >> 1);
-        sbase[1] += (uint32_t)(T >> 1);
-        obase[0] += (uint32_t)((T + 1) >> 1);
-        obase[1] += (uint32_t)(T >> 1);
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        if (pend) epilogue();
     }
     if (timed_out) atomicOr(a.status, 8u);
     tc_fence_before();
@@ -600,7 +716,7 @@ __global__ void __launch_bounds__(128) prefill_merge_kernel(PfArgs a) {
 
 // ---------------------------------------------------------------- host
 struct PfLayout {
-    size_t bitmap, vis, qcount, qlist, prefix, work, part_o, part_ml, total;
+    size_t bitmap, vis, qcount, qlist, prefix, part_o, part_ml, total;
 };
 
 static PfLayout pf_layout(const bsa_kv_desc *d, const bsa_sel_params *p, int Tq) {
@@ -610,7 +726,6 @@ static PfLayout pf_layout(const bsa_kv_desc *d, const bsa_sel_params *p, int Tq)
     L.bitmap = o;  o += align_up((size_t)Tq * H * kPfWords * 4, 256);
     L.vis = o;     o += align_up(H * nb * 4, 256);
     L.qcount = o;  o += align_up(H * nb * 4, 256);
-    L.work = o;    o += 256;
     L.qlist = o;   o += align_up(H * nb * (size_t)Tq * 4, 256);
     L.prefix = o;  o += align_up((H * nb + 1) * 4, 256);
     L.part_o = o;  o += align_up((size_t)Tq * H * kPfSlots * G * d->D * 4, 256);
@@ -630,6 +745,9 @@ bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
                           size_t ws_bytes, cudaStream_t st) {
     const int G = d->Hq / d->Hkv;
     if (p->n_blocks > kPfMaxBlocks || kTile % G != 0 || G > 16) return BSA_ERR_UNSUPPORTED;
+    // query index and slot share a qlist entry; partial records index with int32
+    if (Tq >= (1 << kPfSlotShift) || (int64_t)Tq * d->Hkv * kPfSlots * G >= (int64_t)1 << 31)
+        return BSA_ERR_UNSUPPORTED;
     const PfLayout L = pf_layout(d, p, Tq);
     if (ws_bytes < L.total) return BSA_ERR_WORKSPACE;
     char *w = static_cast<char *>(ws);
@@ -647,7 +765,6 @@ bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
     a.qcount = reinterpret_cast<int32_t *>(w + L.qcount);
     a.qlist = reinterpret_cast<int32_t *>(w + L.qlist);
     a.tile_prefix = reinterpret_cast<int32_t *>(w + L.prefix);
-    a.work = reinterpret_cast<int32_t *>(w + L.work);
     a.part_o = reinterpret_cast<float *>(w + L.part_o);
     a.part_ml = reinterpret_cast<float2 *>(w + L.part_ml);
     a.status = status;
@@ -659,9 +776,8 @@ bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
     if (!make_kv_tmap(&kp, d, K, kTile) || !make_kv_tmap(&vp, d, V, kTile) ||
         !make_kv_tmap(&kl, pd, K_pos, kTile) || !make_kv_tmap(&vl, pd, V_pos, kTile))
         return BSA_ERR_CUDA;
-    // zero the per-block counts and the work counter
+    // zero the per-block counts
     BSA_CUDA_TRY(cudaMemsetAsync(w + L.qcount, 0, (size_t)d->Hkv * p->n_blocks * 4, st));
-    BSA_CUDA_TRY(cudaMemsetAsync(w + L.work, 0, 4, st));
     // P1: selection
     auto smem1_for = [&](int nw) {
         return ((size_t)a.nb * kPfCentStride + (size_t)nw * G * a.D + a.nb) * 4;
