@@ -253,8 +253,9 @@ struct PfSmem {
     static constexpr int kRowQ = kRowPos + 4 * kTile * 4; // int [4][128] row of Q (-1: none)
     static constexpr int kRowRec = kRowQ + 4 * kTile * 4; // int [4][128] partial record (-1: none)
     static constexpr int kDesc = kRowRec + 4 * kTile * 4; // int [4][8]: g, kbeg, kend, T, local, end
-    static constexpr int kPair = kDesc + 4 * 8 * 4;       // float [4][128] quarter-row maxima / sums
-    static constexpr int kBars = kPair + 4 * kTile * 4;   // u64 [23]
+    static constexpr int kPair = kDesc + 4 * 8 * 4;       // float [3][4][128]: quarter-row maxima (by
+                                                          // tile parity), quarter-row sums
+    static constexpr int kBars = kPair + 3 * 4 * kTile * 4;   // u64 [23]
     static constexpr int kMisc = kBars + 23 * 8;          // tmem base
     static constexpr int kPrefix = kMisc + 32;            // int [kPfPrefixCap]
     static constexpr int kBytes = kPrefix + kPfPrefixCap * 4 + 1024;
@@ -545,9 +546,10 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
             const int pend_b = pend_n & 1, pend_m4 = pend_n & 3;
             wait(&odone[pend_u & 1], (pend_u >> 1) & 1);
             tc_fence_after();
-            pairv[cq * kTile + r] = pend_l;
+            float *pl4 = pairv + 8 * kTile;
+            pl4[cq * kTile + r] = pend_l;
             quad_sync(q);
-            const float l_row = (pairv[r] + pairv[kTile + r]) + (pairv[2 * kTile + r] + pairv[3 * kTile + r]);
+            const float l_row = (pl4[r] + pl4[kTile + r]) + (pl4[2 * kTile + r] + pl4[3 * kTile + r]);
             quad_sync(q);
             const int rec = rowrec_s[pend_m4 * kTile + r];
             float *po = rec >= 0 ? a.part_o + (int64_t)rec * D + cq * 32 : nullptr;
@@ -586,31 +588,29 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                 uint32_t sv[32];
                 tmem_ld32(tS + lane_base + cq * 32, sv);
                 tmem_ld_wait();
+                // maxima on the raw logits (the scale is positive); masked
+                // keys become -inf
                 const int key0 = kbeg + t * kTile + cq * 32;
                 float mx = kPfNegInf;
                 if (key0 + 31 < kend && key0 + 31 <= my_pos) {   // every key of the quarter visible
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float v = __uint_as_float(sv[e]) * a.scale_log2;
-                        sv[e] = __float_as_uint(v);
-                        mx = fmaxf(mx, v);
-                    }
+                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int kr = key0 + e;
-                        const bool ok = kr < kend && kr <= my_pos;
-                        const float v = ok ? __uint_as_float(sv[e]) * a.scale_log2 : kPfNegInf;
-                        sv[e] = __float_as_uint(v);
-                        mx = fmaxf(mx, v);
+                        if (!(kr < kend && kr <= my_pos)) sv[e] = __float_as_uint(kPfNegInf);
+                        mx = fmaxf(mx, __uint_as_float(sv[e]));
                     }
                 }
-                // all quarters of the row have read S(u) before any writes P
-                pairv[cq * kTile + r] = mx;
+                // one barrier: the quarters exchange maxima through the tile
+                // parity's buffer, and every quarter has read S(u) before any
+                // writes P into it
+                float *pm = pairv + (st * 4) * kTile;
+                pm[cq * kTile + r] = mx;
                 quad_sync(q);
-                const float m_tile = fmaxf(fmaxf(pairv[r], pairv[kTile + r]),
-                                           fmaxf(pairv[2 * kTile + r], pairv[3 * kTile + r]));
-                quad_sync(q);
+                const float m_tile = fmaxf(fmaxf(pm[r], pm[kTile + r]), fmaxf(pm[2 * kTile + r], pm[3 * kTile + r])) *
+                                     a.scale_log2;
                 // lazy rescale: keep the reference maximum unless this tile
                 // exceeds it by more than 2^8
                 bool rescale = false;
@@ -644,10 +644,13 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                 // the pairs are packed with byte permutes.
                 float lsum = 0.0f;
                 uint32_t ph[16], pl[16];
+                const float neg_m = -m_used;
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const float p0 = m_used == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[e]) - m_used);
-                    const float p1 = m_used == kPfNegInf ? 0.0f : exp2f(__uint_as_float(sv[e + 1]) - m_used);
+                    const float x0 = __fmaf_rn(__uint_as_float(sv[e]), a.scale_log2, neg_m);
+                    const float x1 = __fmaf_rn(__uint_as_float(sv[e + 1]), a.scale_log2, neg_m);
+                    const float p0 = m_used == kPfNegInf ? 0.0f : exp2f(x0);
+                    const float p1 = m_used == kPfNegInf ? 0.0f : exp2f(x1);
                     lsum += p0 + p1;
                     const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
                     const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);
