@@ -170,10 +170,11 @@ class DecodeSession:
         (self.g_refresh if t % self.cfg.refresh == 0 else self.g_plain).replay()
 
     def launches_per_step(self, t: int) -> int:
-        """Library calls one step makes: append, select on refresh steps, and
-        decode; a fused step is one."""
+        """Library kernels one step launches: append, the two selection kernels
+        (scoring, picking) on refresh steps, and the decode; a fused step is one
+        launch."""
         if t % self.cfg.refresh == 0:
-            return 3
+            return 4
         return 1 if self.fused and self.fuses() else 2
 
     def fuses(self) -> bool:
