@@ -505,6 +505,58 @@ def run_reference(args):
     }
 
 
+def run_case(args, device):
+    """A small, fixed invocation of one library call for a profiler to capture
+    (a few launches on a workload of a few GB at most); prints one line.
+      decode   Quest workload: two steps (the second a fused append + decode),
+               then bsa_decode five times, L2 flushed before each
+      select   Quest workload: bsa_select three times, L2 flushed before each
+      prefill  semantic workload at a 65,536-token context: the last chunk of
+               1,024 queries three times"""
+    from block_sparse_long_build_b200 import build as Bld
+    from block_sparse_long_build_b200 import workloads as W
+    from block_sparse_long_build_b200.session import DecodeSession
+    Bld.build()
+    flush = _flusher(device)
+    ev = []
+    if args.case in ("decode", "select"):
+        cfg = W.quest(0)
+        wl = W.Workload(cfg, device)
+        sess = DecodeSession(wl)
+        sess.build_summaries()
+        q = wl.decode_query(0)
+        if args.case == "decode":
+            for t in range(2):
+                q = wl.decode_query(t)
+                k, v = wl.decode_new_kv(t)
+                sess.step(t, q, k, v)
+        for i in range(5 if args.case == "decode" else 3):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sess.decode(q) if args.case == "decode" else sess.select(q)
+            e1.record()
+            ev.append((e0, e1))
+    elif args.case == "prefill":
+        L, Tq = 65536, 1024
+        cfg = W.semantic(0).scaled(L=L, budget_tokens=L // 16, chunk=Tq)
+        wl = W.Workload(cfg, device)
+        sess = DecodeSession(wl)
+        sess.build_summaries()
+        out = torch.empty(Tq, cfg.Hq, cfg.D, device=device)
+        lse = torch.empty(Tq, cfg.Hq, device=device)
+        Q = wl.prefill_queries(L - Tq, Tq)
+        ws = None
+        for i in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ws = sess.prefill_chunk(Q, L - Tq, out, lse, ws)
+            e1.record()
+            ev.append((e0, e1))
+    torch.cuda.synchronize()
+    print(f"case {args.case}: ms per call", [round(a.elapsed_time(b), 4) for a, b in ev], flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -519,7 +571,13 @@ def main():
                     help="context of the prefill run (default: the configuration's 524,288)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--case", choices=["decode", "select", "prefill"], default=None,
+                    help="run one small profiling case instead of the bench (for ncu)")
     args = ap.parse_args()
+    if args.case:
+        torch.cuda.set_device(0)
+        run_case(args, torch.device("cuda", 0))
+        return 0
     if args.warmup < 3:
         args.warmup = 3
     if args.steps is None:
