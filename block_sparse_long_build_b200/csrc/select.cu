@@ -584,6 +584,139 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
 }
 
 
+// The same selection for segments of at most 32 * kPickWarpKeys blocks, by one
+// warp per segment with no CTA barrier: lane l holds blocks l + 32 r; the walk
+// takes the best remaining candidate (highest key, then lowest index; for a
+// budget, the best that still fits) until k blocks or nothing fits; a ballot
+// per r compacts the taken blocks in index order; lane 0 merges the forced
+// ranges and the blocks' ranges.  Shared memory: sel, lo, hi [max_sel] ints.
+__global__ void __launch_bounds__(32) pick_small_kernel(SelArgs a) {
+    extern __shared__ __align__(16) unsigned char psm[];
+    int32_t *sel = reinterpret_cast<int32_t *>(psm);
+    int32_t *slo = sel + a.max_sel, *shi = slo + a.max_sel;
+    const int s = blockIdx.x, b = s / a.Hkv, lane = threadIdx.x;
+    const int nb = a.nb_total;
+    const int32_t *off = a.offsets ? a.offsets + (int64_t)s * (nb + 1) : nullptr;
+    pdl_wait();   // keys and visible counts from score_kernel
+    uint32_t wk[kPickWarpKeys];
+    int wv[kPickWarpKeys];
+#pragma unroll
+    for (int r = 0; r < kPickWarpKeys; ++r) {
+        const int j = lane + 32 * r;
+        wk[r] = j < nb ? a.keys[(int64_t)s * nb + j] : 0u;
+        wv[r] = off && j < nb ? a.vis[(int64_t)s * nb + j] : 0;
+    }
+    // forced token ranges (every lane computes the same), sorted and merged
+    const int n = min(max(a.cur_len[b], 0), a.L_max);
+    int f_lo[3] = {0, 0, 0}, f_hi[3] = {0, 0, 0}, nf = 0;
+    if (off) {
+        if (n > a.local_start) { f_lo[0] = max(a.local_start, 0); f_hi[0] = n; nf = 1; }
+    } else {
+        if (a.sink > 0 && n > 0) { f_lo[0] = 0; f_hi[0] = min(a.sink, n); nf = 1; }
+        int t0 = n;
+        if (a.window > 0) t0 = min(t0, max(0, n - a.window));
+        if (a.keep_current && n > 0) t0 = min(t0, ((n - 1) / a.S) * a.S);
+        if (t0 < n) {
+            if (nf > 0 && t0 <= f_hi[0]) f_hi[0] = n;
+            else if (nf == 0) { f_lo[0] = t0; f_hi[0] = n; nf = 1; }
+            else { f_lo[1] = t0; f_hi[1] = n; nf = 2; }
+        }
+    }
+    // candidates: keys > 0 and (fixed blocks) not wholly inside the forced set
+    int my_c = 0;
+#pragma unroll
+    for (int r = 0; r < kPickWarpKeys; ++r) {
+        if (wk[r] && !off) {
+            const int64_t r0 = (int64_t)(lane + 32 * r) * a.S, r1 = r0 + a.S;
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                if (i < nf && f_lo[i] <= r0 && r1 <= f_hi[i]) wk[r] = 0u;
+        }
+        my_c += wk[r] != 0u;
+    }
+    int n_cand = my_c;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n_cand += __shfl_xor_sync(0xffffffffu, n_cand, o);
+    const bool greedy = off && a.topk < 0;
+    const int limit = greedy ? a.max_sel : min(min(a.topk >= 0 ? a.topk : a.budget / a.S, n_cand), a.max_sel);
+    int remaining = a.budget;
+    uint32_t taken = 0;   // bit r: block lane + 32 r
+    for (int t = 0; t < limit; ++t) {
+        unsigned long long best = 0ull;
+#pragma unroll
+        for (int r = 0; r < kPickWarpKeys; ++r)
+            if (wk[r] && !((taken >> r) & 1u) && (!greedy || wv[r] <= remaining)) {
+                const unsigned long long c =
+                    ((unsigned long long)wk[r] << 32) | (0xffffffffu - (uint32_t)(lane + 32 * r));
+                best = c > best ? c : best;
+            }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other > best ? other : best;
+        }
+        if (best == 0ull) break;
+        const int j = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
+        int vj = 0;
+#pragma unroll
+        for (int r = 0; r < kPickWarpKeys; ++r)
+            if (lane + 32 * r == j) { taken |= 1u << r; vj = wv[r]; }
+        remaining -= __shfl_sync(0xffffffffu, vj, j & 31);
+    }
+    // index-ordered compaction
+    int n_sel = 0;
+#pragma unroll
+    for (int r = 0; r < kPickWarpKeys; ++r) {
+        const uint32_t m = __ballot_sync(0xffffffffu, (taken >> r) & 1u);
+        if ((taken >> r) & 1u) {
+            const int p = n_sel + __popc(m & ((1u << lane) - 1u));
+            const int jj = lane + 32 * r;
+            if (p < a.max_sel) {
+                int lo, hi;
+                if (off) { lo = min(max(off[jj], 0), a.L_max); hi = lo + wv[r]; }
+                else { lo = jj * a.S; hi = lo + a.S; }
+                sel[p] = jj;
+                slo[p] = lo;
+                shi[p] = hi;
+            }
+        }
+        n_sel += __popc(m);
+    }
+    n_sel = min(n_sel, a.max_sel);
+    __syncwarp();
+    for (int i = lane; i < n_sel; i += 32) a.sel_blocks[(int64_t)s * a.max_sel + i] = sel[i];
+    if (lane == 0) {
+        // ranges: forced and selected ranges in start order (forced first on
+        // equal starts); a range grows while the next item starts at or
+        // before its end
+        int32_t *R = a.ranges + (int64_t)s * a.max_ranges * 2;
+        int nr = 0, cs = 0, ce = 0, fi = 0, si = 0;
+        bool open = false;
+        while (fi < nf || si < n_sel) {
+            const int blo = si < n_sel ? slo[si] : 0, bhi = si < n_sel ? shi[si] : 0;
+            const int fl = fi == 0 ? f_lo[0] : f_lo[1], fh = fi == 0 ? f_hi[0] : f_hi[1];
+            int lo, hi;
+            if (fi < nf && (si >= n_sel || fl <= blo)) { lo = fl; hi = fh; ++fi; }
+            else { lo = blo; hi = bhi; ++si; }
+            if (open && lo <= ce) {
+                ce = max(ce, hi);
+            } else {
+                if (open) {
+                    if (nr < a.max_ranges) { R[2 * nr] = cs; R[2 * nr + 1] = ce; }
+                    ++nr;
+                }
+                cs = lo; ce = hi; open = true;
+            }
+        }
+        if (open) {
+            if (nr < a.max_ranges) { R[2 * nr] = cs; R[2 * nr + 1] = ce; }
+            ++nr;
+        }
+        a.n_ranges[s] = min(nr, a.max_ranges);
+        a.sel_count[s] = n_sel;
+    }
+}
+
 bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ, int kind,
                          const bsa_sel_params *p, const int32_t *cur_len, int nb_total,
                          int max_sel, int32_t *sel_blocks, int32_t *sel_count, int max_ranges,
@@ -659,6 +792,11 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
         BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(kPickThreads), smem2, st, a));
         return BSA_OK;
     };
+    if (nb_total <= 32 * kPickWarpKeys) {
+        const size_t smem3 = (size_t)max_sel * 12;
+        BSA_CUDA_TRY(launch_pdl(pick_small_kernel, dim3((unsigned)nseg), dim3(32), smem3, st, a));
+        return BSA_OK;
+    }
     return pick(pick_kernel);
 }
 
