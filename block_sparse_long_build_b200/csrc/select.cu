@@ -792,7 +792,9 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
         BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(kPickThreads), smem2, st, a));
         return BSA_OK;
     };
-    if (nb_total <= 32 * kPickWarpKeys) {
+    // one warp per segment for small top-k problems; the token budget walk
+    // (variable blocks) measured faster in the CTA kernel
+    if (nb_total <= 32 * kPickWarpKeys && !variable) {
         const size_t smem3 = (size_t)max_sel * 12;
         BSA_CUDA_TRY(launch_pdl(pick_small_kernel, dim3((unsigned)nseg), dim3(32), smem3, st, a));
         return BSA_OK;
