@@ -84,6 +84,9 @@ class ClockSampler:
         self.proc = None
 
     def start(self):
+        """Starts sampling and returns once the first sample is in (nvidia-smi
+        takes a moment to start), so that short runs are covered too."""
+        self.first = ""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
@@ -91,6 +94,11 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+        import select
+        ready, _, _ = select.select([self.proc.stdout], [], [], 5.0)
+        if ready:
+            self.first = self.proc.stdout.readline()
 
     def stop(self):
         if self.proc is None:
@@ -103,7 +111,7 @@ class ClockSampler:
             out, _ = self.proc.communicate()
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+        for line in (self.first + out).strip().splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 10:
                 continue
@@ -564,7 +572,7 @@ def main():
                     help="decode steps to time (default: the configuration's own count)")
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="quest", help="tiny | quest | moba | largebatch | semantic")
+    ap.add_argument("--config", default="quest", help="tiny | quest | moba | largebatch | semantic | msa")
     ap.add_argument("--prefill", action="store_true",
                     help="time the block-grouped prefill of the semantic configuration instead")
     ap.add_argument("--prefill-context", type=int, default=0,

@@ -261,6 +261,14 @@ struct PfSmem {
     static constexpr int kBytes = kPrefix + kPfPrefixCap * 4 + 1024;
 };
 
+// 2^x by the MUFU instruction, subnormal results flushed to zero (weights below
+// 2^-126 of the row maximum contribute nothing at fp32 accumulation).
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void quad_sync(int q) {   // the four warps holding rows 32q..32q+31
     asm volatile("bar.sync %0, 128;" ::"r"(1 + q) : "memory");
 }
@@ -649,8 +657,8 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                 for (int e = 0; e < 32; e += 2) {
                     const float x0 = __fmaf_rn(__uint_as_float(sv[e]), a.scale_log2, neg_m);
                     const float x1 = __fmaf_rn(__uint_as_float(sv[e + 1]), a.scale_log2, neg_m);
-                    const float p0 = m_used == kPfNegInf ? 0.0f : exp2f(x0);
-                    const float p1 = m_used == kPfNegInf ? 0.0f : exp2f(x1);
+                    const float p0 = m_used == kPfNegInf ? 0.0f : ex2_ftz(x0);
+                    const float p1 = m_used == kPfNegInf ? 0.0f : ex2_ftz(x1);
                     lsum += p0 + p1;
                     const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
                     const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);

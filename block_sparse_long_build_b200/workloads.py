@@ -124,8 +124,18 @@ def largebatch(seed: int = 0) -> Config:
                   256, 512, False, 1, 256, seed, n_clusters=32)
 
 
+def msa(seed: int = 0) -> Config:
+    """MSA-shaped block decode (Attention mechanisms, MSA: blocks of 128,
+    top-16 per GQA group = 2,048 tokens, the local block always kept):
+    batch 2, 8 KV / 32 query heads, D 128, bf16; 131,072-token cache of 64
+    Gaussian clusters (as quest); mean-pooled block keys; selection every
+    step; 64 decode steps."""
+    return Config("msa", 2, 8, 32, 128, torch.bfloat16, 131072, CENTROID, 128, 16, 0, 0, 0,
+                  True, 1, 64, seed, n_clusters=64)
+
+
 CONFIGS = {"tiny": tiny, "quest": quest, "moba": moba, "semantic": semantic,
-           "largebatch": largebatch}
+           "largebatch": largebatch, "msa": msa}
 
 
 def _gen(device, seed: int) -> torch.Generator:

@@ -39,6 +39,10 @@ CASES = {
     # fp32 cache with D 128 on the CUDA-core path
     "moba_f32": _cfg(W.moba(0), Hkv=1, Hq=4, kv_dtype=torch.float32, L=64 * 50 + 3,
                      block_size=64, topk=5, n_needles=3, steps=2),
+    # MSA-shaped: blocks of 128, top-16, current block, clustered keys
+    "msa_small": _cfg(W.msa(0), B=2, Hkv=2, Hq=8, L=128 * 40 + 50, steps=3),
+    # the same with more than 512 blocks per segment (the CTA-wide radix pick)
+    "msa_many_blocks": _cfg(W.msa(0), B=1, Hkv=2, Hq=8, L=128 * 600 + 17, steps=2),
 }
 
 
