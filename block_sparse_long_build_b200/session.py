@@ -25,6 +25,10 @@ from . import native as N
 from .workloads import Config, Workload
 
 
+def _align(n: int, a: int = 256) -> int:
+    return (n + a - 1) // a * a
+
+
 class DecodeSession:
     def __init__(self, wl: Workload, stream: torch.cuda.Stream | None = None, fused: bool = True):
         self.wl = wl
@@ -58,8 +62,12 @@ class DecodeSession:
         ws = max(N.bsa_workspace_size(self.desc, self.sel, op, 0, self.tokens_hint)
                  for op in (N.BSA_OP_SELECT, N.BSA_OP_DECODE, N.BSA_OP_APPEND))
         self.ws = torch.zeros(ws, dtype=torch.uint8, device=dev)
-        self.out = torch.zeros(c.B, c.Hq, c.D, dtype=torch.float32, device=dev)
-        self.lse = torch.zeros(c.B, c.Hq, dtype=torch.float32, device=dev)
+        # outputs in one buffer (out, then lse) so a step's results leave the
+        # device in one copy
+        n_out = c.B * c.Hq * c.D * 4
+        self.io_out = torch.zeros(_align(n_out) + c.B * c.Hq * 4, dtype=torch.uint8, device=dev)
+        self.out = self.io_out[:n_out].view(torch.float32).view(c.B, c.Hq, c.D)
+        self.lse = self.io_out[_align(n_out):].view(torch.float32).view(c.B, c.Hq)
         self.scale = 1.0 / math.sqrt(c.D)
 
     def token_bound(self) -> int:
@@ -143,15 +151,44 @@ class DecodeSession:
         return ws
 
     # ------------------------------------------------------------ CUDA graphs
+    def io_in_layout(self) -> tuple[int, int, int, int]:
+        """Byte offsets of q, k_new, v_new in the packed step-input buffer, and
+        its size (q fp32 [B, Hq, D], k_new / v_new in the cache dtype
+        [B, Hkv, D], each 256-byte aligned)."""
+        c = self.cfg
+        esz = 2 if c.kv_dtype == torch.bfloat16 else 4
+        nq, nk = c.B * c.Hq * c.D * 4, c.B * c.Hkv * c.D * esz
+        ok = _align(nq)
+        ov = ok + _align(nk)
+        return 0, ok, ov, ov + _align(nk)
+
+    def pack_inputs(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    pin: bool = True) -> torch.Tensor:
+        """One step's inputs packed on the host in the layout of io_in (a
+        single host-to-device copy feeds a step)."""
+        oq, ok, ov, n = self.io_in_layout()
+        buf = torch.zeros(n, dtype=torch.uint8)
+        if pin:
+            buf = buf.pin_memory()
+        for o, x in ((oq, q), (ok, k), (ov, v)):
+            x = x.detach().cpu().contiguous()
+            nbytes = x.numel() * x.element_size()
+            buf[o:o + nbytes].view(x.dtype).copy_(x.view(-1))
+        return buf
+
     def capture(self):
         """Captures one decode step into two CUDA graphs (with and without
         the selection refresh) reading persistent input buffers q_in, k_in,
         v_in.  Launch-bound steps then cost one graph launch each.  Run one
         eager step first so that one-time host setup is not captured."""
         c, dev = self.cfg, self.wl.device
-        self.q_in = torch.zeros(c.B, c.Hq, c.D, dtype=torch.float32, device=dev)
-        self.k_in = torch.zeros(c.B, c.Hkv, c.D, dtype=c.kv_dtype, device=dev)
-        self.v_in = torch.zeros_like(self.k_in)
+        oq, ok, ov, n = self.io_in_layout()
+        esz = 2 if c.kv_dtype == torch.bfloat16 else 4
+        nq, nk = c.B * c.Hq * c.D * 4, c.B * c.Hkv * c.D * esz
+        self.io_in = torch.zeros(n, dtype=torch.uint8, device=dev)
+        self.q_in = self.io_in[oq:oq + nq].view(torch.float32).view(c.B, c.Hq, c.D)
+        self.k_in = self.io_in[ok:ok + nk].view(c.kv_dtype).view(c.B, c.Hkv, c.D)
+        self.v_in = self.io_in[ov:ov + nk].view(c.kv_dtype).view(c.B, c.Hkv, c.D)
         self.g_refresh, self.g_plain = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.g_refresh):
             self.append(self.k_in, self.v_in)
