@@ -331,7 +331,7 @@ bsa_status bsa_prefill_grouped(const bsa_kv_desc *d, const void *K, const void *
     if (!desc_ok(d) || !desc_ok(pd) || !sel_ok(d, p)) return BSA_ERR_ARG;
     if (!K || !V || !summaries || !K_pos || !V_pos || !Q || !out) return BSA_ERR_ARG;
     if (!aligned16(K) || !aligned16(V) || !aligned16(K_pos) || !aligned16(V_pos) || !aligned16(Q) ||
-        !aligned16(out))
+        !aligned16(out) || !aligned16(summaries))
         return BSA_ERR_ARG;
     if (p->block_size != 0 || p->topk >= 0) return BSA_ERR_UNSUPPORTED;
     if (d->B != 1 || pd->B != 1 || d->Hkv != pd->Hkv || d->Hq != pd->Hq || d->D != pd->D)

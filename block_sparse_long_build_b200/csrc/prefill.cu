@@ -33,8 +33,9 @@ constexpr int kPfWords = kPfMaxBlocks / 32;
 constexpr int kPfMaxSel = 64;              // selected blocks kept per (query, KV head)
 constexpr int kPfSlots = kPfMaxSel + 1;    // slot 0 = local part
 constexpr int kPfSlotShift = 24;           // qlist entry: query | slot << 24
-constexpr int kPfSelWarps = 16;            // P1 warps per CTA (8 when shared memory is short)
-constexpr int kPfRowsPerWarp = 8;          // P1 query rows per warp
+constexpr int kPfSelWarps = 16;            // P1 warps per CTA (fewer when shared memory is short)
+constexpr int kPfMergeThreads = 128;       // P4 threads per CTA
+constexpr int kPfD = 128;                  // head dimension of the prefill path
 constexpr int kPfCentStride = 132;         // padded centre row (floats): 16-byte rows, conflict-free
 constexpr int kTile = 128;                 // rows per MMA tile, keys per key tile
 constexpr size_t kMaxSmemPerCta = 227 * 1024;   // opt-in dynamic shared memory per CTA
@@ -59,6 +60,7 @@ struct PfArgs {
     uint32_t *status;
     float *out, *lse;          // [Tq][Hq][D], [Tq][Hq]
     int n_local;               // local work items
+    int sel_rows_per_warp;     // P1: query rows per warp (one wave of CTAs)
 };
 
 __device__ __forceinline__ int pf_visible(const int32_t *pos, int r0, int r1, int lim) {
@@ -77,11 +79,30 @@ __global__ void __launch_bounds__(32 * kPfSelWarps) prefill_select_kernel(PfArgs
     const int nw = blockDim.x >> 5;
     float *cs = psm;                                   // [nb][kPfCentStride]
     float *qv = cs + nb * kPfCentStride;               // [nw][G][D]
-    int *visS = reinterpret_cast<int *>(qv + nw * G * D);   // [nb]
+    uint16_t *qst = reinterpret_cast<uint16_t *>(qv + nw * G * D);   // [nw][G][D] bf16 staging
+    int *visS = reinterpret_cast<int *>(qst + nw * G * D);           // [nb]
     const int g = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rpw = a.sel_rows_per_warp, row0 = (blockIdx.x * nw + warp) * rpw;
+    float *qw = qv + warp * G * D;
+    uint16_t *qs = qst + warp * G * D;
+    // query row i's G heads (bf16) into this warp's staging buffer, 16 bytes a copy
+    auto stage_q = [&](int i) {
+        const uint16_t *qi = a.Q + ((int64_t)i * a.Hq + (int64_t)g * G) * D;
+        for (int e = 8 * lane; e < G * D; e += 256)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(qs + e)), "l"(qi + e)
+                         : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
     pdl_wait();
+    // centres into padded rows, asynchronously, while the visible counts are searched
     const float *cg = a.cent + (int64_t)g * nb * D;
-    for (int e = tid; e < nb * D; e += blockDim.x) cs[(e / D) * kPfCentStride + e % D] = cg[e];
+    for (int e = 4 * tid; e < nb * D; e += 4 * blockDim.x)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                         smem_u32(cs + (e / D) * kPfCentStride + e % D)),
+                     "l"(cg + e)
+                     : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (row0 < a.Tq) stage_q(row0);
     const int32_t *off = a.offsets + (int64_t)g * (nb + 1);
     const int32_t *pos = a.kv_pos + (int64_t)g * a.L_max;
     for (int j = tid; j < nb; j += blockDim.x) {
@@ -90,18 +111,34 @@ __global__ void __launch_bounds__(32 * kPfSelWarps) prefill_select_kernel(PfArgs
         visS[j] = v;
         if (blockIdx.x == 0) a.vis[g * nb + j] = v;
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    float *qw = qv + warp * G * D;
-    for (int r = 0; r < kPfRowsPerWarp; ++r) {
-        const int i = (blockIdx.x * nw + warp) * kPfRowsPerWarp + r;
+    // this lane's centre rows (blocks lane + 32 t)
+    int crow[kPfWords], vr[kPfWords];   // vr: visible rows (INT_MAX past the last block)
+#pragma unroll
+    for (int t = 0; t < kPfWords; ++t) {
+        crow[t] = min(lane + 32 * t, nb - 1) * kPfCentStride;
+        vr[t] = lane + 32 * t < nb ? visS[lane + 32 * t] : 0x7fffffff;
+    }
+    for (int r = 0; r < rpw; ++r) {
+        const int i = row0 + r;
         if (i >= a.Tq) break;
-        const uint16_t *qi = a.Q + ((int64_t)i * a.Hq + (int64_t)g * G) * D;
-        for (int e = lane; e < G * D; e += 32) qw[e] = bf16_to_f32(qi[e]);
+        // row i is staged (the wait covers this lane's copies, the warp
+        // barrier everyone's); widen it, then stage row i + 1 behind the work
+        asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
-        // lane owns blocks lane + 32 t; composite keys (orderable score, ~index).
-        // The (block, head) fma chains are interleaved over d for ILP; each
-        // chain still runs d = 0..D-1 in order.
-        unsigned long long key[kPfWords];
+        for (int e = 4 * lane; e < G * D; e += 128) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(qs + e);
+            *reinterpret_cast<float4 *>(qw + e) =
+                make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                            __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+        }
+        __syncwarp();
+        if (r + 1 < rpw && i + 1 < a.Tq) stage_q(i + 1);
+        // lane owns blocks lane + 32 t; sk[t] = orderable score key of block
+        // lane + 32 t (0: not a candidate). The (block, head) fma chains are
+        // interleaved over d for ILP; each chain still runs d = 0..D-1 in order.
+        uint32_t sk[kPfWords];
         {
             constexpr int kMaxGh = 4;   // heads accumulated together per pass
             float tot[kPfWords];
@@ -111,16 +148,16 @@ __global__ void __launch_bounds__(32 * kPfSelWarps) prefill_select_kernel(PfArgs
                 for (int t = 0; t < kPfWords; ++t)
 #pragma unroll
                     for (int h = 0; h < kMaxGh; ++h) acc[t][h] = 0.0f;
-                for (int d = 0; d < D; d += 4) {
+#pragma unroll 1
+                for (int d = 0; d < kPfD; d += 4) {
                     float4 qd[kMaxGh];
 #pragma unroll
                     for (int h = 0; h < kMaxGh; ++h)
-                        qd[h] = h0 + h < G ? *reinterpret_cast<const float4 *>(qw + (h0 + h) * D + d)
+                        qd[h] = h0 + h < G ? *reinterpret_cast<const float4 *>(qw + (h0 + h) * kPfD + d)
                                            : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                     for (int t = 0; t < kPfWords; ++t) {
-                        const int j = min(lane + 32 * t, nb - 1);
-                        const float4 c = *reinterpret_cast<const float4 *>(cs + j * kPfCentStride + d);
+                        const float4 c = *reinterpret_cast<const float4 *>(cs + crow[t] + d);
 #pragma unroll
                         for (int h = 0; h < kMaxGh; ++h) {
                             acc[t][h] = __fmaf_rn(qd[h].x, c.x, acc[t][h]);
@@ -138,13 +175,11 @@ __global__ void __launch_bounds__(32 * kPfSelWarps) prefill_select_kernel(PfArgs
             }
 #pragma unroll
             for (int t = 0; t < kPfWords; ++t) {
-                key[t] = 0ull;
-                const int j = lane + 32 * t;
+                sk[t] = 0u;
                 // only candidates that can ever fit the budget
-                if (j < nb && visS[j] > 0 && visS[j] <= a.budget) {
-                    uint32_t k32 = f32_order_key(__fadd_rn(tot[t], 0.0f));
-                    if (k32 == 0) k32 = 1;
-                    key[t] = ((unsigned long long)k32 << 32) | (0xffffffffu - (uint32_t)j);
+                if (vr[t] > 0 && vr[t] <= a.budget) {
+                    const uint32_t k32 = f32_order_key(__fadd_rn(tot[t], 0.0f));
+                    sk[t] = k32 ? k32 : 1u;
                 }
             }
         }
@@ -152,27 +187,27 @@ __global__ void __launch_bounds__(32 * kPfSelWarps) prefill_select_kernel(PfArgs
         // What is left of the budget only shrinks, so a block that does not
         // fit now never will: after each take such blocks are dropped, and the
         // best remaining candidate always fits.
+        // The best candidate is the highest key, ties to the lowest block
+        // index: a warp max of the keys, then a warp min of the indices that
+        // hold it.
         uint32_t selbits = 0;   // bit t: block lane + 32 t selected
         int remaining = a.budget, nsel = 0;
         while (nsel < kPfMaxSel) {
-            unsigned long long best = 0ull;
+            uint32_t lm = 0u;
 #pragma unroll
-            for (int t = 0; t < kPfWords; ++t) best = key[t] > best ? key[t] : best;
+            for (int t = 0; t < kPfWords; ++t) lm = max(lm, sk[t]);
+            const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
+            if (m == 0u) break;
+            int cand = 0x7fffffff;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-                best = other > best ? other : best;
-            }
-            if (best == 0ull) break;
-            const int j = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
+            for (int t = kPfWords - 1; t >= 0; --t) cand = sk[t] == m ? lane + 32 * t : cand;
+            const int j = __reduce_min_sync(0xffffffffu, cand);
             remaining -= visS[j];
             ++nsel;
             if (lane == (j & 31)) selbits |= 1u << (j >> 5);
 #pragma unroll
-            for (int t = 0; t < kPfWords; ++t) {
-                const int jj = lane + 32 * t;
-                if (key[t] && (jj == j || visS[jj] > remaining)) key[t] = 0ull;
-            }
+            for (int t = 0; t < kPfWords; ++t)
+                if (lane + 32 * t == j || vr[t] > remaining) sk[t] = 0u;
         }
         if (nsel >= kPfMaxSel && lane == 0) atomicOr(a.status, 4u);
         uint32_t *bm = a.bitmap + ((int64_t)i * a.Hkv + g) * kPfWords;
@@ -690,32 +725,48 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
 }
 
 // ---------------------------------------------------------------- P4
-__global__ void __launch_bounds__(128) prefill_merge_kernel(PfArgs a) {
+__global__ void __launch_bounds__(kPfMergeThreads, 8) prefill_merge_kernel(PfArgs a) {
     pdl_wait();
-    const int i = blockIdx.x, g = blockIdx.y, G = a.G, D = a.D;
-    const uint32_t *bm = a.bitmap + ((int64_t)i * a.Hkv + g) * kPfWords;
-    int nsel = 0;
-    for (int w = 0; w < kPfWords; ++w) nsel += __popc(bm[w]);
-    const int nslot = min(1 + nsel, kPfSlots);
-    const int D4 = D / 4;
-    // one thread per (head, 4 dimensions); slots merged in slot order, with
-    // all of a pass's loads independent of one another
+    const int i = blockIdx.x, g = blockIdx.y, G = a.G, D = a.D, D4 = D / 4;
+    // one thread per (head, 4 dimensions) and pass; the slots are merged in
+    // slot order with a running maximum
     for (int e = threadIdx.x; e < G * D4; e += blockDim.x) {
         const int hh = e / D4, d4 = e % D4;
         const int64_t rec0 = ((int64_t)i * a.Hkv + g) * kPfSlots * G + hh;
-        float M = kPfNegInf;
-#pragma unroll 8
-        for (int s = 0; s < nslot; ++s) M = fmaxf(M, __ldcg(&a.part_ml[rec0 + (int64_t)s * G]).x);
-        float L = 0.0f;
+        // the first slots' records are read before the slot count is known
+        // (every query has kPfSlots records reserved), so the two reads overlap
+        constexpr int kEarly = 4;
+        float2 ml0[kEarly];
+        float4 ov0[kEarly];
+#pragma unroll
+        for (int s = 0; s < kEarly; ++s) {
+            ml0[s] = __ldcg(&a.part_ml[rec0 + (int64_t)s * G]);
+            ov0[s] = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (rec0 + (int64_t)s * G) * D) + d4);
+        }
+        const uint32_t *bm = a.bitmap + ((int64_t)i * a.Hkv + g) * kPfWords;
+        int nsel = 0;
+#pragma unroll
+        for (int w = 0; w < kPfWords; ++w) nsel += __popc(__ldcg(bm + w));
+        const int nslot = min(1 + nsel, kPfSlots);
+        float M = kPfNegInf, L = 0.0f;
         float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int s = 0; s < nslot; ++s) {
+        auto fold = [&](float2 ml, float4 o) {
+            const float mn = fmaxf(M, ml.x);
+            if (mn != kPfNegInf) {
+                const float c = exp2f(M - mn), w = exp2f(ml.x - mn);
+                L = L * c + ml.y * w;
+                O.x = O.x * c + o.x * w; O.y = O.y * c + o.y * w;
+                O.z = O.z * c + o.z * w; O.w = O.w * c + o.w * w;
+                M = mn;
+            }
+        };
+#pragma unroll
+        for (int s = 0; s < kEarly; ++s)
+            if (s < nslot) fold(ml0[s], ov0[s]);
+#pragma unroll 4
+        for (int s = kEarly; s < nslot; ++s) {
             const int64_t rec = rec0 + (int64_t)s * G;
-            const float2 ml = __ldcg(&a.part_ml[rec]);
-            const float4 ov = __ldcg(reinterpret_cast<const float4 *>(a.part_o + rec * D) + d4);
-            const float w = ml.x != kPfNegInf ? exp2f(ml.x - M) : 0.0f;
-            L += ml.y * w;
-            O.x += ov.x * w; O.y += ov.y * w; O.z += ov.z * w; O.w += ov.w * w;
+            fold(__ldcg(&a.part_ml[rec]), __ldcg(reinterpret_cast<const float4 *>(a.part_o + rec * D) + d4));
         }
         const int64_t orow = (int64_t)i * a.Hq + (int64_t)g * G + hh;
         const float inv = L > 0.0f ? 1.0f / L : 0.0f;
@@ -791,14 +842,18 @@ bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
     BSA_CUDA_TRY(cudaMemsetAsync(w + L.qcount, 0, (size_t)d->Hkv * p->n_blocks * 4, st));
     // P1: selection
     auto smem1_for = [&](int nw) {
-        return ((size_t)a.nb * kPfCentStride + (size_t)nw * G * a.D + a.nb) * 4;
+        return ((size_t)a.nb * kPfCentStride + (size_t)nw * G * a.D + a.nb) * 4 + (size_t)nw * G * a.D * 2;
     };
-    const int nw1 = smem1_for(kPfSelWarps) <= kMaxSmemPerCta ? kPfSelWarps : kPfSelWarps / 2;
+    int nw1 = kPfSelWarps;
+    while (nw1 > 1 && smem1_for(nw1) > kMaxSmemPerCta) nw1 /= 2;
     const size_t smem1 = smem1_for(nw1);
     BSA_CUDA_TRY(cudaFuncSetAttribute(prefill_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem1));
+    // one wave: about num_sms / Hkv CTAs per KV head, the rows split evenly
+    const int ctas_per_head = std::max(1, num_sms() / d->Hkv);
+    a.sel_rows_per_warp = std::max(1, (int)div_up(Tq, (int64_t)ctas_per_head * nw1));
     BSA_CUDA_TRY(launch_pdl(prefill_select_kernel,
-                            dim3((unsigned)div_up(Tq, nw1 * kPfRowsPerWarp), (unsigned)d->Hkv),
+                            dim3((unsigned)div_up(Tq, nw1 * a.sel_rows_per_warp), (unsigned)d->Hkv),
                             dim3(32 * nw1), smem1, st, a));
     // P2: tile prefix over (KV head, block)
     prefill_tiles_kernel<<<1, 1024, 0, st>>>(a);
@@ -809,8 +864,8 @@ bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
     prefill_attend_kernel<<<num_sms(), kPfAttThreads, PfSmem::kBytes, st>>>(kp, vp, kl, vl, a);
     BSA_LAUNCH_CHECK();
     // P4: merge of every query's slots
-    BSA_CUDA_TRY(launch_pdl(prefill_merge_kernel, dim3((unsigned)Tq, (unsigned)d->Hkv), dim3(128), 0,
-                            st, a));
+    BSA_CUDA_TRY(launch_pdl(prefill_merge_kernel, dim3((unsigned)Tq, (unsigned)d->Hkv),
+                            dim3(kPfMergeThreads), 0, st, a));
     return BSA_OK;
 }
 

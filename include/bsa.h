@@ -268,8 +268,9 @@ BSA_API bsa_status bsa_decode_step(const bsa_kv_desc *desc, const float *q, void
  * are gathered and contracted against it together on the tensor cores, and
  * the partial results are merged per query by log-sum-exp.
  * Q: device bf16 [Tq][Hq][D]; out: device fp32 [Tq][Hq][D]; lse: device fp32
- * [Tq][Hq] (may be NULL).  pos_limit = 0 makes the call dense causal
- * attention over [0, q_pos0 + i]. */
+ * [Tq][Hq] (may be NULL).  K, V, K_pos, V_pos, Q, out and the CENTROID_NORM
+ * summaries must be 16-byte aligned (BSA_ERR_ARG otherwise).  pos_limit = 0
+ * makes the call dense causal attention over [0, q_pos0 + i]. */
 BSA_API bsa_status bsa_prefill_grouped(const bsa_kv_desc *desc, const void *K, const void *V,
                                const bsa_sel_params *sel, const void *summaries,
                                const bsa_kv_desc *pos_desc, const void *K_pos, const void *V_pos,
