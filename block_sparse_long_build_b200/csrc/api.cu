@@ -20,6 +20,7 @@ bsa_status launch_decode(const bsa_kv_desc *, const float *, const void *, const
                          float *, uint32_t *, uint32_t *, void *, cudaStream_t, const DecAppend *);
 bool decode_can_fuse_append(const bsa_kv_desc *);
 int decode_nsplit(const bsa_kv_desc *, int, int);
+int decode_kernel_count(const bsa_kv_desc *, int, int);
 size_t decode_scratch_bytes(const bsa_kv_desc *, int);
 bsa_status launch_prefill(const bsa_kv_desc *, const void *, const void *, const bsa_sel_params *,
                           const void *, const bsa_kv_desc *, const void *, const void *,
@@ -183,6 +184,11 @@ int32_t bsa_max_selected(const bsa_kv_desc *d, const bsa_sel_params *p) {
 int32_t bsa_max_ranges(const bsa_kv_desc *d, const bsa_sel_params *p) {
     if (!desc_ok(d) || !sel_ok(d, p)) return -1;
     return max_ranges(d, p);
+}
+
+int32_t bsa_decode_kernels(const bsa_kv_desc *d, const bsa_sel_params *p, int32_t tokens_hint) {
+    if (!desc_ok(d) || !sel_ok(d, p) || tokens_hint < 0) return BSA_ERR_ARG;
+    return decode_kernel_count(d, std::max(tokens_hint, 1), max_ranges(d, p));
 }
 
 size_t bsa_workspace_size(const bsa_kv_desc *d, const bsa_sel_params *p, int op, int32_t n_queries,

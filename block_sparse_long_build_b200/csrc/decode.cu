@@ -784,12 +784,27 @@ static bool use_tc(const bsa_kv_desc *d) {
 
 bool decode_can_fuse_append(const bsa_kv_desc *d) { return use_tc(d); }
 
+constexpr int kMinWarpPieces = 8;   // pieces per warp below which more splits stop paying
+
+// Few segments: even the largest clusters would leave SMs idle.  Their splits
+// are not clustered (so there can be more of them) and the merge kernel
+// combines them.
+static bool few_segments(const bsa_kv_desc *d) {
+    return (int64_t)d->B * d->Hkv * kMaxClusterSplits < num_sms();
+}
+
 int decode_nsplit(const bsa_kv_desc *d, int tokens_hint, int max_ranges) {
     const int nseg = d->B * d->Hkv;
     const int64_t pieces = div_up(tokens_hint > 0 ? tokens_hint : 1, kPiece) + max_ranges;
     const int slots = num_sms() * (use_tc(d) ? 2 : 4);
     int nsplit = std::max(1, slots / std::max(nseg, 1));
-    if (use_tc(d)) nsplit = std::min(nsplit, kMaxClusterSplits);   // one cluster per segment
+    if (use_tc(d)) {
+        if (few_segments(d))   // every resident slot, while warps keep enough pieces
+            nsplit = (int)std::min<int64_t>(
+                nsplit, std::max<int64_t>(kMaxClusterSplits, pieces / (kDecWarps * kMinWarpPieces)));
+        else
+            nsplit = std::min(nsplit, kMaxClusterSplits);   // one cluster per segment
+    }
     nsplit = (int)std::min<int64_t>(nsplit, div_up(pieces, kDecWarps));
     return std::max(1, nsplit);
 }
@@ -823,6 +838,37 @@ static int cluster_splits(const void *kern, int smem, int nseg, int max_c, cudaL
     }
     cache.push_back({{kern, smem, nseg, max_c, dev}, best});
     return best;
+}
+
+// Kernels one launch_decode issues: 1 when the splits merge inside clusters
+// (or there is one split), 2 when the merge kernel follows.  Mirrors the
+// choice launch_decode makes.
+int decode_kernel_count(const bsa_kv_desc *d, int tokens_hint, int max_ranges) {
+    const int nsplit = decode_nsplit(d, tokens_hint, max_ranges);
+    if (nsplit <= 1) return 1;
+    if (!use_tc(d) || few_segments(d)) return 2;
+    auto clusters_fit = [&](auto kern_cluster, int smem) -> bool {
+        if (cudaFuncSetAttribute(kern_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(kern_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.blockDim = dim3(kDecThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cluster_splits(reinterpret_cast<const void *>(kern_cluster), smem, d->B * d->Hkv, nsplit,
+                              cfg) > 1;
+    };
+    const bool fit = d->D == 128
+                         ? clusters_fit(decode_tc_kernel<2, kTcStages, true>, TcSmem<2, kTcStages>::kBytes)
+                         : clusters_fit(decode_tc_kernel<1, 2 * kTcStages, true>, TcSmem<1, 2 * kTcStages>::kBytes);
+    return fit ? 1 : 2;
 }
 
 size_t decode_scratch_bytes(const bsa_kv_desc *d, int nsplit) {
@@ -860,7 +906,7 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
         bool clustered = false;
         auto go_tc = [&](auto kern_plain, auto kern_cluster, int smem) -> bsa_status {
             BSA_CUDA_TRY(cudaFuncSetAttribute(kern_plain, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-            if (a.nsplit > 1) {
+            if (a.nsplit > 1 && !few_segments(d)) {
                 BSA_CUDA_TRY(cudaFuncSetAttribute(kern_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
                 BSA_CUDA_TRY(cudaFuncSetAttribute(kern_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
                 cudaLaunchConfig_t cfg = {};

@@ -22,7 +22,7 @@ BSA_F32, BSA_BF16 = 0, 1
 BSA_OP_SELECT, BSA_OP_DECODE, BSA_OP_PREFILL, BSA_OP_APPEND = 0, 1, 2, 3
 
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_summary_blocks", "bsa_summary_bytes",
-            "bsa_max_selected", "bsa_max_ranges", "bsa_workspace_size", "bsa_build_summaries",
+            "bsa_max_selected", "bsa_max_ranges", "bsa_decode_kernels", "bsa_workspace_size", "bsa_build_summaries",
             "bsa_select", "bsa_decode", "bsa_decode_noalloc", "bsa_append_kv", "bsa_decode_step",
             "bsa_prefill_grouped")
 
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
             "bsa_summary_bytes": (SZ, [pd, pp, ctypes.c_int]),
             "bsa_max_selected": (I32, [pd, pp]),
             "bsa_max_ranges": (I32, [pd, pp]),
+            "bsa_decode_kernels": (I32, [pd, pp, I32]),
             "bsa_workspace_size": (SZ, [pd, pp, ctypes.c_int, I32, I32]),
             "bsa_build_summaries": (ctypes.c_int, [pd, P, pp, ctypes.c_int, I32, I32, P, P]),
             "bsa_select": (ctypes.c_int, [pd, P, P, ctypes.c_int, pp, P, I32, P, P, I32, P, P, P,
@@ -145,6 +146,13 @@ def bsa_max_selected(desc, sel) -> int:
 
 def bsa_max_ranges(desc, sel) -> int:
     return lib().bsa_max_ranges(ctypes.byref(desc), ctypes.byref(sel))
+
+
+def bsa_decode_kernels(desc, sel, tokens_hint) -> int:
+    r = lib().bsa_decode_kernels(ctypes.byref(desc), ctypes.byref(sel), tokens_hint)
+    if r < 0:
+        raise BsaError("bsa_decode_kernels", r)
+    return r
 
 
 def bsa_workspace_size(desc, sel, op, n_queries=0, tokens_hint=0) -> int:

@@ -59,6 +59,7 @@ class DecodeSession:
         self.ranges = torch.zeros(nseg, self.max_ranges, 2, dtype=torch.int32, device=dev)
         self.n_ranges = torch.zeros(nseg, dtype=torch.int32, device=dev)
         self.tokens_hint = self.token_bound()
+        self.decode_kernels = N.bsa_decode_kernels(self.desc, self.sel, self.tokens_hint)
         ws = max(N.bsa_workspace_size(self.desc, self.sel, op, 0, self.tokens_hint)
                  for op in (N.BSA_OP_SELECT, N.BSA_OP_DECODE, N.BSA_OP_APPEND))
         self.ws = torch.zeros(ws, dtype=torch.uint8, device=dev)
@@ -208,11 +209,12 @@ class DecodeSession:
 
     def launches_per_step(self, t: int) -> int:
         """Library kernels one step launches: append, the two selection kernels
-        (scoring, picking) on refresh steps, and the decode; a fused step is one
-        launch."""
+        (scoring, picking) on refresh steps, and the decode (one kernel, or two
+        when the split merge is a kernel of its own); a fused step folds the
+        append into the decode."""
         if t % self.cfg.refresh == 0:
-            return 4
-        return 1 if self.fused and self.fuses() else 2
+            return 3 + self.decode_kernels
+        return self.decode_kernels + (0 if self.fused and self.fuses() else 1)
 
     def fuses(self) -> bool:
         """Whether bsa_decode_step runs as one launch for this workload."""

@@ -138,6 +138,15 @@ BSA_API size_t bsa_summary_bytes(const bsa_kv_desc *desc, const bsa_sel_params *
 BSA_API int32_t bsa_max_selected(const bsa_kv_desc *desc, const bsa_sel_params *sel);
 BSA_API int32_t bsa_max_ranges(const bsa_kv_desc *desc, const bsa_sel_params *sel);
 
+/* Kernels one bsa_decode call launches for this geometry and tokens_hint
+ * (the same values bsa_decode gets): 1 when the split-K partials merge
+ * inside the decode grid (one thread-block cluster per segment, or a single
+ * split), 2 when the merge kernel follows.  bsa_decode_step launches as many
+ * when it runs fused (bf16 K/V, D 64 or 128, G <= 8), one more otherwise.
+ * Reads the current device; a negative bsa_status on invalid arguments. */
+BSA_API int32_t bsa_decode_kernels(const bsa_kv_desc *desc, const bsa_sel_params *sel,
+                                   int32_t tokens_hint);
+
 /* Workspace bytes for `op`.  n_queries: query rows per call for
  * BSA_OP_PREFILL (ignored otherwise); tokens_hint: for BSA_OP_DECODE, an
  * upper bound on the tokens any segment's ranges cover (sizes the split-K
