@@ -99,6 +99,9 @@ def test_bad_arguments_rejected_on_host(lib):
     p2 = N.sel_params(16, topk=8, sink=-1)
     assert L.bsa_select(ctypes.byref(d), fake, fake, 2, ctypes.byref(p2), fake, 8, fake, fake,
                         64, fake, fake, fake, 1 << 30, None) == N.BSA_ERR_ARG
+    # kernel-count query: bad descriptor, negative token bound
+    assert L.bsa_decode_kernels(ctypes.byref(_desc(D=96)), ctypes.byref(p), 100) == N.BSA_ERR_ARG
+    assert L.bsa_decode_kernels(ctypes.byref(d), ctypes.byref(p), -1) == N.BSA_ERR_ARG
     # variable blocks without offsets
     p3 = N.sel_params(0, n_blocks=16, topk=-1, budget_tokens=100)
     assert L.bsa_summary_blocks(ctypes.byref(d), ctypes.byref(p3)) == -1

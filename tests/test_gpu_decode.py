@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+from block_sparse_long_build_b200 import native as N
 from block_sparse_long_build_b200 import workloads as W
 
 from gpu_harness import FixedDecodeCheck
@@ -145,3 +146,15 @@ def test_workspace_left_clean():
     nseg = chk.cfg.B * chk.cfg.Hkv
     assert ws[0] == 0                          # no device-side timeout
     assert np.all(ws[1:1 + 2 * nseg] == 0)     # select and decode counters
+
+
+def test_decode_kernel_count():
+    """Many segments merge inside clusters (one kernel); a single sequence of 8
+    KV heads cannot fill the GPU with clusters and takes the merge kernel."""
+    def desc(B):
+        L = 65536
+        return N.KvDesc(B=B, Hq=32, Hkv=8, D=128, kv_dtype=N.BSA_BF16, L_max=L, stride_b=8 * L * 128,
+                        stride_h=L * 128, stride_t=128)
+    p = N.sel_params(16, topk=-1, budget_tokens=4096, sink=256, window=1024)
+    assert N.bsa_decode_kernels(desc(4), p, 5400) == 1
+    assert N.bsa_decode_kernels(desc(1), p, 5400) == 2
