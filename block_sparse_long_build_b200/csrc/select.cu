@@ -316,39 +316,37 @@ struct PickSmem {
 
 // One warp takes, one at a time, the best remaining candidate (highest key,
 // then lowest index) -- that fits in what is left of the budget when
-// `budget` >= 0 -- up to `limit` blocks, marking them in taken[].  Keys and
-// visible counts of blocks lane + 32 r live in registers (nb <= 512).
+// `budget` >= 0 -- up to `limit` blocks, marking them in taken[].  A step is a
+// warp max of the live keys and a warp min of the indices holding it (both
+// redux.sync); a taken block's key is cleared, and under a budget so is every
+// key whose visible rows no longer fit (what is left only shrinks).  Keys
+// and visible counts of blocks lane + 32 r live in registers (nb <= 512).
 __device__ __forceinline__ void warp_walk_regs(const uint32_t *keys, const int32_t *visb, unsigned char *taken,
                                                int nb, int limit, int budget, int lane) {
     uint32_t wk[kPickWarpKeys];
     int wv[kPickWarpKeys];
+    int remaining = budget;
 #pragma unroll
     for (int r = 0; r < kPickWarpKeys; ++r) {
         const int j = lane + 32 * r;
         wk[r] = j < nb ? keys[j] : 0u;
         wv[r] = j < nb && budget >= 0 ? visb[j] : 0;
+        if (budget >= 0 && wv[r] > remaining) wk[r] = 0u;
     }
-    int remaining = budget;
     for (int n = 0; n < limit; ++n) {
-        unsigned long long best = 0ull;
+        uint32_t lm = 0u;
 #pragma unroll
-        for (int r = 0; r < kPickWarpKeys; ++r)
-            if (wk[r] && (budget < 0 || wv[r] <= remaining)) {
-                const unsigned long long c =
-                    ((unsigned long long)wk[r] << 32) | (0xffffffffu - (uint32_t)(lane + 32 * r));
-                best = c > best ? c : best;
-            }
+        for (int r = 0; r < kPickWarpKeys; ++r) lm = max(lm, wk[r]);
+        const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
+        if (m == 0u) break;
+        int cand = 0x7fffffff;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-            best = other > best ? other : best;
-        }
-        if (best == 0ull) break;
-        const int j = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
+        for (int r = kPickWarpKeys - 1; r >= 0; --r) cand = wk[r] == m ? lane + 32 * r : cand;
+        const int j = __reduce_min_sync(0xffffffffu, cand);
         if (budget >= 0) remaining -= visb[j];
 #pragma unroll
         for (int r = 0; r < kPickWarpKeys; ++r)
-            if (lane + 32 * r == j) wk[r] = 0u;
+            if (lane + 32 * r == j || (budget >= 0 && wv[r] > remaining)) wk[r] = 0u;
         if (lane == 0) taken[j] = 1;
     }
 }
@@ -358,19 +356,15 @@ __device__ void warp_walk_smem(const uint32_t *keys, const int32_t *visb, unsign
                                int limit, int budget, int lane) {
     int remaining = budget;
     for (int n = 0; n < limit; ++n) {
-        unsigned long long best = 0ull;
+        uint32_t lm = 0u;
         for (int j = lane; j < nb; j += 32)
-            if (keys[j] && !taken[j] && (budget < 0 || visb[j] <= remaining)) {
-                const unsigned long long c = ((unsigned long long)keys[j] << 32) | (0xffffffffu - (uint32_t)j);
-                best = c > best ? c : best;
-            }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-            best = other > best ? other : best;
-        }
-        if (best == 0ull) break;
-        const int j = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
+            if (keys[j] && !taken[j] && (budget < 0 || visb[j] <= remaining)) lm = max(lm, keys[j]);
+        const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
+        if (m == 0u) break;
+        int cand = 0x7fffffff;
+        for (int j = lane; j < nb && cand == 0x7fffffff; j += 32)
+            if (keys[j] == m && !taken[j] && (budget < 0 || visb[j] <= remaining)) cand = j;
+        const int j = __reduce_min_sync(0xffffffffu, cand);
         if (budget >= 0) remaining -= visb[j];
         if (lane == 0) taken[j] = 1;
         __syncwarp();
@@ -584,31 +578,35 @@ __global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
 }
 
 
-// The same selection for segments of at most 32 * kPickWarpKeys blocks, by one
-// warp per segment with no CTA barrier: lane l holds blocks l + 32 r; the walk
-// takes the best remaining candidate (highest key, then lowest index; for a
-// budget, the best that still fits) until k blocks or nothing fits; a ballot
-// per r compacts the taken blocks in index order; lane 0 merges the forced
-// ranges and the blocks' ranges.  Shared memory: sel, lo, hi [max_sel] ints.
+// The same selection for segments of at most 32 * kPickSmallKeys blocks, by one
+// warp per segment with no CTA barrier: lane l holds blocks l + 32 r in
+// registers; the walk takes the best remaining candidate (highest key, then
+// lowest index; for a budget, the best that still fits: keys that no longer
+// fit are cleared) with a redux.sync max and min per step until k blocks or
+// nothing is left; a ballot per r compacts the taken blocks in index order
+// straight into their place among the forced ranges; the merged ranges come
+// from a warp scan (running maximum of the ends), 32 items per pass.
+// Shared memory: (lo, hi) of max_sel + 2 items.
+constexpr int kPickSmallKeys = 32;
+
 __global__ void __launch_bounds__(32) pick_small_kernel(SelArgs a) {
     extern __shared__ __align__(16) unsigned char psm[];
-    int32_t *sel = reinterpret_cast<int32_t *>(psm);
-    int32_t *slo = sel + a.max_sel, *shi = slo + a.max_sel;
+    int2 *items = reinterpret_cast<int2 *>(psm);
     const int s = blockIdx.x, b = s / a.Hkv, lane = threadIdx.x;
     const int nb = a.nb_total;
     const int32_t *off = a.offsets ? a.offsets + (int64_t)s * (nb + 1) : nullptr;
     pdl_wait();   // keys and visible counts from score_kernel
-    uint32_t wk[kPickWarpKeys];
-    int wv[kPickWarpKeys];
+    uint32_t wk[kPickSmallKeys];
+    int wv[kPickSmallKeys];
 #pragma unroll
-    for (int r = 0; r < kPickWarpKeys; ++r) {
+    for (int r = 0; r < kPickSmallKeys; ++r) {
         const int j = lane + 32 * r;
         wk[r] = j < nb ? a.keys[(int64_t)s * nb + j] : 0u;
         wv[r] = off && j < nb ? a.vis[(int64_t)s * nb + j] : 0;
     }
     // forced token ranges (every lane computes the same), sorted and merged
     const int n = min(max(a.cur_len[b], 0), a.L_max);
-    int f_lo[3] = {0, 0, 0}, f_hi[3] = {0, 0, 0}, nf = 0;
+    int f_lo[2] = {0, 0}, f_hi[2] = {0, 0}, nf = 0;
     if (off) {
         if (n > a.local_start) { f_lo[0] = max(a.local_start, 0); f_hi[0] = n; nf = 1; }
     } else {
@@ -625,7 +623,7 @@ __global__ void __launch_bounds__(32) pick_small_kernel(SelArgs a) {
     // candidates: keys > 0 and (fixed blocks) not wholly inside the forced set
     int my_c = 0;
 #pragma unroll
-    for (int r = 0; r < kPickWarpKeys; ++r) {
+    for (int r = 0; r < kPickSmallKeys; ++r) {
         if (wk[r] && !off) {
             const int64_t r0 = (int64_t)(lane + 32 * r) * a.S, r1 = r0 + a.S;
 #pragma unroll
@@ -634,84 +632,98 @@ __global__ void __launch_bounds__(32) pick_small_kernel(SelArgs a) {
         }
         my_c += wk[r] != 0u;
     }
-    int n_cand = my_c;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n_cand += __shfl_xor_sync(0xffffffffu, n_cand, o);
+    const int n_cand = __reduce_add_sync(0xffffffffu, my_c);
     const bool greedy = off && a.topk < 0;
     const int limit = greedy ? a.max_sel : min(min(a.topk >= 0 ? a.topk : a.budget / a.S, n_cand), a.max_sel);
     int remaining = a.budget;
+    if (greedy) {
+#pragma unroll
+        for (int r = 0; r < kPickSmallKeys; ++r)
+            if (wv[r] > remaining) wk[r] = 0u;
+    }
     uint32_t taken = 0;   // bit r: block lane + 32 r
     for (int t = 0; t < limit; ++t) {
-        unsigned long long best = 0ull;
+        uint32_t lm = 0u;
 #pragma unroll
-        for (int r = 0; r < kPickWarpKeys; ++r)
-            if (wk[r] && !((taken >> r) & 1u) && (!greedy || wv[r] <= remaining)) {
-                const unsigned long long c =
-                    ((unsigned long long)wk[r] << 32) | (0xffffffffu - (uint32_t)(lane + 32 * r));
-                best = c > best ? c : best;
-            }
+        for (int r = 0; r < kPickSmallKeys; ++r) lm = max(lm, wk[r]);
+        const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
+        if (m == 0u) break;
+        int cand = 0x7fffffff;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-            best = other > best ? other : best;
-        }
-        if (best == 0ull) break;
-        const int j = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffu));
+        for (int r = kPickSmallKeys - 1; r >= 0; --r) cand = wk[r] == m ? lane + 32 * r : cand;
+        const int j = __reduce_min_sync(0xffffffffu, cand);
         int vj = 0;
 #pragma unroll
-        for (int r = 0; r < kPickWarpKeys; ++r)
-            if (lane + 32 * r == j) { taken |= 1u << r; vj = wv[r]; }
-        remaining -= __shfl_sync(0xffffffffu, vj, j & 31);
-    }
-    // index-ordered compaction
-    int n_sel = 0;
+        for (int r = 0; r < kPickSmallKeys; ++r)
+            if (lane + 32 * r == j) { taken |= 1u << r; wk[r] = 0u; vj = wv[r]; }
+        if (greedy) {
+            remaining -= __shfl_sync(0xffffffffu, vj, j & 31);
 #pragma unroll
-    for (int r = 0; r < kPickWarpKeys; ++r) {
-        const uint32_t m = __ballot_sync(0xffffffffu, (taken >> r) & 1u);
+            for (int r = 0; r < kPickSmallKeys; ++r)
+                if (wv[r] > remaining) wk[r] = 0u;
+        }
+    }
+    // index-ordered compaction, each block written at its place among the
+    // forced ranges (a forced range comes first on equal starts)
+    int n_sel = 0, below[2] = {0, 0};   // below[f]: taken blocks starting before f_lo[f]
+#pragma unroll
+    for (int r = 0; r < kPickSmallKeys; ++r) {
+        const uint32_t mk = __ballot_sync(0xffffffffu, (taken >> r) & 1u);
         if ((taken >> r) & 1u) {
-            const int p = n_sel + __popc(m & ((1u << lane) - 1u));
+            const int p = n_sel + __popc(mk & ((1u << lane) - 1u));
             const int jj = lane + 32 * r;
+            int lo, hi;
+            if (off) { lo = min(max(off[jj], 0), a.L_max); hi = lo + wv[r]; }
+            else { lo = jj * a.S; hi = lo + a.S; }
+            int before = 0;
+#pragma unroll
+            for (int f = 0; f < 2; ++f) {
+                before += f < nf && f_lo[f] <= lo;
+                below[f] += f < nf && lo < f_lo[f];
+            }
             if (p < a.max_sel) {
-                int lo, hi;
-                if (off) { lo = min(max(off[jj], 0), a.L_max); hi = lo + wv[r]; }
-                else { lo = jj * a.S; hi = lo + a.S; }
-                sel[p] = jj;
-                slo[p] = lo;
-                shi[p] = hi;
+                a.sel_blocks[(int64_t)s * a.max_sel + p] = jj;
+                items[p + before] = make_int2(lo, hi);
             }
         }
-        n_sel += __popc(m);
+        n_sel += __popc(mk);
     }
     n_sel = min(n_sel, a.max_sel);
+#pragma unroll
+    for (int f = 0; f < 2; ++f) {
+        const int nbelow = __reduce_add_sync(0xffffffffu, below[f]);
+        if (f < nf && lane == 0) items[f + nbelow] = make_int2(f_lo[f], f_hi[f]);
+    }
     __syncwarp();
-    for (int i = lane; i < n_sel; i += 32) a.sel_blocks[(int64_t)s * a.max_sel + i] = sel[i];
+    // ranges: item i opens a range when it starts after every earlier item
+    // has ended; a range ends at the running maximum of its last item
+    const int M = n_sel + nf;
+    int32_t *R = a.ranges + (int64_t)s * a.max_ranges * 2;
+    int nr = 0, carry = kIntMin;
+    for (int c0 = 0; c0 < M; c0 += 32) {
+        const int i = c0 + lane;
+        const int2 it = i < M ? items[i] : make_int2(0, kIntMin);
+        int pm = it.y;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, pm, o);
+            if (lane >= o) pm = max(pm, v);
+        }
+        pm = max(pm, carry);
+        int prev = __shfl_up_sync(0xffffffffu, pm, 1);
+        if (lane == 0) prev = carry;
+        const bool start = i < M && (i == 0 || it.x > prev);
+        const uint32_t sm = __ballot_sync(0xffffffffu, start);
+        const int rid = nr + __popc(sm & ((2u << lane) - 1u)) - 1;   // range of item i
+        if (i < M) {
+            if (start && rid < a.max_ranges) R[2 * rid] = it.x;
+            const bool last = i == M - 1 || items[i + 1].x > pm;
+            if (last && rid < a.max_ranges) R[2 * rid + 1] = pm;
+        }
+        nr += __popc(sm);
+        carry = __shfl_sync(0xffffffffu, pm, 31);
+    }
     if (lane == 0) {
-        // ranges: forced and selected ranges in start order (forced first on
-        // equal starts); a range grows while the next item starts at or
-        // before its end
-        int32_t *R = a.ranges + (int64_t)s * a.max_ranges * 2;
-        int nr = 0, cs = 0, ce = 0, fi = 0, si = 0;
-        bool open = false;
-        while (fi < nf || si < n_sel) {
-            const int blo = si < n_sel ? slo[si] : 0, bhi = si < n_sel ? shi[si] : 0;
-            const int fl = fi == 0 ? f_lo[0] : f_lo[1], fh = fi == 0 ? f_hi[0] : f_hi[1];
-            int lo, hi;
-            if (fi < nf && (si >= n_sel || fl <= blo)) { lo = fl; hi = fh; ++fi; }
-            else { lo = blo; hi = bhi; ++si; }
-            if (open && lo <= ce) {
-                ce = max(ce, hi);
-            } else {
-                if (open) {
-                    if (nr < a.max_ranges) { R[2 * nr] = cs; R[2 * nr + 1] = ce; }
-                    ++nr;
-                }
-                cs = lo; ce = hi; open = true;
-            }
-        }
-        if (open) {
-            if (nr < a.max_ranges) { R[2 * nr] = cs; R[2 * nr + 1] = ce; }
-            ++nr;
-        }
         a.n_ranges[s] = min(nr, a.max_ranges);
         a.sel_count[s] = n_sel;
     }
@@ -792,10 +804,12 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
         BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(kPickThreads), smem2, st, a));
         return BSA_OK;
     };
-    // one warp per segment for small top-k problems; the token budget walk
-    // (variable blocks) measured faster in the CTA kernel
-    if (nb_total <= 32 * kPickWarpKeys && !variable) {
-        const size_t smem3 = (size_t)max_sel * 12;
+    // one warp per segment for small top-k problems (a long walk, or the
+    // token budget walk over variable blocks, measured faster in the CTA
+    // kernel)
+    const int64_t k_host = p->topk >= 0 ? p->topk : (p->block_size > 0 ? p->budget_tokens / p->block_size : 0);
+    if (nb_total <= 32 * kPickSmallKeys && !variable && k_host <= 32) {
+        const size_t smem3 = (size_t)(max_sel + 4) * 8;
         BSA_CUDA_TRY(launch_pdl(pick_small_kernel, dim3((unsigned)nseg), dim3(32), smem3, st, a));
         return BSA_OK;
     }

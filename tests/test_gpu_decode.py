@@ -42,8 +42,10 @@ CASES = {
                      block_size=64, topk=5, n_needles=3, steps=2),
     # MSA-shaped: blocks of 128, top-16, current block, clustered keys
     "msa_small": _cfg(W.msa(0), B=2, Hkv=2, Hq=8, L=128 * 40 + 50, steps=3),
-    # the same with more than 512 blocks per segment (the CTA-wide radix pick)
-    "msa_many_blocks": _cfg(W.msa(0), B=1, Hkv=2, Hq=8, L=128 * 600 + 17, steps=2),
+    # 600 blocks per segment: the one-warp pick with keys in every register slot
+    "msa_600_blocks": _cfg(W.msa(0), B=1, Hkv=2, Hq=8, L=128 * 600 + 17, steps=2),
+    # more than 1,024 blocks per segment (the CTA-wide radix pick)
+    "msa_many_blocks": _cfg(W.msa(0), B=1, Hkv=2, Hq=8, L=128 * 1100 + 17, steps=2),
 }
 
 
