@@ -27,6 +27,11 @@ What the oracle computes, with the page (title, section) each step follows:
   the blocks a token budget admits; ties go to the lower block index.
 * Exact softmax attention over the selected tokens in fp64 (Module 14,
   Exercise 14.1, attention with an additive mask).
+* The semantic index ("Semantic blocks for sparse attention", first section):
+  spherical k-means over the unit keys (Lloyd rounds from given starting
+  keys, largest fp32 dot wins, lowest centre on ties, normalised-mean update,
+  an empty cluster keeps its centre) and the block-ordered store (clusters in
+  index order, positions ascending within a cluster).
 
 The fp32 arithmetic that decides the selection follows a fixed order written
 out in ``oracle.c``; everything compared with a tolerance is fp64.
@@ -34,7 +39,10 @@ out in ``oracle.c``; everything compared with a tolerance is fp64.
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 except the semantic-centroid arithmetic's exact fp32 rounding, whose pins are
 invariants only (unit norm, identical-key blocks); no page prints a worked
-example for it.
+example for it.  The k-means is pinned by recovery of well-separated planted
+clusters, agreement with an independent fp64 restatement on an input without
+near ties, and the tie and empty-cluster rules; its exact fp32 rounding is
+likewise unpinned by any printed example.
 """
 from __future__ import annotations
 
@@ -83,6 +91,10 @@ def _lib():
             lib.oracle_block_scores.restype = None
             lib.oracle_attend_rows.argtypes = [P, I, I, P, P, I, L, P, L, D, P, P]
             lib.oracle_attend_rows.restype = None
+            lib.oracle_spherical_kmeans.argtypes = [P, I, L, I, L, I, I, P, P, P, P, P]
+            lib.oracle_spherical_kmeans.restype = None
+            lib.oracle_kmeans_assign.argtypes = [P, I, L, I, P, L, P, I, P]
+            lib.oracle_kmeans_assign.restype = None
             _LIB = lib
     return _LIB
 
@@ -352,3 +364,45 @@ def semantic_select_positions(q_grp, Kpos_seg, labels, n_blocks: int, pos_limit:
     pos = [order[offs[j]:offs[j] + visible[j]] for j in sel]
     pos = np.sort(np.concatenate(pos)) if pos else np.zeros(0, np.int64)
     return sel, pos.astype(np.int64), ties, centroids
+
+
+# --------------------------------------------------------------------------
+# Semantic index: spherical k-means and the block-ordered store
+# --------------------------------------------------------------------------
+
+def spherical_kmeans(K_seg: np.ndarray, k: int, iters: int, init):
+    """Spherical k-means over one segment's keys [L, D] ("Semantic blocks for
+    sparse attention", first section: keys are grouped by spherical k-means
+    and each group is stored together).  Reading taken where the page is
+    silent: start from the unit keys at rows `init` (k distinct rows),
+    `iters` assignments (largest fp32 dot with a unit centre, lowest centre
+    index on ties) with the normalised-mean update between them, an empty
+    cluster keeping its centre.
+
+    Returns (centres [k, D] f32, labels [L] i32, offsets [k+1] i32, order [L]
+    i32): the rows of cluster j in the block-ordered store are
+    offsets[j]..offsets[j+1], and order[i] is the original position of
+    block-ordered row i (clusters in index order, positions ascending)."""
+    K_seg, ld = _rows2d(K_seg)
+    L, D = K_seg.shape
+    init = np.ascontiguousarray(init, dtype=np.int32)
+    assert init.shape == (k,) and len(set(init.tolist())) == k and init.min() >= 0 and init.max() < L
+    C = np.zeros((k, D), np.float32)
+    labels = np.zeros(L, np.int32)
+    offsets = np.zeros(k + 1, np.int32)
+    order = np.zeros(L, np.int32)
+    _lib().oracle_spherical_kmeans(_ptr(K_seg), _kv_dtype(K_seg), ld, D, L, k, iters, _ptr(init),
+                                   _ptr(C), _ptr(labels), _ptr(offsets), _ptr(order))
+    return C, labels, offsets, order
+
+
+def kmeans_assign(K_seg: np.ndarray, rows, C: np.ndarray):
+    """The assignment step alone for the keys at `rows` against unit centres
+    C [k, D] (same arithmetic as ``spherical_kmeans``)."""
+    K_seg, ld = _rows2d(K_seg)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    C = np.ascontiguousarray(C, dtype=np.float32)
+    out = np.zeros(len(rows), np.int32)
+    _lib().oracle_kmeans_assign(_ptr(K_seg), _kv_dtype(K_seg), ld, K_seg.shape[1], _ptr(rows), len(rows),
+                                _ptr(C), C.shape[0], _ptr(out))
+    return out

@@ -201,3 +201,103 @@ void oracle_attend_rows(const float *q /* [G][D] */, int G, int D,
     }
     free(logit);
 }
+
+/* [SEM] "A block groups similar keys from different parts of the request":
+ * the blocks come from spherical k-means over the L2-normalised keys; a
+ * block is one cluster, its keys stored together (sorted by cluster, then by
+ * original position), its centre the normalised mean of its unit keys.
+ *
+ * The page gives no iteration count, start or tie rule; this is the reading
+ * taken (plain Lloyd iterations on the unit sphere):
+ *   u_r     = k_r / ||k_r|| (a zero key stays zero), as in the centres above
+ *   c_j     = u_{init[j]} to start
+ *   iters rounds: every key goes to the centre with the largest u_r . c_j
+ *           (fp32 fma chain over i = 0..D-1; the lowest j on equal dots);
+ *           between rounds each centre becomes the normalised mean of its
+ *           keys' unit vectors summed in position order (the normalised
+ *           centroid arithmetic above); an empty cluster keeps its centre.
+ * So `iters` assignments and iters - 1 updates: the labels returned are
+ * those of the last assignment against the centres returned.
+ * offsets[j] .. offsets[j+1] are cluster j's rows in the block-ordered store;
+ * order[i] is the original position of block-ordered row i. */
+void oracle_spherical_kmeans(const void *K, int dtype, int64_t ld, int D, int64_t L, int k,
+                             int iters, const int32_t *init, float *C /* [k][D] */,
+                             int32_t *labels /* [L] */, int32_t *offsets /* [k+1] */,
+                             int32_t *order /* [L] */) {
+    float *U = (float *)malloc(sizeof(float) * (size_t)L * (size_t)D);
+    float *key = (float *)malloc(sizeof(float) * (size_t)D);
+    float *acc = (float *)malloc(sizeof(float) * (size_t)D);
+    int64_t *cnt = (int64_t *)calloc((size_t)k, sizeof(int64_t));
+    int64_t *fill = (int64_t *)calloc((size_t)k, sizeof(int64_t));
+    for (int64_t r = 0; r < L; ++r) {
+        for (int i = 0; i < D; ++i) key[i] = elem_f(K, dtype, r * ld + i);
+        float nr = norm_f32(key, D);
+        for (int i = 0; i < D; ++i) U[r * D + i] = nr > 0.0f ? key[i] / nr : 0.0f;
+    }
+    for (int j = 0; j < k; ++j)
+        for (int i = 0; i < D; ++i) C[(int64_t)j * D + i] = U[(int64_t)init[j] * D + i];
+    for (int it = 0; it < iters; ++it) {
+        /* assignment */
+        for (int64_t r = 0; r < L; ++r) {
+            float best = -INFINITY;
+            int lab = 0;
+            for (int j = 0; j < k; ++j) {
+                float dot = 0.0f;
+                for (int i = 0; i < D; ++i) dot = fmaf(U[r * D + i], C[(int64_t)j * D + i], dot);
+                if (dot > best) { best = dot; lab = j; }
+            }
+            labels[r] = lab;
+        }
+        if (it == iters - 1) break;
+        /* update: clusters summed over their keys in position order */
+        for (int j = 0; j < k; ++j) {
+            int64_t n = 0;
+            for (int i = 0; i < D; ++i) acc[i] = 0.0f;
+            for (int64_t r = 0; r < L; ++r) {
+                if (labels[r] != j) continue;
+                ++n;
+                for (int i = 0; i < D; ++i) acc[i] = acc[i] + U[r * D + i];
+            }
+            if (n == 0) continue;   /* an empty cluster keeps its centre */
+            float *c = C + (int64_t)j * D;
+            for (int i = 0; i < D; ++i) c[i] = acc[i] / (float)n;
+            float nc = norm_f32(c, D);
+            for (int i = 0; i < D; ++i) c[i] = nc > 0.0f ? c[i] / nc : 0.0f;
+        }
+    }
+    /* block-ordered store: clusters in index order, positions ascending */
+    for (int64_t r = 0; r < L; ++r) ++cnt[labels[r]];
+    offsets[0] = 0;
+    for (int j = 0; j < k; ++j) offsets[j + 1] = offsets[j] + (int32_t)cnt[j];
+    for (int64_t r = 0; r < L; ++r) {
+        const int j = labels[r];
+        order[offsets[j] + fill[j]++] = (int32_t)r;
+    }
+    free(U);
+    free(key);
+    free(acc);
+    free(cnt);
+    free(fill);
+}
+
+/* The assignment alone, for sampled keys against given centres (the same
+ * arithmetic as above): labels[s] = argmax_j u_{rows[s]} . c_j. */
+void oracle_kmeans_assign(const void *K, int dtype, int64_t ld, int D, const int64_t *rows,
+                          int64_t n, const float *C, int k, int32_t *labels) {
+    float *key = (float *)malloc(sizeof(float) * (size_t)D);
+    for (int64_t s = 0; s < n; ++s) {
+        const int64_t r = rows[s];
+        for (int i = 0; i < D; ++i) key[i] = elem_f(K, dtype, r * ld + i);
+        float nr = norm_f32(key, D);
+        for (int i = 0; i < D; ++i) key[i] = nr > 0.0f ? key[i] / nr : 0.0f;
+        float best = -INFINITY;
+        int lab = 0;
+        for (int j = 0; j < k; ++j) {
+            float dot = 0.0f;
+            for (int i = 0; i < D; ++i) dot = fmaf(key[i], C[(int64_t)j * D + i], dot);
+            if (dot > best) { best = dot; lab = j; }
+        }
+        labels[s] = lab;
+    }
+    free(key);
+}

@@ -390,3 +390,86 @@ def test_near_ties_are_listed():
     # and the fp64 scores flag the pair as a near-tie across the cut
     assert s32[1] == s32[2]
     assert sel == [1] and ties == [(1, 2)]
+
+
+# --------------------------------------------------------------------------
+# Semantic index: spherical k-means ("Semantic blocks for sparse attention")
+# --------------------------------------------------------------------------
+
+def _planted(rng, L, k, D, noise):
+    cent = rng.standard_normal((k, D))
+    cent /= np.linalg.norm(cent, axis=1, keepdims=True)
+    lab = rng.integers(0, k, L)
+    X = (cent[lab] + noise * rng.standard_normal((L, D))).astype(np.float32)
+    return X, lab
+
+
+def test_kmeans_recovers_well_separated_clusters_and_stores_them_stably():
+    rng = np.random.default_rng(11)
+    L, k, D = 3000, 12, 64
+    X, lab = _planted(rng, L, k, D, 0.05)
+    init = np.array([np.flatnonzero(lab == j)[3] for j in range(k)])
+    C, labels, off, order = oracle.spherical_kmeans(X, k, 6, init)
+    assert (labels == lab).all()
+    # block-ordered store: a stable sort by cluster, CSR offsets from the counts
+    assert (order == np.argsort(labels, kind="stable")).all()
+    assert (off == np.concatenate([[0], np.cumsum(np.bincount(labels, minlength=k))])).all()
+    # centres are unit vectors near the planted directions
+    assert np.allclose(np.linalg.norm(C.astype(np.float64), axis=1), 1.0, atol=1e-6)
+    U = X / np.linalg.norm(X, axis=1, keepdims=True)
+    for j in range(k):
+        m = U[labels == j].mean(axis=0)
+        assert np.abs(C[j] - m / np.linalg.norm(m)).max() < 1e-5
+
+
+def _kmeans_fp64(X, k, iters, init):
+    """Independent restatement in fp64 with numpy (no fixed order)."""
+    U = X.astype(np.float64)
+    nr = np.linalg.norm(U, axis=1, keepdims=True)
+    U = np.where(nr > 0, U / np.where(nr > 0, nr, 1), 0)
+    C = U[init].copy()
+    margins = []
+    for it in range(iters):
+        dots = U @ C.T
+        lab = np.argmax(dots, axis=1)
+        srt = np.sort(dots, axis=1)
+        margins.append(srt[:, -1] - srt[:, -2])
+        if it == iters - 1:
+            break
+        for j in range(k):
+            if (lab == j).any():
+                m = U[lab == j].mean(axis=0)
+                C[j] = m / np.linalg.norm(m)
+    return C, lab, min(x.min() for x in margins)
+
+
+def test_kmeans_matches_an_fp64_restatement_without_near_ties():
+    rng = np.random.default_rng(5)
+    L, k, D, iters = 400, 5, 16, 4
+    X = rng.standard_normal((L, D)).astype(np.float32)
+    init = rng.choice(L, k, replace=False)
+    C64, lab64, margin = _kmeans_fp64(X, k, iters, init)
+    assert margin > 1e-5, "seed gives a near tie; the fp32 result could differ legitimately"
+    C, labels, _, _ = oracle.spherical_kmeans(X, k, iters, init)
+    assert (labels == lab64).all()
+    assert np.abs(C - C64).max() < 1e-5
+
+
+def test_kmeans_empty_cluster_keeps_its_centre_and_ties_go_low():
+    rng = np.random.default_rng(2)
+    L, D = 300, 32
+    X = rng.standard_normal((L, D)).astype(np.float32)
+    X[1] = X[0]            # two identical starting centres: every tie goes to 0
+    X[7] = 0.0             # a zero key: every dot is 0, so it goes to centre 0
+    init = np.array([0, 1, 2, 3])
+    # one assignment: centre 1 ties with centre 0 everywhere and loses
+    _, lab1, off1, _ = oracle.spherical_kmeans(X, 4, 1, init)
+    assert (lab1 != 1).all() and off1[2] - off1[1] == 0 and lab1[7] == 0
+    # the update in between leaves the empty centre where it was (it may win
+    # keys again once centre 0 has moved)
+    C, labels, _, _ = oracle.spherical_kmeans(X, 4, 2, init)
+    u1 = X[1] / np.float32(np.sqrt(np.sum(X[1].astype(np.float64) ** 2)))
+    assert np.abs(C[1] - u1).max() < 1e-6
+    assert np.abs(C[0] - u1).max() > 1e-3
+    # the assignment helper agrees with the last assignment
+    assert (oracle.kmeans_assign(X, np.arange(L), C) == labels).all()
