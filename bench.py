@@ -468,6 +468,78 @@ def run_prefill(args, device):
     }
 
 
+def run_index(args, device):
+    """The semantic index of the semantic-block configuration: spherical
+    k-means over every KV head's 524,288 position-ordered keys (256 clusters,
+    20 assignment rounds, one starting key per planted cluster) and the
+    block-ordered store gathered from it, one bsa_build_semantic_index call
+    plus one bsa_gather_rows call per run, timed with CUDA events after a
+    warm-up run."""
+    from block_sparse_long_build_b200 import build as Bld
+    from block_sparse_long_build_b200 import native as N
+    from block_sparse_long_build_b200 import workloads as W
+
+    Bld.build()
+    cfg = W.semantic(0)
+    wl = W.Workload(cfg, device)
+    B, H, L, k, D, iters = cfg.B, cfg.Hkv, cfg.L, cfg.n_blocks, cfg.D, 20
+    nseg = B * H
+    lab = wl.labels.reshape(nseg, L)
+    first = torch.full((nseg, k), L, dtype=torch.int64, device=device)
+    first.scatter_reduce_(1, lab, torch.arange(L, device=device).expand(nseg, L), reduce="amin")
+    init = first.to(torch.int32).contiguous()
+    src, dst = N.kv_desc(wl.Kpos, cfg.Hq), N.kv_desc(wl.K, cfg.Hq)
+    ws = torch.zeros(N.bsa_index_workspace_size(src, L, k), dtype=torch.uint8, device=device)
+    C = torch.empty(nseg, k, D, device=device)
+    labels = torch.empty(nseg, L, dtype=torch.int32, device=device)
+    offsets = torch.empty(nseg, k + 1, dtype=torch.int32, device=device)
+    order = torch.empty(nseg, L, dtype=torch.int32, device=device)
+    Kb, Vb = torch.empty_like(wl.K), torch.empty_like(wl.V)
+    flush = _flusher(device)
+
+    def run():
+        N.bsa_build_semantic_index(src, wl.Kpos, L, k, iters, init, C, labels, offsets, order, ws)
+        N.bsa_gather_rows(src, wl.Kpos, wl.Vpos, dst, Kb, Vb, order, L, 0)
+
+    for _ in range(max(1, args.warmup or 1)):
+        run()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    sampler.start()
+    times = []
+    for _ in range(max(1, args.steps or 3)):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    clocks = sampler.stop()
+    ms = float(sum(times) / len(times))
+    recovered = bool(torch.equal(labels.long(), lab))
+    # the assignment rounds dominate: L * k * D fmas per segment per round
+    flops = 2.0 * nseg * L * k * D * iters
+    tflops = flops / (ms / 1e3) / 1e12
+    # fp32 fma peak from the unit counts and the clock: 148 SMs x 128 lanes x
+    # 2 flops x the measured SM clock
+    sm_mhz = clocks.get("sm_mhz") or 1965.0
+    peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    return {
+        "metric": "semantic index build (spherical k-means + block-ordered store), keys per second",
+        "value": nseg * L / (ms / 1e3), "unit": "keys/s", "n_gpus": 1, "steps": len(times),
+        "warmup": max(1, args.warmup or 1), "ms_per_step": ms, "higher_is_better": True,
+        "dtype": "f32", "data": "synthetic", "planted_clusters_recovered": recovered,
+        "config": {"workload": f"semantic blocks: {nseg} KV heads x {L} keys, head_dim {D}, bf16 keys, "
+                               f"{k} clusters, {iters} assignment rounds",
+                   "l2": "flushed before each run"},
+        "roofline": {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x SM clock",
+                     "traffic": None},
+        "clocks": clocks,
+    }
+
+
 def _bf16_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -575,6 +647,8 @@ def main():
                     help="context of the prefill run (default: the configuration's 524,288)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--index", action="store_true",
+                    help="time the semantic index build (k-means + block-ordered store)")
     ap.add_argument("--case", choices=["decode", "select", "prefill"], default=None,
                     help="run one small profiling case instead of the bench (for ncu)")
     args = ap.parse_args()
@@ -594,6 +668,12 @@ def main():
             local = int(os.environ.get("LOCAL_RANK", "0"))
             torch.cuda.set_device(local)
             print(json.dumps(run_prefill(args, torch.device("cuda", local))), flush=True)
+        return 0
+    if args.index:
+        if rank == 0:
+            local = int(os.environ.get("LOCAL_RANK", "0"))
+            torch.cuda.set_device(local)
+            print(json.dumps(run_index(args, torch.device("cuda", local))), flush=True)
         return 0
     if args.impl == "reference":
         if rank != 0:

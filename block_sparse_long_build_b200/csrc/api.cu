@@ -27,6 +27,12 @@ bsa_status launch_prefill(const bsa_kv_desc *, const void *, const void *, const
                           const void *, int, int, float, float *, float *, uint32_t *, void *,
                           size_t, cudaStream_t);
 size_t prefill_ws_bytes(const bsa_kv_desc *, const bsa_sel_params *, int);
+size_t kmeans_ws_bytes(const bsa_kv_desc *, int64_t, int);
+bool kmeans_supported(const bsa_kv_desc *, int);
+bsa_status launch_kmeans(const bsa_kv_desc *, const void *, int64_t, int, int, const int32_t *, float *,
+                         int32_t *, int32_t *, int32_t *, void *, cudaStream_t);
+bsa_status launch_gather_rows(const bsa_kv_desc *, const void *, const void *, const bsa_kv_desc *, void *,
+                              void *, const int32_t *, int64_t, int64_t, cudaStream_t);
 
 int num_sms() {
     static int n = 0;
@@ -184,6 +190,35 @@ int32_t bsa_max_selected(const bsa_kv_desc *d, const bsa_sel_params *p) {
 int32_t bsa_max_ranges(const bsa_kv_desc *d, const bsa_sel_params *p) {
     if (!desc_ok(d) || !sel_ok(d, p)) return -1;
     return max_ranges(d, p);
+}
+
+size_t bsa_index_workspace_size(const bsa_kv_desc *d, int64_t L, int32_t k) {
+    if (!desc_ok(d) || L < 1 || L > d->L_max || L > 0x7fffffffLL || k < 1 || k > L) return 0;
+    return kmeans_ws_bytes(d, L, k);
+}
+
+bsa_status bsa_build_semantic_index(const bsa_kv_desc *d, const void *K, int64_t L, int32_t k,
+                                    int32_t iters, const int32_t *init, float *centres, int32_t *labels,
+                                    int32_t *offsets, int32_t *order, void *ws, size_t ws_bytes,
+                                    bsa_stream_t stream) {
+    if (!desc_ok(d) || !K || !init || !centres || !labels || !offsets || !order) return BSA_ERR_ARG;
+    if (L < 1 || L > d->L_max || L > 0x7fffffffLL || k < 1 || k > L || iters < 1) return BSA_ERR_ARG;
+    if (!aligned16(K) || !aligned16(centres)) return BSA_ERR_ARG;
+    if (!kmeans_supported(d, k)) return BSA_ERR_UNSUPPORTED;
+    if (!ws_ok(ws, ws_bytes, kmeans_ws_bytes(d, L, k))) return BSA_ERR_WORKSPACE;
+    return launch_kmeans(d, K, L, k, iters, init, centres, labels, offsets, order, ws, (cudaStream_t)stream);
+}
+
+bsa_status bsa_gather_rows(const bsa_kv_desc *src, const void *K, const void *V, const bsa_kv_desc *dst,
+                           void *K_out, void *V_out, const int32_t *rows, int64_t n, int64_t dst_row0,
+                           bsa_stream_t stream) {
+    if (!desc_ok(src) || !desc_ok(dst) || !K || !V || !K_out || !V_out || !rows) return BSA_ERR_ARG;
+    if (src->B != dst->B || src->Hkv != dst->Hkv || src->D != dst->D || src->kv_dtype != dst->kv_dtype)
+        return BSA_ERR_ARG;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(K_out) || !aligned16(V_out)) return BSA_ERR_ARG;
+    if (n < 0 || dst_row0 < 0 || dst_row0 + n > dst->L_max) return BSA_ERR_ARG;
+    if (n == 0) return BSA_OK;
+    return launch_gather_rows(src, K, V, dst, K_out, V_out, rows, n, dst_row0, (cudaStream_t)stream);
 }
 
 int32_t bsa_decode_kernels(const bsa_kv_desc *d, const bsa_sel_params *p, int32_t tokens_hint) {

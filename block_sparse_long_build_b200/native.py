@@ -24,7 +24,8 @@ BSA_OP_SELECT, BSA_OP_DECODE, BSA_OP_PREFILL, BSA_OP_APPEND = 0, 1, 2, 3
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_summary_blocks", "bsa_summary_bytes",
             "bsa_max_selected", "bsa_max_ranges", "bsa_decode_kernels", "bsa_workspace_size", "bsa_build_summaries",
             "bsa_select", "bsa_decode", "bsa_decode_noalloc", "bsa_append_kv", "bsa_decode_step",
-            "bsa_prefill_grouped")
+            "bsa_prefill_grouped", "bsa_index_workspace_size", "bsa_build_semantic_index",
+            "bsa_gather_rows")
 
 
 class BsaError(RuntimeError):
@@ -70,6 +71,9 @@ def lib() -> ctypes.CDLL:
             "bsa_max_selected": (I32, [pd, pp]),
             "bsa_max_ranges": (I32, [pd, pp]),
             "bsa_decode_kernels": (I32, [pd, pp, I32]),
+            "bsa_index_workspace_size": (SZ, [pd, ctypes.c_int64, I32]),
+            "bsa_build_semantic_index": (ctypes.c_int, [pd, P, ctypes.c_int64, I32, I32, P, P, P, P, P, P, SZ, P]),
+            "bsa_gather_rows": (ctypes.c_int, [pd, P, P, pd, P, P, P, ctypes.c_int64, ctypes.c_int64, P]),
             "bsa_workspace_size": (SZ, [pd, pp, ctypes.c_int, I32, I32]),
             "bsa_build_summaries": (ctypes.c_int, [pd, P, pp, ctypes.c_int, I32, I32, P, P]),
             "bsa_select": (ctypes.c_int, [pd, P, P, ctypes.c_int, pp, P, I32, P, P, I32, P, P, P,
@@ -219,3 +223,21 @@ def bsa_prefill_grouped(desc, K, V, sel, summaries, pos_desc, K_pos, V_pos, Q, q
                                      _p(summaries), ctypes.byref(pos_desc), _p(K_pos), _p(V_pos),
                                      _p(Q), q_pos0, Tq, scale, _p(out), _p(lse), _p(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def bsa_index_workspace_size(desc, L, n_clusters) -> int:
+    return lib().bsa_index_workspace_size(ctypes.byref(desc), L, n_clusters)
+
+
+def bsa_build_semantic_index(desc, K, L, n_clusters, iters, init, centres, labels, offsets, order, ws,
+                             stream=None):
+    _check("bsa_build_semantic_index",
+           lib().bsa_build_semantic_index(ctypes.byref(desc), _p(K), L, n_clusters, iters, _p(init),
+                                          _p(centres), _p(labels), _p(offsets), _p(order), _p(ws),
+                                          ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def bsa_gather_rows(src, K, V, dst, K_out, V_out, rows, n, dst_row0=0, stream=None):
+    _check("bsa_gather_rows",
+           lib().bsa_gather_rows(ctypes.byref(src), _p(K), _p(V), ctypes.byref(dst), _p(K_out), _p(V_out),
+                                 _p(rows), n, dst_row0, _stream(stream)))

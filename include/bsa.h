@@ -287,6 +287,45 @@ BSA_API bsa_status bsa_prefill_grouped(const bsa_kv_desc *desc, const void *K, c
                                float *out, float *lse, void *ws, size_t ws_bytes,
                                bsa_stream_t stream);
 
+/* The semantic index ("Semantic blocks for sparse attention", first section:
+ * similar keys from anywhere in the request form one block, stored together
+ * and scored through its centre): spherical k-means over rows [0, L) of each
+ * segment of K (desc geometry, bf16 or fp32, D 64 or 128), then the
+ * block-ordered store.  Arithmetic, fixed so that labels compare bit for bit:
+ *   u_r = k_r / ||k_r|| (fp32; ||.|| = sqrt of an fma chain over i; a zero
+ *         key stays zero); c_j = u_{init[j]} to start;
+ *   `iters` assignment rounds: label_r = argmax_j of the fp32 fma chain over
+ *         i of u_r[i] * c_j[i], the lowest j on equal values; between rounds
+ *         c_j = m / ||m||, m = (u summed over cluster j in position order) /
+ *         n_j (the CENTROID_NORM arithmetic); an empty cluster keeps c_j.
+ * Outputs (device, [B*Hkv] segments each): centres [k][D] fp32 (those of the
+ * last assignment), labels [L], offsets [k+1] (cluster j is rows
+ * offsets[j] .. offsets[j+1] of the block-ordered store) and order [L] (the
+ * original position of block-ordered row i: clusters in index order,
+ * positions ascending), which is the kv_pos a grouped prefill takes and the
+ * row list bsa_gather_rows takes.  init [B*Hkv][k]: starting rows (entries
+ * outside [0, L) are clamped).  1 <= k <= min(L, 1024) and k * D <= 49,152;
+ * the workspace (bsa_index_workspace_size bytes, 16-byte aligned) needs no
+ * zeroing.  BSA_ERR_ARG / BSA_ERR_UNSUPPORTED / BSA_ERR_WORKSPACE before any
+ * launch. */
+BSA_API size_t bsa_index_workspace_size(const bsa_kv_desc *desc, int64_t L, int32_t n_clusters);
+BSA_API bsa_status bsa_build_semantic_index(const bsa_kv_desc *desc, const void *K, int64_t L,
+                                            int32_t n_clusters, int32_t iters, const int32_t *init,
+                                            float *centres, int32_t *labels, int32_t *offsets,
+                                            int32_t *order, void *ws, size_t ws_bytes,
+                                            bsa_stream_t stream);
+
+/* Row gather between two caches of the same B, Hkv, D and dtype (strides may
+ * differ): for every segment, rows dst_row0 + i of K_out / V_out take rows
+ * rows[seg][i] of K / V, i < n (rows: device int32 [B*Hkv][n]; an entry
+ * outside [0, src L_max) leaves its destination row as it was; rows past the
+ * destination's L_max are BSA_ERR_ARG).  Builds the
+ * block-ordered store from `order`.  All four caches 16-byte aligned. */
+BSA_API bsa_status bsa_gather_rows(const bsa_kv_desc *src, const void *K, const void *V,
+                                   const bsa_kv_desc *dst, void *K_out, void *V_out,
+                                   const int32_t *rows, int64_t n, int64_t dst_row0,
+                                   bsa_stream_t stream);
+
 /* Static text for a status code. */
 BSA_API const char *bsa_status_string(bsa_status status);
 
