@@ -58,9 +58,12 @@ def _kernel_sha() -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def _profiled_traffic():
+def _profiled_traffic(config: str):
     """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source (else None)."""
+    taken on the current kernel source and covers this workload (the summary
+    is a capture of the Quest-style decode), else None."""
+    if config != "quest":
+        return None
     if not os.path.exists(PROFILE):
         return None
     txt = open(PROFILE).read()
@@ -333,7 +336,7 @@ def run_ours(args, rank: int, world: int, device):
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)" if peak_src == "measured" else "fallback 6.65 TB/s",
             "unit": "GB/s",
             "frac": achieved / peak,
-            "traffic": _profiled_traffic(),
+            "traffic": _profiled_traffic(cfg.name),
             "algorithmic_bytes_per_launch": kbytes,
             "launch_ms": k_ms,
         },
@@ -481,6 +484,8 @@ def run_index(args, device):
 
     Bld.build()
     cfg = W.semantic(0)
+    if args.index_keys:
+        cfg = cfg.scaled(L=args.index_keys, budget_tokens=args.index_keys // 16)
     wl = W.Workload(cfg, device)
     B, H, L, k, D, iters = cfg.B, cfg.Hkv, cfg.L, cfg.n_blocks, cfg.D, 20
     nseg = B * H
@@ -649,6 +654,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--index", action="store_true",
                     help="time the semantic index build (k-means + block-ordered store)")
+    ap.add_argument("--index-keys", type=int, default=0,
+                    help="keys per KV head for --index (a smaller case for profiling)")
     ap.add_argument("--case", choices=["decode", "select", "prefill"], default=None,
                     help="run one small profiling case instead of the bench (for ncu)")
     args = ap.parse_args()

@@ -130,6 +130,97 @@ __global__ void __launch_bounds__(kKmAssignThreads) km_assign_kernel(KmArgs a) {
     for (int j = threadIdx.x; j < k; j += blockDim.x) h[j] = hist[j];
 }
 
+// The same labels, register-blocked for k <= 256 (the common case): a tile of
+// 64 keys at a time, their unit vectors transposed in shared memory
+// uT[d][key] next to the centres cT[d][j]; warp w owns keys 8w .. 8w+7 of the
+// tile and lane l the centres 4l .. 4l+3 and 128 + 4l .. 128 + 4l+3, so each
+// d step is two broadcast loads of u, two conflict-free loads of c and 64
+// fmas into acc[key][centre] -- every (key, centre) chain still runs over
+// d = 0 .. D-1 in order.  Each lane keeps its best centre per key (lowest
+// index on equal dots); the warp then takes the largest dot (redux.sync max
+// of its orderable key, -0 folded into +0) and the lowest centre holding it.
+constexpr int kKmTile = 64;
+constexpr int kKmTiledMaxK = 256;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) km_assign_tiled_kernel(KmArgs a) {
+    extern __shared__ __align__(16) float kms[];
+    float *cT = kms;                       // [D][256]
+    float *uT = cT + D * kKmTiledMaxK;     // [D][kKmTile]
+    int *hist = reinterpret_cast<int *>(uT + D * kKmTile);   // [k]
+    const int s = blockIdx.y, c = blockIdx.x, k = a.k;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float *Cg = a.C + (int64_t)s * k * D;
+    for (int e = tid; e < D * kKmTiledMaxK; e += blockDim.x) {
+        const int d = e / kKmTiledMaxK, j = e % kKmTiledMaxK;
+        cT[e] = j < k ? Cg[(int64_t)j * D + d] : 0.0f;
+    }
+    for (int j = tid; j < k; j += blockDim.x) hist[j] = 0;
+    const int64_t key0 = (int64_t)c * kKmChunk;
+    for (int t0 = 0; t0 < kKmChunk; t0 += kKmTile) {
+        __syncthreads();   // centres in place / the previous tile's u consumed
+        {   // unit vectors of the tile's keys, transposed: thread = (key, quarter of D)
+            const int kk = tid >> 2, part = tid & 3;
+            const int64_t r = key0 + t0 + kk;
+            constexpr int Q = D / 4;
+            if (r < a.L) {
+                const T *row = km_row<T>(a, s, r);
+                const float nr = a.norms[(int64_t)s * a.L + r];
+#pragma unroll 8
+                for (int d = part * Q; d < part * Q + Q; ++d) {
+                    const float v = load_elem(row, d);
+                    uT[d * kKmTile + kk] = nr > 0.0f ? __fdiv_rn(v, nr) : 0.0f;
+                }
+            } else {
+                for (int d = part * Q; d < part * Q + Q; ++d) uT[d * kKmTile + kk] = 0.0f;
+            }
+        }
+        __syncthreads();
+        float acc[8][8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+#pragma unroll
+            for (int y = 0; y < 8; ++y) acc[x][y] = 0.0f;
+        const float *up = uT + warp * 8;
+        const float *cp = cT + lane * 4;
+#pragma unroll 4
+        for (int d = 0; d < D; ++d) {
+            const float4 u0 = *reinterpret_cast<const float4 *>(up + d * kKmTile);
+            const float4 u1 = *reinterpret_cast<const float4 *>(up + d * kKmTile + 4);
+            const float4 c0 = *reinterpret_cast<const float4 *>(cp + d * kKmTiledMaxK);
+            const float4 c1 = *reinterpret_cast<const float4 *>(cp + d * kKmTiledMaxK + 128);
+            const float uu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+#pragma unroll
+                for (int y = 0; y < 8; ++y) acc[x][y] = __fmaf_rn(uu[x], cc[y], acc[x][y]);
+        }
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+            // this lane's best centre for key x (its centres in increasing order)
+            float best = 0.0f;
+            int lab = -1;
+#pragma unroll
+            for (int y = 0; y < 8; ++y) {
+                const int j = (y < 4 ? 0 : 128) + lane * 4 + (y & 3);
+                if (j < k && (lab < 0 || acc[x][y] > best)) { best = acc[x][y]; lab = j; }
+            }
+            const uint32_t ok = lab >= 0 ? f32_order_key(__fadd_rn(best, 0.0f)) : 0u;
+            const uint32_t m = __reduce_max_sync(0xffffffffu, ok);
+            const int win = __reduce_min_sync(0xffffffffu, ok == m && lab >= 0 ? lab : 0x7fffffff);
+            const int64_t r = key0 + t0 + warp * 8 + x;
+            if (lane == 0 && r < a.L) {
+                a.labels[(int64_t)s * a.L + r] = win;
+                atomicAdd(&hist[win], 1);
+            }
+        }
+    }
+    __syncthreads();
+    int32_t *h = a.chist + ((int64_t)s * a.nchunk + c) * k;
+    for (int j = tid; j < k; j += blockDim.x) h[j] = hist[j];
+}
+
 // Cluster sizes -> offsets; chist[c][j] becomes the first slot of chunk c's
 // keys of cluster j.  One CTA per segment, thread j per cluster.
 __global__ void __launch_bounds__(kKmMaxK) km_scan_kernel(KmArgs a) {
@@ -219,15 +310,19 @@ __global__ void __launch_bounds__(128) km_update_kernel(KmArgs a) {
     float acc = 0.0f;
     if (i < D) {
         int p = beg;
-        for (; p + 4 <= end; p += 4) {   // loads batched, adds in order
-            const int r0 = ord[p], r1 = ord[p + 1], r2 = ord[p + 2], r3 = ord[p + 3];
-            const float v0 = load_elem(km_row<T>(a, s, r0), i), v1 = load_elem(km_row<T>(a, s, r1), i);
-            const float v2 = load_elem(km_row<T>(a, s, r2), i), v3 = load_elem(km_row<T>(a, s, r3), i);
-            const float n0 = nrm[r0], n1 = nrm[r1], n2 = nrm[r2], n3 = nrm[r3];
-            acc = __fadd_rn(acc, n0 > 0.0f ? __fdiv_rn(v0, n0) : 0.0f);
-            acc = __fadd_rn(acc, n1 > 0.0f ? __fdiv_rn(v1, n1) : 0.0f);
-            acc = __fadd_rn(acc, n2 > 0.0f ? __fdiv_rn(v2, n2) : 0.0f);
-            acc = __fadd_rn(acc, n3 > 0.0f ? __fdiv_rn(v3, n3) : 0.0f);
+        constexpr int kB = 16;   // rows in flight; the adds stay in order
+        for (; p + kB <= end; p += kB) {
+            int r[kB];
+            float v[kB], n[kB];
+#pragma unroll
+            for (int q = 0; q < kB; ++q) r[q] = ord[p + q];
+#pragma unroll
+            for (int q = 0; q < kB; ++q) {
+                v[q] = load_elem(km_row<T>(a, s, r[q]), i);
+                n[q] = nrm[r[q]];
+            }
+#pragma unroll
+            for (int q = 0; q < kB; ++q) acc = __fadd_rn(acc, n[q] > 0.0f ? __fdiv_rn(v[q], n[q]) : 0.0f);
         }
         for (; p < end; ++p) {
             const int r0 = ord[p];
@@ -278,8 +373,10 @@ bsa_status launch_kmeans(const bsa_kv_desc *d, const void *K, int64_t L, int k, 
     auto run = [&](auto tag, auto dtag) -> bsa_status {
         using T = decltype(tag);
         constexpr int DD = decltype(dtag)::value;
-        auto assign = km_assign_kernel<T, DD>;
-        BSA_CUDA_TRY(cudaFuncSetAttribute(assign, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_assign));
+        const bool tiled = k <= kKmTiledMaxK;
+        auto assign = tiled ? km_assign_tiled_kernel<T, DD> : km_assign_kernel<T, DD>;
+        const size_t smem_a = tiled ? (size_t)DD * (kKmTiledMaxK + kKmTile) * 4 + (size_t)k * 4 : smem_assign;
+        BSA_CUDA_TRY(cudaFuncSetAttribute(assign, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a));
         BSA_CUDA_TRY(cudaFuncSetAttribute(km_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)smem_scatter));
         km_norms_kernel<T><<<gkeys, 256, 0, st>>>(a);
@@ -287,7 +384,7 @@ bsa_status launch_kmeans(const bsa_kv_desc *d, const void *K, int64_t L, int k, 
         km_init_kernel<T><<<gclusters, DD, 0, st>>>(a);
         BSA_LAUNCH_CHECK();
         for (int it = 0; it < iters; ++it) {
-            assign<<<gchunks, kKmAssignThreads, smem_assign, st>>>(a);
+            assign<<<gchunks, kKmAssignThreads, smem_a, st>>>(a);
             BSA_LAUNCH_CHECK();
             km_scan_kernel<<<(unsigned)nseg, kKmMaxK, 0, st>>>(a);
             BSA_LAUNCH_CHECK();

@@ -47,6 +47,7 @@ def _run_index(K, L, k, iters, init):
     (torch.bfloat16, 128, 5000 + 37, 22, 5, 0.35),   # ragged chunk, k not a multiple of 4
     (torch.float32, 64, 3000, 16, 4, 0.5),
     (torch.bfloat16, 128, 1024, 1, 2, 0.3),          # one cluster
+    (torch.bfloat16, 128, 4096 + 3, 300, 3, 0.4),    # more than 256 clusters (untiled assignment)
 ])
 def test_index_matches_oracle_bit_for_bit(dtype, D, L, k, iters, noise):
     rng = np.random.default_rng(L + k)
