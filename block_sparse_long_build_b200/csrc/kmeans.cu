@@ -157,25 +157,46 @@ __global__ void __launch_bounds__(256) km_assign_tiled_kernel(KmArgs a) {
     }
     for (int j = tid; j < k; j += blockDim.x) hist[j] = 0;
     const int64_t key0 = (int64_t)c * kKmChunk;
+    // the tile's rows: thread = (key kk, quarter part of D); the next tile's
+    // raw rows are fetched (16-byte loads) while the current tile computes
+    constexpr int Q = D / 4, EPV = 16 / (int)sizeof(T), NV = Q / EPV;
+    const int kk = tid >> 2, part = tid & 3;
+    uint4 raw[NV];
+    float nrr = 0.0f;
+    auto fetch = [&](int t0) {
+        const int64_t r = key0 + t0 + kk;
+        if (r < a.L) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(km_row<T>(a, s, r) + part * Q);
+#pragma unroll
+            for (int v = 0; v < NV; ++v) raw[v] = __ldg(src + v);
+            nrr = a.norms[(int64_t)s * a.L + r];
+        } else {
+#pragma unroll
+            for (int v = 0; v < NV; ++v) raw[v] = make_uint4(0u, 0u, 0u, 0u);
+            nrr = 0.0f;
+        }
+    };
+    fetch(0);
     for (int t0 = 0; t0 < kKmChunk; t0 += kKmTile) {
         __syncthreads();   // centres in place / the previous tile's u consumed
-        {   // unit vectors of the tile's keys, transposed: thread = (key, quarter of D)
-            const int kk = tid >> 2, part = tid & 3;
-            const int64_t r = key0 + t0 + kk;
-            constexpr int Q = D / 4;
-            if (r < a.L) {
-                const T *row = km_row<T>(a, s, r);
-                const float nr = a.norms[(int64_t)s * a.L + r];
-#pragma unroll 8
-                for (int d = part * Q; d < part * Q + Q; ++d) {
-                    const float v = load_elem(row, d);
-                    uT[d * kKmTile + kk] = nr > 0.0f ? __fdiv_rn(v, nr) : 0.0f;
+        {   // unit vectors of the tile's keys, transposed
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                const uint32_t w[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) {
+                    float x;
+                    if constexpr (sizeof(T) == 2)
+                        x = __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+                    else
+                        x = __uint_as_float(w[e]);
+                    const int d = part * Q + v * EPV + e;
+                    uT[d * kKmTile + kk] = nrr > 0.0f ? __fdiv_rn(x, nrr) : 0.0f;
                 }
-            } else {
-                for (int d = part * Q; d < part * Q + Q; ++d) uT[d * kKmTile + kk] = 0.0f;
             }
         }
         __syncthreads();
+        if (t0 + kKmTile < kKmChunk) fetch(t0 + kKmTile);
         float acc[8][8];
 #pragma unroll
         for (int x = 0; x < 8; ++x)

@@ -375,7 +375,7 @@ __device__ void warp_walk_smem(const uint32_t *keys, const int32_t *visb, unsign
 // owns the contiguous blocks [t kpt, t kpt + kpt) for the index-ordered
 // compactions.  Loops stay rolled (short unrolls batch the loads): the
 // kernel runs once per selection, so compact code beats straight-line code.
-__global__ void __launch_bounds__(kPickThreads) pick_kernel(SelArgs a) {
+__global__ void __launch_bounds__(kPickThreads, 2) pick_kernel(SelArgs a) {
     extern __shared__ __align__(16) unsigned char psm[];
     const int nb = a.nb_total;
     uint32_t *keys = reinterpret_cast<uint32_t *>(psm + PickSmem::keys(nb));
