@@ -136,7 +136,8 @@ __global__ void __launch_bounds__(kKmAssignThreads) km_assign_kernel(KmArgs a) {
 // tile and lane l the centres 4l .. 4l+3 and 128 + 4l .. 128 + 4l+3, so each
 // d step is two broadcast loads of u, two conflict-free loads of c and 64
 // fmas into acc[key][centre] -- every (key, centre) chain still runs over
-// d = 0 .. D-1 in order.  Each lane keeps its best centre per key (lowest
+// d = 0 .. D-1 in order (two chains per fma.rn.f32x2: each half is its own
+// fused multiply-add, rounded once).  Each lane keeps its best centre per key (lowest
 // index on equal dots); the warp then takes the largest dot (redux.sync max
 // of its orderable key, -0 folded into +0) and the lowest centre holding it.
 constexpr int kKmTile = 64;
@@ -215,7 +216,12 @@ __global__ void __launch_bounds__(256) km_assign_tiled_kernel(KmArgs a) {
 #pragma unroll
             for (int x = 0; x < 8; ++x)
 #pragma unroll
-                for (int y = 0; y < 8; ++y) acc[x][y] = __fmaf_rn(uu[x], cc[y], acc[x][y]);
+                for (int y = 0; y < 8; y += 2)
+                    asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+                        "mov.b64 pa, {%2, %2};\n\tmov.b64 pb, {%3, %4};\n\tmov.b64 pc, {%0, %1};\n\t"
+                        "fma.rn.f32x2 pc, pa, pb, pc;\n\tmov.b64 {%0, %1}, pc;\n\t}"
+                        : "+f"(acc[x][y]), "+f"(acc[x][y + 1])
+                        : "f"(uu[x]), "f"(cc[y]), "f"(cc[y + 1]));
         }
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
