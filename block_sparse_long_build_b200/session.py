@@ -196,16 +196,41 @@ class DecodeSession:
             self.select(self.q_in)
             self.decode(self.q_in)
         with torch.cuda.graph(self.g_plain):
-            if self.fused:
-                self.decode_step(self.q_in, self.k_in, self.v_in)
-            else:
-                self.append(self.k_in, self.v_in)
-                self.decode(self.q_in)
+            self._plain_step()
+        # the same two steps with their host traffic inside the graph: the
+        # packed inputs in from the pinned staging buffer host_in, the packed
+        # outputs (out, lse) back to the pinned host_out
+        self.host_in = torch.zeros(n, dtype=torch.uint8).pin_memory()
+        self.host_out = torch.zeros(self.io_out.numel(), dtype=torch.uint8).pin_memory()
+        self.g_refresh_io, self.g_plain_io = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_refresh_io):
+            self.io_in.copy_(self.host_in, non_blocking=True)
+            self.append(self.k_in, self.v_in)
+            self.select(self.q_in)
+            self.decode(self.q_in)
+            self.host_out.copy_(self.io_out, non_blocking=True)
+        with torch.cuda.graph(self.g_plain_io):
+            self.io_in.copy_(self.host_in, non_blocking=True)
+            self._plain_step()
+            self.host_out.copy_(self.io_out, non_blocking=True)
+
+    def _plain_step(self):
+        if self.fused:
+            self.decode_step(self.q_in, self.k_in, self.v_in)
+        else:
+            self.append(self.k_in, self.v_in)
+            self.decode(self.q_in)
 
     def replay(self, t: int):
         """Decode step t from the captured graphs (inputs already in q_in,
         k_in, v_in)."""
         (self.g_refresh if t % self.cfg.refresh == 0 else self.g_plain).replay()
+
+    def replay_io(self, t: int):
+        """Decode step t with its host traffic: the packed inputs staged in
+        host_in (pinned) go in, the packed outputs come back to host_out, all in
+        one graph launch."""
+        (self.g_refresh_io if t % self.cfg.refresh == 0 else self.g_plain_io).replay()
 
     def launches_per_step(self, t: int) -> int:
         """Library kernels one step launches: append, the two selection kernels
