@@ -120,3 +120,32 @@ def test_product_path_has_no_oracle_import():
                 src = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), f
                 assert "oracle.c" not in src and "_oracle.so" not in src, f
+
+
+def test_semantic_index_arguments_rejected_on_host(lib):
+    """The index and gather entry points validate on the host and launch
+    nothing when an argument is out of range."""
+    L = N.lib()
+    d = _desc(B=1, Hkv=2, Hq=8, L_max=4096, stride_b=2 * 4096 * 128, stride_h=4096 * 128)
+    fake = 1 << 20
+    assert N.bsa_index_workspace_size(d, 4096, 64) > 0
+    assert N.bsa_index_workspace_size(d, 4097, 64) == 0          # more keys than the cache holds
+    assert N.bsa_index_workspace_size(d, 100, 101) == 0           # more clusters than keys
+    args = lambda Lk, k, it, ws_bytes: (ctypes.byref(d), fake, Lk, k, it, fake, fake, fake, fake, fake,
+                                        fake, ws_bytes, None)
+    assert L.bsa_build_semantic_index(*args(4096, 64, 0, 1 << 30)) == N.BSA_ERR_ARG      # no round
+    assert L.bsa_build_semantic_index(*args(4096, 0, 5, 1 << 30)) == N.BSA_ERR_ARG       # no cluster
+    assert L.bsa_build_semantic_index(*args(4096, 2048, 5, 1 << 30)) == N.BSA_ERR_UNSUPPORTED
+    assert L.bsa_build_semantic_index(*args(4096, 64, 5, 16)) == N.BSA_ERR_WORKSPACE
+    assert L.bsa_build_semantic_index(ctypes.byref(d), fake, 4096, 64, 5, None, fake, fake, fake, fake,
+                                      fake, 1 << 30, None) == N.BSA_ERR_ARG              # no starting rows
+    # gather: geometry mismatch, destination overflow, misaligned cache
+    d2 = _desc(B=1, Hkv=4, Hq=8, L_max=4096, stride_b=4 * 4096 * 128, stride_h=4096 * 128)
+    assert L.bsa_gather_rows(ctypes.byref(d), fake, fake, ctypes.byref(d2), fake, fake, fake, 10, 0,
+                             None) == N.BSA_ERR_ARG
+    assert L.bsa_gather_rows(ctypes.byref(d), fake, fake, ctypes.byref(d), fake, fake, fake, 100, 4000,
+                             None) == N.BSA_ERR_ARG
+    assert L.bsa_gather_rows(ctypes.byref(d), fake + 2, fake, ctypes.byref(d), fake, fake, fake, 10, 0,
+                             None) == N.BSA_ERR_ARG
+    assert L.bsa_gather_rows(ctypes.byref(d), fake, fake, ctypes.byref(d), fake, fake, fake, 0, 0,
+                             None) == N.BSA_OK                                           # nothing to do
