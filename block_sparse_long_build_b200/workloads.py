@@ -25,8 +25,10 @@ Readings taken where the workload descriptions leave a choice open:
 * Semantic workload: the planted clusters are the blocks.  Keys are
   normalise(centre + 0.05 * xi); block sizes are log-normal (sigma 0.5)
   rescaled to sum to the context; positions are assigned to blocks by a
-  random shuffle.  The planted assignment stands in for the spherical k-means
-  index, which this module does not run.
+  random shuffle.  The store is built here from the planted assignment; the
+  library's spherical k-means (bsa_build_semantic_index), started from the
+  first key of each planted cluster, recovers exactly that assignment, so
+  bsa_gather_rows over its order gives the same block-ordered store.
 """
 from __future__ import annotations
 
