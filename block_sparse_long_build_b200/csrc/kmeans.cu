@@ -12,10 +12,12 @@
 //   `iters` rounds of assignment, iters - 1 updates between them.
 //
 // Kernels, per round (every segment at once):
-//   km_assign_kernel    a CTA per 1,024 keys of a segment: the centres in
-//                       shared memory, one key's unit vector per thread in
-//                       registers, four centres' fma chains at a time; the
-//                       chunk's label histogram
+//   km_assign_tiled_kernel  (k <= 256) a CTA per 1,024 keys of a segment, 64
+//                       keys at a time: unit keys and centres transposed in
+//                       shared memory, 8 keys x 8 centres of fma chains per
+//                       thread, a warp argmax; the chunk's label histogram
+//   km_assign_kernel    (k > 256) the same with one key's unit vector per
+//                       thread in registers, four centres' chains at a time
 //   km_scan_kernel      a CTA per segment: cluster sizes, CSR offsets and each
 //                       chunk's first slot per cluster
 //   km_scatter_kernel   a CTA per chunk: stable slots (rank among equal labels
