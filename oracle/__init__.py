@@ -32,6 +32,9 @@ What the oracle computes, with the page (title, section) each step follows:
   keys, largest fp32 dot wins, lowest centre on ties, normalised-mean update,
   an empty cluster keeps its centre) and the block-ordered store (clusters in
   index order, positions ascending within a cluster).
+* A paged cache ("Sparse long-context inference with self-indexing attention",
+  "How much memory the KV cache takes"): pages gathered back into the
+  sequence's cache through its page table.
 
 The fp32 arithmetic that decides the selection follows a fixed order written
 out in ``oracle.c``; everything compared with a tolerance is fp64.
@@ -406,3 +409,24 @@ def kmeans_assign(K_seg: np.ndarray, rows, C: np.ndarray):
     _lib().oracle_kmeans_assign(_ptr(K_seg), _kv_dtype(K_seg), ld, K_seg.shape[1], _ptr(rows), len(rows),
                                 _ptr(C), C.shape[0], _ptr(out))
     return out
+
+
+# --------------------------------------------------------------------------
+# Paged KV ("Sparse long-context inference with self-indexing attention",
+# "How much memory the KV cache takes": the cache as fixed-size pages)
+# --------------------------------------------------------------------------
+
+def paged_to_contiguous(pool: np.ndarray, page_table, page_size: int, n_tokens: int) -> np.ndarray:
+    """One sequence's cache rows [Hkv, n_tokens, D] from a page pool
+    [n_pages, Hkv, page_size, D] and its page table (logical page i of the
+    sequence is physical page page_table[i]): token t sits in page
+    page_table[t // page_size] at row t % page_size.  Attention over a paged
+    cache is attention over this gathered cache, so the contiguous oracle
+    applies unchanged."""
+    page_table = np.asarray(page_table, dtype=np.int64)
+    n_pages = -(-n_tokens // page_size)
+    assert len(page_table) >= n_pages and (page_table[:n_pages] >= 0).all()
+    assert (page_table[:n_pages] < pool.shape[0]).all()
+    t = np.arange(n_tokens)
+    rows = pool[page_table[t // page_size], :, t % page_size, :]   # [n_tokens, Hkv, D]
+    return np.ascontiguousarray(rows.transpose(1, 0, 2))

@@ -473,3 +473,36 @@ def test_kmeans_empty_cluster_keeps_its_centre_and_ties_go_low():
     assert np.abs(C[0] - u1).max() > 1e-3
     # the assignment helper agrees with the last assignment
     assert (oracle.kmeans_assign(X, np.arange(L), C) == labels).all()
+
+
+def test_paged_cache_gathers_to_the_contiguous_cache():
+    """A cache cut into pages and scattered over a pool by a random page table
+    reads back as the original cache, and attention over it is unchanged."""
+    rng = np.random.default_rng(4)
+    H, D, P, n = 2, 16, 16, 16 * 7 + 5
+    K = rng.standard_normal((H, n, D)).astype(np.float32)
+    n_pages = -(-n // P)
+    pool = np.zeros((n_pages + 3, H, P, D), np.float32)
+    table = rng.permutation(n_pages + 3)[:n_pages]
+    for i in range(n_pages):
+        rows = K[:, i * P:min((i + 1) * P, n)]
+        pool[table[i], :, :rows.shape[1]] = rows
+    back = oracle.paged_to_contiguous(pool, table, P, n)
+    assert back.shape == K.shape and (back == K).all()
+    # identity table over an in-order pool is a reshape
+    pool2 = np.zeros((n_pages, H, P, D), np.float32)
+    for i in range(n_pages):
+        rows = K[:, i * P:min((i + 1) * P, n)]
+        pool2[i, :, :rows.shape[1]] = rows
+    assert (oracle.paged_to_contiguous(pool2, np.arange(n_pages), P, n) == K).all()
+    q = rng.standard_normal((1, D)).astype(np.float32)
+    V = rng.standard_normal((H, n, D)).astype(np.float32)
+    poolv = np.zeros_like(pool)
+    for i in range(n_pages):
+        rows = V[:, i * P:min((i + 1) * P, n)]
+        poolv[table[i], :, :rows.shape[1]] = rows
+    Vb = oracle.paged_to_contiguous(poolv, table, P, n)
+    rows = np.arange(n)
+    o1, l1 = oracle.attend(q, K[0], V[0], rows, 0.25)
+    o2, l2 = oracle.attend(q, back[0], Vb[0], rows, 0.25)
+    assert (o1 == o2).all() and (l1 == l2).all()
