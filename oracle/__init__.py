@@ -35,6 +35,8 @@ What the oracle computes, with the page (title, section) each step follows:
 * A paged cache ("Sparse long-context inference with self-indexing attention",
   "How much memory the KV cache takes"): pages gathered back into the
   sequence's cache through its page table.
+* FP8 (E4M3) cache codes decoded exactly ("Attention mechanisms in modern
+  LLMs", basic maths and real cost: narrow KV formats such as FP8).
 
 The fp32 arithmetic that decides the selection follows a fixed order written
 out in ``oracle.c``; everything compared with a tolerance is fp64.
@@ -430,3 +432,24 @@ def paged_to_contiguous(pool: np.ndarray, page_table, page_size: int, n_tokens: 
     t = np.arange(n_tokens)
     rows = pool[page_table[t // page_size], :, t % page_size, :]   # [n_tokens, Hkv, D]
     return np.ascontiguousarray(rows.transpose(1, 0, 2))
+
+
+# --------------------------------------------------------------------------
+# FP8 K/V ("Attention mechanisms in modern LLMs", section on the basic maths
+# and the real cost: the KV cache may be kept in FP8 and other narrow formats)
+# --------------------------------------------------------------------------
+
+def fp8_e4m3_to_f32(codes) -> np.ndarray:
+    """Exact values of FP8 E4M3 codes (1 sign bit, 4 exponent bits with bias 7,
+    3 mantissa bits; exponent 0 is subnormal, m * 2^-9; S.1111.111 is NaN and
+    there is no infinity, so the largest finite value is 448).  The page says
+    only "FP8"; E4M3, the usual format for cached keys and values, is the
+    reading taken.  An FP8 cache is read through this table, then the
+    fp32/fp64 oracle applies unchanged."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where((e == 0xF) & (m == 0x7), np.nan, val)
+    return (sign * val).astype(np.float32)

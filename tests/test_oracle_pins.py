@@ -506,3 +506,15 @@ def test_paged_cache_gathers_to_the_contiguous_cache():
     o1, l1 = oracle.attend(q, K[0], V[0], rows, 0.25)
     o2, l2 = oracle.attend(q, back[0], Vb[0], rows, 0.25)
     assert (o1 == o2).all() and (l1 == l2).all()
+
+
+def test_fp8_e4m3_decoding_matches_torch_and_the_format_limits():
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.fp8_e4m3_to_f32(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    both_nan = np.isnan(ours) & np.isnan(ref)
+    assert (both_nan | (ours == ref)).all()
+    assert np.isnan(ours).sum() == 2                       # S.1111.111
+    assert ours[0x38] == 1.0 and ours[0x7E] == 448.0 and ours[0x01] == 2.0 ** -9
+    assert ours[0x80] == 0.0 and np.signbit(ours[0x80])    # negative zero
