@@ -151,6 +151,29 @@ static bool ws_ok(const void *ws, size_t have, size_t need) {
     return ws && aligned16(ws) && have >= need;
 }
 
+// Host-side checks shared by every decode entry point (bsa_decode,
+// bsa_decode_step, bsa_decode_noalloc): BSA_OK or the error to return before
+// anything touches device memory.
+bsa_status decode_check_args(const bsa_kv_desc *d, const float *q, const void *K, const void *V,
+                             const int32_t *ranges, const int32_t *n_ranges, int32_t max_r,
+                             const int32_t *cur_len, int32_t tokens_hint, float scale,
+                             const float *out) {
+    if (!desc_ok(d)) return BSA_ERR_ARG;
+    if (!q || !K || !V || !ranges || !n_ranges || !cur_len || !out) return BSA_ERR_ARG;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(q)) return BSA_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(ranges) % 8) return BSA_ERR_ARG;
+    if (max_r < 1 || max_r > 4096 || tokens_hint < 0) return BSA_ERR_ARG;
+    if (d->Hq / d->Hkv > kMaxG) return BSA_ERR_UNSUPPORTED;
+    if (!(scale > 0.0f) || scale != scale) return BSA_ERR_ARG;
+    return BSA_OK;
+}
+
+// Bytes of the status word + counters area at the start of a workspace.
+size_t ws_counters_bytes(const bsa_kv_desc *d) { return counters_bytes(d); }
+
+void *noalloc_scratch_on_current_context();
+void arm_decode_wait_limit(uint32_t limit_ns);
+
 }  // namespace bsa
 
 using namespace bsa;
@@ -167,8 +190,38 @@ const char *bsa_status_string(bsa_status s) {
         case BSA_ERR_CUDA: return "CUDA error";
         case BSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case BSA_ERR_TIMEOUT: return "device-side wait timed out";
+        case BSA_ERR_CAPACITY: return "a per-query limit was reached; result truncated";
     }
     return "unknown status";
+}
+
+bsa_status bsa_workspace_status(const void *ws, size_t ws_bytes, int32_t clear, uint32_t *bits,
+                                bsa_stream_t stream) {
+    void *word = const_cast<void *>(ws);
+    if (!word) {
+        word = noalloc_scratch_on_current_context();
+        if (!word) return BSA_ERR_CUDA;
+    } else if (ws_bytes < 4 || (reinterpret_cast<uintptr_t>(ws) & 3)) {
+        return BSA_ERR_WORKSPACE;
+    }
+    const cudaStream_t st = (cudaStream_t)stream;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, word, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        (clear && cudaMemsetAsync(word, 0, 4, st) != cudaSuccess) ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return BSA_ERR_CUDA;
+    }
+    if (bits) *bits = v;
+    if (v & (1u | 2u | 8u)) return BSA_ERR_TIMEOUT;
+    if (v) return BSA_ERR_CAPACITY;
+    return BSA_OK;
+}
+
+bsa_status bsa_test_arm_wait_limit(int32_t limit_us) {
+    if (limit_us < 0 || limit_us > 100000) return BSA_ERR_ARG;
+    arm_decode_wait_limit((uint32_t)limit_us * 1000u);
+    return BSA_OK;
 }
 
 int32_t bsa_summary_blocks(const bsa_kv_desc *d, const bsa_sel_params *p) {
@@ -292,13 +345,9 @@ bsa_status bsa_decode(const bsa_kv_desc *d, const float *q, const void *K, const
                       const int32_t *ranges, const int32_t *n_ranges, int32_t max_r,
                       const int32_t *cur_len, int32_t tokens_hint, float scale, float *out,
                       float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream) {
-    if (!desc_ok(d)) return BSA_ERR_ARG;
-    if (!q || !K || !V || !ranges || !n_ranges || !cur_len || !out) return BSA_ERR_ARG;
-    if (!aligned16(K) || !aligned16(V) || !aligned16(q)) return BSA_ERR_ARG;
-    if (reinterpret_cast<uintptr_t>(ranges) % 8) return BSA_ERR_ARG;
-    if (max_r < 1 || max_r > 4096 || tokens_hint < 0) return BSA_ERR_ARG;
-    if (d->Hq / d->Hkv > kMaxG) return BSA_ERR_UNSUPPORTED;
-    if (!(scale > 0.0f) || scale != scale) return BSA_ERR_ARG;
+    const bsa_status chk =
+        decode_check_args(d, q, K, V, ranges, n_ranges, max_r, cur_len, tokens_hint, scale, out);
+    if (chk != BSA_OK) return chk;
     const int nsplit = decode_nsplit(d, std::max(tokens_hint, 1), max_r);
     const size_t need = counters_bytes(d) + decode_scratch_bytes(d, nsplit);
     if (!ws_ok(ws, ws_bytes, need)) return BSA_ERR_WORKSPACE;
@@ -319,12 +368,9 @@ bsa_status bsa_decode_step(const bsa_kv_desc *d, const float *q, void *K, void *
     if (!desc_ok(d) || !K || !V || !k_new || !v_new || !cur_len) return BSA_ERR_ARG;
     if (p && !sel_ok(d, p)) return BSA_ERR_ARG;
     if (summaries && (!p || kind < BSA_SUM_CENTROID || kind > BSA_SUM_MINMAX)) return BSA_ERR_ARG;
-    if (!q || !ranges || !n_ranges || !out) return BSA_ERR_ARG;
-    if (!aligned16(K) || !aligned16(V) || !aligned16(q)) return BSA_ERR_ARG;
-    if (reinterpret_cast<uintptr_t>(ranges) % 8) return BSA_ERR_ARG;
-    if (max_r < 1 || max_r > 4096 || tokens_hint < 0) return BSA_ERR_ARG;
-    if (d->Hq / d->Hkv > kMaxG) return BSA_ERR_UNSUPPORTED;
-    if (!(scale > 0.0f) || scale != scale) return BSA_ERR_ARG;
+    const bsa_status chk =
+        decode_check_args(d, q, K, V, ranges, n_ranges, max_r, cur_len, tokens_hint, scale, out);
+    if (chk != BSA_OK) return chk;
     const int nsplit = decode_nsplit(d, std::max(tokens_hint, 1), max_r);
     const size_t need = counters_bytes(d) + decode_scratch_bytes(d, nsplit);
     if (!ws_ok(ws, ws_bytes, need)) return BSA_ERR_WORKSPACE;

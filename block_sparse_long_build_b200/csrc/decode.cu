@@ -21,6 +21,7 @@
 // q_lo = q - q_hi (rows 8-15), so one m16n8k16 bf16 MMA gives the logits to
 // ~2^-17 relative; the softmax weights are split the same way for P.V.
 // Accumulation is fp32.
+#include <atomic>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -53,8 +54,14 @@ struct DecArgs {
     float2 *part_ml;      // [nseg][nsplit][G]
     uint32_t *counters;   // [nseg]; entry b * Hkv counts the CTAs of sequence b (fused append)
     uint32_t *status;     // sticky error bits
+    uint32_t stall_ns;    // test hook: a wait of this bound on a barrier nothing completes
     DecAppend app;
 };
+
+// Limit of the test stall armed for the next decode launch (0: none).
+static std::atomic<uint32_t> g_armed_stall_ns{0};
+
+void arm_decode_wait_limit(uint32_t limit_ns) { g_armed_stall_ns.store(limit_ns); }
 
 // Exclusive scan over the CTA (blockDim.x a multiple of 32, <= 1024).
 __device__ __forceinline__ int block_excl_scan(int v, int *tmp, int *total) {
@@ -441,7 +448,8 @@ struct TcSmem {
     static constexpr int kBars = kInfo + kDecWarps * NST * 8;         // u64  [warps][NST]
     static constexpr int kMisc = kBars + kDecWarps * NST * 8;         // float sml[2*kMaxG], int tmp[36]
     static constexpr int kPtab = kMisc + 2 * kMaxG * 4 + 36 * 4;      // int2 [warps][kWarpCap]
-    static constexpr int kBytes = kPtab + kDecWarps * kWarpCap * 8 + 1024;
+    static constexpr int kStall = kPtab + kDecWarps * kWarpCap * 8;   // u64: test-hook barrier
+    static constexpr int kBytes = kStall + 8 + 1024;
     static_assert(kRing >= kDecWarps * kMaxG * (2 + 64 * NH) * 4,
                   "per-warp partials must fit in the ring");
 };
@@ -479,6 +487,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (lane == 0) {
         for (int i = 0; i < NST; ++i) mbar_init(&wfull[i], 1);
         fence_mbar_init();
+    }
+    if (a.stall_ns && c == 0 && s == 0 && tid == 0) {
+        // test hook: a bounded wait on a barrier that nothing completes, before
+        // any copy is issued; it gives up after stall_ns and reports a timeout
+        uint64_t *bar = reinterpret_cast<uint64_t *>(dsm + L::kStall);
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        if (!mbar_wait_bounded(bar, 0u, a.stall_ns)) atomicOr(a.status, 1u);
     }
     pdl_wait();   // ranges, lengths and the cache come from earlier kernels
     // fused append: lanes 0.. hold 16-byte chunks of the new key, lanes 16..
@@ -897,6 +913,7 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
                                            align_up(nseg * a.nsplit * a.G * d->D * 4, 256));
     a.counters = counters;
     a.status = status;
+    a.stall_ns = use_tc(d) ? g_armed_stall_ns.exchange(0u) : 0u;
     dim3 grid(a.nsplit, (unsigned)nseg);
     if (use_tc(d)) {
         CUtensorMap tk, tv;

@@ -209,7 +209,12 @@ __global__ void __launch_bounds__(32 * kPfSelWarps) prefill_select_kernel(PfArgs
             for (int t = 0; t < kPfWords; ++t)
                 if (lane + 32 * t == j || vr[t] > remaining) sk[t] = 0u;
         }
-        if (nsel >= kPfMaxSel && lane == 0) atomicOr(a.status, 4u);
+        if (nsel >= kPfMaxSel) {   // capacity reached: report it only if a block still fits
+            uint32_t lm = 0u;
+#pragma unroll
+            for (int t = 0; t < kPfWords; ++t) lm = max(lm, sk[t]);
+            if (__reduce_max_sync(0xffffffffu, lm) != 0u && lane == 0) atomicOr(a.status, 4u);
+        }
         uint32_t *bm = a.bitmap + ((int64_t)i * a.Hkv + g) * kPfWords;
         uint32_t words[kPfWords];
 #pragma unroll

@@ -15,8 +15,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbsa.so")
 
-BSA_OK, BSA_ERR_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA, BSA_ERR_WORKSPACE, BSA_ERR_TIMEOUT = (
-    0, -1, -2, -3, -4, -5)
+(BSA_OK, BSA_ERR_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA, BSA_ERR_WORKSPACE, BSA_ERR_TIMEOUT,
+ BSA_ERR_CAPACITY) = (0, -1, -2, -3, -4, -5, -6)
 BSA_SUM_CENTROID, BSA_SUM_CENTROID_NORM, BSA_SUM_MINMAX = 0, 1, 2
 BSA_F32, BSA_BF16 = 0, 1
 BSA_OP_SELECT, BSA_OP_DECODE, BSA_OP_PREFILL, BSA_OP_APPEND = 0, 1, 2, 3
@@ -25,7 +25,7 @@ EXPORTED = ("bsa_version", "bsa_status_string", "bsa_summary_blocks", "bsa_summa
             "bsa_max_selected", "bsa_max_ranges", "bsa_decode_kernels", "bsa_workspace_size", "bsa_build_summaries",
             "bsa_select", "bsa_decode", "bsa_decode_noalloc", "bsa_append_kv", "bsa_decode_step",
             "bsa_prefill_grouped", "bsa_index_workspace_size", "bsa_build_semantic_index",
-            "bsa_gather_rows")
+            "bsa_gather_rows", "bsa_workspace_status", "bsa_test_arm_wait_limit")
 
 
 class BsaError(RuntimeError):
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
                                                I32, F, P, P, P, SZ, P]),
             "bsa_prefill_grouped": (ctypes.c_int, [pd, P, P, pp, P, pd, P, P, P, I32, I32, F, P, P,
                                                    P, SZ, P]),
+            "bsa_workspace_status": (ctypes.c_int, [P, SZ, I32, ctypes.POINTER(ctypes.c_uint32), P]),
+            "bsa_test_arm_wait_limit": (ctypes.c_int, [I32]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -241,3 +243,24 @@ def bsa_gather_rows(src, K, V, dst, K_out, V_out, rows, n, dst_row0=0, stream=No
     _check("bsa_gather_rows",
            lib().bsa_gather_rows(ctypes.byref(src), _p(K), _p(V), ctypes.byref(dst), _p(K_out), _p(V_out),
                                  _p(rows), n, dst_row0, _stream(stream)))
+
+
+def bsa_workspace_status(ws, clear=True, stream=None) -> tuple[int, int]:
+    """Waits for `stream`, reads (and by default clears) the sticky device-side
+    status word of a workspace tensor; ws=None reads the scratch built into
+    the library for bsa_decode_noalloc.  Returns (status, raw bits) without
+    raising: BSA_OK, BSA_ERR_TIMEOUT or BSA_ERR_CAPACITY."""
+    bits = ctypes.c_uint32(0)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    r = lib().bsa_workspace_status(_p(ws), nbytes, int(bool(clear)), ctypes.byref(bits),
+                                   _stream(stream))
+    if r not in (BSA_OK, BSA_ERR_TIMEOUT, BSA_ERR_CAPACITY):
+        raise BsaError("bsa_workspace_status", r)
+    return r, bits.value
+
+
+def bsa_test_arm_wait_limit(limit_us: int):
+    """Test hook: the next tensor-core decode launch makes one warp wait on a
+    barrier nothing completes, for at most limit_us microseconds, and report
+    it as a timeout (see include/bsa.h)."""
+    _check("bsa_test_arm_wait_limit", lib().bsa_test_arm_wait_limit(limit_us))

@@ -27,7 +27,10 @@
  *  - Pointers named d_* or documented "device" are CUDA device pointers;
  *    descriptors and parameter structs are host pointers read during the call
  *    only.  The caller owns every buffer, including the workspace; the
- *    library allocates nothing and keeps no state between calls.
+ *    library allocates nothing.  Between calls it keeps only per-process
+ *    caches of device properties (SM count, cluster occupancy, the tensor-map
+ *    encoder) and, for bsa_decode_noalloc, its built-in scratch array and
+ *    that array's address per CUDA context.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream).  BSA_OK means "validated and launched"; a failed launch returns
  *    BSA_ERR_CUDA.  Results are ready when the stream reaches them.
@@ -44,6 +47,13 @@
  *    before its first use.  Every call leaves its counters at zero again, so
  *    one workspace can serve any sequence of calls on one stream.  Calls that
  *    may overlap on the GPU need separate workspaces.
+ *  - Device-side errors: the first 4 bytes of a workspace are a sticky status
+ *    word that kernels set and never clear: bit 0 a decode wait for a tile
+ *    copy gave up, bit 1 a selection wait gave up, bit 3 a prefill wait gave
+ *    up (each BSA_ERR_TIMEOUT; the call finished with partial data), bit 2 a
+ *    prefill query had more blocks within its budget than the 64 this build
+ *    keeps (BSA_ERR_CAPACITY; that query's block list was cut at 64).  Read
+ *    and clear it with bsa_workspace_status().
  */
 #ifndef BSA_H
 #define BSA_H
@@ -69,7 +79,9 @@ typedef enum {
     BSA_ERR_UNSUPPORTED = -2,  /* valid, but a shape this build does not cover  */
     BSA_ERR_CUDA = -3,         /* a CUDA call or launch failed                  */
     BSA_ERR_WORKSPACE = -4,    /* workspace missing, misaligned or too small    */
-    BSA_ERR_TIMEOUT = -5       /* a bounded device-side wait gave up            */
+    BSA_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up            */
+    BSA_ERR_CAPACITY = -6      /* a per-query limit of this build was reached
+                                  and the result was truncated                 */
 } bsa_status;
 
 typedef enum {
@@ -218,15 +230,21 @@ BSA_API bsa_status bsa_decode(const bsa_kv_desc *desc, const float *q, const voi
  * ws_bytes, using a 4 MiB scratch array built into the library (a
  * file-scope device array: every GPU that loads the library holds it until
  * the process exits).  It allocates nothing.
- *  - The first call on a device looks up the array's device address with
- *    cudaGetSymbolAddress (with that device current) and caches it; make
- *    that first call before any stream capture.
- *  - Every call shares the one array and zeroes its counters first, on
- *    `stream`.  Calls that may overlap on the GPU (other streams, other host
- *    threads) race on it and give wrong results: serialise them.
+ *  - The first call in each CUDA context (per device, and again after a
+ *    device reset) looks up the array's device address with
+ *    cudaGetSymbolAddress, with that device current, and caches it under the
+ *    context's unique id; make that first call before any stream capture.
+ *  - Every call shares the one array and zeroes its status word and counters
+ *    first, on `stream`, after its arguments have been checked (a rejected
+ *    call touches nothing).  Calls that may overlap on the GPU (other
+ *    streams, other host threads) race on it and give wrong results:
+ *    serialise them.
+ *  - The status word of a call (a timed-out wait) stays readable until the
+ *    next call zeroes it: bsa_workspace_status(NULL, 0, ...).
  *  - A problem that needs more scratch than 4 MiB (what bsa_workspace_size
- *    reports for BSA_OP_DECODE with these sizes) is rejected with
- *    BSA_ERR_WORKSPACE before anything is launched. */
+ *    reports for BSA_OP_DECODE with these sizes and the selection parameters
+ *    whose bsa_max_ranges() is max_ranges) is rejected with BSA_ERR_WORKSPACE
+ *    before anything is launched. */
 BSA_API bsa_status bsa_decode_noalloc(const bsa_kv_desc *desc, const float *q, const void *K,
                                       const void *V, const int32_t *ranges,
                                       const int32_t *n_ranges, int32_t max_ranges,
@@ -325,6 +343,32 @@ BSA_API bsa_status bsa_gather_rows(const bsa_kv_desc *src, const void *K, const 
                                    const bsa_kv_desc *dst, void *K_out, void *V_out,
                                    const int32_t *rows, int64_t n, int64_t dst_row0,
                                    bsa_stream_t stream);
+
+/* Reads the sticky device-side status word of a workspace (see the
+ * conventions above) once the work enqueued on `stream` so far has finished:
+ * the call waits for the stream, so it must not be made while the stream is
+ * being captured into a CUDA graph (it then returns BSA_ERR_CUDA).
+ * ws == NULL reads the scratch built into the library for
+ * bsa_decode_noalloc on the current device (ws_bytes is then ignored).
+ * When clear != 0 the word is reset to zero afterwards.  bits (host, may be
+ * NULL) receives the raw word.  Returns BSA_OK when no bit is set,
+ * BSA_ERR_TIMEOUT when a wait bit (0, 1 or 3) is set, otherwise
+ * BSA_ERR_CAPACITY; BSA_ERR_WORKSPACE for a workspace smaller than 4 bytes or
+ * misaligned; BSA_ERR_CUDA when the stream or the copy fails. */
+BSA_API bsa_status bsa_workspace_status(const void *ws, size_t ws_bytes, int32_t clear,
+                                        uint32_t *bits, bsa_stream_t stream);
+
+/* Test hook, not part of the method: the next decode launch of this process
+ * (bsa_decode, bsa_decode_step or bsa_decode_noalloc on the tensor-core path)
+ * makes one warp of its first CTA wait, before any tile copy is issued, on a
+ * barrier that nothing completes, giving up after limit_us microseconds
+ * (1 <= limit_us <= 100,000; 0 disarms).  The wait ends by its limit, sets
+ * the timeout bit of the status word as a real stalled copy would, and the
+ * launch then runs to completion with correct results, so a caller can check
+ * that a wait which gives up is reported (bsa_workspace_status returns
+ * BSA_ERR_TIMEOUT) without stalling anything.  BSA_ERR_ARG for a limit out of
+ * range. */
+BSA_API bsa_status bsa_test_arm_wait_limit(int32_t limit_us);
 
 /* Static text for a status code. */
 BSA_API const char *bsa_status_string(bsa_status status);

@@ -348,15 +348,18 @@ def decode_fixed_segment(q_grp, K_seg, V_seg, n_sel: int, n_now: int, kind: int,
 
 
 def semantic_select_positions(q_grp, Kpos_seg, labels, n_blocks: int, pos_limit: int,
-                              budget_tokens: int, centroids=None):
+                              budget_tokens: int, centroids=None, order=None):
     """Semantic-block selection for one query group, in ORIGINAL positions.
 
     labels[p] = block of position p.  A block's centre is computed over all
     its keys in ascending position order (the block's stored order); a query
-    may read a block's positions below pos_limit.  Returns (selected block
-    ids, selected positions ascending, ties, centroids)."""
+    may read a block's positions below pos_limit.  `centroids` and `order`
+    (the stable sort of the positions by label) may be passed in when the
+    same labels are reused.  Returns (selected block ids, selected positions
+    ascending, ties, centroids)."""
     labels = np.asarray(labels)
-    order = np.argsort(labels, kind="stable")            # (block, position)
+    if order is None:
+        order = np.argsort(labels, kind="stable")        # (block, position)
     counts = np.bincount(labels, minlength=n_blocks)
     offs = np.zeros(n_blocks + 1, np.int64)
     offs[1:] = np.cumsum(counts)

@@ -11,3 +11,18 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size parity cases")
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Near-ties across the selection cut (fp64 scores within 1e-6 relative),
+    per test that compared selections with the oracle."""
+    h = sys.modules.get("gpu_harness")
+    if h is None or not h.NEAR_TIES:
+        return
+    tr = terminalreporter
+    tr.section("near-ties at the selection cut (fp64, 1e-6 relative)")
+    tot = [0, 0, 0]
+    for label, (n, with_ties, pairs) in sorted(h.NEAR_TIES.items()):
+        tr.write_line(f"{label}: {n} selections compared, {with_ties} with near-ties, {pairs} pairs")
+        tot = [a + b for a, b in zip(tot, (n, with_ties, pairs))]
+    tr.write_line(f"total: {tot[0]} selections compared, {tot[1]} with near-ties, {tot[2]} pairs")

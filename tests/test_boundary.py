@@ -35,8 +35,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_status_strings(lib):
     assert N.bsa_version() >= 100
-    for s in (0, -1, -2, -3, -4, -5):
-        assert N.status_string(s)
+    for s in (0, -1, -2, -3, -4, -5, -6):
+        assert N.status_string(s) and N.status_string(s) != "unknown status"
 
 
 def _desc(**kw):
@@ -149,3 +149,33 @@ def test_semantic_index_arguments_rejected_on_host(lib):
                              None) == N.BSA_ERR_ARG
     assert L.bsa_gather_rows(ctypes.byref(d), fake, fake, ctypes.byref(d), fake, fake, fake, 0, 0,
                              None) == N.BSA_OK                                           # nothing to do
+
+
+def test_noalloc_checks_arguments_before_touching_its_scratch(lib):
+    """bsa_decode_noalloc makes every check bsa_decode makes before it clears
+    its built-in scratch: on a machine without a GPU, a call that got past the
+    checks would fail in the CUDA runtime (BSA_ERR_CUDA), so BSA_ERR_ARG here
+    shows the rejection came first."""
+    L = N.lib()
+    d = _desc()
+    fake = 1 << 20
+    call = lambda q, K, out, scale, max_r: L.bsa_decode_noalloc(
+        ctypes.byref(d), q, K, fake, fake, fake, max_r, fake, 100, scale, out, None, None)
+    assert call(None, fake, fake, 0.1, 16) == N.BSA_ERR_ARG          # no queries
+    assert call(fake, fake + 2, fake, 0.1, 16) == N.BSA_ERR_ARG      # misaligned K
+    assert call(fake, fake, None, 0.1, 16) == N.BSA_ERR_ARG          # no output
+    assert call(fake, fake, fake, float("nan"), 16) == N.BSA_ERR_ARG
+    assert call(fake, fake, fake, 0.1, 0) == N.BSA_ERR_ARG           # no range slot
+    g16 = _desc(Hq=8 * 16)
+    assert L.bsa_decode_noalloc(ctypes.byref(g16), fake, fake, fake, fake, fake, 16, fake, 100, 0.1,
+                                fake, None, None) == N.BSA_ERR_UNSUPPORTED
+
+
+def test_status_reader_and_test_hook_arguments(lib):
+    L = N.lib()
+    bits = ctypes.c_uint32(7)
+    assert L.bsa_workspace_status(1 << 20, 2, 0, ctypes.byref(bits), None) == N.BSA_ERR_WORKSPACE
+    assert L.bsa_workspace_status((1 << 20) + 2, 64, 0, ctypes.byref(bits), None) == N.BSA_ERR_WORKSPACE
+    assert L.bsa_test_arm_wait_limit(-1) == N.BSA_ERR_ARG
+    assert L.bsa_test_arm_wait_limit(100001) == N.BSA_ERR_ARG
+    assert L.bsa_test_arm_wait_limit(0) == N.BSA_OK                  # disarmed

@@ -16,7 +16,7 @@ import oracle
 from block_sparse_long_build_b200 import workloads as W
 from block_sparse_long_build_b200.session import DecodeSession
 
-from gpu_harness import ATOL, host
+from gpu_harness import ATOL, current_label, host, record_ties
 
 pytestmark = pytest.mark.gpu
 
@@ -56,6 +56,7 @@ def _check_chunk(cfg, wl, sess, p, Tq, rows):
                 sel, pos, ties, _ = oracle.semantic_select_positions(
                     qg, Kpos[0, g, :cfg.L], labels[0, g], cfg.n_blocks, p, p // 16)
                 got = [j for j in range(cfg.n_blocks) if (bitmap[i, g, j // 32] >> (j % 32)) & 1]
+                record_ties(current_label(), ties)
                 assert got == sel, f"chunk {p} row {i} head {g}: selection differs; ties {ties}"
                 rws = np.concatenate([pos, np.arange(p, P + 1)])
             else:

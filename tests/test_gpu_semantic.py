@@ -15,7 +15,7 @@ import oracle
 from block_sparse_long_build_b200 import workloads as W
 from block_sparse_long_build_b200.session import DecodeSession
 
-from gpu_harness import ATOL, host
+from gpu_harness import ATOL, assert_status_clean, current_label, host, record_ties
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +48,7 @@ def test_semantic_decode_matches_oracle(cfg):
         Vpos[0, :, L + t] = host(v)[0]
         sess.step(t, q, k, v)
         torch.cuda.synchronize()
+        assert_status_clean(sess.ws, f"after step {t}")
         qh = host(q)
         out = sess.out.cpu().numpy()
         sel = sess.sel_blocks.cpu().numpy()
@@ -56,6 +57,7 @@ def test_semantic_decode_matches_oracle(cfg):
             qg = qh[0, g * cfg.G:(g + 1) * cfg.G]
             ref_sel, pos, ties, _ = oracle.semantic_select_positions(
                 qg, Kpos[0, g, :L], labels[0, g], cfg.n_blocks, L - loc, cfg.budget_tokens)
+            record_ties(current_label(), ties)
             assert sel[g, :cnt[g]].tolist() == ref_sel, f"step {t} head {g}: near-ties {ties}"
             rows = np.concatenate([pos, np.arange(L - loc, L + t + 1)])
             ref, _ = oracle.attend(qg, Kpos[0, g], Vpos[0, g], rows, 1 / math.sqrt(cfg.D))
