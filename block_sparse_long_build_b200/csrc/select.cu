@@ -578,39 +578,35 @@ __global__ void __launch_bounds__(kPickThreads, 2) pick_kernel(SelArgs a) {
 }
 
 
-// The same selection for segments of at most 32 * kPickSmallKeys blocks, by one
-// warp per segment with no CTA barrier: lane l holds blocks l + 32 r in
-// registers; the walk takes the best remaining candidate (highest key, then
-// lowest index; for a budget, the best that still fits: keys that no longer
-// fit are cleared) with a redux.sync max and min per step until k blocks or
-// nothing is left; a ballot per r compacts the taken blocks in index order
-// straight into their place among the forced ranges; the merged ranges come
-// from a warp scan (running maximum of the ends), 32 items per pass.
-// Shared memory: (lo, hi) of max_sel + 2 items.
-constexpr int kPickSmallKeys = 32;
-
-__global__ void __launch_bounds__(32) pick_small_kernel(SelArgs a) {
+// The same selection for fixed blocks, segments of at most 32 * NK blocks,
+// by one warp per segment with no CTA barrier: lane l holds the keys of
+// blocks l + 32 r in registers.  The k-th largest key T is found bit by bit
+// from the top (T gains bit b when at least k candidate keys are >= T | b: one
+// warp-wide count per bit); the selected blocks are those with key > T and,
+// among the keys equal to T, the k - count(> T) of lowest index (ballots in
+// index order).  A ballot per r compacts them in index order straight into
+// their place among the forced ranges; the merged ranges come from a warp
+// scan (running maximum of the ends), 32 items per pass.  Shared memory:
+// (lo, hi) of max_sel + 2 items.
+template <int NK>
+__global__ void __launch_bounds__(32) pick_warp_kernel(SelArgs a) {
+    static_assert(NK >= 1 && NK <= 64, "taken[] holds 64 bits");
     extern __shared__ __align__(16) unsigned char psm[];
     int2 *items = reinterpret_cast<int2 *>(psm);
     const int s = blockIdx.x, b = s / a.Hkv, lane = threadIdx.x;
     const int nb = a.nb_total;
-    const int32_t *off = a.offsets ? a.offsets + (int64_t)s * (nb + 1) : nullptr;
-    pdl_wait();   // keys and visible counts from score_kernel
-    uint32_t wk[kPickSmallKeys];
-    int wv[kPickSmallKeys];
+    pdl_wait();   // keys from score_kernel
+    uint32_t wk[NK];
 #pragma unroll
-    for (int r = 0; r < kPickSmallKeys; ++r) {
+    for (int r = 0; r < NK; ++r) {
         const int j = lane + 32 * r;
         wk[r] = j < nb ? a.keys[(int64_t)s * nb + j] : 0u;
-        wv[r] = off && j < nb ? a.vis[(int64_t)s * nb + j] : 0;
     }
     // forced token ranges (every lane computes the same), sorted and merged
     const int n = min(max(a.cur_len[b], 0), a.L_max);
     int f_lo[2] = {0, 0}, f_hi[2] = {0, 0}, nf = 0;
-    if (off) {
-        if (n > a.local_start) { f_lo[0] = max(a.local_start, 0); f_hi[0] = n; nf = 1; }
-    } else {
-        if (a.sink > 0 && n > 0) { f_lo[0] = 0; f_hi[0] = min(a.sink, n); nf = 1; }
+    if (a.sink > 0 && n > 0) { f_lo[0] = 0; f_hi[0] = min(a.sink, n); nf = 1; }
+    {
         int t0 = n;
         if (a.window > 0) t0 = min(t0, max(0, n - a.window));
         if (a.keep_current && n > 0) t0 = min(t0, ((n - 1) / a.S) * a.S);
@@ -620,11 +616,11 @@ __global__ void __launch_bounds__(32) pick_small_kernel(SelArgs a) {
             else { f_lo[1] = t0; f_hi[1] = n; nf = 2; }
         }
     }
-    // candidates: keys > 0 and (fixed blocks) not wholly inside the forced set
+    // candidates: keys > 0 and not wholly inside the forced set
     int my_c = 0;
 #pragma unroll
-    for (int r = 0; r < kPickSmallKeys; ++r) {
-        if (wk[r] && !off) {
+    for (int r = 0; r < NK; ++r) {
+        if (wk[r]) {
             const int64_t r0 = (int64_t)(lane + 32 * r) * a.S, r1 = r0 + a.S;
 #pragma unroll
             for (int i = 0; i < 2; ++i)
@@ -633,48 +629,41 @@ __global__ void __launch_bounds__(32) pick_small_kernel(SelArgs a) {
         my_c += wk[r] != 0u;
     }
     const int n_cand = __reduce_add_sync(0xffffffffu, my_c);
-    const bool greedy = off && a.topk < 0;
-    const int limit = greedy ? a.max_sel : min(min(a.topk >= 0 ? a.topk : a.budget / a.S, n_cand), a.max_sel);
-    int remaining = a.budget;
-    if (greedy) {
+    const int k = min(min(a.topk >= 0 ? a.topk : a.budget / a.S, n_cand), a.max_sel);
+    uint64_t taken = 0;   // bit r: block lane + 32 r (NK <= 64)
+    if (k > 0) {
+        // T = the k-th largest candidate key (>= 1, since k <= n_cand)
+        uint32_t T = 0u;
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t c = T | (1u << bit);
+            int cnt = 0;
 #pragma unroll
-        for (int r = 0; r < kPickSmallKeys; ++r)
-            if (wv[r] > remaining) wk[r] = 0u;
-    }
-    uint32_t taken = 0;   // bit r: block lane + 32 r
-    for (int t = 0; t < limit; ++t) {
-        uint32_t lm = 0u;
+            for (int r = 0; r < NK; ++r) cnt += wk[r] >= c;
+            if (__reduce_add_sync(0xffffffffu, cnt) >= k) T = c;
+        }
+        int gt = 0;
 #pragma unroll
-        for (int r = 0; r < kPickSmallKeys; ++r) lm = max(lm, wk[r]);
-        const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
-        if (m == 0u) break;
-        int cand = 0x7fffffff;
+        for (int r = 0; r < NK; ++r) gt += wk[r] > T;
+        const int need_eq = k - __reduce_add_sync(0xffffffffu, gt);
+        int eq_seen = 0;
 #pragma unroll
-        for (int r = kPickSmallKeys - 1; r >= 0; --r) cand = wk[r] == m ? lane + 32 * r : cand;
-        const int j = __reduce_min_sync(0xffffffffu, cand);
-        int vj = 0;
-#pragma unroll
-        for (int r = 0; r < kPickSmallKeys; ++r)
-            if (lane + 32 * r == j) { taken |= 1u << r; wk[r] = 0u; vj = wv[r]; }
-        if (greedy) {
-            remaining -= __shfl_sync(0xffffffffu, vj, j & 31);
-#pragma unroll
-            for (int r = 0; r < kPickSmallKeys; ++r)
-                if (wv[r] > remaining) wk[r] = 0u;
+        for (int r = 0; r < NK; ++r) {
+            const uint32_t eqm = __ballot_sync(0xffffffffu, wk[r] == T);
+            const int rank = eq_seen + __popc(eqm & ((1u << lane) - 1u));
+            if (wk[r] > T || (wk[r] == T && rank < need_eq)) taken |= 1ull << r;
+            eq_seen += __popc(eqm);
         }
     }
     // index-ordered compaction, each block written at its place among the
     // forced ranges (a forced range comes first on equal starts)
     int n_sel = 0, below[2] = {0, 0};   // below[f]: taken blocks starting before f_lo[f]
 #pragma unroll
-    for (int r = 0; r < kPickSmallKeys; ++r) {
-        const uint32_t mk = __ballot_sync(0xffffffffu, (taken >> r) & 1u);
-        if ((taken >> r) & 1u) {
+    for (int r = 0; r < NK; ++r) {
+        const uint32_t mk = __ballot_sync(0xffffffffu, (uint32_t)(taken >> r) & 1u);
+        if ((taken >> r) & 1ull) {
             const int p = n_sel + __popc(mk & ((1u << lane) - 1u));
             const int jj = lane + 32 * r;
-            int lo, hi;
-            if (off) { lo = min(max(off[jj], 0), a.L_max); hi = lo + wv[r]; }
-            else { lo = jj * a.S; hi = lo + a.S; }
+            const int lo = jj * a.S, hi = lo + a.S;
             int before = 0;
 #pragma unroll
             for (int f = 0; f < 2; ++f) {
@@ -804,14 +793,19 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
         BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(kPickThreads), smem2, st, a));
         return BSA_OK;
     };
-    // one warp per segment for small top-k problems (a long walk, or the
-    // token budget walk over variable blocks, measured faster in the CTA
-    // kernel)
-    const int64_t k_host = p->topk >= 0 ? p->topk : (p->block_size > 0 ? p->budget_tokens / p->block_size : 0);
-    if (nb_total <= 32 * kPickSmallKeys && !variable && k_host <= 32) {
+    // fixed blocks, up to 2,048 per segment: one warp per segment with the
+    // keys in registers (the token-budget walk over variable blocks measured
+    // faster in the CTA kernel)
+    if (!variable && nb_total <= 32 * 64) {
         const size_t smem3 = (size_t)(max_sel + 4) * 8;
-        BSA_CUDA_TRY(launch_pdl(pick_small_kernel, dim3((unsigned)nseg), dim3(32), smem3, st, a));
-        return BSA_OK;
+        auto warp_pick = [&](auto kern) -> bsa_status {
+            BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(32), smem3, st, a));
+            return BSA_OK;
+        };
+        if (nb_total <= 32 * 16) return warp_pick(pick_warp_kernel<16>);
+        if (nb_total <= 32 * 32) return warp_pick(pick_warp_kernel<32>);
+        if (nb_total <= 32 * 48) return warp_pick(pick_warp_kernel<48>);
+        return warp_pick(pick_warp_kernel<64>);
     }
     return pick(pick_kernel);
 }
