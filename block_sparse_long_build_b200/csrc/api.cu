@@ -72,8 +72,9 @@ static EncodeTiledFn encode_fn() {
 bool make_kv_tmap(CUtensorMap *map, const bsa_kv_desc *d, const void *base, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[4] = {(cuuint64_t)d->D, (cuuint64_t)d->L_max, (cuuint64_t)d->Hkv,
-                                (cuuint64_t)d->B};
+    const bool paged = d->page_rows > 0;
+    const cuuint64_t dims[4] = {(cuuint64_t)d->D, (cuuint64_t)(paged ? d->page_rows : d->L_max),
+                                (cuuint64_t)d->Hkv, (cuuint64_t)(paged ? d->n_pages : d->B)};
     const cuuint64_t strides[3] = {(cuuint64_t)d->stride_t * 2, (cuuint64_t)d->stride_h * 2,
                                    (cuuint64_t)d->stride_b * 2};
     const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
@@ -112,6 +113,12 @@ static bool desc_ok(const bsa_kv_desc *d) {
     if (d->stride_t < d->D || d->stride_h < 1 || d->stride_b < 1) return false;
     const int64_t es = elem_size(d);
     if ((d->stride_t * es) % 16 || (d->stride_h * es) % 16 || (d->stride_b * es) % 16) return false;
+    if (d->page_rows < 0) return false;
+    if (d->page_rows > 0) {   // paged pool
+        if (d->page_rows % 16 || d->pages_per_seq < 1 || !d->page_table || d->n_pages < 1 ||
+            d->n_pages > 0x7fffffffLL || (int64_t)d->pages_per_seq * d->page_rows != d->L_max)
+            return false;
+    }
     return true;
 }
 
@@ -257,7 +264,7 @@ bsa_status bsa_build_semantic_index(const bsa_kv_desc *d, const void *K, int64_t
     if (!desc_ok(d) || !K || !init || !centres || !labels || !offsets || !order) return BSA_ERR_ARG;
     if (L < 1 || L > d->L_max || L > 0x7fffffffLL || k < 1 || k > L || iters < 1) return BSA_ERR_ARG;
     if (!aligned16(K) || !aligned16(centres)) return BSA_ERR_ARG;
-    if (!kmeans_supported(d, k)) return BSA_ERR_UNSUPPORTED;
+    if (d->page_rows > 0 || !kmeans_supported(d, k)) return BSA_ERR_UNSUPPORTED;
     if (!ws_ok(ws, ws_bytes, kmeans_ws_bytes(d, L, k))) return BSA_ERR_WORKSPACE;
     return launch_kmeans(d, K, L, k, iters, init, centres, labels, offsets, order, ws, (cudaStream_t)stream);
 }
@@ -269,6 +276,7 @@ bsa_status bsa_gather_rows(const bsa_kv_desc *src, const void *K, const void *V,
     if (src->B != dst->B || src->Hkv != dst->Hkv || src->D != dst->D || src->kv_dtype != dst->kv_dtype)
         return BSA_ERR_ARG;
     if (!aligned16(K) || !aligned16(V) || !aligned16(K_out) || !aligned16(V_out)) return BSA_ERR_ARG;
+    if (src->page_rows > 0 || dst->page_rows > 0) return BSA_ERR_UNSUPPORTED;
     if (n < 0 || dst_row0 < 0 || dst_row0 + n > dst->L_max) return BSA_ERR_ARG;
     if (n == 0) return BSA_OK;
     return launch_gather_rows(src, K, V, dst, K_out, V_out, rows, n, dst_row0, (cudaStream_t)stream);
@@ -421,6 +429,7 @@ bsa_status bsa_prefill_grouped(const bsa_kv_desc *d, const void *K, const void *
         !aligned16(out) || !aligned16(summaries))
         return BSA_ERR_ARG;
     if (p->block_size != 0 || p->topk >= 0) return BSA_ERR_UNSUPPORTED;
+    if (d->page_rows > 0 || pd->page_rows > 0) return BSA_ERR_UNSUPPORTED;
     if (d->B != 1 || pd->B != 1 || d->Hkv != pd->Hkv || d->Hq != pd->Hq || d->D != pd->D)
         return BSA_ERR_ARG;
     if (d->kv_dtype != BSA_BF16 || pd->kv_dtype != BSA_BF16 || d->D != 128) return BSA_ERR_UNSUPPORTED;

@@ -378,7 +378,8 @@ inline size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 int num_sms();
 
 // Encodes a 4-D bf16 tensor map over a KV cache: dims (D, L_max, Hkv, B),
-// box (64, rows, 1, 1), 128-byte swizzle, zero fill out of bounds.
+// or (D, page rows, Hkv, pages) for a paged pool; box (64, rows, 1, 1),
+// 128-byte swizzle, zero fill out of bounds.
 bool make_kv_tmap(CUtensorMap *map, const bsa_kv_desc *desc, const void *base, int box_rows);
 
 // Encodes a 2-D tensor map over `rows` rows of `row_bytes` bytes holding
@@ -394,6 +395,35 @@ struct WsLayout {
     size_t scratch = 0;    // offset of the op's scratch
     size_t total = 0;
 };
+
+// Where the rows of a cache live: contiguous [B][Hkv][L_max][D], or paged (a
+// pool [pages][Hkv][P][D] reached through a page table per sequence).
+struct KvRows {
+    int64_t stride_b, stride_h, stride_t;   // paged: stride_b is between pages
+    const int32_t *table;                   // nullptr: contiguous
+    int32_t P, pps;                         // paged: rows per page, table entries per sequence
+    int64_t n_pages;
+    // Element offset of logical row r of segment (b, g), or -1 when the row's
+    // page is outside the pool.
+    __device__ __forceinline__ int64_t off(int b, int g, int64_t r) const {
+        if (!table) return b * stride_b + g * stride_h + r * stride_t;
+        const int64_t pg = __ldg(table + (int64_t)b * pps + r / P);
+        if (pg < 0 || pg >= n_pages) return -1;
+        return pg * stride_b + g * stride_h + (r % P) * stride_t;
+    }
+};
+
+inline KvRows kv_rows(const bsa_kv_desc *d) {
+    KvRows r;
+    r.stride_b = d->stride_b;
+    r.stride_h = d->stride_h;
+    r.stride_t = d->stride_t;
+    r.table = d->page_rows > 0 ? d->page_table : nullptr;
+    r.P = d->page_rows > 0 ? d->page_rows : 1;
+    r.pps = d->pages_per_seq;
+    r.n_pages = d->n_pages;
+    return r;
+}
 
 // Fused append of the step's new row (k_new == nullptr: none): the same
 // bookkeeping as the append kernel, done inside the decode grid.

@@ -47,7 +47,8 @@ struct DecArgs {
     int max_ranges;
     const int32_t *cur_len;
     const void *K, *V;
-    int64_t stride_b, stride_h, stride_t;
+    KvRows rows;          // where each logical row lives (contiguous or paged)
+    int aligned;          // pieces cut at multiples of 16 rows (paged pools)
     int B, Hq, Hkv, G, D, L_max, nsplit;
     float scale_log2;
     float *part_o;        // [nseg][nsplit][G][D]
@@ -139,6 +140,26 @@ __device__ __forceinline__ int2 clamp_range(const DecArgs &a, int2 v, bool last,
     return make_int2(lo, hi);
 }
 
+// 16-row pieces of range x.  A contiguous cache cuts the range from its
+// start; a paged pool cuts it at multiples of 16 rows so that no piece
+// straddles a page (the first and last pieces may then use part of their
+// 16-row box).
+__device__ __forceinline__ int piece_count(int2 x, bool al) {
+    if (x.y <= x.x) return 0;
+    return al ? (x.y + kPiece - 1) / kPiece - x.x / kPiece : (x.y - x.x + kPiece - 1) / kPiece;
+}
+
+// Piece q of range x: (first row of its 16-row box, valid rows lo | hi << 8
+// of the box).
+__device__ __forceinline__ int2 piece_of(int2 x, int q, bool al) {
+    if (al) {
+        const int row = (x.x / kPiece + q) * kPiece;
+        return make_int2(row, max(x.x - row, 0) | (min(x.y - row, kPiece) << 8));
+    }
+    const int row = x.x + q * kPiece;
+    return make_int2(row, min(kPiece, x.y - row) << 8);
+}
+
 // Warp-local view of a segment's range table (no CTA-wide barrier): lane l
 // owns the slots [r0, r1) = [l k, l k + k), k = ceil(max_ranges / 32), and
 // pbase is the number of 16-row pieces in the slots before r0.  The CTA's
@@ -150,24 +171,41 @@ struct WarpRanges {
 };
 
 // Writes the table entries of range x (first piece pp) for warp-local
-// indices i in [i0, i0 + kWarpCap).
+// indices i in [i0, i0 + kWarpCap): (box row, valid rows, TMA row coordinate,
+// TMA outer coordinate); a paged pool's coordinates are filled in by
+// warp_translate.
 __device__ __forceinline__ void fill_range(const WarpRanges &w, int2 x, int pp, int warp, int i0,
-                                           int2 *tab) {
-    const int cnt = (x.y - x.x + kPiece - 1) / kPiece;
+                                           int b, bool al, int4 *tab) {
+    const int cnt = piece_count(x, al);
     const int lo_p = pp - w.first - warp;                       // i >= ceil(lo_p / 4)
     const int hi_p = min(pp + cnt, w.last) - w.first - warp;    // i <  ceil(hi_p / 4)
     const int ia = max(lo_p > 0 ? (lo_p + kDecWarps - 1) / kDecWarps : 0, i0);
     const int ib = min(hi_p > 0 ? (hi_p + kDecWarps - 1) / kDecWarps : 0, i0 + kWarpCap);
     for (int i = ia; i < ib; ++i) {
-        const int row = x.x + (w.first + warp + kDecWarps * i - pp) * kPiece;
-        tab[i - i0] = make_int2(row, min(kPiece, x.y - row));
+        const int2 pr = piece_of(x, w.first + warp + kDecWarps * i - pp, al);
+        tab[i - i0] = make_int4(pr.x, pr.y, pr.x, b);
+    }
+}
+
+// Paged pool: the TMA coordinates (row in page, page) of the table entries
+// [0, n), looked up in the sequence's page table by all lanes together.  An
+// entry outside the pool gives an out-of-bounds box, which reads zeros.
+__device__ __forceinline__ void warp_translate(const DecArgs &a, int b, int lane, int n, int4 *tab) {
+    if (!a.rows.table) return;
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+        int4 e = tab[i];
+        e.z = e.x % a.rows.P;
+        e.w = __ldg(a.rows.table + (int64_t)b * a.rows.pps + e.x / a.rows.P);
+        tab[i] = e;
     }
 }
 
 // Scans the range table and fills the first window of this warp's piece
 // table (the caller syncs the warp before reading it).
 __device__ __forceinline__ WarpRanges warp_ranges(const DecArgs &a, int s, int b, int c, int warp,
-                                                  int lane, int2 *tab) {
+                                                  int lane, int4 *tab) {
+    const bool al = a.aligned != 0;
     WarpRanges w;
     w.R = a.ranges + (int64_t)s * a.max_ranges * 2;
     const int k = (a.max_ranges + 31) >> 5;
@@ -187,11 +225,11 @@ __device__ __forceinline__ WarpRanges warp_ranges(const DecArgs &a, int s, int b
 #pragma unroll
     for (int j = 0; j < kRegRanges; ++j) {
         rv[j] = clamp_range(a, rv[j], w.r0 + j == w.nr - 1, w.cl);
-        if (w.r0 + j < end) cnt += (rv[j].y - rv[j].x + kPiece - 1) / kPiece;
+        if (w.r0 + j < end) cnt += piece_count(rv[j], al);
     }
     for (int r = w.r0 + kRegRanges; r < end; ++r) {
         const int2 x = clamp_range(a, __ldg(R2 + r), r == w.nr - 1, w.cl);
-        cnt += (x.y - x.x + kPiece - 1) / kPiece;
+        cnt += piece_count(x, al);
     }
     int incl = cnt;
 #pragma unroll
@@ -209,25 +247,27 @@ __device__ __forceinline__ WarpRanges warp_ranges(const DecArgs &a, int s, int b
 #pragma unroll
     for (int j = 0; j < kRegRanges; ++j)
         if (w.r0 + j < end && pp < w.last) {
-            fill_range(w, rv[j], pp, warp, 0, tab);
-            pp += (rv[j].y - rv[j].x + kPiece - 1) / kPiece;
+            fill_range(w, rv[j], pp, warp, 0, b, al, tab);
+            pp += piece_count(rv[j], al);
         }
     for (int r = w.r0 + kRegRanges; r < end && pp < w.last; ++r) {
         const int2 x = clamp_range(a, __ldg(R2 + r), r == w.nr - 1, w.cl);
-        fill_range(w, x, pp, warp, 0, tab);
-        pp += (x.y - x.x + kPiece - 1) / kPiece;
+        fill_range(w, x, pp, warp, 0, b, al, tab);
+        pp += piece_count(x, al);
     }
     return w;
 }
 
 // Refills the table with the window i in [i0, i0 + kWarpCap).
-__device__ __forceinline__ void warp_refill(const DecArgs &a, const WarpRanges &w, int warp, int i0, int2 *tab) {
+__device__ __forceinline__ void warp_refill(const DecArgs &a, const WarpRanges &w, int warp, int i0,
+                                            int b, int4 *tab) {
+    const bool al = a.aligned != 0;
     int pp = w.pbase;
     const int end = min(w.r1, w.nr);
     for (int r = w.r0; r < end && pp < w.last; ++r) {
         const int2 x = clamp_range(a, __ldg(reinterpret_cast<const int2 *>(w.R) + r), r == w.nr - 1, w.cl);
-        fill_range(w, x, pp, warp, i0, tab);
-        pp += (x.y - x.x + kPiece - 1) / kPiece;
+        fill_range(w, x, pp, warp, i0, b, al, tab);
+        pp += piece_count(x, al);
     }
 }
 
@@ -416,14 +456,14 @@ __device__ __forceinline__ void finish_append(const DecArgs &a, int b, int g, in
     const DecAppend &p = a.app;
     if (owner && p.summ && p.S > 0 && (n + 1) % p.S == 0) {
         const int j = (n + 1) / p.S - 1;
-        const uint16_t *Kseg = static_cast<const uint16_t *>(a.K) + b * a.stride_b + g * a.stride_h;
+        const uint16_t *K = static_cast<const uint16_t *>(a.K);
         char *out = static_cast<char *>(p.summ) + ((int64_t)(b * a.Hkv + g) * p.nb_total + j) * p.row_bytes;
         if (p.kind == BSA_SUM_MINMAX)
-            summarize_minmax<uint16_t>(Kseg, a.stride_t, a.D, (int64_t)j * p.S, (int64_t)(j + 1) * p.S,
+            summarize_minmax<uint16_t>(K, a.rows, b, g, a.D, (int64_t)j * p.S, (int64_t)(j + 1) * p.S,
                                        reinterpret_cast<uint16_t *>(out));
         else
-            summarize_centroid<uint16_t>(Kseg, a.stride_t, a.D, (int64_t)j * p.S,
-                                         (int64_t)(j + 1) * p.S, reinterpret_cast<float *>(out));
+            summarize_centroid<uint16_t>(K, a.rows, b, g, a.D, (int64_t)j * p.S, (int64_t)(j + 1) * p.S,
+                                         reinterpret_cast<float *>(out));
     }
     if (threadIdx.x == 0) {
         __threadfence();
@@ -444,11 +484,11 @@ template <int NH, int NST>
 struct TcSmem {
     static constexpr int kPieceBytes = 2 * NH * kBoxBytes;
     static constexpr int kRing = kDecWarps * NST * kPieceBytes;
-    static constexpr int kInfo = kRing;                               // int2 [warps][NST]
+    static constexpr int kInfo = kRing;                               // int [warps][NST], 8-B slots
     static constexpr int kBars = kInfo + kDecWarps * NST * 8;         // u64  [warps][NST]
     static constexpr int kMisc = kBars + kDecWarps * NST * 8;         // float sml[2*kMaxG], int tmp[36]
-    static constexpr int kPtab = kMisc + 2 * kMaxG * 4 + 36 * 4;      // int2 [warps][kWarpCap]
-    static constexpr int kStall = kPtab + kDecWarps * kWarpCap * 8;   // u64: test-hook barrier
+    static constexpr int kPtab = kMisc + 2 * kMaxG * 4 + 36 * 4;      // int4 [warps][kWarpCap]
+    static constexpr int kStall = kPtab + kDecWarps * kWarpCap * 16;  // u64: test-hook barrier
     static constexpr int kBytes = kStall + 8 + 1024;
     static_assert(kRing >= kDecWarps * kMaxG * (2 + 64 * NH) * 4,
                   "per-warp partials must fit in the ring");
@@ -467,7 +507,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     int2 *info = reinterpret_cast<int2 *>(dsm + L::kInfo);
     uint64_t *full = reinterpret_cast<uint64_t *>(dsm + L::kBars);
     float *sml = reinterpret_cast<float *>(dsm + L::kMisc);
-    int2 *ptab = reinterpret_cast<int2 *>(dsm + L::kPtab);
+    int4 *ptab = reinterpret_cast<int4 *>(dsm + L::kPtab);
 
     const int c = blockIdx.x, s = blockIdx.y;
     const int b = s / a.Hkv, g = s % a.Hkv;
@@ -478,8 +518,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // first load.
     unsigned char *ring = dsm + warp * NST * L::kPieceBytes;
     uint64_t *wfull = full + warp * NST;
-    int2 *winfo = info + warp * NST;
-    int2 *wtab = ptab + warp * kWarpCap;
+    int2 *winfo = info + warp * NST;   // .x: valid rows of the stage's piece
+    int4 *wtab = ptab + warp * kWarpCap;
     if (tid == 0) {
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
@@ -511,16 +551,17 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     const int n_my = wr.last - wr.first;
     // this warp's pieces: CTA-local indices warp, warp + 4, warp + 8, ...
     const int my_count = n_my > warp ? (n_my - warp + kDecWarps - 1) / kDecWarps : 0;
+    warp_translate(a, b, lane, min(my_count, kWarpCap), wtab);
     __syncwarp();
     auto issue = [&](int idx, int st) {   // lane 0 only
-        const int2 pr = wtab[idx % kWarpCap];
-        winfo[st] = pr;
+        const int4 pr = wtab[idx % kWarpCap];
+        winfo[st].x = pr.y;
         mbar_arrive_expect_tx(&wfull[st], (uint32_t)(2 * NH * kBoxBytes));
         unsigned char *dst = ring + st * L::kPieceBytes;
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-            tma_load_4d(dst + h * kBoxBytes, &tmK, &wfull[st], h * 64, pr.x, g, b);
-            tma_load_4d(dst + (NH + h) * kBoxBytes, &tmV, &wfull[st], h * 64, pr.x, g, b);
+            tma_load_4d(dst + h * kBoxBytes, &tmK, &wfull[st], h * 64, pr.z, g, pr.w);
+            tma_load_4d(dst + (NH + h) * kBoxBytes, &tmV, &wfull[st], h * 64, pr.z, g, pr.w);
         }
     };
     // Warp-collective, before piece idx is issued: if the piece holds the
@@ -528,14 +569,16 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     bool wrote = false;
     auto maybe_append = [&](int idx) {
         if (wr.app < 0) return;
-        const int2 pr = wtab[idx % kWarpCap];
-        if (pr.x <= wr.app && wr.app < pr.x + pr.y) {
-            const int64_t off = b * a.stride_b + g * a.stride_h + (int64_t)wr.app * a.stride_t;
-            if (lane < kChunks)
-                reinterpret_cast<uint4 *>(static_cast<uint16_t *>(const_cast<void *>(a.K)) + off)[lane] = nkv;
-            else if (lane >= 16 && lane - 16 < kChunks)
-                reinterpret_cast<uint4 *>(static_cast<uint16_t *>(const_cast<void *>(a.V)) + off)[lane - 16] = nkv;
-            asm volatile("fence.proxy.async.global;" ::: "memory");
+        const int4 pr = wtab[idx % kWarpCap];
+        if (pr.x + (pr.y & 255) <= wr.app && wr.app < pr.x + (pr.y >> 8)) {
+            const int64_t off = a.rows.off(b, g, wr.app);
+            if (off >= 0) {   // (a row whose page is outside the pool is not written)
+                if (lane < kChunks)
+                    reinterpret_cast<uint4 *>(static_cast<uint16_t *>(const_cast<void *>(a.K)) + off)[lane] = nkv;
+                else if (lane >= 16 && lane - 16 < kChunks)
+                    reinterpret_cast<uint4 *>(static_cast<uint16_t *>(const_cast<void *>(a.V)) + off)[lane - 16] = nkv;
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+            }
             __syncwarp();
             wrote = true;
         }
@@ -580,14 +623,16 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     for (int idx = 0; idx < my_count; ++idx) {
         const int st = idx % NST;
         if (!timed_out && !mbar_wait_bounded(&wfull[st], (uint32_t)((idx / NST) & 1))) timed_out = true;
-        const int nv = winfo[st].y;
+        const int vr = winfo[st].x;
+        const int vlo = vr & 255, vhi = vr >> 8;   // valid rows [vlo, vhi) of the box
         unsigned char *kp = ring + st * L::kPieceBytes;
         unsigned char *vp = kp + NH * kBoxBytes;
-        if (nv < kPiece) {   // rows past the range end: zero V so 0 * junk stays 0
-            for (int e = lane; e < (kPiece - nv) * NH * 8; e += 32) {
-                const int r = nv + e / (NH * 8), h = (e / 8) % NH, ch = e % 8;
-                *reinterpret_cast<uint4 *>(vp + h * kBoxBytes + r * 128 + ch * 16) =
-                    make_uint4(0, 0, 0, 0);
+        if (vlo > 0 || vhi < kPiece) {   // rows outside the range: zero V so 0 * junk stays 0
+            for (int e = lane; e < kPiece * NH * 8; e += 32) {
+                const int r = e / (NH * 8), h = (e / 8) % NH, ch = e % 8;
+                if (r < vlo || r >= vhi)
+                    *reinterpret_cast<uint4 *>(vp + h * kBoxBytes + r * 128 + ch * 16) =
+                        make_uint4(0, 0, 0, 0);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -619,7 +664,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             for (int e = 0; e < 2; ++e) {
                 const int tok = n * 8 + 2 * tig + e;
                 const float v = (sa[n][e] + sb[n][e]) + (sa[n][2 + e] + sb[n][2 + e]);
-                lg[n * 2 + e] = tok < nv ? v * a.scale_log2 : kNegInf;
+                lg[n * 2 + e] = tok >= vlo && tok < vhi ? v * a.scale_log2 : kNegInf;
             }
         float mx = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -668,7 +713,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         __syncwarp();
         if (idx + NST < my_count) {
             if ((idx + NST) % kWarpCap == 0) {   // next window of this warp's pieces
-                warp_refill(a, wr, warp, idx + NST, wtab);
+                warp_refill(a, wr, warp, idx + NST, b, wtab);
+                warp_translate(a, b, lane, min(my_count - (idx + NST), kWarpCap), wtab);
                 __syncwarp();
             }
             maybe_append(idx + NST);
@@ -744,16 +790,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_generic_kernel(DecArgs a) 
 #pragma unroll
         for (int k = 0; k < PER; ++k) o[h][k] = 0.0f;
     }
-    const T *Ks = static_cast<const T *>(a.K) + b * a.stride_b + g * a.stride_h;
-    const T *Vs = static_cast<const T *>(a.V) + b * a.stride_b + g * a.stride_h;
+    const T *Ks = static_cast<const T *>(a.K);
+    const T *Vs = static_cast<const T *>(a.V);
     for (int p = first + warp; p < last; p += kDecWarps) {
         const int2 pr = piece_rows(p, rs, re, ps, nr);
         for (int r = pr.x; r < pr.x + pr.y; ++r) {
+            const int64_t ro = a.rows.off(b, g, r);   // < 0: the row's page is outside the pool
             float kv[PER], vv[PER];
 #pragma unroll
             for (int k = 0; k < PER; ++k) {
-                kv[k] = load_elem(Ks, (int64_t)r * a.stride_t + lane + 32 * k);
-                vv[k] = load_elem(Vs, (int64_t)r * a.stride_t + lane + 32 * k);
+                kv[k] = ro < 0 ? 0.0f : load_elem(Ks, ro + lane + 32 * k);
+                vv[k] = ro < 0 ? 0.0f : load_elem(Vs, ro + lane + 32 * k);
             }
 #pragma unroll
             for (int h = 0; h < kMaxG; ++h) {
@@ -902,7 +949,8 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
     a.app = app ? *app : DecAppend{};
     a.q = q; a.out = out; a.lse = lse; a.ranges = ranges; a.n_ranges = n_ranges;
     a.max_ranges = max_ranges; a.cur_len = cur_len; a.K = K; a.V = V;
-    a.stride_b = d->stride_b; a.stride_h = d->stride_h; a.stride_t = d->stride_t;
+    a.rows = kv_rows(d);
+    a.aligned = d->page_rows > 0;
     a.B = d->B; a.Hq = d->Hq; a.Hkv = d->Hkv; a.G = d->Hq / d->Hkv; a.D = d->D;
     a.L_max = d->L_max;
     a.nsplit = decode_nsplit(d, tokens_hint, max_ranges);

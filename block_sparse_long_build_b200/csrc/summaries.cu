@@ -14,7 +14,7 @@ struct SumArgs {
     const void *K;
     void *summ;
     const int32_t *offsets;   // variable blocks or nullptr
-    int64_t stride_b, stride_h, stride_t;
+    KvRows rows;
     int Hkv, D, L_max, S, nb_total, first_block, kind;
     size_t row_bytes;
 };
@@ -25,7 +25,6 @@ __global__ void __launch_bounds__(128) build_summaries_kernel(SumArgs a) {
     const int j = a.first_block + blockIdx.x;
     const int s = blockIdx.y;
     const int b = s / a.Hkv, g = s % a.Hkv;
-    const T *Kseg = static_cast<const T *>(a.K) + b * a.stride_b + g * a.stride_h;
     int64_t r0, r1;
     if (a.offsets) {
         const int32_t *off = a.offsets + (int64_t)s * (a.nb_total + 1);
@@ -36,7 +35,7 @@ __global__ void __launch_bounds__(128) build_summaries_kernel(SumArgs a) {
         r1 = r0 + a.S;
     }
     char *out = static_cast<char *>(a.summ) + ((int64_t)s * a.nb_total + j) * a.row_bytes;
-    summarize_rows<T>(Kseg, a.stride_t, a.D, r0, r1, a.kind, out, sm);
+    summarize_rows<T>(static_cast<const T *>(a.K), a.rows, b, g, a.D, r0, r1, a.kind, out, sm);
 }
 
 struct AppendArgs {
@@ -44,7 +43,7 @@ struct AppendArgs {
     const void *k_new, *v_new;
     int32_t *cur_len;
     void *summ;
-    int64_t stride_b, stride_h, stride_t;
+    KvRows rows;
     int Hkv, D, L_max, S, nb_total, kind;
     size_t row_bytes;
 };
@@ -57,14 +56,16 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
     const int b = blockIdx.x;
     const int n = a.cur_len[b];
     if (n < 0 || n >= a.L_max) return;
-    T *K = static_cast<T *>(a.K) + b * a.stride_b;
-    T *V = static_cast<T *>(a.V) + b * a.stride_b;
+    T *K = static_cast<T *>(a.K);
+    T *V = static_cast<T *>(a.V);
     const T *kn = static_cast<const T *>(a.k_new) + (int64_t)b * a.Hkv * a.D;
     const T *vn = static_cast<const T *>(a.v_new) + (int64_t)b * a.Hkv * a.D;
     for (int e = threadIdx.x; e < a.Hkv * a.D; e += blockDim.x) {
-        int g = e / a.D, i = e % a.D;
-        K[g * a.stride_h + (int64_t)n * a.stride_t + i] = kn[e];
-        V[g * a.stride_h + (int64_t)n * a.stride_t + i] = vn[e];
+        const int g = e / a.D, i = e % a.D;
+        const int64_t o = a.rows.off(b, g, n);
+        if (o < 0) continue;   // the row's page is outside the pool
+        K[o + i] = kn[e];
+        V[o + i] = vn[e];
     }
     __syncthreads();
     if (a.summ && a.S > 0 && (n + 1) % a.S == 0) {
@@ -72,8 +73,8 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
         for (int g = 0; g < a.Hkv; ++g) {
             const int s = b * a.Hkv + g;
             char *out = static_cast<char *>(a.summ) + ((int64_t)s * a.nb_total + j) * a.row_bytes;
-            summarize_rows<T>(K + g * a.stride_h, a.stride_t, a.D, (int64_t)j * a.S,
-                              (int64_t)(j + 1) * a.S, a.kind, out, sm);
+            summarize_rows<T>(K, a.rows, b, g, a.D, (int64_t)j * a.S, (int64_t)(j + 1) * a.S,
+                              a.kind, out, sm);
             __syncthreads();
         }
     }
@@ -91,7 +92,7 @@ bsa_status launch_build_summaries(const bsa_kv_desc *d, const void *K, const bsa
     SumArgs a;
     a.K = K; a.summ = summ;
     a.offsets = p->block_size == 0 ? p->block_offsets : nullptr;
-    a.stride_b = d->stride_b; a.stride_h = d->stride_h; a.stride_t = d->stride_t;
+    a.rows = kv_rows(d);
     a.Hkv = d->Hkv; a.D = d->D; a.L_max = d->L_max; a.S = p->block_size;
     a.nb_total = nb_total; a.first_block = first_block; a.kind = kind;
     a.row_bytes = summary_row_bytes(kind, d->D, d->kv_dtype);
@@ -111,7 +112,7 @@ bsa_status launch_append(const bsa_kv_desc *d, void *K, void *V, const void *kn,
     AppendArgs a;
     a.K = K; a.V = V; a.k_new = kn; a.v_new = vn; a.cur_len = cur_len;
     a.summ = (p && p->block_size > 0) ? summ : nullptr;
-    a.stride_b = d->stride_b; a.stride_h = d->stride_h; a.stride_t = d->stride_t;
+    a.rows = kv_rows(d);
     a.Hkv = d->Hkv; a.D = d->D; a.L_max = d->L_max; a.S = p ? p->block_size : 0;
     a.nb_total = nb_total; a.kind = kind;
     a.row_bytes = summary_row_bytes(kind, d->D, d->kv_dtype);

@@ -21,24 +21,33 @@ __device__ __forceinline__ float row_norm_f32(const float *x, int D) {
     return __fsqrt_rn(acc);
 }
 
+// Element i of logical row r of segment (b, g); zero for a row whose page
+// is outside the pool.
+template <typename T>
+__device__ __forceinline__ float row_elem(const T *K, const KvRows &kr, int b, int g, int64_t r,
+                                          int i) {
+    const int64_t o = kr.off(b, g, r);
+    return o < 0 ? 0.0f : load_elem(K, o + i);
+}
+
 // Centroid of rows [r0, r1): thread i < D sums dimension i in row order.
 template <typename T>
-__device__ __forceinline__ void summarize_centroid(const T *Kseg, int64_t st, int D, int64_t r0,
-                                                   int64_t r1, float *out) {
+__device__ __forceinline__ void summarize_centroid(const T *K, const KvRows &kr, int b, int g, int D,
+                                                   int64_t r0, int64_t r1, float *out) {
     const int i = threadIdx.x;
     const int64_t n = r1 - r0;
     if (i < D) {
         float acc = 0.0f;
         int64_t r = r0;
         for (; r + 4 <= r1; r += 4) {   // loads batched, adds stay in order
-            float v0 = load_elem(Kseg, r * st + i), v1 = load_elem(Kseg, (r + 1) * st + i);
-            float v2 = load_elem(Kseg, (r + 2) * st + i), v3 = load_elem(Kseg, (r + 3) * st + i);
+            float v0 = row_elem(K, kr, b, g, r, i), v1 = row_elem(K, kr, b, g, r + 1, i);
+            float v2 = row_elem(K, kr, b, g, r + 2, i), v3 = row_elem(K, kr, b, g, r + 3, i);
             acc = __fadd_rn(acc, v0);
             acc = __fadd_rn(acc, v1);
             acc = __fadd_rn(acc, v2);
             acc = __fadd_rn(acc, v3);
         }
-        for (; r < r1; ++r) acc = __fadd_rn(acc, load_elem(Kseg, r * st + i));
+        for (; r < r1; ++r) acc = __fadd_rn(acc, row_elem(K, kr, b, g, r, i));
         out[i] = n > 0 ? __fdiv_rn(acc, (float)n) : 0.0f;
     }
 }
@@ -46,14 +55,14 @@ __device__ __forceinline__ void summarize_centroid(const T *Kseg, int64_t st, in
 // Min/max of rows [r0, r1) in the cache dtype, stored as (min, max) pairs
 // per dimension: thread i < D scans dimension i in row order.
 template <typename T>
-__device__ __forceinline__ void summarize_minmax(const T *Kseg, int64_t st, int D, int64_t r0,
-                                                 int64_t r1, T *o) {
+__device__ __forceinline__ void summarize_minmax(const T *K, const KvRows &kr, int b, int g, int D,
+                                                 int64_t r0, int64_t r1, T *o) {
     const int i = threadIdx.x;
     const int64_t n = r1 - r0;
     if (i < D) {
         float lo = __int_as_float(0x7f800000), hi = __int_as_float(0xff800000);  // +inf, -inf
         for (int64_t r = r0; r < r1; ++r) {
-            float v = load_elem(Kseg, r * st + i);
+            float v = row_elem(K, kr, b, g, r, i);
             if (v < lo) lo = v;
             if (v > hi) hi = v;
         }
@@ -68,21 +77,21 @@ __device__ __forceinline__ void summarize_minmax(const T *Kseg, int64_t st, int 
     }
 }
 
-// Summary of rows [r0, r1) of one segment, computed by the whole CTA
+// Summary of rows [r0, r1) of segment (b, g), computed by the whole CTA
 // (blockDim.x >= D).  `out` points at this block's summary: D floats for the
 // centroid kinds, D (min, max) pairs of cache elements for MINMAX.
 // `sm` must hold kNormChunk*(D+1) + D + 1 floats.
 template <typename T>
-__device__ void summarize_rows(const T *Kseg, int64_t st, int D, int64_t r0, int64_t r1,
-                               int kind, void *out, float *sm) {
+__device__ void summarize_rows(const T *K, const KvRows &kr, int b, int g, int D, int64_t r0,
+                               int64_t r1, int kind, void *out, float *sm) {
     const int i = threadIdx.x;
     const int64_t n = r1 - r0;
     if (kind == BSA_SUM_CENTROID) {
-        summarize_centroid<T>(Kseg, st, D, r0, r1, static_cast<float *>(out));
+        summarize_centroid<T>(K, kr, b, g, D, r0, r1, static_cast<float *>(out));
         return;
     }
     if (kind == BSA_SUM_MINMAX) {
-        summarize_minmax<T>(Kseg, st, D, r0, r1, static_cast<T *>(out));
+        summarize_minmax<T>(K, kr, b, g, D, r0, r1, static_cast<T *>(out));
         return;
     }
     // BSA_SUM_CENTROID_NORM
@@ -94,7 +103,7 @@ __device__ void summarize_rows(const T *Kseg, int64_t st, int D, int64_t r0, int
         __syncthreads();
         for (int e = threadIdx.x; e < cn * D; e += blockDim.x) {
             int rr = e / D, ii = e % D;
-            rows[rr * (D + 1) + ii] = load_elem(Kseg, (c0 + rr) * st + ii);
+            rows[rr * (D + 1) + ii] = row_elem(K, kr, b, g, c0 + rr, ii);
         }
         __syncthreads();
         if (threadIdx.x < cn) nrm[threadIdx.x] = row_norm_f32(rows + threadIdx.x * (D + 1), D);

@@ -38,7 +38,9 @@ class KvDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("kv_dtype", ctypes.c_int32), ("L_max", ctypes.c_int32),
                 ("stride_b", ctypes.c_int64), ("stride_h", ctypes.c_int64),
-                ("stride_t", ctypes.c_int64)]
+                ("stride_t", ctypes.c_int64), ("page_rows", ctypes.c_int32),
+                ("pages_per_seq", ctypes.c_int32), ("page_table", ctypes.c_void_p),
+                ("n_pages", ctypes.c_int64)]
 
 
 class SelParams(ctypes.Structure):
@@ -124,7 +126,19 @@ def kv_desc(K: torch.Tensor, Hq: int) -> KvDesc:
     assert K.dim() == 4 and K.stride(3) == 1
     dt = {torch.float32: BSA_F32, torch.bfloat16: BSA_BF16}[K.dtype]
     B, H, L, D = K.shape
-    return KvDesc(B, Hq, H, D, dt, L, K.stride(0), K.stride(1), K.stride(2))
+    return KvDesc(B, Hq, H, D, dt, L, K.stride(0), K.stride(1), K.stride(2), 0, 0, None, 0)
+
+
+def paged_kv_desc(pool: torch.Tensor, Hq: int, page_table: torch.Tensor) -> KvDesc:
+    """Descriptor of a paged cache: pool [n_pages, Hkv, page_rows, D] (D
+    contiguous) and page_table int32 [B, pages_per_seq] on the device."""
+    assert pool.dim() == 4 and pool.stride(3) == 1
+    assert page_table.dtype == torch.int32 and page_table.dim() == 2 and page_table.is_contiguous()
+    dt = {torch.float32: BSA_F32, torch.bfloat16: BSA_BF16}[pool.dtype]
+    n_pages, H, P, D = pool.shape
+    B, pps = page_table.shape
+    return KvDesc(B, Hq, H, D, dt, pps * P, pool.stride(0), pool.stride(1), pool.stride(2), P, pps,
+                  page_table.data_ptr(), n_pages)
 
 
 def sel_params(block_size=0, n_blocks=0, block_offsets=None, kv_pos=None, topk=-1,

@@ -30,13 +30,22 @@ def _align(n: int, a: int = 256) -> int:
 
 
 class DecodeSession:
-    def __init__(self, wl: Workload, stream: torch.cuda.Stream | None = None, fused: bool = True):
+    """page_rows > 0 keeps the cache as a page pool (Workload.paged) instead
+    of the workload's contiguous [B, Hkv, L_max, D] tensors."""
+
+    def __init__(self, wl: Workload, stream: torch.cuda.Stream | None = None, fused: bool = True,
+                 page_rows: int = 0, spare_pages: int = 0):
         self.wl = wl
         self.fused = fused
         c = self.cfg = wl.cfg
         dev = wl.device
         self.stream = stream
-        self.desc = N.kv_desc(wl.K, c.Hq)
+        if page_rows:
+            self.K, self.V, self.page_table = wl.paged(page_rows, spare_pages)
+            self.desc = N.paged_kv_desc(self.K, c.Hq, self.page_table)
+        else:
+            self.K, self.V, self.page_table = wl.K, wl.V, None
+            self.desc = N.kv_desc(wl.K, c.Hq)
         if c.block_size == 0:
             self.sel = N.sel_params(0, c.n_blocks, wl.block_offsets, wl.kv_pos, topk=-1,
                                     budget_tokens=c.budget_tokens, local_start=wl.local_start,
@@ -88,11 +97,11 @@ class DecodeSession:
             nb = self.nb
         else:
             nb = (n_tokens if n_tokens is not None else c.L) // c.block_size
-        N.bsa_build_summaries(self.desc, self.wl.K, self.sel, self.kind, 0, nb, self.summaries,
+        N.bsa_build_summaries(self.desc, self.K, self.sel, self.kind, 0, nb, self.summaries,
                               self.stream)
 
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor):
-        N.bsa_append_kv(self.desc, self.wl.K, self.wl.V, k_new, v_new, self.wl.cur_len, self.sel,
+        N.bsa_append_kv(self.desc, self.K, self.V, k_new, v_new, self.wl.cur_len, self.sel,
                         self.kind, self.summaries if self.cfg.block_size > 0 else None,
                         self.stream)
 
@@ -103,14 +112,14 @@ class DecodeSession:
 
     def decode(self, q: torch.Tensor, out: torch.Tensor | None = None,
                lse: torch.Tensor | None = None):
-        N.bsa_decode(self.desc, q, self.wl.K, self.wl.V, self.ranges, self.n_ranges,
+        N.bsa_decode(self.desc, q, self.K, self.V, self.ranges, self.n_ranges,
                      self.max_ranges, self.wl.cur_len, self.tokens_hint, self.scale,
                      self.out if out is None else out, self.lse if lse is None else lse,
                      self.ws, self.stream)
 
     def decode_step(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor):
         """Append the new row and attend (no selection refresh)."""
-        N.bsa_decode_step(self.desc, q, self.wl.K, self.wl.V, k_new, v_new, self.wl.cur_len,
+        N.bsa_decode_step(self.desc, q, self.K, self.V, k_new, v_new, self.wl.cur_len,
                           self.sel, self.kind,
                           self.summaries if self.cfg.block_size > 0 else None, self.ranges,
                           self.n_ranges, self.max_ranges, self.tokens_hint, self.scale, self.out,

@@ -253,6 +253,31 @@ class Workload:
         self.local_start = L                    # first row of the local part
         self.cur_len = torch.full((B,), L + c.chunk, dtype=torch.int32, device=dev)
 
+    # ---------------------------------------------------------------- paged
+    def paged(self, page_rows: int, spare_pages: int = 0, seed_offset: int = 7_000_001):
+        """The cache laid out as a page pool ("Sparse long-context inference
+        with self-indexing attention": the KV cache held as fixed-size pages):
+        every sequence's rows cut into pages of `page_rows`, the pages placed
+        at seeded random slots of a pool with `spare_pages` unused slots.
+        Returns (K_pool, V_pool [n_pages, Hkv, page_rows, D], page_table int32
+        [B, pages_per_seq]); logical page i of sequence b is pool page
+        page_table[b, i]."""
+        c, dev = self.cfg, self.device
+        B, H, Lm, D = self.K.shape
+        pps = -(-Lm // page_rows)
+        n_pages = B * pps + spare_pages
+        g = _gen(dev, c.seed + seed_offset)
+        slots = torch.randperm(n_pages, generator=g, device=dev)[: B * pps]
+        table = slots.view(B, pps).to(torch.int32).contiguous()
+        Kp = torch.zeros(n_pages, H, page_rows, D, dtype=self.K.dtype, device=dev)
+        Vp = torch.zeros_like(Kp)
+        for b in range(B):
+            for i in range(pps):
+                r0, r1 = i * page_rows, min((i + 1) * page_rows, Lm)
+                Kp[table[b, i], :, : r1 - r0] = self.K[b, :, r0:r1]
+                Vp[table[b, i], :, : r1 - r0] = self.V[b, :, r0:r1]
+        return Kp, Vp, table
+
     # --------------------------------------------------------------- inputs
     def decode_query(self, step: int) -> torch.Tensor:
         """Step `step`'s queries [B, Hq, D] fp32."""

@@ -94,12 +94,31 @@ typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype;
 
 typedef enum { BSA_OP_SELECT = 0, BSA_OP_DECODE = 1, BSA_OP_PREFILL = 2, BSA_OP_APPEND = 3 } bsa_op;
 
-/* KV-cache geometry. */
+/* KV-cache geometry.
+ *
+ * Contiguous cache (page_rows = 0): K and V are [B][Hkv][L_max][D] with
+ * element strides stride_b, stride_h, stride_t.
+ *
+ * Paged cache (page_rows > 0; "Sparse long-context inference with
+ * self-indexing attention", "How much memory the KV cache takes": the cache
+ * held as fixed-size pages): K and V point at a pool of n_pages pages,
+ * [n_pages][Hkv][page_rows][D] with element strides stride_b (between
+ * pages), stride_h, stride_t.  Logical row r of sequence b, KV head g lives in
+ * page page_table[b * pages_per_seq + r / page_rows] at row r % page_rows.
+ * page_rows is a multiple of 16, L_max = pages_per_seq * page_rows, and every
+ * table entry a sequence's rows [0, L_max) can reach must be in
+ * [0, n_pages): a decode reads zeros for rows whose entry is outside, and
+ * appends skip them.  Sequences may share pages.  The page table is device
+ * memory the caller owns; selection outputs stay in logical rows. */
 typedef struct {
     int32_t B, Hq, Hkv, D;     /* D in {64, 128}; Hq a multiple of Hkv            */
     int32_t kv_dtype;          /* bsa_dtype of K and V                             */
     int32_t L_max;             /* rows per segment                                 */
     int64_t stride_b, stride_h, stride_t;   /* element strides of K and V          */
+    int32_t page_rows;         /* 0: contiguous; else rows per page               */
+    int32_t pages_per_seq;     /* paged: table entries per sequence               */
+    const int32_t *page_table; /* paged: device int32 [B][pages_per_seq]          */
+    int64_t n_pages;           /* paged: pages in the pool                        */
 } bsa_kv_desc;
 
 /* Selection parameters, in the pages' terms.

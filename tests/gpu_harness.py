@@ -75,17 +75,34 @@ class FixedDecodeCheck:
 
     segments: the (b, g) pairs compared (default: all); only their caches are
     copied to the host.  run(check_steps=...) compares only those steps (the
-    GPU runs every step in between, as a real decode would)."""
+    GPU runs every step in between, as a real decode would).  page_rows > 0
+    runs the library on a page pool (seeded random page table); the oracle
+    then reads each sequence's cache back through that table with its own
+    paged_to_contiguous."""
 
-    def __init__(self, cfg, device="cuda", fused=True, segments=None):
+    def __init__(self, cfg, device="cuda", fused=True, segments=None, page_rows=0,
+                 spare_pages=0):
         self.cfg = cfg
         self.wl = Workload(cfg, device)
-        self.sess = DecodeSession(self.wl, fused=fused)
+        self.sess = DecodeSession(self.wl, fused=fused, page_rows=page_rows,
+                                  spare_pages=spare_pages)
+        self.L_max = self.sess.desc.L_max
         self.segs = segments if segments is not None else [
             (b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
         # the oracle's own copy of each compared segment's cache
-        self.K = {(b, g): host(self.wl.K[b, g]) for b, g in self.segs}
-        self.V = {(b, g): host(self.wl.V[b, g]) for b, g in self.segs}
+        if page_rows:
+            Kp, Vp = host(self.sess.K), host(self.sess.V)
+            table = self.sess.page_table.cpu().numpy()
+            self.K, self.V = {}, {}
+            for b in sorted({b for b, _ in self.segs}):
+                kb = oracle.paged_to_contiguous(Kp, table[b], page_rows, self.L_max)
+                vb = oracle.paged_to_contiguous(Vp, table[b], page_rows, self.L_max)
+                for bb, g in self.segs:
+                    if bb == b:
+                        self.K[(b, g)], self.V[(b, g)] = kb[g].copy(), vb[g].copy()
+        else:
+            self.K = {(b, g): host(self.wl.K[b, g]) for b, g in self.segs}
+            self.V = {(b, g): host(self.wl.V[b, g]) for b, g in self.segs}
         self.n = [int(x) for x in self.wl.cur_len.cpu()]
         self.n_sel = list(self.n)
         self.q_sel = None       # queries of the last refresh step
@@ -103,7 +120,7 @@ class FixedDecodeCheck:
                 k, v = self.wl.decode_new_kv(t)
                 kh, vh = host(k), host(v)
                 for b in range(c.B):
-                    if self.n[b] < c.L_max:
+                    if self.n[b] < self.L_max:
                         for bb, g in self.segs:
                             if bb == b:
                                 self.K[(b, g)][self.n[b]] = kh[b, g]
