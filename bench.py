@@ -824,10 +824,12 @@ def run_case(args, device):
     (a few launches on a workload of a few GB at most); prints one line.
       decode      Quest workload: two steps (the second a fused append + decode),
                   then bsa_decode five times, L2 flushed before each
-      decode_lb   large-batch workload cut to 8 sequences (1.1 GB of cache):
-                  one step, then bsa_decode five times, L2 flushed before each
+      decode_lb   large-batch workload cut to --case-batch sequences (default
+                  8: 1.1 GB of cache): one step, then bsa_decode five times, L2
+                  flushed before each
       select      Quest workload: bsa_select three times, L2 flushed before each
-      select_lb   large-batch workload cut to 8 sequences: bsa_select three times
+      select_lb   large-batch workload cut to --case-batch sequences: bsa_select
+                  three times
       prefill     semantic workload at a 65,536-token context: the last chunk of
                   1,024 queries three times"""
     from block_sparse_long_build_b200 import build as Bld
@@ -837,7 +839,8 @@ def run_case(args, device):
     flush = _flusher(device)
     ev = []
     if args.case in ("decode", "select", "decode_lb", "select_lb"):
-        cfg = W.quest(0) if args.case in ("decode", "select") else W.largebatch(0).scaled(B=8)
+        cfg = (W.quest(0) if args.case in ("decode", "select")
+               else W.largebatch(0).scaled(B=args.case_batch))
         wl = W.Workload(cfg, device)
         sess = DecodeSession(wl)
         sess.build_summaries()
@@ -916,6 +919,8 @@ def main():
                     help="keys per KV head for --index (a smaller case for profiling)")
     ap.add_argument("--case", choices=["decode", "select", "decode_lb", "select_lb", "prefill"],
                     default=None, help="run one small profiling case instead of the bench (for ncu)")
+    ap.add_argument("--case-batch", type=int, default=8,
+                    help="sequences of the large-batch profiling cases")
     args = ap.parse_args()
     if args.case:
         torch.cuda.set_device(0)

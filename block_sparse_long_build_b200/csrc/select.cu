@@ -578,31 +578,35 @@ __global__ void __launch_bounds__(kPickThreads, 2) pick_kernel(SelArgs a) {
 }
 
 
-// The same selection for fixed blocks, segments of at most 32 * NK blocks,
-// by one warp per segment with no CTA barrier: lane l holds the keys of
-// blocks l + 32 r in registers.  The k-th largest key T is found bit by bit
-// from the top (T gains bit b when at least k candidate keys are >= T | b: one
-// warp-wide count per bit); the selected blocks are those with key > T and,
-// among the keys equal to T, the k - count(> T) of lowest index (ballots in
-// index order).  A ballot per r compacts them in index order straight into
-// their place among the forced ranges; the merged ranges come from a warp
-// scan (running maximum of the ends), 32 items per pass.  Shared memory:
-// (lo, hi) of max_sel + 2 items.
+// The same selection for fixed blocks, segments of at most 128 * NK blocks,
+// by one 128-thread CTA per segment: thread t holds the keys of blocks
+// [t NK, t NK + NK) in registers, so the threads' runs are in index order.
+// The k-th largest key T is found bit by bit from the top: T gains bit b when
+// at least k candidate keys are >= T | b (a warp count, then the four warps'
+// counts through shared memory: one barrier per bit, the counts double-
+// buffered by bit parity).  The selected blocks are those with key > T and,
+// among the keys equal to T, the k - count(> T) of lowest index; exclusive
+// scans over the threads give each taken block its place in index order and
+// among the forced ranges, and the merged ranges come from scans of the
+// running maximum of the ends.  Shared memory: (lo, hi) of max_sel + 2
+// items and their running maxima.
+constexpr int kPickFixedThreads = 128;
+
 template <int NK>
-__global__ void __launch_bounds__(32) pick_warp_kernel(SelArgs a) {
-    static_assert(NK >= 1 && NK <= 64, "taken[] holds 64 bits");
+__global__ void __launch_bounds__(kPickFixedThreads) pick_fixed_kernel(SelArgs a) {
     extern __shared__ __align__(16) unsigned char psm[];
     int2 *items = reinterpret_cast<int2 *>(psm);
-    const int s = blockIdx.x, b = s / a.Hkv, lane = threadIdx.x;
-    const int nb = a.nb_total;
+    int *pmax = reinterpret_cast<int *>(psm + (size_t)(a.max_sel + 4) * 8);
+    __shared__ int cnt2[2][kPickFixedThreads / 32];
+    __shared__ int tmp[40];
+    const int s = blockIdx.x, b = s / a.Hkv;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nb = a.nb_total, j0 = tid * NK;
     pdl_wait();   // keys from score_kernel
     uint32_t wk[NK];
 #pragma unroll
-    for (int r = 0; r < NK; ++r) {
-        const int j = lane + 32 * r;
-        wk[r] = j < nb ? a.keys[(int64_t)s * nb + j] : 0u;
-    }
-    // forced token ranges (every lane computes the same), sorted and merged
+    for (int r = 0; r < NK; ++r) wk[r] = j0 + r < nb ? a.keys[(int64_t)s * nb + j0 + r] : 0u;
+    // forced token ranges (every thread computes the same), sorted and merged
     const int n = min(max(a.cur_len[b], 0), a.L_max);
     int f_lo[2] = {0, 0}, f_hi[2] = {0, 0}, nf = 0;
     if (a.sink > 0 && n > 0) { f_lo[0] = 0; f_hi[0] = min(a.sink, n); nf = 1; }
@@ -621,16 +625,28 @@ __global__ void __launch_bounds__(32) pick_warp_kernel(SelArgs a) {
 #pragma unroll
     for (int r = 0; r < NK; ++r) {
         if (wk[r]) {
-            const int64_t r0 = (int64_t)(lane + 32 * r) * a.S, r1 = r0 + a.S;
+            const int64_t r0 = (int64_t)(j0 + r) * a.S, r1 = r0 + a.S;
 #pragma unroll
             for (int i = 0; i < 2; ++i)
                 if (i < nf && f_lo[i] <= r0 && r1 <= f_hi[i]) wk[r] = 0u;
         }
         my_c += wk[r] != 0u;
     }
-    const int n_cand = __reduce_add_sync(0xffffffffu, my_c);
+    // CTA sum through the parity-buffered warp counts (one barrier each)
+    int par = 0;
+    auto cta_sum = [&](int v) -> int {
+        v = __reduce_add_sync(0xffffffffu, v);
+        if (lane == 0) cnt2[par][warp] = v;
+        __syncthreads();
+        int t = 0;
+#pragma unroll
+        for (int w = 0; w < kPickFixedThreads / 32; ++w) t += cnt2[par][w];
+        par ^= 1;
+        return t;
+    };
+    const int n_cand = cta_sum(my_c);
     const int k = min(min(a.topk >= 0 ? a.topk : a.budget / a.S, n_cand), a.max_sel);
-    uint64_t taken = 0;   // bit r: block lane + 32 r (NK <= 64)
+    uint32_t taken = 0;   // bit r: block j0 + r
     if (k > 0) {
         // T = the k-th largest candidate key (>= 1, since k <= n_cand)
         uint32_t T = 0u;
@@ -639,30 +655,31 @@ __global__ void __launch_bounds__(32) pick_warp_kernel(SelArgs a) {
             int cnt = 0;
 #pragma unroll
             for (int r = 0; r < NK; ++r) cnt += wk[r] >= c;
-            if (__reduce_add_sync(0xffffffffu, cnt) >= k) T = c;
+            if (cta_sum(cnt) >= k) T = c;
         }
-        int gt = 0;
-#pragma unroll
-        for (int r = 0; r < NK; ++r) gt += wk[r] > T;
-        const int need_eq = k - __reduce_add_sync(0xffffffffu, gt);
-        int eq_seen = 0;
+        int gt = 0, eq = 0;
 #pragma unroll
         for (int r = 0; r < NK; ++r) {
-            const uint32_t eqm = __ballot_sync(0xffffffffu, wk[r] == T);
-            const int rank = eq_seen + __popc(eqm & ((1u << lane) - 1u));
-            if (wk[r] > T || (wk[r] == T && rank < need_eq)) taken |= 1ull << r;
-            eq_seen += __popc(eqm);
+            gt += wk[r] > T;
+            eq += wk[r] == T;
         }
+        const int need_eq = k - cta_sum(gt);
+        int tot;
+        int eq_rank = cta_excl_sum(eq, tmp, &tot);   // keys equal to T before this thread's
+#pragma unroll
+        for (int r = 0; r < NK; ++r)
+            if (wk[r] > T || (wk[r] == T && eq_rank++ < need_eq)) taken |= 1u << r;
     }
     // index-ordered compaction, each block written at its place among the
     // forced ranges (a forced range comes first on equal starts)
-    int n_sel = 0, below[2] = {0, 0};   // below[f]: taken blocks starting before f_lo[f]
+    int tot;
+    int p = cta_excl_sum(__popc(taken), tmp, &tot);
+    const int n_sel = min(tot, a.max_sel);
+    int below[2] = {0, 0};   // taken blocks starting before f_lo[f]
 #pragma unroll
     for (int r = 0; r < NK; ++r) {
-        const uint32_t mk = __ballot_sync(0xffffffffu, (uint32_t)(taken >> r) & 1u);
-        if ((taken >> r) & 1ull) {
-            const int p = n_sel + __popc(mk & ((1u << lane) - 1u));
-            const int jj = lane + 32 * r;
+        if ((taken >> r) & 1u) {
+            const int jj = j0 + r;
             const int lo = jj * a.S, hi = lo + a.S;
             int before = 0;
 #pragma unroll
@@ -674,45 +691,40 @@ __global__ void __launch_bounds__(32) pick_warp_kernel(SelArgs a) {
                 a.sel_blocks[(int64_t)s * a.max_sel + p] = jj;
                 items[p + before] = make_int2(lo, hi);
             }
+            ++p;
         }
-        n_sel += __popc(mk);
     }
-    n_sel = min(n_sel, a.max_sel);
 #pragma unroll
     for (int f = 0; f < 2; ++f) {
-        const int nbelow = __reduce_add_sync(0xffffffffu, below[f]);
-        if (f < nf && lane == 0) items[f + nbelow] = make_int2(f_lo[f], f_hi[f]);
+        const int nbelow = cta_sum(below[f]);
+        if (f < nf && tid == 0) items[f + nbelow] = make_int2(f_lo[f], f_hi[f]);
     }
-    __syncwarp();
+    __syncthreads();
     // ranges: item i opens a range when it starts after every earlier item
     // has ended; a range ends at the running maximum of its last item
     const int M = n_sel + nf;
-    int32_t *R = a.ranges + (int64_t)s * a.max_ranges * 2;
-    int nr = 0, carry = kIntMin;
-    for (int c0 = 0; c0 < M; c0 += 32) {
-        const int i = c0 + lane;
-        const int2 it = i < M ? items[i] : make_int2(0, kIntMin);
-        int pm = it.y;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, pm, o);
-            if (lane >= o) pm = max(pm, v);
-        }
-        pm = max(pm, carry);
-        int prev = __shfl_up_sync(0xffffffffu, pm, 1);
-        if (lane == 0) prev = carry;
-        const bool start = i < M && (i == 0 || it.x > prev);
-        const uint32_t sm = __ballot_sync(0xffffffffu, start);
-        const int rid = nr + __popc(sm & ((2u << lane) - 1u)) - 1;   // range of item i
-        if (i < M) {
-            if (start && rid < a.max_ranges) R[2 * rid] = it.x;
-            const bool last = i == M - 1 || items[i + 1].x > pm;
-            if (last && rid < a.max_ranges) R[2 * rid + 1] = pm;
-        }
-        nr += __popc(sm);
-        carry = __shfl_sync(0xffffffffu, pm, 31);
+    int carry = kIntMin;
+    for (int t0 = 0; t0 < M; t0 += kPickFixedThreads) {
+        const int i = t0 + tid;
+        const int pm = max(cta_incl_max(i < M ? items[i].y : kIntMin, tmp, &tot), carry);
+        if (i < M) pmax[i] = pm;
+        carry = max(carry, tot);
     }
-    if (lane == 0) {
+    __syncthreads();
+    int32_t *R = a.ranges + (int64_t)s * a.max_ranges * 2;
+    int nr = 0;
+    for (int t0 = 0; t0 < M; t0 += kPickFixedThreads) {
+        const int i = t0 + tid;
+        const int start = i < M && (i == 0 || items[i].x > pmax[i - 1]);
+        const int rid = nr + cta_excl_sum(start, tmp, &tot) + start - 1;   // range of item i
+        if (i < M) {
+            if (start && rid < a.max_ranges) R[2 * rid] = items[i].x;
+            const bool last = i == M - 1 || items[i + 1].x > pmax[i];
+            if (last && rid < a.max_ranges) R[2 * rid + 1] = pmax[i];
+        }
+        nr += tot;
+    }
+    if (tid == 0) {
         a.n_ranges[s] = min(nr, a.max_ranges);
         a.sel_count[s] = n_sel;
     }
@@ -793,19 +805,20 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
         BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(kPickThreads), smem2, st, a));
         return BSA_OK;
     };
-    // fixed blocks, up to 2,048 per segment: one warp per segment with the
-    // keys in registers (the token-budget walk over variable blocks measured
-    // faster in the CTA kernel)
-    if (!variable && nb_total <= 32 * 64) {
-        const size_t smem3 = (size_t)(max_sel + 4) * 8;
-        auto warp_pick = [&](auto kern) -> bsa_status {
-            BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(32), smem3, st, a));
+    // fixed blocks, up to 4,096 per segment: 128 threads per segment with
+    // the keys in registers (the token-budget walk over variable blocks
+    // measured faster in the 512-thread kernel)
+    if (!variable && nb_total <= kPickFixedThreads * 32) {
+        const size_t smem3 = (size_t)(max_sel + 4) * 12;
+        auto fixed_pick = [&](auto kern) -> bsa_status {
+            BSA_CUDA_TRY(launch_pdl(kern, dim3((unsigned)nseg), dim3(kPickFixedThreads), smem3, st, a));
             return BSA_OK;
         };
-        if (nb_total <= 32 * 16) return warp_pick(pick_warp_kernel<16>);
-        if (nb_total <= 32 * 32) return warp_pick(pick_warp_kernel<32>);
-        if (nb_total <= 32 * 48) return warp_pick(pick_warp_kernel<48>);
-        return warp_pick(pick_warp_kernel<64>);
+        if (nb_total <= kPickFixedThreads * 4) return fixed_pick(pick_fixed_kernel<4>);
+        if (nb_total <= kPickFixedThreads * 8) return fixed_pick(pick_fixed_kernel<8>);
+        if (nb_total <= kPickFixedThreads * 12) return fixed_pick(pick_fixed_kernel<12>);
+        if (nb_total <= kPickFixedThreads * 16) return fixed_pick(pick_fixed_kernel<16>);
+        return fixed_pick(pick_fixed_kernel<32>);
     }
     return pick(pick_kernel);
 }
