@@ -55,7 +55,8 @@ FALLBACK_HBM_GBS = 6650.0
 METRIC = "sparse-decode tokens/s and effective KV GB/s vs 8 TB/s HBM roofline"
 CSRC = os.path.join(ROOT, "block_sparse_long_build_b200", "csrc")
 HEADLINE = "largebatch"
-ALSO_DECODE = ("quest", "moba", "msa", "semantic")
+ALSO_DECODE = ("quest", "moba", "msa", "semantic", "largebatch_fp8", "quest_fp8")
+DTYPE_NAMES = {torch.bfloat16: "bf16", torch.float32: "f32", torch.float8_e4m3fn: "e4m3"}
 ATOL = 2e-3
 
 
@@ -178,7 +179,8 @@ def _step_bytes(sess, t: int) -> tuple[int, int]:
     ranges = sess.ranges.cpu().numpy()
     nr = sess.n_ranges.cpu().numpy()
     cur = sess.wl.cur_len.cpu().numpy()
-    esz = 2 if c.kv_dtype == torch.bfloat16 else 4
+    esz = torch.empty(0, dtype=c.kv_dtype).element_size()
+    sesz = 4 if c.kv_dtype == torch.float32 else 2   # min/max summaries: bf16 for bf16 and FP8
     tokens = 0
     for s in range(c.B * c.Hkv):
         r = ranges[s, :nr[s]].astype(np.int64)
@@ -193,7 +195,7 @@ def _step_bytes(sess, t: int) -> tuple[int, int]:
             rows = sum(int(x) // c.block_size for x in cur) * c.Hkv
         else:
             rows = c.n_blocks * c.B * c.Hkv
-        row_bytes = 2 * c.D * esz if c.kind == 2 else c.D * 4
+        row_bytes = 2 * c.D * sesz if c.kind == 2 else c.D * 4
         tot += rows * row_bytes
     tot += c.B * c.Hkv * c.D * 2 * esz   # appended row
     return tot, dec
@@ -360,7 +362,7 @@ def decode_line(name: str, K_steps: int, W_steps: int, rank: int, world: int, de
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if cfg.kv_dtype == torch.bfloat16 else "f32",
+        "dtype": DTYPE_NAMES[cfg.kv_dtype],
         "data": "synthetic",
         "effective_kv_gbs": eff_gbs,
         "effective_kv_frac_of_8tbs": eff_gbs / 8000.0,
@@ -400,10 +402,20 @@ def decode_line(name: str, K_steps: int, W_steps: int, rank: int, world: int, de
 
 
 def _host(t):
+    """bf16 as uint16 bit patterns, FP8 as uint8 codes, fp32 as float32."""
     t = t.detach().cpu().contiguous()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     return t.numpy()
+
+
+def _oracle_kv(a):
+    """FP8 codes decoded by the oracle's own E4M3 table (it reads fp32 or
+    bf16 bits); other arrays as they are."""
+    import oracle
+    return oracle.fp8_e4m3_to_f32(a) if a.dtype == np.uint8 else a
 
 
 def _host_cores() -> int:
@@ -448,7 +460,7 @@ def cpu_baseline_decode(cfg, wl, inputs0, step0, budget_s):
             out, lse = oracle.attend(qg, Kpos[b, g], Vpos[b, g], rows, 1 / math.sqrt(cfg.D))
             t_acc += time.perf_counter() - t0
         else:
-            K, V = _host(wl.K[b, g]), _host(wl.V[b, g])
+            K, V = _oracle_kv(_host(wl.K[b, g])), _oracle_kv(_host(wl.V[b, g]))
             t0 = time.perf_counter()
             ref = oracle.decode_fixed_segment(qg, K, V, n, n, cfg.kind, cfg.block_size, cfg.topk,
                                               cfg.budget_tokens, cfg.sink, cfg.window,
@@ -787,7 +799,7 @@ def run_reference(args):
         done, t_acc, i = 0, 0.0, t
         while True:
             b, g = segs[i % len(segs)]
-            K, V = _host(wl.K[b, g]), _host(wl.V[b, g])
+            K, V = _oracle_kv(_host(wl.K[b, g])), _oracle_kv(_host(wl.V[b, g]))
             t0 = time.perf_counter()
             oracle.decode_fixed_segment(q[b, g * cfg.G:(g + 1) * cfg.G], K, V, cfg.L, cfg.L,
                                         cfg.kind, cfg.block_size, cfg.topk, cfg.budget_tokens,

@@ -75,11 +75,13 @@ bool make_kv_tmap(CUtensorMap *map, const bsa_kv_desc *d, const void *base, int 
     const bool paged = d->page_rows > 0;
     const cuuint64_t dims[4] = {(cuuint64_t)d->D, (cuuint64_t)(paged ? d->page_rows : d->L_max),
                                 (cuuint64_t)d->Hkv, (cuuint64_t)(paged ? d->n_pages : d->B)};
-    const cuuint64_t strides[3] = {(cuuint64_t)d->stride_t * 2, (cuuint64_t)d->stride_h * 2,
-                                   (cuuint64_t)d->stride_b * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+    const cuuint64_t es = d->kv_dtype == BSA_FP8_E4M3 ? 1 : 2;   // bf16 or FP8 codes
+    const cuuint64_t strides[3] = {(cuuint64_t)d->stride_t * es, (cuuint64_t)d->stride_h * es,
+                                   (cuuint64_t)d->stride_b * es};
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / es), (cuuint32_t)box_rows, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+    CUresult r = fn(map, es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                    const_cast<void *>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -102,13 +104,15 @@ bool make_rows_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int esize, cons
 // ------------------------------------------------------------- validation
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-static int elem_size(const bsa_kv_desc *d) { return d->kv_dtype == BSA_BF16 ? 2 : 4; }
+static int elem_size(const bsa_kv_desc *d) {
+    return d->kv_dtype == BSA_F32 ? 4 : d->kv_dtype == BSA_BF16 ? 2 : 1;
+}
 
 static bool desc_ok(const bsa_kv_desc *d) {
     if (!d) return false;
     if (d->B < 1 || d->Hkv < 1 || d->Hq < d->Hkv || d->Hq % d->Hkv != 0) return false;
     if (d->D != 64 && d->D != 128) return false;
-    if (d->kv_dtype != BSA_F32 && d->kv_dtype != BSA_BF16) return false;
+    if (d->kv_dtype != BSA_F32 && d->kv_dtype != BSA_BF16 && d->kv_dtype != BSA_FP8_E4M3) return false;
     if (d->L_max < 1) return false;
     if (d->stride_t < d->D || d->stride_h < 1 || d->stride_b < 1) return false;
     const int64_t es = elem_size(d);
@@ -238,8 +242,9 @@ int32_t bsa_summary_blocks(const bsa_kv_desc *d, const bsa_sel_params *p) {
 
 size_t bsa_summary_bytes(const bsa_kv_desc *d, const bsa_sel_params *p, bsa_summary_kind kind) {
     if (!desc_ok(d) || !sel_ok(d, p)) return 0;
-    const size_t row = kind == BSA_SUM_MINMAX ? (size_t)2 * d->D * elem_size(d) : (size_t)d->D * 4;
-    return (size_t)d->B * d->Hkv * nb_total(d, p) * row;
+    if (kind < BSA_SUM_CENTROID || kind > BSA_SUM_MINMAX) return 0;
+    // the row size the kernels write: bf16 bounds for bf16 and FP8 caches
+    return (size_t)d->B * d->Hkv * nb_total(d, p) * summary_row_bytes(kind, d->D, d->kv_dtype);
 }
 
 int32_t bsa_max_selected(const bsa_kv_desc *d, const bsa_sel_params *p) {
@@ -264,7 +269,8 @@ bsa_status bsa_build_semantic_index(const bsa_kv_desc *d, const void *K, int64_t
     if (!desc_ok(d) || !K || !init || !centres || !labels || !offsets || !order) return BSA_ERR_ARG;
     if (L < 1 || L > d->L_max || L > 0x7fffffffLL || k < 1 || k > L || iters < 1) return BSA_ERR_ARG;
     if (!aligned16(K) || !aligned16(centres)) return BSA_ERR_ARG;
-    if (d->page_rows > 0 || !kmeans_supported(d, k)) return BSA_ERR_UNSUPPORTED;
+    if (d->page_rows > 0 || d->kv_dtype == BSA_FP8_E4M3 || !kmeans_supported(d, k))
+        return BSA_ERR_UNSUPPORTED;
     if (!ws_ok(ws, ws_bytes, kmeans_ws_bytes(d, L, k))) return BSA_ERR_WORKSPACE;
     return launch_kmeans(d, K, L, k, iters, init, centres, labels, offsets, order, ws, (cudaStream_t)stream);
 }

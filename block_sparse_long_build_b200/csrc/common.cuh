@@ -3,6 +3,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -27,6 +29,28 @@ template <> __device__ __forceinline__ float load_elem<uint16_t>(const uint16_t 
     return bf16_to_f32(p[i]);
 }
 
+// FP8 E4M3 code -> its exact fp32 value.  The code's seven magnitude bits
+// (4 exponent, 3 mantissa), placed at the bottom of an fp32 exponent and
+// mantissa field, read as the value times 2^-120 -- normal codes and
+// subnormal ones (exponent 0: m * 2^-9) alike -- so one exact multiply by
+// 2^120 rescales (denormals must not be flushed).  S.1111.111 is NaN.
+__device__ __forceinline__ float fp8e4m3_to_f32(uint32_t code) {
+    const uint32_t mag = code & 0x7fu;
+    if (mag == 0x7fu) return __int_as_float(0x7fc00000);
+    const float v = __uint_as_float(mag << 20) * 0x1p120f;
+    return (code & 0x80u) ? -v : v;
+}
+template <> __device__ __forceinline__ float load_elem<uint8_t>(const uint8_t *p, int64_t i) {
+    return fp8e4m3_to_f32(p[i]);
+}
+
+// Two FP8 E4M3 codes (low byte first) -> an f16x2 register (low half first),
+// exact: every E4M3 value is an f16 value.
+__device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint16_t pair) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
 // fp32 -> orderable uint32: larger float -> larger key (no NaNs expected).
 __device__ __forceinline__ uint32_t f32_order_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -43,6 +67,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_round(float x) {
     return __bfloat162float(__float2bfloat16_rn(x));
 }
+
+// Packs two floats into an f16x2 register, round to nearest even; `lo` in
+// the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float f16_round(float x) { return __half2float(__float2half_rn(x)); }
 
 // ---------------------------------------------------------------- smem/ptx
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -153,6 +186,16 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
                                                uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D = A(16x16 f16, row) * B(16x8 f16, col) + D, fp32 accumulators.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -377,9 +420,9 @@ inline size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 // Number of SMs of the current device (cached per process on first use).
 int num_sms();
 
-// Encodes a 4-D bf16 tensor map over a KV cache: dims (D, L_max, Hkv, B),
-// or (D, page rows, Hkv, pages) for a paged pool; box (64, rows, 1, 1),
-// 128-byte swizzle, zero fill out of bounds.
+// Encodes a 4-D tensor map over a bf16 or FP8 KV cache: dims (D, L_max, Hkv,
+// B), or (D, page rows, Hkv, pages) for a paged pool; box (128 bytes of
+// columns, rows, 1, 1), 128-byte swizzle, zero fill out of bounds.
 bool make_kv_tmap(CUtensorMap *map, const bsa_kv_desc *desc, const void *base, int box_rows);
 
 // Encodes a 2-D tensor map over `rows` rows of `row_bytes` bytes holding

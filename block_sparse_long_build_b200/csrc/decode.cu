@@ -451,19 +451,20 @@ __global__ void __launch_bounds__(128) lse_merge_kernel(DecArgs a) {
 // builds the summary of the fixed block that row completes; the last CTA of
 // sequence b to get here (every CTA of it has read cur_len by then) sets
 // cur_len[b] = n + 1 and resets the counter.
+template <typename T>
 __device__ __forceinline__ void finish_append(const DecArgs &a, int b, int g, int n, bool owner) {
     if (n < 0) return;
     const DecAppend &p = a.app;
     if (owner && p.summ && p.S > 0 && (n + 1) % p.S == 0) {
         const int j = (n + 1) / p.S - 1;
-        const uint16_t *K = static_cast<const uint16_t *>(a.K);
+        const T *K = static_cast<const T *>(a.K);
         char *out = static_cast<char *>(p.summ) + ((int64_t)(b * a.Hkv + g) * p.nb_total + j) * p.row_bytes;
         if (p.kind == BSA_SUM_MINMAX)
-            summarize_minmax<uint16_t>(K, a.rows, b, g, a.D, (int64_t)j * p.S, (int64_t)(j + 1) * p.S,
-                                       reinterpret_cast<uint16_t *>(out));
+            summarize_minmax<T>(K, a.rows, b, g, a.D, (int64_t)j * p.S, (int64_t)(j + 1) * p.S,
+                                reinterpret_cast<minmax_t<T> *>(out));
         else
-            summarize_centroid<uint16_t>(K, a.rows, b, g, a.D, (int64_t)j * p.S, (int64_t)(j + 1) * p.S,
-                                         reinterpret_cast<float *>(out));
+            summarize_centroid<T>(K, a.rows, b, g, a.D, (int64_t)j * p.S, (int64_t)(j + 1) * p.S,
+                                  reinterpret_cast<float *>(out));
     }
     if (threadIdx.x == 0) {
         __threadfence();
@@ -478,27 +479,34 @@ __device__ __forceinline__ void finish_append(const DecArgs &a, int b, int g, in
 // ======================================================================
 // Tensor-core path
 // ======================================================================
-// Shared memory: one ring per warp, NST stages of one piece each (K then V,
-// NH boxes of 16 rows x 64 columns apiece).
-template <int NH, int NST>
+// Shared memory: one ring per warp, NST stages of one piece each (K then V:
+// NH boxes of 16 rows x 64 bf16 columns apiece, or for an FP8 cache one box
+// of 16 rows x 128 FP8 columns apiece), then for an FP8 cache one f16 piece
+// per warp (the bf16 layout) that each stage is converted into.
+template <int NH, int NST, bool F8 = false>
 struct TcSmem {
-    static constexpr int kPieceBytes = 2 * NH * kBoxBytes;
+    static constexpr int kPieceBytes = F8 ? 2 * kBoxBytes : 2 * NH * kBoxBytes;
     static constexpr int kRing = kDecWarps * NST * kPieceBytes;
-    static constexpr int kInfo = kRing;                               // int [warps][NST], 8-B slots
+    static constexpr int kConv = kRing;                               // FP8: f16 piece [warps]
+    static constexpr int kConvBytes = F8 ? kDecWarps * 2 * NH * kBoxBytes : 0;
+    static constexpr int kInfo = kConv + kConvBytes;                  // int [warps][NST], 8-B slots
     static constexpr int kBars = kInfo + kDecWarps * NST * 8;         // u64  [warps][NST]
     static constexpr int kMisc = kBars + kDecWarps * NST * 8;         // float sml[2*kMaxG], int tmp[36]
     static constexpr int kPtab = kMisc + 2 * kMaxG * 4 + 36 * 4;      // int4 [warps][kWarpCap]
     static constexpr int kStall = kPtab + kDecWarps * kWarpCap * 16;  // u64: test-hook barrier
     static constexpr int kBytes = kStall + 8 + 1024;
-    static_assert(kRing >= kDecWarps * kMaxG * (2 + 64 * NH) * 4,
+    static_assert(kRing + kConvBytes >= kDecWarps * kMaxG * (2 + 64 * NH) * 4,
                   "per-warp partials must fit in the ring");
+    static_assert(kInfo >= 32768 + kMaxG * 64 * NH * 4, "the cluster merge's partial must fit below the tables");
+    static_assert(!F8 || NH == 2, "FP8 pieces are 128 columns");
 };
 
-template <int NH, int NST, bool CLUSTER>
+template <int NH, int NST, bool CLUSTER, bool F8 = false>
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      DecArgs a) {
-    using L = TcSmem<NH, NST>;
+    using L = TcSmem<NH, NST, F8>;
+    using T = std::conditional_t<F8, uint8_t, uint16_t>;   // cache element
     constexpr int D = 64 * NH;
     constexpr int NT = D / 8;   // 8-column MMA tiles across D
     extern __shared__ unsigned char dsm_raw[];
@@ -517,6 +525,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // Every warp works out its own pieces: no CTA-wide barrier before the
     // first load.
     unsigned char *ring = dsm + warp * NST * L::kPieceBytes;
+    unsigned char *conv = dsm + L::kConv + warp * 2 * NH * kBoxBytes;   // FP8 only
     uint64_t *wfull = full + warp * NST;
     int2 *winfo = info + warp * NST;   // .x: valid rows of the stage's piece
     int4 *wtab = ptab + warp * kWarpCap;
@@ -539,7 +548,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     pdl_wait();   // ranges, lengths and the cache come from earlier kernels
     // fused append: lanes 0.. hold 16-byte chunks of the new key, lanes 16..
     // of the new value
-    constexpr int kChunks = D / 8;
+    constexpr int kChunks = D * (int)sizeof(T) / 16;
     uint4 nkv = make_uint4(0u, 0u, 0u, 0u);
     if (a.app.k_new) {
         if (lane < kChunks)
@@ -556,12 +565,17 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     auto issue = [&](int idx, int st) {   // lane 0 only
         const int4 pr = wtab[idx % kWarpCap];
         winfo[st].x = pr.y;
-        mbar_arrive_expect_tx(&wfull[st], (uint32_t)(2 * NH * kBoxBytes));
+        mbar_arrive_expect_tx(&wfull[st], (uint32_t)L::kPieceBytes);
         unsigned char *dst = ring + st * L::kPieceBytes;
+        if constexpr (F8) {
+            tma_load_4d(dst, &tmK, &wfull[st], 0, pr.z, g, pr.w);
+            tma_load_4d(dst + kBoxBytes, &tmV, &wfull[st], 0, pr.z, g, pr.w);
+        } else {
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-            tma_load_4d(dst + h * kBoxBytes, &tmK, &wfull[st], h * 64, pr.z, g, pr.w);
-            tma_load_4d(dst + (NH + h) * kBoxBytes, &tmV, &wfull[st], h * 64, pr.z, g, pr.w);
+            for (int h = 0; h < NH; ++h) {
+                tma_load_4d(dst + h * kBoxBytes, &tmK, &wfull[st], h * 64, pr.z, g, pr.w);
+                tma_load_4d(dst + (NH + h) * kBoxBytes, &tmV, &wfull[st], h * 64, pr.z, g, pr.w);
+            }
         }
     };
     // Warp-collective, before piece idx is issued: if the piece holds the
@@ -574,9 +588,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             const int64_t off = a.rows.off(b, g, wr.app);
             if (off >= 0) {   // (a row whose page is outside the pool is not written)
                 if (lane < kChunks)
-                    reinterpret_cast<uint4 *>(static_cast<uint16_t *>(const_cast<void *>(a.K)) + off)[lane] = nkv;
+                    reinterpret_cast<uint4 *>(static_cast<T *>(const_cast<void *>(a.K)) + off)[lane] = nkv;
                 else if (lane >= 16 && lane - 16 < kChunks)
-                    reinterpret_cast<uint4 *>(static_cast<uint16_t *>(const_cast<void *>(a.V)) + off)[lane - 16] = nkv;
+                    reinterpret_cast<uint4 *>(static_cast<T *>(const_cast<void *>(a.V)) + off)[lane - 16] = nkv;
                 asm volatile("fence.proxy.async.global;" ::: "memory");
             }
             __syncwarp();
@@ -604,13 +618,20 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             float hi[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                hi[e] = bf16_round(x[e]);
+                hi[e] = F8 ? f16_round(x[e]) : bf16_round(x[e]);
                 lo[e] = x[e] - hi[e];
             }
-            qa[kk][0] = pack_bf16x2(hi[0], hi[1]);
-            qa[kk][1] = pack_bf16x2(lo[0], lo[1]);
-            qa[kk][2] = pack_bf16x2(hi[2], hi[3]);
-            qa[kk][3] = pack_bf16x2(lo[2], lo[3]);
+            if constexpr (F8) {
+                qa[kk][0] = pack_f16x2(hi[0], hi[1]);
+                qa[kk][1] = pack_f16x2(lo[0], lo[1]);
+                qa[kk][2] = pack_f16x2(hi[2], hi[3]);
+                qa[kk][3] = pack_f16x2(lo[2], lo[3]);
+            } else {
+                qa[kk][0] = pack_bf16x2(hi[0], hi[1]);
+                qa[kk][1] = pack_bf16x2(lo[0], lo[1]);
+                qa[kk][2] = pack_bf16x2(hi[2], hi[3]);
+                qa[kk][3] = pack_bf16x2(lo[2], lo[3]);
+            }
         }
     }
 
@@ -627,7 +648,50 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const int vlo = vr & 255, vhi = vr >> 8;   // valid rows [vlo, vhi) of the box
         unsigned char *kp = ring + st * L::kPieceBytes;
         unsigned char *vp = kp + NH * kBoxBytes;
-        if (vlo > 0 || vhi < kPiece) {   // rows outside the range: zero V so 0 * junk stays 0
+        bool issued_early = false;
+        if constexpr (F8) {
+            // the stage's FP8 K and V boxes -> this warp's f16 piece in the
+            // bf16 layout (FP8 chunk c of a row: columns 16c .. 16c+15, i.e.
+            // f16 box c / 4, chunks 2 (c % 4) and 2 (c % 4) + 1); V rows outside
+            // [vlo, vhi) become zeros so that 0 * junk stays 0
+            const unsigned char *src = kp;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int u = lane + 32 * k;
+                const int kv = u >> 7, r = (u >> 3) & 15, cc = u & 7;
+                const uint4 w = *reinterpret_cast<const uint4 *>(src + kv * kBoxBytes + r * 128 +
+                                                                 ((cc ^ (r & 7)) << 4));
+                uint32_t h[8];
+                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    h[2 * e] = fp8x2_to_f16x2((uint16_t)(wv[e] & 0xffffu));
+                    h[2 * e + 1] = fp8x2_to_f16x2((uint16_t)(wv[e] >> 16));
+                }
+                if (kv == 1 && (r < vlo || r >= vhi))
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) h[e] = 0u;
+                unsigned char *row = conv + (kv * NH + (cc >> 2)) * kBoxBytes + r * 128;
+                const int c0 = 2 * (cc & 3);
+                *reinterpret_cast<uint4 *>(row + ((c0 ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4 *>(row + (((c0 + 1) ^ (r & 7)) << 4)) =
+                    make_uint4(h[4], h[5], h[6], h[7]);
+            }
+            __syncwarp();
+            // the stage has been read: its next copy can start now
+            if (idx + NST < my_count) {
+                if ((idx + NST) % kWarpCap == 0) {   // next window of this warp's pieces
+                    warp_refill(a, wr, warp, idx + NST, b, wtab);
+                    warp_translate(a, b, lane, min(my_count - (idx + NST), kWarpCap), wtab);
+                    __syncwarp();
+                }
+                maybe_append(idx + NST);
+                if (lane == 0) issue(idx + NST, st);
+            }
+            issued_early = true;
+            kp = conv;
+            vp = conv + NH * kBoxBytes;
+        } else if (vlo > 0 || vhi < kPiece) {   // rows outside the range: zero V so 0 * junk stays 0
             for (int e = lane; e < kPiece * NH * 8; e += 32) {
                 const int r = e / (NH * 8), h = (e / 8) % NH, ch = e % 8;
                 if (r < vlo || r >= vhi)
@@ -649,7 +713,15 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             const int ch = ch0 + ((lane >> 3) & 1);
             uint32_t b0, b1, b2, b3;
             ldmatrix_x4(kbase + half * kBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4), b0, b1, b2, b3);
-            if (kk & 1) {
+            if constexpr (F8) {
+                if (kk & 1) {
+                    mma_f16_16816(sb[0], qa[kk], b0, b1);
+                    mma_f16_16816(sb[1], qa[kk], b2, b3);
+                } else {
+                    mma_f16_16816(sa[0], qa[kk], b0, b1);
+                    mma_f16_16816(sa[1], qa[kk], b2, b3);
+                }
+            } else if (kk & 1) {
                 mma_bf16_16816(sb[0], qa[kk], b0, b1);
                 mma_bf16_16816(sb[1], qa[kk], b2, b3);
             } else {
@@ -691,13 +763,20 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             float ph[4], pl[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                ph[e] = bf16_round(p[e]);
+                ph[e] = F8 ? f16_round(p[e]) : bf16_round(p[e]);
                 pl[e] = p[e] - ph[e];
             }
-            pa[0] = pack_bf16x2(ph[0], ph[1]);
-            pa[1] = pack_bf16x2(pl[0], pl[1]);
-            pa[2] = pack_bf16x2(ph[2], ph[3]);
-            pa[3] = pack_bf16x2(pl[2], pl[3]);
+            if constexpr (F8) {
+                pa[0] = pack_f16x2(ph[0], ph[1]);
+                pa[1] = pack_f16x2(pl[0], pl[1]);
+                pa[2] = pack_f16x2(ph[2], ph[3]);
+                pa[3] = pack_f16x2(pl[2], pl[3]);
+            } else {
+                pa[0] = pack_bf16x2(ph[0], ph[1]);
+                pa[1] = pack_bf16x2(pl[0], pl[1]);
+                pa[2] = pack_bf16x2(ph[2], ph[3]);
+                pa[3] = pack_bf16x2(pl[2], pl[3]);
+            }
         }
         // O += P V
 #pragma unroll
@@ -707,11 +786,16 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             const int ch = ch0 + (lane >> 4);
             uint32_t r0, r1, r2, r3;
             ldmatrix_x4_trans(vbase + half * kBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4), r0, r1, r2, r3);
-            mma_bf16_16816(o[2 * cp], pa, r0, r1);
-            mma_bf16_16816(o[2 * cp + 1], pa, r2, r3);
+            if constexpr (F8) {
+                mma_f16_16816(o[2 * cp], pa, r0, r1);
+                mma_f16_16816(o[2 * cp + 1], pa, r2, r3);
+            } else {
+                mma_bf16_16816(o[2 * cp], pa, r0, r1);
+                mma_bf16_16816(o[2 * cp + 1], pa, r2, r3);
+            }
         }
         __syncwarp();
-        if (idx + NST < my_count) {
+        if (!issued_early && idx + NST < my_count) {
             if ((idx + NST) % kWarpCap == 0) {   // next window of this warp's pieces
                 warp_refill(a, wr, warp, idx + NST, b, wtab);
                 warp_translate(a, b, lane, min(my_count - (idx + NST), kWarpCap), wtab);
@@ -747,7 +831,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         cluster_finish(a, b, g, wm, wl, wo, sml, reinterpret_cast<float *>(dsm + 32768));
     else
         finish(a, s, b, g, c, wm, wl, wo, sml);
-    if (a.app.k_new) finish_append(a, b, g, wr.app, cta_wrote);
+    if (a.app.k_new) finish_append<T>(a, b, g, wr.app, cta_wrote);
 }
 
 // ======================================================================
@@ -838,11 +922,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_generic_kernel(DecArgs a) 
 // ======================================================================
 // Host side
 // ======================================================================
-constexpr int kTcStages = 3;   // pieces in flight per warp
+constexpr int kTcStages = 3;   // pieces in flight per warp (bf16)
+constexpr int kF8Stages = 4;   // pieces in flight per warp (FP8: half the bytes per piece)
 
 static bool use_tc(const bsa_kv_desc *d) {
-    return d->kv_dtype == BSA_BF16 && (d->D == 64 || d->D == 128) && d->Hq / d->Hkv <= kMaxG &&
-           d->stride_t == d->D;
+    const bool dt = d->kv_dtype == BSA_BF16 ? (d->D == 64 || d->D == 128)
+                                            : d->kv_dtype == BSA_FP8_E4M3 && d->D == 128;
+    return dt && d->Hq / d->Hkv <= kMaxG && d->stride_t == d->D;
 }
 
 bool decode_can_fuse_append(const bsa_kv_desc *d) { return use_tc(d); }
@@ -928,9 +1014,12 @@ int decode_kernel_count(const bsa_kv_desc *d, int tokens_hint, int max_ranges) {
         return cluster_splits(reinterpret_cast<const void *>(kern_cluster), smem, d->B * d->Hkv, nsplit,
                               cfg) > 1;
     };
-    const bool fit = d->D == 128
-                         ? clusters_fit(decode_tc_kernel<2, kTcStages, true>, TcSmem<2, kTcStages>::kBytes)
-                         : clusters_fit(decode_tc_kernel<1, 2 * kTcStages, true>, TcSmem<1, 2 * kTcStages>::kBytes);
+    const bool fit =
+        d->kv_dtype == BSA_FP8_E4M3
+            ? clusters_fit(decode_tc_kernel<2, kF8Stages, true, true>, TcSmem<2, kF8Stages, true>::kBytes)
+        : d->D == 128
+            ? clusters_fit(decode_tc_kernel<2, kTcStages, true>, TcSmem<2, kTcStages>::kBytes)
+            : clusters_fit(decode_tc_kernel<1, 2 * kTcStages, true>, TcSmem<1, 2 * kTcStages>::kBytes);
     return fit ? 1 : 2;
 }
 
@@ -1001,7 +1090,10 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
             return BSA_OK;
         };
         bsa_status r;
-        if (d->D == 128)
+        if (d->kv_dtype == BSA_FP8_E4M3)
+            r = go_tc(decode_tc_kernel<2, kF8Stages, false, true>, decode_tc_kernel<2, kF8Stages, true, true>,
+                      TcSmem<2, kF8Stages, true>::kBytes);
+        else if (d->D == 128)
             r = go_tc(decode_tc_kernel<2, kTcStages, false>, decode_tc_kernel<2, kTcStages, true>,
                       TcSmem<2, kTcStages>::kBytes);
         else   // D = 64
@@ -1022,6 +1114,8 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
         bsa_status r;
         if (d->kv_dtype == BSA_BF16)
             r = d->D == 128 ? go(decode_generic_kernel<uint16_t, 128>) : go(decode_generic_kernel<uint16_t, 64>);
+        else if (d->kv_dtype == BSA_FP8_E4M3)
+            r = d->D == 128 ? go(decode_generic_kernel<uint8_t, 128>) : go(decode_generic_kernel<uint8_t, 64>);
         else
             r = d->D == 128 ? go(decode_generic_kernel<float, 128>) : go(decode_generic_kernel<float, 64>);
         if (r != BSA_OK) return r;

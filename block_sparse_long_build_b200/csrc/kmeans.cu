@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const char *K, const c
 bsa_status launch_gather_rows(const bsa_kv_desc *src, const void *K, const void *V, const bsa_kv_desc *dst,
                               void *K_out, void *V_out, const int32_t *rows, int64_t n, int64_t dst_row0,
                               cudaStream_t st) {
-    const int64_t es = src->kv_dtype == BSA_BF16 ? 2 : 4;
+    const int64_t es = src->kv_dtype == BSA_F32 ? 4 : src->kv_dtype == BSA_BF16 ? 2 : 1;
     const dim3 grid((unsigned)div_up(n, 8), (unsigned)(src->B * src->Hkv));
     gather_rows_kernel<<<grid, 256, 0, st>>>(
         static_cast<const char *>(K), static_cast<const char *>(V), static_cast<char *>(K_out),

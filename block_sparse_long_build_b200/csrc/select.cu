@@ -748,7 +748,7 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
     a.topk = p->topk; a.budget = p->budget_tokens; a.sink = p->sink; a.window = p->window;
     a.keep_current = p->keep_current_block; a.local_start = p->local_start;
     a.pos_limit = p->pos_limit; a.max_sel = max_sel; a.max_ranges = max_ranges;
-    const bool bf = kind == BSA_SUM_MINMAX && d->kv_dtype == BSA_BF16;
+    const bool bf = kind == BSA_SUM_MINMAX && d->kv_dtype != BSA_F32;   // bf16 bounds (FP8: exact)
     const int esz = bf ? 2 : 4;
     const int cols = kind == BSA_SUM_MINMAX ? 2 * d->D : d->D;
     a.row_bytes = cols * esz;

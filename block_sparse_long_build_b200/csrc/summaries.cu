@@ -100,6 +100,8 @@ bsa_status launch_build_summaries(const bsa_kv_desc *d, const void *K, const bsa
     size_t smem = summary_smem(kind, d->D);
     if (d->kv_dtype == BSA_BF16)
         build_summaries_kernel<uint16_t><<<grid, 128, smem, st>>>(a);
+    else if (d->kv_dtype == BSA_FP8_E4M3)
+        build_summaries_kernel<uint8_t><<<grid, 128, smem, st>>>(a);
     else
         build_summaries_kernel<float><<<grid, 128, smem, st>>>(a);
     BSA_LAUNCH_CHECK();
@@ -119,6 +121,8 @@ bsa_status launch_append(const bsa_kv_desc *d, void *K, void *V, const void *kn,
     size_t smem = summary_smem(kind, d->D);
     if (d->kv_dtype == BSA_BF16)
         BSA_CUDA_TRY(launch_pdl(append_kernel<uint16_t>, dim3(d->B), dim3(256), smem, st, a));
+    else if (d->kv_dtype == BSA_FP8_E4M3)
+        BSA_CUDA_TRY(launch_pdl(append_kernel<uint8_t>, dim3(d->B), dim3(256), smem, st, a));
     else
         BSA_CUDA_TRY(launch_pdl(append_kernel<float>, dim3(d->B), dim3(256), smem, st, a));
     BSA_LAUNCH_CHECK();

@@ -8,6 +8,8 @@
 //                  m = mean of u_r as above, c = m / ||m||
 //   minmax         running min / max over rows in order (first wins on ties)
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace bsa {
@@ -52,11 +54,16 @@ __device__ __forceinline__ void summarize_centroid(const T *K, const KvRows &kr,
     }
 }
 
-// Min/max of rows [r0, r1) in the cache dtype, stored as (min, max) pairs
-// per dimension: thread i < D scans dimension i in row order.
+// Element type of MINMAX summaries for a cache of T: the cache dtype, bf16
+// (exact) for an FP8 cache.
+template <typename T>
+using minmax_t = std::conditional_t<sizeof(T) == 4, float, uint16_t>;
+
+// Min/max of rows [r0, r1), stored as (min, max) pairs per dimension (fp32
+// or bf16 bits): thread i < D scans dimension i in row order.
 template <typename T>
 __device__ __forceinline__ void summarize_minmax(const T *K, const KvRows &kr, int b, int g, int D,
-                                                 int64_t r0, int64_t r1, T *o) {
+                                                 int64_t r0, int64_t r1, minmax_t<T> *o) {
     const int i = threadIdx.x;
     const int64_t n = r1 - r0;
     if (i < D) {
@@ -67,7 +74,7 @@ __device__ __forceinline__ void summarize_minmax(const T *K, const KvRows &kr, i
             if (v > hi) hi = v;
         }
         if (n <= 0) lo = hi = 0.0f;
-        if constexpr (sizeof(T) == 2) {
+        if constexpr (sizeof(T) <= 2) {   // bf16 and FP8 values are bf16 values: exact
             o[2 * i] = static_cast<uint16_t>(__float_as_uint(lo) >> 16);
             o[2 * i + 1] = static_cast<uint16_t>(__float_as_uint(hi) >> 16);
         } else {
@@ -91,7 +98,7 @@ __device__ void summarize_rows(const T *K, const KvRows &kr, int b, int g, int D
         return;
     }
     if (kind == BSA_SUM_MINMAX) {
-        summarize_minmax<T>(K, kr, b, g, D, r0, r1, static_cast<T *>(out));
+        summarize_minmax<T>(K, kr, b, g, D, r0, r1, static_cast<minmax_t<T> *>(out));
         return;
     }
     // BSA_SUM_CENTROID_NORM
@@ -129,7 +136,7 @@ __device__ void summarize_rows(const T *K, const KvRows &kr, int b, int g, int D
 }
 
 __host__ __device__ inline size_t summary_row_bytes(int kind, int D, int kv_dtype) {
-    return kind == BSA_SUM_MINMAX ? (size_t)2 * D * (kv_dtype == BSA_BF16 ? 2 : 4)
+    return kind == BSA_SUM_MINMAX ? (size_t)2 * D * (kv_dtype == BSA_F32 ? 4 : 2)
                                   : (size_t)D * 4;
 }
 

@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_PKG, "libbsa.so")
 (BSA_OK, BSA_ERR_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA, BSA_ERR_WORKSPACE, BSA_ERR_TIMEOUT,
  BSA_ERR_CAPACITY) = (0, -1, -2, -3, -4, -5, -6)
 BSA_SUM_CENTROID, BSA_SUM_CENTROID_NORM, BSA_SUM_MINMAX = 0, 1, 2
-BSA_F32, BSA_BF16 = 0, 1
+BSA_F32, BSA_BF16, BSA_FP8_E4M3 = 0, 1, 2
+_DTYPES = {torch.float32: BSA_F32, torch.bfloat16: BSA_BF16, torch.float8_e4m3fn: BSA_FP8_E4M3}
 BSA_OP_SELECT, BSA_OP_DECODE, BSA_OP_PREFILL, BSA_OP_APPEND = 0, 1, 2, 3
 
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_summary_blocks", "bsa_summary_bytes",
@@ -124,7 +125,7 @@ def _stream(stream):
 def kv_desc(K: torch.Tensor, Hq: int) -> KvDesc:
     """Descriptor of a [B, Hkv, L_max, D] cache (D contiguous)."""
     assert K.dim() == 4 and K.stride(3) == 1
-    dt = {torch.float32: BSA_F32, torch.bfloat16: BSA_BF16}[K.dtype]
+    dt = _DTYPES[K.dtype]
     B, H, L, D = K.shape
     return KvDesc(B, Hq, H, D, dt, L, K.stride(0), K.stride(1), K.stride(2), 0, 0, None, 0)
 
@@ -134,7 +135,7 @@ def paged_kv_desc(pool: torch.Tensor, Hq: int, page_table: torch.Tensor) -> KvDe
     contiguous) and page_table int32 [B, pages_per_seq] on the device."""
     assert pool.dim() == 4 and pool.stride(3) == 1
     assert page_table.dtype == torch.int32 and page_table.dim() == 2 and page_table.is_contiguous()
-    dt = {torch.float32: BSA_F32, torch.bfloat16: BSA_BF16}[pool.dtype]
+    dt = _DTYPES[pool.dtype]
     n_pages, H, P, D = pool.shape
     B, pps = page_table.shape
     return KvDesc(B, Hq, H, D, dt, pps * P, pool.stride(0), pool.stride(1), pool.stride(2), P, pps,

@@ -166,7 +166,7 @@ class DecodeSession:
         its size (q fp32 [B, Hq, D], k_new / v_new in the cache dtype
         [B, Hkv, D], each 256-byte aligned)."""
         c = self.cfg
-        esz = 2 if c.kv_dtype == torch.bfloat16 else 4
+        esz = torch.empty(0, dtype=c.kv_dtype).element_size()
         nq, nk = c.B * c.Hq * c.D * 4, c.B * c.Hkv * c.D * esz
         ok = _align(nq)
         ov = ok + _align(nk)
@@ -193,7 +193,7 @@ class DecodeSession:
         eager step first so that one-time host setup is not captured."""
         c, dev = self.cfg, self.wl.device
         oq, ok, ov, n = self.io_in_layout()
-        esz = 2 if c.kv_dtype == torch.bfloat16 else 4
+        esz = torch.empty(0, dtype=c.kv_dtype).element_size()
         nq, nk = c.B * c.Hq * c.D * 4, c.B * c.Hkv * c.D * esz
         self.io_in = torch.zeros(n, dtype=torch.uint8, device=dev)
         self.q_in = self.io_in[oq:oq + nq].view(torch.float32).view(c.B, c.Hq, c.D)
@@ -253,5 +253,6 @@ class DecodeSession:
     def fuses(self) -> bool:
         """Whether bsa_decode_step runs as one launch for this workload."""
         c = self.cfg
-        return (c.kv_dtype == torch.bfloat16 and c.D in (64, 128) and c.G <= 8
-                and not (c.block_size > 0 and self.kind == N.BSA_SUM_CENTROID_NORM))
+        tc = (c.kv_dtype == torch.bfloat16 and c.D in (64, 128)) or \
+            (c.kv_dtype == torch.float8_e4m3fn and c.D == 128)
+        return tc and c.G <= 8 and not (c.block_size > 0 and self.kind == N.BSA_SUM_CENTROID_NORM)

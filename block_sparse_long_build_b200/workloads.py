@@ -136,8 +136,26 @@ def msa(seed: int = 0) -> Config:
                   True, 1, 64, seed, n_clusters=64)
 
 
+def quest_fp8(seed: int = 0) -> Config:
+    """The Quest-style paged decode with the cache in FP8 (E4M3; Attention
+    mechanisms, basic maths and the real cost: FP8 among the cache formats):
+    batch 4, 8 KV / 32 query heads, D 128; 65,536-token cache of 64 Gaussian
+    clusters; pages of 16 with min/max bounds; budget 4096 tokens; sink 256;
+    window 1024; selection refreshed every 32 steps; 128 decode steps."""
+    return replace(quest(seed), name="quest_fp8", kv_dtype=torch.float8_e4m3fn)
+
+
+def largebatch_fp8(seed: int = 0) -> Config:
+    """The large-batch decode with the cache in FP8 (E4M3): batch 64, 32 query
+    / 8 KV heads, D 128; 32,768 tokens of 32 clusters per sequence; pages of
+    32 with min/max; budget 8192; sink 256; window 512; selection every
+    step; 256 steps."""
+    return replace(largebatch(seed), name="largebatch_fp8", kv_dtype=torch.float8_e4m3fn)
+
+
 CONFIGS = {"tiny": tiny, "quest": quest, "moba": moba, "semantic": semantic,
-           "largebatch": largebatch, "msa": msa}
+           "largebatch": largebatch, "msa": msa, "quest_fp8": quest_fp8,
+           "largebatch_fp8": largebatch_fp8}
 
 
 def _gen(device, seed: int) -> torch.Generator:

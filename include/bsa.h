@@ -90,7 +90,13 @@ typedef enum {
     BSA_SUM_MINMAX = 2          /* elementwise (min, max) pairs, cache dtype      */
 } bsa_summary_kind;
 
-typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype;
+/* Element types of K and V.  BSA_FP8_E4M3 ("Attention mechanisms in modern
+ * LLMs", basic maths and the real cost: the cache may be kept in FP8):
+ * 1 sign, 4 exponent (bias 7) and 3 mantissa bits, exponent 0 subnormal,
+ * S.1111.111 NaN, no infinity (largest finite 448).  For an FP8 cache, MINMAX
+ * summaries hold the bounds as bf16 (exact), and the decode reads 1 byte per
+ * element; D must be 128 on the tensor-core path (D 64 runs on CUDA cores). */
+typedef enum { BSA_F32 = 0, BSA_BF16 = 1, BSA_FP8_E4M3 = 2 } bsa_dtype;
 
 typedef enum { BSA_OP_SELECT = 0, BSA_OP_DECODE = 1, BSA_OP_PREFILL = 2, BSA_OP_APPEND = 3 } bsa_op;
 
@@ -159,9 +165,10 @@ typedef struct {
 BSA_API int32_t bsa_summary_blocks(const bsa_kv_desc *desc, const bsa_sel_params *sel);
 
 /* Bytes of the summaries buffer: segments x blocks x (D fp32 for the centroid
- * kinds | D (min, max) pairs of cache elements for MINMAX: element 2i is the
- * block's minimum of dimension i, element 2i + 1 its maximum, so that one
- * byte permute picks and widens the bound a query's sign selects). */
+ * kinds | D (min, max) pairs for MINMAX, in the cache dtype (bf16 for an FP8
+ * cache): element 2i is the block's minimum of dimension i, element 2i + 1 its
+ * maximum, so that one byte permute picks and widens the bound a query's sign
+ * selects). */
 BSA_API size_t bsa_summary_bytes(const bsa_kv_desc *desc, const bsa_sel_params *sel,
                          bsa_summary_kind kind);
 

@@ -41,11 +41,20 @@ def current_label() -> str:
 
 
 def host(t: torch.Tensor) -> np.ndarray:
-    """Device tensor -> numpy: bf16 as uint16 bit patterns, fp32 as float32."""
+    """Device tensor -> numpy: bf16 as uint16 bit patterns, FP8 as uint8
+    codes, fp32 as float32."""
     t = t.detach().cpu().contiguous()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     return t.numpy()
+
+
+def oracle_kv(a: np.ndarray) -> np.ndarray:
+    """A host cache array in a type the oracle reads: FP8 codes decoded by the
+    oracle's own fp8_e4m3_to_f32 (exact values as float32), others as is."""
+    return oracle.fp8_e4m3_to_f32(a) if a.dtype == np.uint8 else a
 
 
 def assert_status_clean(ws: torch.Tensor | None, what: str = "") -> None:
@@ -57,7 +66,7 @@ def gpu_summaries(raw: np.ndarray, sess: DecodeSession, s: int, nb: int):
     """Segment s's first nb summaries from the raw summaries buffer."""
     c = sess.cfg
     if sess.kind == N.BSA_SUM_MINMAX:
-        esz = 2 if c.kv_dtype == torch.bfloat16 else 4
+        esz = 4 if c.kv_dtype == torch.float32 else 2   # bf16 bounds for bf16 and FP8 caches
         row = 2 * c.D * esz
         seg = raw[s * sess.nb * row:(s * sess.nb + nb) * row]
         # (min, max) pairs per dimension
@@ -91,7 +100,7 @@ class FixedDecodeCheck:
             (b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
         # the oracle's own copy of each compared segment's cache
         if page_rows:
-            Kp, Vp = host(self.sess.K), host(self.sess.V)
+            Kp, Vp = oracle_kv(host(self.sess.K)), oracle_kv(host(self.sess.V))
             table = self.sess.page_table.cpu().numpy()
             self.K, self.V = {}, {}
             for b in sorted({b for b, _ in self.segs}):
@@ -101,8 +110,8 @@ class FixedDecodeCheck:
                     if bb == b:
                         self.K[(b, g)], self.V[(b, g)] = kb[g].copy(), vb[g].copy()
         else:
-            self.K = {(b, g): host(self.wl.K[b, g]) for b, g in self.segs}
-            self.V = {(b, g): host(self.wl.V[b, g]) for b, g in self.segs}
+            self.K = {(b, g): oracle_kv(host(self.wl.K[b, g])) for b, g in self.segs}
+            self.V = {(b, g): oracle_kv(host(self.wl.V[b, g])) for b, g in self.segs}
         self.n = [int(x) for x in self.wl.cur_len.cpu()]
         self.n_sel = list(self.n)
         self.q_sel = None       # queries of the last refresh step
@@ -118,7 +127,7 @@ class FixedDecodeCheck:
             q = self.wl.decode_query(t)
             if t > 0 or c.name != "tiny":
                 k, v = self.wl.decode_new_kv(t)
-                kh, vh = host(k), host(v)
+                kh, vh = oracle_kv(host(k)), oracle_kv(host(v))
                 for b in range(c.B):
                     if self.n[b] < self.L_max:
                         for bb, g in self.segs:

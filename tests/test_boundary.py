@@ -179,3 +179,35 @@ def test_status_reader_and_test_hook_arguments(lib):
     assert L.bsa_test_arm_wait_limit(-1) == N.BSA_ERR_ARG
     assert L.bsa_test_arm_wait_limit(100001) == N.BSA_ERR_ARG
     assert L.bsa_test_arm_wait_limit(0) == N.BSA_OK                  # disarmed
+
+
+def test_fp8_summary_rows_are_bf16(lib):
+    """An FP8 cache's min/max page bounds are stored as exact bf16 pairs: the
+    summaries buffer must hold 2 * D * 2 bytes per page (the kernels' rows),
+    not 2 * D * 1."""
+    d = _desc(kv_dtype=N.BSA_FP8_E4M3)
+    p = N.sel_params(16, topk=-1, budget_tokens=4096, sink=256, window=1024)
+    nb = 65664 // 16
+    assert N.bsa_summary_bytes(d, p, N.BSA_SUM_MINMAX) == 32 * nb * 2 * 128 * 2
+    assert N.bsa_summary_bytes(d, p, N.BSA_SUM_CENTROID) == 32 * nb * 128 * 4
+    assert N.bsa_summary_bytes(d, p, 7) == 0
+
+
+def test_paged_descriptor_validation(lib):
+    """A paged descriptor needs a table, pages of a multiple of 16 rows and
+    L_max = pages_per_seq * page_rows; entry points without a paged path
+    refuse it on the host."""
+    fake = 1 << 20
+    good = dict(B=2, Hkv=2, Hq=8, L_max=64 * 10, stride_b=2 * 64 * 128, stride_h=64 * 128,
+                page_rows=64, pages_per_seq=10, page_table=fake, n_pages=25)
+    p = N.sel_params(16, topk=4, sink=16, window=32)
+    assert N.bsa_summary_blocks(_desc(**good), p) == 40
+    for bad in (dict(page_rows=24), dict(page_table=None), dict(L_max=64 * 10 + 16),
+                dict(n_pages=0), dict(page_rows=-16)):
+        assert N.bsa_summary_blocks(_desc(**{**good, **bad}), p) == -1, bad
+    L = N.lib()
+    d = _desc(**good)
+    assert L.bsa_gather_rows(ctypes.byref(d), fake, fake, ctypes.byref(d), fake, fake, fake, 10, 0,
+                             None) == N.BSA_ERR_UNSUPPORTED
+    assert L.bsa_build_semantic_index(ctypes.byref(d), fake, 100, 8, 2, fake, fake, fake, fake,
+                                      fake, fake, 1 << 30, None) == N.BSA_ERR_UNSUPPORTED
