@@ -853,6 +853,8 @@ def run_case(args, device):
     if args.case in ("decode", "select", "decode_lb", "select_lb"):
         cfg = (W.quest(0) if args.case in ("decode", "select")
                else W.largebatch(0).scaled(B=args.case_batch))
+        if args.case_fp8:
+            cfg = cfg.scaled(kv_dtype=torch.float8_e4m3fn)
         wl = W.Workload(cfg, device)
         sess = DecodeSession(wl)
         sess.build_summaries()
@@ -893,7 +895,7 @@ def run_case(args, device):
 
 def _compact(line: dict) -> dict:
     """A secondary line without the keys it shares with the headline."""
-    keep = ("metric", "value", "unit", "steps", "warmup", "ms_per_step", "ms_total",
+    keep = ("metric", "value", "unit", "dtype", "steps", "warmup", "ms_per_step", "ms_total",
             "effective_kv_gbs", "effective_kv_frac_of_8tbs", "algorithmic_tflops",
             "planted_clusters_recovered", "config", "roofline", "e2e", "gpu_launches",
             "cpu_baseline", "parity_sample", "clocks")
@@ -933,6 +935,8 @@ def main():
                     default=None, help="run one small profiling case instead of the bench (for ncu)")
     ap.add_argument("--case-batch", type=int, default=8,
                     help="sequences of the large-batch profiling cases")
+    ap.add_argument("--case-fp8", action="store_true",
+                    help="the decode and select profiling cases on an FP8 cache")
     args = ap.parse_args()
     if args.case:
         torch.cuda.set_device(0)

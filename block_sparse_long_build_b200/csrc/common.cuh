@@ -450,9 +450,10 @@ struct KvRows {
     // page is outside the pool.
     __device__ __forceinline__ int64_t off(int b, int g, int64_t r) const {
         if (!table) return b * stride_b + g * stride_h + r * stride_t;
-        const int64_t pg = __ldg(table + (int64_t)b * pps + r / P);
+        const int32_t rr = (int32_t)r;   // rows of a segment fit in 32 bits
+        const int64_t pg = __ldg(table + (int64_t)b * pps + rr / P);
         if (pg < 0 || pg >= n_pages) return -1;
-        return pg * stride_b + g * stride_h + (r % P) * stride_t;
+        return pg * stride_b + g * stride_h + (int64_t)(rr % P) * stride_t;
     }
 };
 

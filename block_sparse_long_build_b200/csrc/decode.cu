@@ -48,7 +48,6 @@ struct DecArgs {
     const int32_t *cur_len;
     const void *K, *V;
     KvRows rows;          // where each logical row lives (contiguous or paged)
-    int aligned;          // pieces cut at multiples of 16 rows (paged pools)
     int B, Hq, Hkv, G, D, L_max, nsplit;
     float scale_log2;
     float *part_o;        // [nseg][nsplit][G][D]
@@ -144,15 +143,17 @@ __device__ __forceinline__ int2 clamp_range(const DecArgs &a, int2 v, bool last,
 // start; a paged pool cuts it at multiples of 16 rows so that no piece
 // straddles a page (the first and last pieces may then use part of their
 // 16-row box).
-__device__ __forceinline__ int piece_count(int2 x, bool al) {
+template <bool AL>
+__device__ __forceinline__ int piece_count(int2 x) {
     if (x.y <= x.x) return 0;
-    return al ? (x.y + kPiece - 1) / kPiece - x.x / kPiece : (x.y - x.x + kPiece - 1) / kPiece;
+    return AL ? (x.y + kPiece - 1) / kPiece - x.x / kPiece : (x.y - x.x + kPiece - 1) / kPiece;
 }
 
 // Piece q of range x: (first row of its 16-row box, valid rows lo | hi << 8
 // of the box).
-__device__ __forceinline__ int2 piece_of(int2 x, int q, bool al) {
-    if (al) {
+template <bool AL>
+__device__ __forceinline__ int2 piece_of(int2 x, int q) {
+    if constexpr (AL) {
         const int row = (x.x / kPiece + q) * kPiece;
         return make_int2(row, max(x.x - row, 0) | (min(x.y - row, kPiece) << 8));
     }
@@ -174,15 +175,16 @@ struct WarpRanges {
 // indices i in [i0, i0 + kWarpCap): (box row, valid rows, TMA row coordinate,
 // TMA outer coordinate); a paged pool's coordinates are filled in by
 // warp_translate.
+template <bool AL>
 __device__ __forceinline__ void fill_range(const WarpRanges &w, int2 x, int pp, int warp, int i0,
-                                           int b, bool al, int4 *tab) {
-    const int cnt = piece_count(x, al);
+                                           int b, int4 *tab) {
+    const int cnt = piece_count<AL>(x);
     const int lo_p = pp - w.first - warp;                       // i >= ceil(lo_p / 4)
     const int hi_p = min(pp + cnt, w.last) - w.first - warp;    // i <  ceil(hi_p / 4)
     const int ia = max(lo_p > 0 ? (lo_p + kDecWarps - 1) / kDecWarps : 0, i0);
     const int ib = min(hi_p > 0 ? (hi_p + kDecWarps - 1) / kDecWarps : 0, i0 + kWarpCap);
     for (int i = ia; i < ib; ++i) {
-        const int2 pr = piece_of(x, w.first + warp + kDecWarps * i - pp, al);
+        const int2 pr = piece_of<AL>(x, w.first + warp + kDecWarps * i - pp);
         tab[i - i0] = make_int4(pr.x, pr.y, pr.x, b);
     }
 }
@@ -191,7 +193,6 @@ __device__ __forceinline__ void fill_range(const WarpRanges &w, int2 x, int pp, 
 // [0, n), looked up in the sequence's page table by all lanes together.  An
 // entry outside the pool gives an out-of-bounds box, which reads zeros.
 __device__ __forceinline__ void warp_translate(const DecArgs &a, int b, int lane, int n, int4 *tab) {
-    if (!a.rows.table) return;
     __syncwarp();
     for (int i = lane; i < n; i += 32) {
         int4 e = tab[i];
@@ -201,11 +202,16 @@ __device__ __forceinline__ void warp_translate(const DecArgs &a, int b, int lane
     }
 }
 
+template <bool AL>
+__device__ __forceinline__ void warp_refill(const DecArgs &a, const WarpRanges &w, int warp, int i0,
+                                            int b, int4 *tab);
+
 // Scans the range table and fills the first window of this warp's piece
-// table (the caller syncs the warp before reading it).
+// table (the caller syncs the warp before reading it).  AL: pieces cut at
+// multiples of 16 rows (paged pools).
+template <bool AL>
 __device__ __forceinline__ WarpRanges warp_ranges(const DecArgs &a, int s, int b, int c, int warp,
                                                   int lane, int4 *tab) {
-    const bool al = a.aligned != 0;
     WarpRanges w;
     w.R = a.ranges + (int64_t)s * a.max_ranges * 2;
     const int k = (a.max_ranges + 31) >> 5;
@@ -225,11 +231,11 @@ __device__ __forceinline__ WarpRanges warp_ranges(const DecArgs &a, int s, int b
 #pragma unroll
     for (int j = 0; j < kRegRanges; ++j) {
         rv[j] = clamp_range(a, rv[j], w.r0 + j == w.nr - 1, w.cl);
-        if (w.r0 + j < end) cnt += piece_count(rv[j], al);
+        if (w.r0 + j < end) cnt += piece_count<AL>(rv[j]);
     }
     for (int r = w.r0 + kRegRanges; r < end; ++r) {
         const int2 x = clamp_range(a, __ldg(R2 + r), r == w.nr - 1, w.cl);
-        cnt += piece_count(x, al);
+        cnt += piece_count<AL>(x);
     }
     int incl = cnt;
 #pragma unroll
@@ -243,31 +249,23 @@ __device__ __forceinline__ WarpRanges warp_ranges(const DecArgs &a, int s, int b
     per = (per + kDecWarps - 1) / kDecWarps * kDecWarps;
     w.first = min(c * per, w.P);
     w.last = min(w.P, w.first + per);
-    int pp = w.pbase;
-#pragma unroll
-    for (int j = 0; j < kRegRanges; ++j)
-        if (w.r0 + j < end && pp < w.last) {
-            fill_range(w, rv[j], pp, warp, 0, b, al, tab);
-            pp += piece_count(rv[j], al);
-        }
-    for (int r = w.r0 + kRegRanges; r < end && pp < w.last; ++r) {
-        const int2 x = clamp_range(a, __ldg(R2 + r), r == w.nr - 1, w.cl);
-        fill_range(w, x, pp, warp, 0, b, al, tab);
-        pp += piece_count(x, al);
-    }
+    // the first window, from the same slots (now in L1) in a rolled loop: this
+    // code runs once per warp, so it stays short
+    warp_refill<AL>(a, w, warp, 0, b, tab);
     return w;
 }
 
-// Refills the table with the window i in [i0, i0 + kWarpCap).
+// Fills the table with the window i in [i0, i0 + kWarpCap).
+template <bool AL>
 __device__ __forceinline__ void warp_refill(const DecArgs &a, const WarpRanges &w, int warp, int i0,
                                             int b, int4 *tab) {
-    const bool al = a.aligned != 0;
     int pp = w.pbase;
     const int end = min(w.r1, w.nr);
+#pragma unroll 1
     for (int r = w.r0; r < end && pp < w.last; ++r) {
         const int2 x = clamp_range(a, __ldg(reinterpret_cast<const int2 *>(w.R) + r), r == w.nr - 1, w.cl);
-        fill_range(w, x, pp, warp, i0, b, al, tab);
-        pp += piece_count(x, al);
+        fill_range<AL>(w, x, pp, warp, i0, b, tab);
+        pp += piece_count<AL>(x);
     }
 }
 
@@ -501,7 +499,7 @@ struct TcSmem {
     static_assert(!F8 || NH == 2, "FP8 pieces are 128 columns");
 };
 
-template <int NH, int NST, bool CLUSTER, bool F8 = false>
+template <int NH, int NST, bool CLUSTER, bool F8, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      DecArgs a) {
@@ -556,11 +554,11 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         else if (lane >= 16 && lane - 16 < kChunks)
             nkv = __ldg(static_cast<const uint4 *>(a.app.v_new) + (int64_t)s * kChunks + lane - 16);
     }
-    const WarpRanges wr = warp_ranges(a, s, b, c, warp, lane, wtab);
+    const WarpRanges wr = warp_ranges<PAGED>(a, s, b, c, warp, lane, wtab);
     const int n_my = wr.last - wr.first;
     // this warp's pieces: CTA-local indices warp, warp + 4, warp + 8, ...
     const int my_count = n_my > warp ? (n_my - warp + kDecWarps - 1) / kDecWarps : 0;
-    warp_translate(a, b, lane, min(my_count, kWarpCap), wtab);
+    if constexpr (PAGED) warp_translate(a, b, lane, min(my_count, kWarpCap), wtab);
     __syncwarp();
     auto issue = [&](int idx, int st) {   // lane 0 only
         const int4 pr = wtab[idx % kWarpCap];
@@ -585,7 +583,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         if (wr.app < 0) return;
         const int4 pr = wtab[idx % kWarpCap];
         if (pr.x + (pr.y & 255) <= wr.app && wr.app < pr.x + (pr.y >> 8)) {
-            const int64_t off = a.rows.off(b, g, wr.app);
+            const int64_t off = PAGED ? a.rows.off(b, g, wr.app)
+                                      : b * a.rows.stride_b + g * a.rows.stride_h + (int64_t)wr.app * a.rows.stride_t;
             if (off >= 0) {   // (a row whose page is outside the pool is not written)
                 if (lane < kChunks)
                     reinterpret_cast<uint4 *>(static_cast<T *>(const_cast<void *>(a.K)) + off)[lane] = nkv;
@@ -681,8 +680,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             // the stage has been read: its next copy can start now
             if (idx + NST < my_count) {
                 if ((idx + NST) % kWarpCap == 0) {   // next window of this warp's pieces
-                    warp_refill(a, wr, warp, idx + NST, b, wtab);
-                    warp_translate(a, b, lane, min(my_count - (idx + NST), kWarpCap), wtab);
+                    warp_refill<PAGED>(a, wr, warp, idx + NST, b, wtab);
+                    if constexpr (PAGED) warp_translate(a, b, lane, min(my_count - (idx + NST), kWarpCap), wtab);
                     __syncwarp();
                 }
                 maybe_append(idx + NST);
@@ -797,8 +796,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         __syncwarp();
         if (!issued_early && idx + NST < my_count) {
             if ((idx + NST) % kWarpCap == 0) {   // next window of this warp's pieces
-                warp_refill(a, wr, warp, idx + NST, b, wtab);
-                warp_translate(a, b, lane, min(my_count - (idx + NST), kWarpCap), wtab);
+                warp_refill<PAGED>(a, wr, warp, idx + NST, b, wtab);
+                if constexpr (PAGED) warp_translate(a, b, lane, min(my_count - (idx + NST), kWarpCap), wtab);
                 __syncwarp();
             }
             maybe_append(idx + NST);
@@ -1014,12 +1013,15 @@ int decode_kernel_count(const bsa_kv_desc *d, int tokens_hint, int max_ranges) {
         return cluster_splits(reinterpret_cast<const void *>(kern_cluster), smem, d->B * d->Hkv, nsplit,
                               cfg) > 1;
     };
-    const bool fit =
-        d->kv_dtype == BSA_FP8_E4M3
-            ? clusters_fit(decode_tc_kernel<2, kF8Stages, true, true>, TcSmem<2, kF8Stages, true>::kBytes)
-        : d->D == 128
-            ? clusters_fit(decode_tc_kernel<2, kTcStages, true>, TcSmem<2, kTcStages>::kBytes)
-            : clusters_fit(decode_tc_kernel<1, 2 * kTcStages, true>, TcSmem<1, 2 * kTcStages>::kBytes);
+    auto fits = [&](auto paged) -> bool {
+        constexpr bool PG = decltype(paged)::value;
+        if (d->kv_dtype == BSA_FP8_E4M3)
+            return clusters_fit(decode_tc_kernel<2, kF8Stages, true, true, PG>, TcSmem<2, kF8Stages, true>::kBytes);
+        if (d->D == 128)
+            return clusters_fit(decode_tc_kernel<2, kTcStages, true, false, PG>, TcSmem<2, kTcStages>::kBytes);
+        return clusters_fit(decode_tc_kernel<1, 2 * kTcStages, true, false, PG>, TcSmem<1, 2 * kTcStages>::kBytes);
+    };
+    const bool fit = d->page_rows > 0 ? fits(std::true_type()) : fits(std::false_type());
     return fit ? 1 : 2;
 }
 
@@ -1039,7 +1041,6 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
     a.q = q; a.out = out; a.lse = lse; a.ranges = ranges; a.n_ranges = n_ranges;
     a.max_ranges = max_ranges; a.cur_len = cur_len; a.K = K; a.V = V;
     a.rows = kv_rows(d);
-    a.aligned = d->page_rows > 0;
     a.B = d->B; a.Hq = d->Hq; a.Hkv = d->Hkv; a.G = d->Hq / d->Hkv; a.D = d->D;
     a.L_max = d->L_max;
     a.nsplit = decode_nsplit(d, tokens_hint, max_ranges);
@@ -1089,16 +1090,18 @@ bsa_status launch_decode(const bsa_kv_desc *d, const float *q, const void *K, co
             BSA_CUDA_TRY(launch_pdl(kern_plain, grid, dim3(kDecThreads), smem, st, tk, tv, a));
             return BSA_OK;
         };
-        bsa_status r;
-        if (d->kv_dtype == BSA_FP8_E4M3)
-            r = go_tc(decode_tc_kernel<2, kF8Stages, false, true>, decode_tc_kernel<2, kF8Stages, true, true>,
-                      TcSmem<2, kF8Stages, true>::kBytes);
-        else if (d->D == 128)
-            r = go_tc(decode_tc_kernel<2, kTcStages, false>, decode_tc_kernel<2, kTcStages, true>,
-                      TcSmem<2, kTcStages>::kBytes);
-        else   // D = 64
-            r = go_tc(decode_tc_kernel<1, 2 * kTcStages, false>, decode_tc_kernel<1, 2 * kTcStages, true>,
-                      TcSmem<1, 2 * kTcStages>::kBytes);
+        auto by_layout = [&](auto paged) -> bsa_status {
+            constexpr bool PG = decltype(paged)::value;
+            if (d->kv_dtype == BSA_FP8_E4M3)
+                return go_tc(decode_tc_kernel<2, kF8Stages, false, true, PG>,
+                             decode_tc_kernel<2, kF8Stages, true, true, PG>, TcSmem<2, kF8Stages, true>::kBytes);
+            if (d->D == 128)
+                return go_tc(decode_tc_kernel<2, kTcStages, false, false, PG>,
+                             decode_tc_kernel<2, kTcStages, true, false, PG>, TcSmem<2, kTcStages>::kBytes);
+            return go_tc(decode_tc_kernel<1, 2 * kTcStages, false, false, PG>,   // D = 64
+                         decode_tc_kernel<1, 2 * kTcStages, true, false, PG>, TcSmem<1, 2 * kTcStages>::kBytes);
+        };
+        const bsa_status r = d->page_rows > 0 ? by_layout(std::true_type()) : by_layout(std::false_type());
         if (r != BSA_OK) return r;
         BSA_LAUNCH_CHECK();
         if (clustered) return BSA_OK;

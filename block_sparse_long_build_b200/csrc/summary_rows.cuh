@@ -32,6 +32,20 @@ __device__ __forceinline__ float row_elem(const T *K, const KvRows &kr, int b, i
     return o < 0 ? 0.0f : load_elem(K, o + i);
 }
 
+// Element i of rows r .. r + 3 of segment (b, g), the loads issued together.
+template <typename T>
+__device__ __forceinline__ void row_elems4(const T *K, const KvRows &kr, int b, int g, int64_t r,
+                                           int i, float (&v)[4]) {
+    if (!kr.table) {   // contiguous: one base, a fixed row stride
+        const T *p = K + b * kr.stride_b + g * kr.stride_h + r * kr.stride_t + i;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = load_elem(p, e * kr.stride_t);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = row_elem(K, kr, b, g, r + e, i);
+    }
+}
+
 // Centroid of rows [r0, r1): thread i < D sums dimension i in row order.
 template <typename T>
 __device__ __forceinline__ void summarize_centroid(const T *K, const KvRows &kr, int b, int g, int D,
@@ -42,12 +56,12 @@ __device__ __forceinline__ void summarize_centroid(const T *K, const KvRows &kr,
         float acc = 0.0f;
         int64_t r = r0;
         for (; r + 4 <= r1; r += 4) {   // loads batched, adds stay in order
-            float v0 = row_elem(K, kr, b, g, r, i), v1 = row_elem(K, kr, b, g, r + 1, i);
-            float v2 = row_elem(K, kr, b, g, r + 2, i), v3 = row_elem(K, kr, b, g, r + 3, i);
-            acc = __fadd_rn(acc, v0);
-            acc = __fadd_rn(acc, v1);
-            acc = __fadd_rn(acc, v2);
-            acc = __fadd_rn(acc, v3);
+            float v[4];
+            row_elems4(K, kr, b, g, r, i, v);
+            acc = __fadd_rn(acc, v[0]);
+            acc = __fadd_rn(acc, v[1]);
+            acc = __fadd_rn(acc, v[2]);
+            acc = __fadd_rn(acc, v[3]);
         }
         for (; r < r1; ++r) acc = __fadd_rn(acc, row_elem(K, kr, b, g, r, i));
         out[i] = n > 0 ? __fdiv_rn(acc, (float)n) : 0.0f;
@@ -68,8 +82,18 @@ __device__ __forceinline__ void summarize_minmax(const T *K, const KvRows &kr, i
     const int64_t n = r1 - r0;
     if (i < D) {
         float lo = __int_as_float(0x7f800000), hi = __int_as_float(0xff800000);  // +inf, -inf
-        for (int64_t r = r0; r < r1; ++r) {
-            float v = row_elem(K, kr, b, g, r, i);
+        int64_t r = r0;
+        for (; r + 4 <= r1; r += 4) {   // loads batched, rows scanned in order
+            float v[4];
+            row_elems4(K, kr, b, g, r, i, v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (v[e] < lo) lo = v[e];
+                if (v[e] > hi) hi = v[e];
+            }
+        }
+        for (; r < r1; ++r) {
+            const float v = row_elem(K, kr, b, g, r, i);
             if (v < lo) lo = v;
             if (v > hi) hi = v;
         }
