@@ -117,13 +117,15 @@ class DecodeSession:
                      self.out if out is None else out, self.lse if lse is None else lse,
                      self.ws, self.stream)
 
-    def decode_step(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor):
+    def decode_step(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                    out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
         """Append the new row and attend (no selection refresh)."""
         N.bsa_decode_step(self.desc, q, self.K, self.V, k_new, v_new, self.wl.cur_len,
                           self.sel, self.kind,
                           self.summaries if self.cfg.block_size > 0 else None, self.ranges,
-                          self.n_ranges, self.max_ranges, self.tokens_hint, self.scale, self.out,
-                          self.lse, self.ws, self.stream)
+                          self.n_ranges, self.max_ranges, self.tokens_hint, self.scale,
+                          self.out if out is None else out, self.lse if lse is None else lse,
+                          self.ws, self.stream)
 
     def step(self, t: int, q: torch.Tensor, k_new: torch.Tensor | None, v_new: torch.Tensor | None):
         """Decode step t: append (when new K/V are given), select on refresh
@@ -223,12 +225,56 @@ class DecodeSession:
             self._plain_step()
             self.host_out.copy_(self.io_out, non_blocking=True)
 
-    def _plain_step(self):
+    def _plain_step(self, q=None, k=None, v=None, out=None, lse=None):
+        q = self.q_in if q is None else q
+        k = self.k_in if k is None else k
+        v = self.v_in if v is None else v
         if self.fused:
-            self.decode_step(self.q_in, self.k_in, self.v_in)
+            self.decode_step(q, k, v, out, lse)
         else:
-            self.append(self.k_in, self.v_in)
-            self.decode(self.q_in)
+            self.append(k, v)
+            self.decode(q, out, lse)
+
+    def _io_views(self, io_in: torch.Tensor, io_out: torch.Tensor):
+        c = self.cfg
+        oq, ok, ov, _ = self.io_in_layout()
+        esz = torch.empty(0, dtype=c.kv_dtype).element_size()
+        nq, nk = c.B * c.Hq * c.D * 4, c.B * c.Hkv * c.D * esz
+        q = io_in[oq:oq + nq].view(torch.float32).view(c.B, c.Hq, c.D)
+        k = io_in[ok:ok + nk].view(c.kv_dtype).view(c.B, c.Hkv, c.D)
+        v = io_in[ov:ov + nk].view(c.kv_dtype).view(c.B, c.Hkv, c.D)
+        n_out = c.B * c.Hq * c.D * 4
+        out = io_out[:n_out].view(torch.float32).view(c.B, c.Hq, c.D)
+        lse = io_out[_align(n_out):].view(torch.float32).view(c.B, c.Hq)
+        return q, k, v, out, lse
+
+    def capture_pipelined(self):
+        """Graphs for a pipelined step loop: two device input buffers and two
+        output buffers (step t uses pair t % 2), so that a copy stream can
+        bring step t+1's inputs in and take step t-1's outputs out while step
+        t computes.  Four graphs: (refresh or not) x (buffer pair)."""
+        dev = self.wl.device
+        _, _, _, n = self.io_in_layout()
+        self.pipe_in = [torch.zeros(n, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.pipe_out = [torch.zeros(self.io_out.numel(), dtype=torch.uint8, device=dev)
+                         for _ in range(2)]
+        self.g_pipe = {}
+        for p in range(2):
+            q, k, v, out, lse = self._io_views(self.pipe_in[p], self.pipe_out[p])
+            for refresh in (True, False):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    if refresh:
+                        self.append(k, v)
+                        self.select(q)
+                        self.decode(q, out, lse)
+                    else:
+                        self._plain_step(q, k, v, out, lse)
+                self.g_pipe[(refresh, p)] = g
+
+    def replay_pipelined(self, t: int):
+        """Decode step t from buffer pair t % 2 (inputs already in pipe_in)."""
+        self.g_pipe[(t % self.cfg.refresh == 0, t % 2)].replay()
 
     def replay(self, t: int):
         """Decode step t from the captured graphs (inputs already in q_in,
