@@ -291,6 +291,183 @@ __global__ void __launch_bounds__(kSelThreads * score_tpb(GT), 3)
     pdl_trigger();
 }
 
+// Two fused multiply-adds in one instruction, each rounded once:
+// c0 = a * b0 + c0, c1 = a * b1 + c1 (bit-identical to two __fmaf_rn).
+__device__ __forceinline__ void fma2_shared_a(float &c0, float &c1, float a, float b0, float b1) {
+    asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+        "mov.b64 pa, {%2, %2};\n\tmov.b64 pb, {%3, %4};\n\tmov.b64 pc, {%0, %1};\n\t"
+        "fma.rn.f32x2 pc, pa, pb, pc;\n\tmov.b64 {%0, %1}, pc;\n\t}"
+        : "+f"(c0), "+f"(c1)
+        : "f"(a), "f"(b0), "f"(b1));
+}
+
+// Scoring with two block rows per thread, for G = 4, 8 or 16 and D = 64 or
+// 128 (min/max bf16 bounds or fp32 centroids).  A tile is 128 rows; lanes 2p
+// and 2p + 1 take rows p and p + 64 of it, lane 2p the first G/2 heads and
+// lane 2p + 1 the others.  Each head's score is still one fp32 fma chain over
+// i = 0..D-1, the two rows' chains advanced together by fma.rn.f32x2 (each
+// half rounded once, as fmaf); the query values and bound selectors a step
+// needs are read once for both rows.  Head sums in head order: lane 2p adds
+// its heads, lane 2p + 1 continues from that sum with its own.
+constexpr int kPairThreads = 128;
+
+template <int SK, int G, int D>
+__global__ void __launch_bounds__(kPairThreads, 3)
+    score_pair_kernel(const __grid_constant__ CUtensorMap tmS, SelArgs a) {
+    constexpr int HPT = G / 2;
+    static_assert(G % 2 == 0 && G <= kSelMaxG, "pairs of head slices");
+    extern __shared__ unsigned char dsm_raw[];
+    unsigned char *ring = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    const int nb = a.nb_total;
+    constexpr int QS = D + 4;                                                       // floats per head row
+    float *qbuf = reinterpret_cast<float *>(ring + (size_t)a.nst * a.tile_bytes);   // [nst][G][D+4]
+    uint32_t *selb = reinterpret_cast<uint32_t *>(qbuf + (size_t)a.nst * G * QS);   // [G][D+4]
+    __shared__ uint64_t full[kSelMaxStages];
+    const int tid = threadIdx.x;
+    const int pr = tid >> 1, part = tid & 1;   // row pair (rows pr, pr + 64), head half
+    const int my_items =
+        a.n_items > (int)blockIdx.x ? (a.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+    if (tid == 0) {
+        prefetch_tmap(&tmS);
+        for (int i = 0; i < a.nst; ++i) mbar_init(&full[i], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_wait();   // queries, lengths and summaries come from earlier kernels
+    constexpr int esz = SK == kScoreMinmaxBf16 ? 2 : 4;
+    auto issue = [&](int k) {   // thread 0: item k of this CTA into stage k % nst
+        const int item = (int)blockIdx.x + k * (int)gridDim.x;
+        const int s = item / a.tiles_per_seg, t = item % a.tiles_per_seg;
+        const int st = k % a.nst;
+        const int b = s / a.Hkv, g = s % a.Hkv;
+        unsigned char *dst = ring + (size_t)st * a.tile_bytes;
+        mbar_arrive_expect_tx(&full[st], a.tile_bytes + (uint32_t)(G * D * 4));
+        for (int bx = 0; bx < a.nbox; ++bx)
+            tma_load_2d(dst + bx * (kSelThreads * 128), &tmS, &full[st], bx * (128 / esz),
+                        s * nb + t * kSelThreads);
+        const float *qg = a.q + ((int64_t)b * a.Hq + (int64_t)g * G) * D;
+        for (int h = 0; h < G; ++h)
+            bulk_load(qbuf + (size_t)st * G * QS + h * QS, qg + h * D, (uint32_t)(D * 4), &full[st]);
+    };
+    if (tid == 0)
+        for (int k = 0; k < a.nst && k < my_items; ++k) issue(k);
+    bool timed_out = false;
+    for (int k = 0; k < my_items; ++k) {
+        const int item = (int)blockIdx.x + k * (int)gridDim.x;
+        const int s = item / a.tiles_per_seg, t = item % a.tiles_per_seg;
+        const int b = s / a.Hkv;
+        const int j0 = t * kSelThreads + pr, j1 = j0 + kSelThreads / 2;
+        const bool writer = part == 1;
+        // candidacy needs no summary: worked out while the tile is in flight
+        int vis0 = 0, vis1 = 0;
+        bool valid0 = false, valid1 = false;
+        if (writer) {
+            if (a.offsets) {
+                const int32_t *off = a.offsets + (int64_t)s * (nb + 1);
+                const int32_t *pos = a.kv_pos + (int64_t)s * a.L_max;
+                if (j0 < nb) {
+                    const int r0 = min(max(off[j0], 0), a.L_max), r1 = min(max(off[j0 + 1], r0), a.L_max);
+                    vis0 = visible_prefix(pos, r0, r1, a.pos_limit);
+                    valid0 = vis0 > 0;
+                }
+                if (j1 < nb) {
+                    const int r0 = min(max(off[j1], 0), a.L_max), r1 = min(max(off[j1 + 1], r0), a.L_max);
+                    vis1 = visible_prefix(pos, r0, r1, a.pos_limit);
+                    valid1 = vis1 > 0;
+                }
+            } else {
+                const int n = min(max(a.cur_len[b], 0), a.L_max);
+                valid0 = j0 < nb && (int64_t)(j0 + 1) * a.S <= n;
+                valid1 = j1 < nb && (int64_t)(j1 + 1) * a.S <= n;
+            }
+        }
+        const int st = k % a.nst;
+        if (!timed_out && !mbar_wait_bounded(&full[st], (uint32_t)((k / a.nst) & 1))) {
+            timed_out = true;
+            atomicOr(a.status, 2u);
+        }
+        const float *qs = qbuf + (size_t)st * G * QS;
+        if constexpr (SK == kScoreMinmaxBf16) {
+            // per (head, dimension): which bound the query's sign picks
+            for (int e = tid; e < G * D; e += blockDim.x) {
+                const int h = e / D, i = e % D;
+                selb[h * QS + i] = qs[h * QS + i] < 0.0f ? kPickMin : kPickMax;
+            }
+            __syncthreads();
+        }
+        const unsigned char *tile = ring + (size_t)st * a.tile_bytes;
+        const unsigned char *rowA = tile + pr * 128;
+        const unsigned char *rowB = tile + (pr + kSelThreads / 2) * 128;
+        uint32_t sw[8];   // swizzled chunk offsets; rows pr and pr + 64 share them
+#pragma unroll
+        for (int c = 0; c < 8; ++c) sw[c] = (uint32_t)((c ^ (pr & 7)) << 4);
+        float acc0[HPT], acc1[HPT];
+#pragma unroll
+        for (int h = 0; h < HPT; ++h) acc0[h] = acc1[h] = 0.0f;
+        const int h0 = part * HPT;
+        constexpr int W = 4;   // dimensions per 16-byte chunk (bf16 pairs or fp32)
+#pragma unroll
+        for (int i = 0; i < D; i += W) {
+            const int off = SK == kScoreMinmaxBf16 ? i * 4 : i * 4;   // bytes into the row
+            const int box = off >> 7, c = (off >> 4) & 7;
+            const uint4 wa = *reinterpret_cast<const uint4 *>(rowA + box * (kSelThreads * 128) + sw[c]);
+            const uint4 wb = *reinterpret_cast<const uint4 *>(rowB + box * (kSelThreads * 128) + sw[c]);
+            const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xb[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int h = 0; h < HPT; ++h) {
+                const float4 q4 = *reinterpret_cast<const float4 *>(qs + (h0 + h) * QS + i);
+                const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+                if constexpr (SK == kScoreMinmaxBf16) {
+                    const uint4 s4 = *reinterpret_cast<const uint4 *>(selb + (h0 + h) * QS + i);
+                    const uint32_t sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        fma2_shared_a(acc0[h], acc1[h], qv[e], widen_bf16(xa[e], sv[e]),
+                                      widen_bf16(xb[e], sv[e]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        fma2_shared_a(acc0[h], acc1[h], qv[e], __uint_as_float(xa[e]), __uint_as_float(xb[e]));
+                }
+            }
+        }
+        // heads summed in head order: lane 2p's heads, then lane 2p + 1's
+        float run0 = acc0[0], run1 = acc1[0];
+#pragma unroll
+        for (int h = 1; h < HPT; ++h) {
+            run0 = __fadd_rn(run0, acc0[h]);
+            run1 = __fadd_rn(run1, acc1[h]);
+        }
+        const float prev0 = __shfl_up_sync(0xffffffffu, run0, 1);
+        const float prev1 = __shfl_up_sync(0xffffffffu, run1, 1);
+        if (writer) {
+            run0 = prev0;
+            run1 = prev1;
+#pragma unroll
+            for (int h = 0; h < HPT; ++h) {
+                run0 = __fadd_rn(run0, acc0[h]);
+                run1 = __fadd_rn(run1, acc1[h]);
+            }
+            auto put = [&](int j, bool valid, int vis, float run) {
+                if (j >= nb) return;
+                uint32_t key = 0;
+                if (valid) {
+                    key = f32_order_key(__fadd_rn(run, 0.0f));
+                    if (key == 0) key = 1;   // 0 marks "not a candidate"
+                }
+                a.keys[(int64_t)s * nb + j] = key;
+                if (a.offsets) a.vis[(int64_t)s * nb + j] = vis;
+            };
+            put(j0, valid0, vis0, run0);
+            put(j1, valid1, vis1, run1);
+        }
+        __syncthreads();   // stage st has been read by every thread
+        if (tid == 0 && k + a.nst < my_items) issue(k + a.nst);
+    }
+    pdl_trigger();
+}
+
 // ---------------------------------------------------------------- picking
 constexpr int kPickWarpKeys = 16;   // keys per lane of the one-warp walks (nb <= 512)
 
@@ -779,6 +956,14 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
     };
     auto by_gd = [&](auto sk, auto dt) -> bsa_status {
         constexpr int SK = decltype(sk)::value, DT = decltype(dt)::value;
+        if constexpr (SK != kScoreMinmaxF32 && DT > 0) {   // two rows per thread
+            switch (a.G) {
+                case 4: return launch(score_pair_kernel<SK, 4, DT>, kPairThreads / kSelThreads);
+                case 8: return launch(score_pair_kernel<SK, 8, DT>, kPairThreads / kSelThreads);
+                case 16: return launch(score_pair_kernel<SK, 16, DT>, kPairThreads / kSelThreads);
+                default: break;
+            }
+        }
         switch (a.G) {
             case 1: return launch(score_kernel<SK, 1, DT>, score_tpb(1));
             case 2: return launch(score_kernel<SK, 2, DT>, score_tpb(2));
