@@ -23,7 +23,7 @@ int decode_nsplit(const bsa_kv_desc *, int, int);
 int decode_kernel_count(const bsa_kv_desc *, int, int);
 size_t decode_scratch_bytes(const bsa_kv_desc *, int);
 bsa_status launch_prefill(const bsa_kv_desc *, const void *, const void *, const bsa_sel_params *,
-                          const void *, const bsa_kv_desc *, const void *, const void *,
+                          const void *, const bsa_kv_desc *, const void *, const void *, int,
                           const void *, int, int, float, float *, float *, uint32_t *, void *,
                           size_t, cudaStream_t);
 size_t prefill_ws_bytes(const bsa_kv_desc *, const bsa_sel_params *, int);
@@ -427,8 +427,9 @@ bsa_status bsa_append_kv(const bsa_kv_desc *d, void *K, void *V, const void *k_n
 bsa_status bsa_prefill_grouped(const bsa_kv_desc *d, const void *K, const void *V,
                                const bsa_sel_params *p, const void *summaries,
                                const bsa_kv_desc *pd, const void *K_pos, const void *V_pos,
-                               const void *Q, int32_t q_pos0, int32_t Tq, float scale, float *out,
-                               float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream) {
+                               int32_t pos_base, const void *Q, int32_t q_pos0, int32_t Tq,
+                               float scale, float *out, float *lse, void *ws, size_t ws_bytes,
+                               bsa_stream_t stream) {
     if (!desc_ok(d) || !desc_ok(pd) || !sel_ok(d, p)) return BSA_ERR_ARG;
     if (!K || !V || !summaries || !K_pos || !V_pos || !Q || !out) return BSA_ERR_ARG;
     if (!aligned16(K) || !aligned16(V) || !aligned16(K_pos) || !aligned16(V_pos) || !aligned16(Q) ||
@@ -440,13 +441,15 @@ bsa_status bsa_prefill_grouped(const bsa_kv_desc *d, const void *K, const void *
         return BSA_ERR_ARG;
     if (d->kv_dtype != BSA_BF16 || pd->kv_dtype != BSA_BF16 || d->D != 128) return BSA_ERR_UNSUPPORTED;
     if (d->stride_t != d->D || pd->stride_t != pd->D) return BSA_ERR_UNSUPPORTED;
-    if (Tq < 1 || q_pos0 < 0 || (int64_t)q_pos0 + Tq > pd->L_max || p->pos_limit < 0 ||
-        p->pos_limit > q_pos0)
+    // the window K_pos/V_pos holds positions [pos_base, pos_base + pd->L_max): every
+    // local key, [pos_limit, q_pos0 + Tq), must be in it
+    if (Tq < 1 || q_pos0 < 0 || p->pos_limit < 0 || p->pos_limit > q_pos0 || pos_base < 0 ||
+        pos_base > p->pos_limit || (int64_t)q_pos0 + Tq - pos_base > pd->L_max)
         return BSA_ERR_ARG;
     if (!(scale > 0.0f)) return BSA_ERR_ARG;
     const size_t need = bsa_workspace_size(d, p, BSA_OP_PREFILL, Tq, 0);
     if (!ws_ok(ws, ws_bytes, need)) return BSA_ERR_WORKSPACE;
-    return launch_prefill(d, K, V, p, summaries, pd, K_pos, V_pos, Q, q_pos0, Tq, scale, out, lse,
+    return launch_prefill(d, K, V, p, summaries, pd, K_pos, V_pos, pos_base, Q, q_pos0, Tq, scale, out, lse,
                           static_cast<uint32_t *>(ws), static_cast<char *>(ws) + counters_bytes(d),
                           ws_bytes - counters_bytes(d), (cudaStream_t)stream);
 }

@@ -45,6 +45,7 @@ constexpr float kPfLn2 = 0.69314718055994530942f;
 struct PfArgs {
     int Hq, Hkv, G, D, nb, L_max, Lpos;
     int Tq, q_pos0, pos_limit, budget;
+    int pos_base;              // position of row 0 of the position-ordered K/V
     float scale_log2;
     const uint16_t *Q;         // [Tq][Hq][D] bf16
     const float *cent;         // [Hkv][nb][D]
@@ -498,7 +499,9 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                 wait(&qready[m], (n >> 2) & 1);
                 const int *desc = desc_s + m * 8;
                 if (timed_out || desc[5]) break;
-                const int g = desc[0], kbeg = desc[1], T = desc[3];
+                const int g = desc[0], T = desc[3];
+                // local items address the position-ordered window from its base
+                const int kbeg = desc[1] - (desc[4] ? a.pos_base : 0);
                 const CUtensorMap *map = desc[4] ? (isk ? &tmKl : &tmVl) : (isk ? &tmKp : &tmVp);
                 for (int t = 0; t < T; ++t, ++u) {
                     const int st = u & 1;
@@ -807,7 +810,7 @@ size_t prefill_ws_bytes(const bsa_kv_desc *d, const bsa_sel_params *p, int Tq) {
 
 bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
                           const bsa_sel_params *p, const void *summaries, const bsa_kv_desc *pd,
-                          const void *K_pos, const void *V_pos, const void *Q, int q_pos0, int Tq,
+                          const void *K_pos, const void *V_pos, int pos_base, const void *Q, int q_pos0, int Tq,
                           float scale, float *out, float *lse, uint32_t *status, void *ws,
                           size_t ws_bytes, cudaStream_t st) {
     const int G = d->Hq / d->Hkv;
@@ -822,6 +825,7 @@ bsa_status launch_prefill(const bsa_kv_desc *d, const void *K, const void *V,
     a.Hq = d->Hq; a.Hkv = d->Hkv; a.G = G; a.D = d->D; a.nb = p->n_blocks;
     a.L_max = d->L_max; a.Lpos = pd->L_max;
     a.Tq = Tq; a.q_pos0 = q_pos0; a.pos_limit = p->pos_limit; a.budget = p->budget_tokens;
+    a.pos_base = pos_base;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.Q = static_cast<const uint16_t *>(Q);
     a.cent = static_cast<const float *>(summaries);

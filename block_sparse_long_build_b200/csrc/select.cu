@@ -376,12 +376,10 @@ __global__ void __launch_bounds__(kPairThreads, 3)
                     vis1 = visible_prefix(pos, r0, r1, a.pos_limit);
                     valid1 = vis1 > 0;
                 }
-            } else {
-                const int n = min(max(a.cur_len[b], 0), a.L_max);
-                valid0 = j0 < nb && (int64_t)(j0 + 1) * a.S <= n;
-                valid1 = j1 < nb && (int64_t)(j1 + 1) * a.S <= n;
             }
         }
+        // fixed blocks: the length is loaded now and compared after the scoring
+        const int n_fixed = !a.offsets && writer ? __ldg(a.cur_len + b) : 0;
         const int st = k % a.nst;
         if (!timed_out && !mbar_wait_bounded(&full[st], (uint32_t)((k / a.nst) & 1))) {
             timed_out = true;
@@ -442,6 +440,11 @@ __global__ void __launch_bounds__(kPairThreads, 3)
         const float prev0 = __shfl_up_sync(0xffffffffu, run0, 1);
         const float prev1 = __shfl_up_sync(0xffffffffu, run1, 1);
         if (writer) {
+            if (!a.offsets) {
+                const int n = min(max(n_fixed, 0), a.L_max);
+                valid0 = j0 < nb && (int64_t)(j0 + 1) * a.S <= n;
+                valid1 = j1 < nb && (int64_t)(j1 + 1) * a.S <= n;
+            }
             run0 = prev0;
             run1 = prev1;
 #pragma unroll

@@ -86,8 +86,8 @@ def lib() -> ctypes.CDLL:
             "bsa_append_kv": (ctypes.c_int, [pd, P, P, P, P, P, pp, ctypes.c_int, P, P]),
             "bsa_decode_step": (ctypes.c_int, [pd, P, P, P, P, P, P, pp, ctypes.c_int, P, P, P, I32,
                                                I32, F, P, P, P, SZ, P]),
-            "bsa_prefill_grouped": (ctypes.c_int, [pd, P, P, pp, P, pd, P, P, P, I32, I32, F, P, P,
-                                                   P, SZ, P]),
+            "bsa_prefill_grouped": (ctypes.c_int, [pd, P, P, pp, P, pd, P, P, I32, P, I32, I32, F, P,
+                                                   P, P, SZ, P]),
             "bsa_workspace_status": (ctypes.c_int, [P, SZ, I32, ctypes.POINTER(ctypes.c_uint32), P]),
             "bsa_test_arm_wait_limit": (ctypes.c_int, [I32]),
         }
@@ -233,12 +233,12 @@ def bsa_decode_step(desc, q, K, V, k_new, v_new, cur_len, sel, kind, summaries, 
                                  ws.numel() * ws.element_size(), _stream(stream)))
 
 
-def bsa_prefill_grouped(desc, K, V, sel, summaries, pos_desc, K_pos, V_pos, Q, q_pos0, Tq, scale,
-                        out, lse, ws, stream=None):
+def bsa_prefill_grouped(desc, K, V, sel, summaries, pos_desc, K_pos, V_pos, pos_base, Q, q_pos0,
+                        Tq, scale, out, lse, ws, stream=None):
     _check("bsa_prefill_grouped",
            lib().bsa_prefill_grouped(ctypes.byref(desc), _p(K), _p(V), ctypes.byref(sel),
                                      _p(summaries), ctypes.byref(pos_desc), _p(K_pos), _p(V_pos),
-                                     _p(Q), q_pos0, Tq, scale, _p(out), _p(lse), _p(ws),
+                                     pos_base, _p(Q), q_pos0, Tq, scale, _p(out), _p(lse), _p(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)))
 
 

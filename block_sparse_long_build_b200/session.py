@@ -154,12 +154,17 @@ class DecodeSession:
         sel = N.sel_params(0, c.n_blocks, wl.block_offsets, wl.kv_pos, topk=-1,
                            budget_tokens=q_pos0 // 16 if sparse else 0,
                            local_start=wl.local_start, pos_limit=q_pos0 if sparse else 0)
-        pos_desc = N.kv_desc(wl.Kpos, c.Hq)
+        # the position-ordered window the local part reads: the chunk's own
+        # rows past the dense limit, the whole prefix below it
+        base = q_pos0 if sparse else 0
+        Kw = wl.Kpos[:, :, base:q_pos0 + Tq]
+        Vw = wl.Vpos[:, :, base:q_pos0 + Tq]
+        pos_desc = N.kv_desc(Kw, c.Hq)
         need = N.bsa_workspace_size(self.desc, sel, N.BSA_OP_PREFILL, Tq, 0)
         if ws is None or ws.numel() < need:
             ws = torch.zeros(need, dtype=torch.uint8, device=wl.device)
-        N.bsa_prefill_grouped(self.desc, wl.K, wl.V, sel, self.summaries, pos_desc, wl.Kpos,
-                              wl.Vpos, Q, q_pos0, Tq, self.scale, out, lse, ws, self.stream)
+        N.bsa_prefill_grouped(self.desc, wl.K, wl.V, sel, self.summaries, pos_desc, Kw, Vw, base,
+                              Q, q_pos0, Tq, self.scale, out, lse, ws, self.stream)
         return ws
 
     # ------------------------------------------------------------ CUDA graphs

@@ -313,7 +313,10 @@ BSA_API bsa_status bsa_decode_step(const bsa_kv_desc *desc, const float *q, void
 /* Block-grouped prefill for variable (semantic) blocks, batch 1.
  * Query row i sits at position q_pos0 + i and reads
  *   (a) the positions [pos_limit, q_pos0 + i] densely and causally from the
- *       position-ordered cache K_pos / V_pos (pos_desc geometry), and
+ *       position-ordered keys and values K_pos / V_pos (pos_desc geometry),
+ *       whose row r holds position pos_base + r -- for a chunk past the dense
+ *       limit (pos_limit = q_pos0) just the chunk's own rows, pos_base =
+ *       q_pos0; it must cover [pos_limit, q_pos0 + Tq), and
  *   (b) the visible prefixes (kv_pos < pos_limit) of the blocks its group
  *       selects from the block-ordered store K / V (desc geometry) with the
  *       variable-block rules above (budget_tokens, CENTROID_NORM summaries).
@@ -327,8 +330,8 @@ BSA_API bsa_status bsa_decode_step(const bsa_kv_desc *desc, const float *q, void
 BSA_API bsa_status bsa_prefill_grouped(const bsa_kv_desc *desc, const void *K, const void *V,
                                const bsa_sel_params *sel, const void *summaries,
                                const bsa_kv_desc *pos_desc, const void *K_pos, const void *V_pos,
-                               const void *Q, int32_t q_pos0, int32_t Tq, float scale,
-                               float *out, float *lse, void *ws, size_t ws_bytes,
+                               int32_t pos_base, const void *Q, int32_t q_pos0, int32_t Tq,
+                               float scale, float *out, float *lse, void *ws, size_t ws_bytes,
                                bsa_stream_t stream);
 
 /* The semantic index ("Semantic blocks for sparse attention", first section:

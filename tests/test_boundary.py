@@ -107,7 +107,7 @@ def test_bad_arguments_rejected_on_host(lib):
     assert L.bsa_summary_blocks(ctypes.byref(d), ctypes.byref(p3)) == -1
     # grouped prefill outside its domain (fixed blocks)
     assert L.bsa_prefill_grouped(ctypes.byref(d), fake, fake, ctypes.byref(p), fake,
-                                 ctypes.byref(d), fake, fake, fake, 0, 16, 0.1, fake, None, fake,
+                                 ctypes.byref(d), fake, fake, 0, fake, 0, 16, 0.1, fake, None, fake,
                                  1 << 30, None) in (N.BSA_ERR_ARG, N.BSA_ERR_UNSUPPORTED)
 
 
@@ -211,3 +211,26 @@ def test_paged_descriptor_validation(lib):
                              None) == N.BSA_ERR_UNSUPPORTED
     assert L.bsa_build_semantic_index(ctypes.byref(d), fake, 100, 8, 2, fake, fake, fake, fake,
                                       fake, fake, 1 << 30, None) == N.BSA_ERR_UNSUPPORTED
+
+
+def test_prefill_position_window_rules(lib):
+    """The position-ordered window must start at or before pos_limit and cover
+    every local key up to q_pos0 + Tq; otherwise the call is refused on the
+    host."""
+    L = N.lib()
+    fake = 1 << 20
+    blk = _desc(B=1, Hkv=2, Hq=8, L_max=8192, stride_b=2 * 8192 * 128, stride_h=8192 * 128)
+    p = N.sel_params(0, n_blocks=16, block_offsets=fake, kv_pos=fake, topk=-1,
+                     budget_tokens=256, pos_limit=4096)
+    win = _desc(B=1, Hkv=2, Hq=8, L_max=1024, stride_b=2 * 8192 * 128, stride_h=8192 * 128)
+
+    def call(pos_base, q_pos0, Tq):
+        return L.bsa_prefill_grouped(ctypes.byref(blk), fake, fake, ctypes.byref(p), fake,
+                                     ctypes.byref(win), fake, fake, pos_base, fake, q_pos0, Tq,
+                                     0.1, fake, None, fake, 16, None)
+
+    # valid windows reach the workspace check (too small here)
+    assert call(4096, 4096, 1024) == N.BSA_ERR_WORKSPACE
+    assert call(4096, 4096, 1025) == N.BSA_ERR_ARG      # past the window's end
+    assert call(4097, 4097, 512) == N.BSA_ERR_ARG       # base after pos_limit
+    assert call(-1, 4096, 16) == N.BSA_ERR_ARG

@@ -90,8 +90,9 @@ def _prefill(cfg, wl, sess, p, budget):
     out = torch.empty(Tq, cfg.Hq, cfg.D, device="cuda")
     lse = torch.empty(Tq, cfg.Hq, device="cuda")
     Q = wl.prefill_queries(p, Tq)
-    N.bsa_prefill_grouped(sess.desc, wl.K, wl.V, sel, sess.summaries, N.kv_desc(wl.Kpos, cfg.Hq),
-                          wl.Kpos, wl.Vpos, Q, p, Tq, 1 / math.sqrt(cfg.D), out, lse, ws)
+    Kw, Vw = wl.Kpos[:, :, p:p + Tq], wl.Vpos[:, :, p:p + Tq]   # the chunk's own rows
+    N.bsa_prefill_grouped(sess.desc, wl.K, wl.V, sel, sess.summaries, N.kv_desc(Kw, cfg.Hq), Kw, Vw,
+                          p, Q, p, Tq, 1 / math.sqrt(cfg.D), out, lse, ws)
     return N.bsa_workspace_status(ws), out
 
 
