@@ -302,17 +302,24 @@ __device__ __forceinline__ void fma2_shared_a(float &c0, float &c1, float a, flo
 }
 
 // Scoring with two block rows per thread, for G = 4, 8 or 16 and D = 64 or
-// 128 (min/max bf16 bounds or fp32 centroids).  A tile is 128 rows; lanes 2p
-// and 2p + 1 take rows p and p + 64 of it, lane 2p the first G/2 heads and
+// 128 (min/max bf16 bounds or fp32 centroids).  A tile is R = kPairRows rows
+// and the CTA R threads; lanes 2p and 2p + 1 take rows p and p + R/2 of it, lane 2p the first G/2 heads and
 // lane 2p + 1 the others.  Each head's score is still one fp32 fma chain over
 // i = 0..D-1, the two rows' chains advanced together by fma.rn.f32x2 (each
 // half rounded once, as fmaf); the query values and bound selectors a step
 // needs are read once for both rows.  Head sums in head order: lane 2p adds
 // its heads, lane 2p + 1 continues from that sum with its own.
-constexpr int kPairThreads = 128;
+#ifndef BSA_SCORE_PAIR_ROWS
+#define BSA_SCORE_PAIR_ROWS 64
+#endif
+#ifndef BSA_SCORE_PAIR_STAGES
+#define BSA_SCORE_PAIR_STAGES 1
+#endif
+constexpr int kPairRows = BSA_SCORE_PAIR_ROWS;   // rows per tile = threads per CTA
+static_assert(kPairRows == 64 || kPairRows == 128, "tile of 64 or 128 rows");
 
 template <int SK, int G, int D>
-__global__ void __launch_bounds__(kPairThreads, 3)
+__global__ void __launch_bounds__(kPairRows, 384 / kPairRows)
     score_pair_kernel(const __grid_constant__ CUtensorMap tmS, SelArgs a) {
     constexpr int HPT = G / 2;
     static_assert(G % 2 == 0 && G <= kSelMaxG, "pairs of head slices");
@@ -344,8 +351,8 @@ __global__ void __launch_bounds__(kPairThreads, 3)
         unsigned char *dst = ring + (size_t)st * a.tile_bytes;
         mbar_arrive_expect_tx(&full[st], a.tile_bytes + (uint32_t)(G * D * 4));
         for (int bx = 0; bx < a.nbox; ++bx)
-            tma_load_2d(dst + bx * (kSelThreads * 128), &tmS, &full[st], bx * (128 / esz),
-                        s * nb + t * kSelThreads);
+            tma_load_2d(dst + bx * (kPairRows * 128), &tmS, &full[st], bx * (128 / esz),
+                        s * nb + t * kPairRows);
         const float *qg = a.q + ((int64_t)b * a.Hq + (int64_t)g * G) * D;
         for (int h = 0; h < G; ++h)
             bulk_load(qbuf + (size_t)st * G * QS + h * QS, qg + h * D, (uint32_t)(D * 4), &full[st]);
@@ -357,7 +364,7 @@ __global__ void __launch_bounds__(kPairThreads, 3)
         const int item = (int)blockIdx.x + k * (int)gridDim.x;
         const int s = item / a.tiles_per_seg, t = item % a.tiles_per_seg;
         const int b = s / a.Hkv;
-        const int j0 = t * kSelThreads + pr, j1 = j0 + kSelThreads / 2;
+        const int j0 = t * kPairRows + pr, j1 = j0 + kPairRows / 2;
         const bool writer = part == 1;
         // candidacy needs no summary: worked out while the tile is in flight
         int vis0 = 0, vis1 = 0;
@@ -396,7 +403,7 @@ __global__ void __launch_bounds__(kPairThreads, 3)
         }
         const unsigned char *tile = ring + (size_t)st * a.tile_bytes;
         const unsigned char *rowA = tile + pr * 128;
-        const unsigned char *rowB = tile + (pr + kSelThreads / 2) * 128;
+        const unsigned char *rowB = tile + (pr + kPairRows / 2) * 128;
         uint32_t sw[8];   // swizzled chunk offsets; rows pr and pr + 64 share them
 #pragma unroll
         for (int c = 0; c < 8; ++c) sw[c] = (uint32_t)((c ^ (pr & 7)) << 4);
@@ -409,8 +416,8 @@ __global__ void __launch_bounds__(kPairThreads, 3)
         for (int i = 0; i < D; i += W) {
             const int off = SK == kScoreMinmaxBf16 ? i * 4 : i * 4;   // bytes into the row
             const int box = off >> 7, c = (off >> 4) & 7;
-            const uint4 wa = *reinterpret_cast<const uint4 *>(rowA + box * (kSelThreads * 128) + sw[c]);
-            const uint4 wb = *reinterpret_cast<const uint4 *>(rowB + box * (kSelThreads * 128) + sw[c]);
+            const uint4 wa = *reinterpret_cast<const uint4 *>(rowA + box * (kPairRows * 128) + sw[c]);
+            const uint4 wb = *reinterpret_cast<const uint4 *>(rowB + box * (kPairRows * 128) + sw[c]);
             const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
             for (int h = 0; h < HPT; ++h) {
@@ -933,24 +940,28 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
     const int cols = kind == BSA_SUM_MINMAX ? 2 * d->D : d->D;
     a.row_bytes = cols * esz;
     a.nbox = a.row_bytes / 128;
-    a.tile_bytes = (uint32_t)(a.nbox * kSelThreads * 128);
+    // two rows per thread where the group size and head_dim allow
+    const bool pair = (kind != BSA_SUM_MINMAX || bf) && (d->D == 64 || d->D == 128) &&
+                      (a.G == 4 || a.G == 8 || a.G == 16);
+    const int tile_rows = pair ? kPairRows : kSelThreads;
+    a.tile_bytes = (uint32_t)(a.nbox * tile_rows * 128);
     const size_t qbytes = (size_t)a.G * (d->D + 4) * 4;
     const size_t cap = 227 * 1024 - 1024;
-    a.nst = (int)std::min<size_t>(kScoreStages, (cap - qbytes) / (a.tile_bytes + qbytes));
+    a.nst = (int)std::min<size_t>(pair ? BSA_SCORE_PAIR_STAGES : kScoreStages,
+                                  (cap - qbytes) / (a.tile_bytes + qbytes));
     if (a.nst < 1) return BSA_ERR_UNSUPPORTED;
     const size_t smem1 = 1024 + (size_t)a.nst * (a.tile_bytes + qbytes) + qbytes;   // + selectors
     const size_t smem2 = PickSmem::bytes(nb_total, max_sel);
     if (smem2 > cap) return BSA_ERR_UNSUPPORTED;
-    a.tiles_per_seg = (int)div_up(nb_total, kSelThreads);
+    a.tiles_per_seg = (int)div_up(nb_total, tile_rows);
     const int nseg = d->B * d->Hkv;
     a.n_items = nseg * a.tiles_per_seg;
     CUtensorMap tm;
     if (!make_rows_tmap(&tm, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                        esz, summ, cols, (int64_t)nseg * nb_total, a.row_bytes, kSelThreads))
+                        esz, summ, cols, (int64_t)nseg * nb_total, a.row_bytes, tile_rows))
         return BSA_ERR_CUDA;
-    auto launch = [&](auto kern, int tpb) -> bsa_status {
+    auto launch = [&](auto kern, int threads) -> bsa_status {
         BSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1));
-        const int threads = kSelThreads * tpb;
         int per_sm = 0;
         BSA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem1));
         const int grid = std::max(1, std::min(a.n_items, num_sms() * std::max(per_sm, 1)));
@@ -960,20 +971,20 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
     auto by_gd = [&](auto sk, auto dt) -> bsa_status {
         constexpr int SK = decltype(sk)::value, DT = decltype(dt)::value;
         if constexpr (SK != kScoreMinmaxF32 && DT > 0) {   // two rows per thread
-            switch (a.G) {
-                case 4: return launch(score_pair_kernel<SK, 4, DT>, kPairThreads / kSelThreads);
-                case 8: return launch(score_pair_kernel<SK, 8, DT>, kPairThreads / kSelThreads);
-                case 16: return launch(score_pair_kernel<SK, 16, DT>, kPairThreads / kSelThreads);
+            if (pair) switch (a.G) {
+                case 4: return launch(score_pair_kernel<SK, 4, DT>, kPairRows);
+                case 8: return launch(score_pair_kernel<SK, 8, DT>, kPairRows);
+                case 16: return launch(score_pair_kernel<SK, 16, DT>, kPairRows);
                 default: break;
             }
         }
         switch (a.G) {
-            case 1: return launch(score_kernel<SK, 1, DT>, score_tpb(1));
-            case 2: return launch(score_kernel<SK, 2, DT>, score_tpb(2));
-            case 4: return launch(score_kernel<SK, 4, DT>, score_tpb(4));
-            case 8: return launch(score_kernel<SK, 8, DT>, score_tpb(8));
-            case 16: return launch(score_kernel<SK, 16, DT>, score_tpb(16));
-            default: return launch(score_kernel<SK, 0, 0>, score_tpb(0));
+            case 1: return launch(score_kernel<SK, 1, DT>, kSelThreads * score_tpb(1));
+            case 2: return launch(score_kernel<SK, 2, DT>, kSelThreads * score_tpb(2));
+            case 4: return launch(score_kernel<SK, 4, DT>, kSelThreads * score_tpb(4));
+            case 8: return launch(score_kernel<SK, 8, DT>, kSelThreads * score_tpb(8));
+            case 16: return launch(score_kernel<SK, 16, DT>, kSelThreads * score_tpb(16));
+            default: return launch(score_kernel<SK, 0, 0>, kSelThreads * score_tpb(0));
         }
     };
     auto by_g = [&](auto sk) -> bsa_status {
