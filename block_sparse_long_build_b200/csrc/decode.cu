@@ -479,14 +479,14 @@ __device__ __forceinline__ void finish_append(const DecArgs &a, int b, int g, in
 // ======================================================================
 // Shared memory: one ring per warp, NST stages of one piece each (K then V:
 // NH boxes of 16 rows x 64 bf16 columns apiece, or for an FP8 cache one box
-// of 16 rows x 128 FP8 columns apiece), then for an FP8 cache one f16 piece
-// per warp (the bf16 layout) that each stage is converted into.
+// of 16 rows x 128 FP8 columns apiece), then for an FP8 cache one f16 V box
+// per warp (the bf16 layout) that each stage's V is widened into.
 template <int NH, int NST, bool F8 = false>
 struct TcSmem {
     static constexpr int kPieceBytes = F8 ? 2 * kBoxBytes : 2 * NH * kBoxBytes;
     static constexpr int kRing = kDecWarps * NST * kPieceBytes;
-    static constexpr int kConv = kRing;                               // FP8: f16 piece [warps]
-    static constexpr int kConvBytes = F8 ? kDecWarps * 2 * NH * kBoxBytes : 0;
+    static constexpr int kConv = kRing;                               // FP8: f16 V [warps]
+    static constexpr int kConvBytes = F8 ? kDecWarps * NH * kBoxBytes : 0;
     static constexpr int kInfo = kConv + kConvBytes;                  // int [warps][NST], 8-B slots
     static constexpr int kBars = kInfo + kDecWarps * NST * 8;         // u64  [warps][NST]
     static constexpr int kMisc = kBars + kDecWarps * NST * 8;         // float sml[2*kMaxG], int tmp[36]
@@ -523,7 +523,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // Every warp works out its own pieces: no CTA-wide barrier before the
     // first load.
     unsigned char *ring = dsm + warp * NST * L::kPieceBytes;
-    unsigned char *conv = dsm + L::kConv + warp * 2 * NH * kBoxBytes;   // FP8 only
+    unsigned char *conv = dsm + L::kConv + warp * NH * kBoxBytes;   // FP8 only: f16 V
     uint64_t *wfull = full + warp * NST;
     int2 *winfo = info + warp * NST;   // .x: valid rows of the stage's piece
     int4 *wtab = ptab + warp * kWarpCap;
@@ -609,11 +609,15 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
             float x[4];
-            const int k0 = kk * 16 + 2 * tig;
+            // logical columns 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9 of the
+            // 16-wide step; an FP8 cache pairs them with physical columns
+            // 4 tig .. 4 tig + 3 (its K fragments are four consecutive codes),
+            // the dot product being the same sum in another order of terms
+            const int k0 = kk * 16 + (F8 ? 4 * tig : 2 * tig);
             x[0] = live ? qg[k0] : 0.0f;
             x[1] = live ? qg[k0 + 1] : 0.0f;
-            x[2] = live ? qg[k0 + 8] : 0.0f;
-            x[3] = live ? qg[k0 + 9] : 0.0f;
+            x[2] = live ? qg[k0 + (F8 ? 2 : 8)] : 0.0f;
+            x[3] = live ? qg[k0 + (F8 ? 3 : 9)] : 0.0f;
             float hi[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -648,18 +652,21 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         unsigned char *kp = ring + st * L::kPieceBytes;
         unsigned char *vp = kp + NH * kBoxBytes;
         bool issued_early = false;
+        // S = Q K^T for the piece's 16 rows: two 8-row MMA tiles, even and odd
+        // k-steps in separate accumulators (shorter dependency chains)
+        float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         if constexpr (F8) {
-            // the stage's FP8 K and V boxes -> this warp's f16 piece in the
-            // bf16 layout (FP8 chunk c of a row: columns 16c .. 16c+15, i.e.
-            // f16 box c / 4, chunks 2 (c % 4) and 2 (c % 4) + 1); V rows outside
-            // [vlo, vhi) become zeros so that 0 * junk stays 0
-            const unsigned char *src = kp;
+            // V: the stage's FP8 box -> this warp's f16 box in the bf16 layout
+            // (FP8 chunk c of a row: columns 16c .. 16c+15, i.e. f16 box c / 4,
+            // chunks 2 (c % 4) and 2 (c % 4) + 1); rows outside [vlo, vhi)
+            // become zeros so that 0 * junk stays 0
+            const unsigned char *vsrc = kp + kBoxBytes;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < 4; ++k) {
                 const int u = lane + 32 * k;
-                const int kv = u >> 7, r = (u >> 3) & 15, cc = u & 7;
-                const uint4 w = *reinterpret_cast<const uint4 *>(src + kv * kBoxBytes + r * 128 +
-                                                                 ((cc ^ (r & 7)) << 4));
+                const int r = u >> 3, cc = u & 7;
+                const uint4 w = *reinterpret_cast<const uint4 *>(vsrc + r * 128 + ((cc ^ (r & 7)) << 4));
                 uint32_t h[8];
                 const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -667,15 +674,28 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                     h[2 * e] = fp8x2_to_f16x2((uint16_t)(wv[e] & 0xffffu));
                     h[2 * e + 1] = fp8x2_to_f16x2((uint16_t)(wv[e] >> 16));
                 }
-                if (kv == 1 && (r < vlo || r >= vhi))
+                if (r < vlo || r >= vhi)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) h[e] = 0u;
-                unsigned char *row = conv + (kv * NH + (cc >> 2)) * kBoxBytes + r * 128;
+                unsigned char *row = conv + (cc >> 2) * kBoxBytes + r * 128;
                 const int c0 = 2 * (cc & 3);
                 *reinterpret_cast<uint4 *>(row + ((c0 ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
                 *reinterpret_cast<uint4 *>(row + (((c0 + 1) ^ (r & 7)) << 4)) =
                     make_uint4(h[4], h[5], h[6], h[7]);
             }
+            // K fragments straight from the FP8 box: row gid (+8), four codes
+            // at columns 16 kk + 4 tig widened to two f16 pairs
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int r = gid + 8 * nt;
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(
+                        kp + r * 128 + ((kk ^ (r & 7)) << 4) + 4 * tig);
+                    const uint32_t b0 = fp8x2_to_f16x2((uint16_t)(w & 0xffffu));
+                    const uint32_t b1 = fp8x2_to_f16x2((uint16_t)(w >> 16));
+                    mma_f16_16816(kk & 1 ? sb[nt] : sa[nt], qa[kk], b0, b1);
+                }
             __syncwarp();
             // the stage has been read: its next copy can start now
             if (idx + NST < my_count) {
@@ -688,8 +708,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                 if (lane == 0) issue(idx + NST, st);
             }
             issued_early = true;
-            kp = conv;
-            vp = conv + NH * kBoxBytes;
+            vp = conv;
         } else if (vlo > 0 || vhi < kPiece) {   // rows outside the range: zero V so 0 * junk stays 0
             for (int e = lane; e < kPiece * NH * 8; e += 32) {
                 const int r = e / (NH * 8), h = (e / 8) % NH, ch = e % 8;
@@ -701,26 +720,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             __syncwarp();
         }
         const uint32_t kbase = smem_u32(kp), vbase = smem_u32(vp);
-        // S = Q K^T for the piece's 16 rows: two 8-row MMA tiles, even and odd
-        // k-steps in separate accumulators (shorter dependency chains)
-        float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < (F8 ? 0 : D / 16); ++kk) {   // bf16: K fragments by ldmatrix
             const int half = kk / 4, ch0 = (kk % 4) * 2;
             const int r = (lane >> 4) * 8 + (lane & 7);
             const int ch = ch0 + ((lane >> 3) & 1);
             uint32_t b0, b1, b2, b3;
             ldmatrix_x4(kbase + half * kBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4), b0, b1, b2, b3);
-            if constexpr (F8) {
-                if (kk & 1) {
-                    mma_f16_16816(sb[0], qa[kk], b0, b1);
-                    mma_f16_16816(sb[1], qa[kk], b2, b3);
-                } else {
-                    mma_f16_16816(sa[0], qa[kk], b0, b1);
-                    mma_f16_16816(sa[1], qa[kk], b2, b3);
-                }
-            } else if (kk & 1) {
+            if (kk & 1) {
                 mma_bf16_16816(sb[0], qa[kk], b0, b1);
                 mma_bf16_16816(sb[1], qa[kk], b2, b3);
             } else {

@@ -102,6 +102,12 @@ EDGE = {
     # G = 1 (multi-head), pages of 16
     "g1": _cfg(W.quest(0), B=2, Hkv=4, Hq=4, L=2048 + 3, budget_tokens=256, sink=16, window=64,
                refresh=1, steps=2),
+    # G = 2: one row per thread in the scoring kernel
+    "g2": _cfg(W.quest(0), B=2, Hkv=4, Hq=8, L=2048 + 3, budget_tokens=256, sink=16, window=64,
+               refresh=1, steps=2),
+    # fp32 cache with min/max page bounds (fp32 pairs, the per-row scoring kernel)
+    "minmax_f32": _cfg(W.quest(0), B=2, Hkv=2, Hq=8, kv_dtype=torch.float32, L=2048 + 5,
+                       budget_tokens=256, sink=16, window=64, refresh=2, steps=3),
 }
 
 
@@ -159,3 +165,34 @@ def test_decode_kernel_count():
     p = N.sel_params(16, topk=-1, budget_tokens=4096, sink=256, window=1024)
     assert N.bsa_decode_kernels(desc(4), p, 5400) == 1
     assert N.bsa_decode_kernels(desc(1), p, 5400) == 2
+
+
+def test_selection_g16_matches_oracle():
+    """G = 16 (the decode stops at 8 query heads per KV head; selection goes to
+    16): the paired-row scorer with eight heads per thread, selections and
+    ranges bit for bit."""
+    import oracle
+    from gpu_harness import host, record_ties, current_label
+    cfg = _cfg(W.moba(0), Hkv=2, Hq=32, L=128 * 30 + 11, block_size=128, topk=6, n_needles=4,
+               steps=1)
+    wl = W.Workload(cfg, "cuda")
+    from block_sparse_long_build_b200.session import DecodeSession
+    sess = DecodeSession(wl)
+    sess.build_summaries()
+    q = wl.decode_query(0)
+    sess.select(q)
+    torch.cuda.synchronize()
+    qh, K = host(q), host(wl.K)
+    n = cfg.L
+    sel, cnt = host(sess.sel_blocks), host(sess.sel_count)
+    ranges, nr = host(sess.ranges), host(sess.n_ranges)
+    for g in range(cfg.Hkv):
+        beg, end = oracle.fixed_block_bounds(n, cfg.block_size)
+        summ = oracle.block_summaries(K[0, g], beg, end, cfg.kind)
+        s32, s64 = oracle.block_scores(qh[0, g * cfg.G:(g + 1) * cfg.G], summ, cfg.kind)
+        want, want_r, ties = oracle.select_fixed(s32, s64, n, cfg.block_size, cfg.topk,
+                                                 cfg.budget_tokens, cfg.sink, cfg.window,
+                                                 cfg.keep_current)
+        record_ties(current_label(), ties)
+        assert sel[g, :cnt[g]].tolist() == want
+        assert [tuple(x) for x in ranges[g, :nr[g]].tolist()] == want_r
