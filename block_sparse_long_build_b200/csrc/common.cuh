@@ -181,6 +181,16 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t &r0, u
                  : "r"(addr));
 }
 
+// Two fused multiply-adds in one instruction, each rounded once:
+// c0 = a * b0 + c0, c1 = a * b1 + c1 (bit-identical to two __fmaf_rn).
+__device__ __forceinline__ void fma2_shared_a(float &c0, float &c1, float a, float b0, float b1) {
+    asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+        "mov.b64 pa, {%2, %2};\n\tmov.b64 pb, {%3, %4};\n\tmov.b64 pc, {%0, %1};\n\t"
+        "fma.rn.f32x2 pc, pa, pb, pc;\n\tmov.b64 {%0, %1}, pc;\n\t}"
+        : "+f"(c0), "+f"(c1)
+        : "f"(a), "f"(b0), "f"(b1));
+}
+
 // D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulators.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
                                                uint32_t b0, uint32_t b1) {

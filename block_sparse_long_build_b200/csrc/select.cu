@@ -291,16 +291,6 @@ __global__ void __launch_bounds__(kSelThreads * score_tpb(GT), 3)
     pdl_trigger();
 }
 
-// Two fused multiply-adds in one instruction, each rounded once:
-// c0 = a * b0 + c0, c1 = a * b1 + c1 (bit-identical to two __fmaf_rn).
-__device__ __forceinline__ void fma2_shared_a(float &c0, float &c1, float a, float b0, float b1) {
-    asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
-        "mov.b64 pa, {%2, %2};\n\tmov.b64 pb, {%3, %4};\n\tmov.b64 pc, {%0, %1};\n\t"
-        "fma.rn.f32x2 pc, pa, pb, pc;\n\tmov.b64 {%0, %1}, pc;\n\t}"
-        : "+f"(c0), "+f"(c1)
-        : "f"(a), "f"(b0), "f"(b1));
-}
-
 // Scoring with two block rows per thread, for G = 4, 8 or 16 and D = 64 or
 // 128 (min/max bf16 bounds or fp32 centroids).  A tile is R = kPairRows rows
 // and the CTA R threads; lanes 2p and 2p + 1 take rows p and p + R/2 of it, lane 2p the first G/2 heads and
