@@ -17,6 +17,8 @@ benchmark takes.
   blocks (so the merge runs over many partial slots).
 * A small Quest-shaped case with enough segments for the clustered decode
   grid, where a page completes inside a fused (clustered) step.
+* The FP8 cache at the large-batch size and the Quest configuration on a
+  page pool (sampled segments / every segment at chosen steps).
 
 Selections are compared bit for bit, outputs and log-sum-exp within max-abs
 2e-3 of the fp64 oracle.  Sampling keeps the oracle's time to seconds per
@@ -76,6 +78,29 @@ def test_largebatch_full_size():
     chk = FixedDecodeCheck(cfg, segments=segs)
     chk.run(20, check_steps={0, 1, 19})
     assert chk.compared == 3 * len(segs)
+    del chk
+    _free()
+
+
+def test_largebatch_fp8_full_size():
+    """The FP8 (E4M3) cache at the large-batch size, sampled segments."""
+    cfg = W.largebatch_fp8(0)
+    segs = [(0, 0), (5, 3), (31, 7), (63, 1)]
+    chk = FixedDecodeCheck(cfg, segments=segs)
+    chk.run(6, check_steps={0, 5})
+    assert chk.compared == 2 * len(segs)
+    del chk
+    _free()
+
+
+def test_quest_paged_full_size():
+    """The Quest-style configuration on a page pool (pages of 256 rows at
+    random slots): every segment at a refresh and at the fused steps after it."""
+    cfg = W.quest(0)
+    chk = FixedDecodeCheck(cfg, page_rows=256, spare_pages=16)
+    assert chk.sess.fuses() and chk.sess.decode_kernels == 1
+    chk.run(3, check_steps={0, 2})
+    assert chk.compared == 2 * cfg.B * cfg.Hkv
     del chk
     _free()
 
