@@ -18,9 +18,10 @@
 //      [pos_limit, q], causal) and grouped (the gathered rows of one block
 //      against its visible prefix).  Q rows are gathered into 128-byte-
 //      swizzled shared memory, K/V tiles arrive by TMA (no multicast),
-//      S = Q K^T accumulates in TMEM (tcgen05.mma, bf16 in, fp32 out), one
-//      thread per row runs the online softmax and writes P (bf16) back to
-//      TMEM, O += P V reads P from TMEM.  Each item leaves an unnormalised
+//      S = Q K^T accumulates in TMEM (tcgen05.mma, bf16 in, fp32 out), four
+//      threads per row run the online softmax and write P (fp16) back to
+//      TMEM, and O += P V reads P from TMEM with the V tile converted to
+//      fp16 in shared memory (the two operands of one product share a type).  Each item leaves an unnormalised
 //      partial (o, m, l) in its (query, KV head, slot) record.
 //   P4 prefill_merge_kernel   log-sum-exp merge of a query's slots (local
 //      first, then blocks in index order).
@@ -259,7 +260,9 @@ __global__ void __launch_bounds__(1024) prefill_tiles_kernel(PfArgs a) {
 // ---------------------------------------------------------------- P3
 // Warp-specialised and pipelined across work items:
 //   warps 0-15  softmax + epilogue, four threads per row (warp w owns TMEM
-//               lanes 32 (w % 4).. and the column quarter w / 4)
+//               lanes 32 (w % 4).. and the column quarter w / 4); each warp
+//               also converts its 2 KiB slice of every V tile to fp16 while
+//               the tile's S is computed
 //   warp 16     lane 0 issues every tcgen05.mma
 //   warp 17     lane 0 streams the K tiles, lane 1 the V tiles by TMA (no
 //               multicast); the two lanes wait on different barriers
@@ -277,9 +280,11 @@ __global__ void __launch_bounds__(1024) prefill_tiles_kernel(PfArgs a) {
 //   qready[m] item n (m = n & 3) described, Q gathered (32) parity (n >> 2) & 1
 //   qfree[b]  item n's last S complete (b = n & 1)          parity (n >> 1) & 1
 //   efree[b]  item n's epilogue done, 16 softmax warps      parity (n >> 1) & 1
-//   kfull/vfull[s] tile u (s = u & 1), TMA bytes           parity (u >> 1) & 1
+//   kfull/vfull[s] tile u (s = u & 1), TMA bytes (vfull also awaited by the
+//             softmax warps, which convert V)         parity (u >> 1) & 1
 //   kfree/vfree[s] S(u) / P.V(u) complete (tcgen05.commit) parity (u >> 1) & 1
-//   sfull[s]  S(u) complete; pfull[s] P(u) in TMEM (16 warps); odone[s] P.V(u)
+//   sfull[s]  S(u) complete; pfull[s] P(u) in TMEM and V(u) in fp16 (16
+//             warps); odone[s] P.V(u) complete
 constexpr int kPfSoftWarps = 16;
 constexpr int kPfMmaWarp = 16, kPfLoadWarp = 17, kPfProdWarp = 18;
 constexpr int kPfAttThreads = 32 * 20;
@@ -312,6 +317,67 @@ __device__ __forceinline__ float ex2_ftz(float x) {
 
 __device__ __forceinline__ void quad_sync(int q) {   // the four warps holding rows 32q..32q+31
     asm volatile("bar.sync %0, 128;" ::"r"(1 + q) : "memory");
+}
+// the same barrier, returning whether any of the 128 threads passed true
+__device__ __forceinline__ bool quad_any(int q, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.or.pred po, %2, 128, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(1 + q)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ float fmax3(float x, float y, float z) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(x), "f"(y), "f"(z));
+    return d;
+}
+// largest of 32 values, as a tree of depth four
+__device__ __forceinline__ float max32(const uint32_t (&v)[32]) {
+    float m[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i)
+        m[i] = fmax3(__uint_as_float(v[3 * i]), __uint_as_float(v[3 * i + 1]), __uint_as_float(v[3 * i + 2]));
+    m[10] = fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31]));
+    return fmaxf(fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmax3(m[6], m[7], m[8])),
+                 fmaxf(m[9], m[10]));
+}
+
+// This warp's 2 KiB slice of a 32 KiB V stage, bf16 to fp16 in place (the
+// 128-byte swizzle moves whole 16-byte chunks, so the layout is unchanged).
+// Magnitudes beyond the fp16 range saturate to +-65504.
+__device__ __forceinline__ void v_to_f16(unsigned char *stage, int warp, int lane) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint4 *p = reinterpret_cast<uint4 *>(stage + warp * 2048 + (lane + 32 * i) * 16);
+        uint4 x = *p;
+        uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xffff0000u);
+            asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(w[j]) : "f"(hi), "f"(lo));
+        }
+        *p = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// Pairs of fp32 operations in one instruction each: ffma2 gives
+// (x0 y0 + z0, x1 y1 + z1); fadd2 adds (x0, x1) into (d0, d1).
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float x0, float x1, float y0, float y1, float z0,
+                                      float z1) {
+    asm("{\n\t.reg .b64 px, py, pz;\n\tmov.b64 px, {%2, %3};\n\tmov.b64 py, {%4, %5};\n\t"
+        "mov.b64 pz, {%6, %7};\n\tfma.rn.f32x2 pz, px, py, pz;\n\tmov.b64 {%0, %1}, pz;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(x0), "f"(x1), "f"(y0), "f"(y1), "f"(z0), "f"(z1));
+}
+__device__ __forceinline__ void fadd2(float &d0, float &d1, float x0, float x1) {
+    asm("{\n\t.reg .b64 px, pd;\n\tmov.b64 px, {%2, %3};\n\tmov.b64 pd, {%0, %1};\n\t"
+        "add.rn.f32x2 pd, pd, px;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(x0), "f"(x1));
 }
 
 __global__ void __launch_bounds__(kPfAttThreads, 1)
@@ -523,7 +589,7 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
         // ================= tcgen05.mma issue (one lane)
         if (lane == 0) {
             constexpr uint32_t kIdescQK = umma_idesc_bf16(128, 128, 0, 0);
-            constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 128, 0, 1);
+            constexpr uint32_t kIdescPV = umma_idesc_f16(128, 128, 0, 1);   // P and V in fp16
             int pend_u = -1, pend_n = 0;
             bool pend_first = false;
             auto pv = [&](int v, int pn, bool first) {   // O[pn & 1] (+)= P(v) V(v)
@@ -538,7 +604,6 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                 for (int k = 0; k < 8; ++k) {
                     const uint64_t vd = umma_sdesc_sw128(v0 + k * 2048, 16384, 1024);
                     umma_ts(tO, tP + k * 8, vd, kIdescPV, (!first || k > 0) ? 1u : 0u);
-                    umma_ts(tO, tP + 64 + k * 8, vd, kIdescPV, 1u);
                 }
                 umma_commit(&odone[st]);
                 umma_commit(&vfree[st]);
@@ -633,6 +698,11 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
             float m_used = kPfNegInf, l_part = 0.0f;
             for (int t = 0; t < T; ++t, ++u) {
                 const int st = u & 1;
+                // V(u) to fp16, while S(u) is computed; P(u)'s arrival below
+                // also tells the MMA lane that this warp's slice is converted
+                wait(&vfull[st], (u >> 1) & 1);
+                v_to_f16(sm + PfSmem::kV + st * 32768, warp, lane);
+                fence_proxy_async_smem();
                 wait(&sfull[st], (u >> 1) & 1);
                 tc_fence_after();
                 const uint32_t tS = tmem + st * 128;
@@ -642,76 +712,79 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                 // maxima on the raw logits (the scale is positive); masked
                 // keys become -inf
                 const int key0 = kbeg + t * kTile + cq * 32;
-                float mx = kPfNegInf;
-                if (key0 + 31 < kend && key0 + 31 <= my_pos) {   // every key of the quarter visible
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
-                } else {
+                if (!(key0 + 31 < kend && key0 + 31 <= my_pos)) {   // some key of the quarter hidden
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int kr = key0 + e;
                         if (!(kr < kend && kr <= my_pos)) sv[e] = __float_as_uint(kPfNegInf);
-                        mx = fmaxf(mx, __uint_as_float(sv[e]));
                     }
                 }
-                // one barrier: the quarters exchange maxima through the tile
-                // parity's buffer, and every quarter has read S(u) before any
-                // writes P into it
-                float *pm = pairv + (st * 4) * kTile;
-                pm[cq * kTile + r] = mx;
-                quad_sync(q);
-                const float m_tile = fmaxf(fmaxf(pm[r], pm[kTile + r]), fmaxf(pm[2 * kTile + r], pm[3 * kTile + r])) *
-                                     a.scale_log2;
-                // lazy rescale: keep the reference maximum unless this tile
-                // exceeds it by more than 2^8
-                bool rescale = false;
-                float factor = 1.0f, m_ref = m_used;
-                if (m_tile != kPfNegInf) {
-                    if (m_used == kPfNegInf) {
-                        m_ref = m_tile;   // nothing accumulated yet for this row
-                    } else if (m_tile > m_used + kPfRescale) {
-                        rescale = true;
-                        factor = exp2f(m_used - m_tile);
-                        m_ref = m_tile;
+                const float qmax = max32(sv);
+                // Lazy rescale: a row keeps its reference maximum unless this
+                // tile exceeds it by more than 2^8 (or it has none yet and the
+                // tile has a visible key).  The tile's row maximum is over all
+                // four quarters, and it exceeds a bound exactly when one
+                // quarter's does, so the quarters first agree, in one barrier,
+                // on whether any row must move; only then are maxima exchanged.
+                // The barrier also orders every quarter's read of S(u) before
+                // any quarter writes P into it.
+                const float qm = qmax * a.scale_log2;
+                const bool need = qm != kPfNegInf && (m_used == kPfNegInf || qm > m_used + kPfRescale);
+                float factor = 1.0f;
+                if (quad_any(q, need)) {
+                    float *pm = pairv + (st * 4) * kTile;
+                    pm[cq * kTile + r] = qmax;
+                    quad_sync(q);
+                    const float m_tile =
+                        fmaxf(fmaxf(pm[r], pm[kTile + r]), fmaxf(pm[2 * kTile + r], pm[3 * kTile + r])) * a.scale_log2;
+                    bool rescale = false;
+                    float m_ref = m_used;
+                    if (m_tile != kPfNegInf) {
+                        if (m_used == kPfNegInf) {
+                            m_ref = m_tile;   // nothing accumulated yet for this row
+                        } else if (m_tile > m_used + kPfRescale) {
+                            rescale = true;
+                            factor = exp2f(m_used - m_tile);
+                            m_ref = m_tile;
+                        }
                     }
-                }
-                if (t > 0 && __any_sync(0xffffffffu, rescale)) {
-                    // O must hold P.V(u-1) before it is scaled
-                    wait(&odone[(u - 1) & 1], ((u - 1) >> 1) & 1);
-                    tc_fence_after();
-                    uint32_t ov[32];
-                    tmem_ld32(tO + lane_base + cq * 32, ov);
-                    tmem_ld_wait();
+                    if (t > 0 && __any_sync(0xffffffffu, rescale)) {
+                        // O must hold P.V(u-1) before it is scaled
+                        wait(&odone[(u - 1) & 1], ((u - 1) >> 1) & 1);
+                        tc_fence_after();
+                        uint32_t ov[32];
+                        tmem_ld32(tO + lane_base + cq * 32, ov);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
-                    tmem_st32(tO + lane_base + cq * 32, ov);
+                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+                        tmem_st32(tO + lane_base + cq * 32, ov);
+                    }
+                    m_used = m_ref;
                 }
                 l_part *= factor;
-                m_used = m_ref;
-                // P = P_hi + P_lo over this quarter's 32 keys: P_hi in the
-                // tile's S columns 16 cq.., P_lo in 64 + 16 cq..  P_hi is p cut
-                // to bf16 (its top 16 bits), P_lo = p - P_hi (exact in fp32) cut
-                // the same way, so P_hi + P_lo matches p to 2^-15 relative;
-                // the pairs are packed with byte permutes.
-                float lsum = 0.0f;
-                uint32_t ph[16], pl[16];
-                const float neg_m = -m_used;
+                // P in fp16 over this quarter's 32 keys, written to the tile's S
+                // columns 16 cq..  (two keys a column).  The row sum l adds the
+                // rounded weights, so O / l is a weighted mean of V with weights
+                // that sum to one: each fp16 half is read back exactly as its
+                // bits shifted into an fp32 2^-112 times its value, and the sum
+                // is scaled by 2^112 at the end.  A row with no visible key so
+                // far has only -inf logits, which give 0 with any finite offset.
+                float ls0 = 0.0f, ls1 = 0.0f;
+                uint32_t ph[16];
+                const float neg_m = m_used == kPfNegInf ? 0.0f : -m_used;
+                const float sc = a.scale_log2;
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const float x0 = __fmaf_rn(__uint_as_float(sv[e]), a.scale_log2, neg_m);
-                    const float x1 = __fmaf_rn(__uint_as_float(sv[e + 1]), a.scale_log2, neg_m);
-                    const float p0 = m_used == kPfNegInf ? 0.0f : ex2_ftz(x0);
-                    const float p1 = m_used == kPfNegInf ? 0.0f : ex2_ftz(x1);
-                    lsum += p0 + p1;
-                    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-                    const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);
-                    const float r1 = p1 - __uint_as_float(b1 & 0xffff0000u);
-                    ph[e / 2] = __byte_perm(b0, b1, 0x7632);
-                    pl[e / 2] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+                    float x0, x1;
+                    ffma2(x0, x1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), sc, sc, neg_m, neg_m);
+                    const float p0 = ex2_ftz(x0), p1 = ex2_ftz(x1);
+                    uint32_t w;
+                    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(p1), "f"(p0));
+                    ph[e / 2] = w;
+                    fadd2(ls0, ls1, __uint_as_float((w & 0xffffu) << 13), __uint_as_float((w >> 16) << 13));
                 }
                 tmem_st16(tS + lane_base + cq * 16, ph);
-                tmem_st16(tS + lane_base + 64 + cq * 16, pl);
-                l_part += lsum;
+                l_part += (ls0 + ls1) * 0x1p112f;
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();

@@ -15,11 +15,18 @@ def pytest_configure(config):
 
 def pytest_terminal_summary(terminalreporter, exitstatus, config):
     """Near-ties across the selection cut (fp64 scores within 1e-6 relative),
-    per test that compared selections with the oracle."""
+    per test that compared selections with the oracle, and the largest
+    |GPU - oracle| of each test that compared outputs."""
     h = sys.modules.get("gpu_harness")
-    if h is None or not h.NEAR_TIES:
+    if h is None:
         return
     tr = terminalreporter
+    if h.MAX_ERR:
+        tr.section("largest |GPU - oracle| over outputs and log-sum-exp (bar 2e-3)")
+        for label, e in sorted(h.MAX_ERR.items()):
+            tr.write_line(f"{label}: {e:.2e}")
+    if not h.NEAR_TIES:
+        return
     tr.section("near-ties at the selection cut (fp64, 1e-6 relative)")
     tot = [0, 0, 0]
     for label, (n, with_ties, pairs) in sorted(h.NEAR_TIES.items()):

@@ -26,6 +26,12 @@ ATOL = 2e-3
 
 # test label -> [selections compared, selections with a near-tie, near-tie pairs]
 NEAR_TIES: dict[str, list[int]] = {}
+# largest |GPU - oracle| over outputs and log-sum-exp, per test
+MAX_ERR: dict[str, float] = {}
+
+
+def record_err(label: str, *errs) -> None:
+    MAX_ERR[label] = max([MAX_ERR.get(label, 0.0)] + [float(e) for e in errs])
 
 
 def record_ties(label: str, ties) -> None:
@@ -189,6 +195,7 @@ class FixedDecodeCheck:
             err = np.abs(out[b, g * c.G:(g + 1) * c.G] - ref["out"]).max()
             lerr = np.abs(lse[b, g * c.G:(g + 1) * c.G] - ref["lse"]).max()
             worst = max(worst, float(err), float(lerr))
+            record_err(current_label(), err, lerr)
             assert err <= ATOL, f"segment {s}: max |out - oracle| = {err:.3e}"
             assert lerr <= ATOL, f"segment {s}: max |lse - oracle| = {lerr:.3e}"
             self.compared += 1

@@ -36,7 +36,7 @@ from block_sparse_long_build_b200 import workloads as W
 from block_sparse_long_build_b200.session import DecodeSession
 
 from gpu_harness import (ATOL, FixedDecodeCheck, assert_status_clean, current_label, host,
-                         record_ties)
+                         record_err, record_ties)
 
 pytestmark = pytest.mark.gpu
 
@@ -174,6 +174,7 @@ def test_semantic_decode_full_size(semantic_full):
             ref, ref_lse = oracle.attend(qg, Kp[0, g], Vp[0, g], rows, 1 / math.sqrt(cfg.D))
             err = np.abs(out[0, g * cfg.G:(g + 1) * cfg.G] - ref).max()
             lerr = np.abs(lse[0, g * cfg.G:(g + 1) * cfg.G] - ref_lse).max()
+            record_err(current_label(), err, lerr)
             assert err <= ATOL, f"step {t} head {g}: max |out - oracle| = {err:.3e}"
             assert lerr <= ATOL, f"step {t} head {g}: max |lse - oracle| = {lerr:.3e}"
     # put the cache length back for the prefill tests sharing the fixture
@@ -222,6 +223,7 @@ def _check_prefill(cfg, wl, sess, Kpos, Vpos, labels, orders, cents, p, Tq, head
             ref, ref_lse = oracle.attend(qg, Kpos[0, g], Vpos[0, g], rws, 1 / math.sqrt(cfg.D))
             err = np.abs(out_h[i, g * cfg.G:(g + 1) * cfg.G] - ref).max()
             lerr = np.abs(lse_h[i, g * cfg.G:(g + 1) * cfg.G] - ref_lse).max()
+            record_err(current_label(), err, lerr)
             assert err <= ATOL, f"chunk {p} row {i} head {g}: max |out - oracle| = {err:.3e}"
             assert lerr <= ATOL, f"chunk {p} row {i} head {g}: max |lse - oracle| = {lerr:.3e}"
     return most

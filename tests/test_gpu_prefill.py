@@ -16,7 +16,7 @@ import oracle
 from block_sparse_long_build_b200 import workloads as W
 from block_sparse_long_build_b200.session import DecodeSession
 
-from gpu_harness import ATOL, current_label, host, record_ties
+from gpu_harness import ATOL, current_label, host, record_err, record_ties
 
 pytestmark = pytest.mark.gpu
 
@@ -66,6 +66,7 @@ def _check_chunk(cfg, wl, sess, p, Tq, rows):
             err = np.abs(out_h[i, g * cfg.G:(g + 1) * cfg.G] - ref).max()
             lerr = np.abs(lse_h[i, g * cfg.G:(g + 1) * cfg.G] - ref_lse).max()
             worst = max(worst, float(err), float(lerr))
+            record_err(current_label(), err, lerr)
             assert err <= ATOL, f"chunk {p} row {i} head {g}: max |out - oracle| = {err:.3e}"
             assert lerr <= ATOL, f"chunk {p} row {i} head {g}: max |lse - oracle| = {lerr:.3e}"
     return worst

@@ -15,7 +15,7 @@ import oracle
 from block_sparse_long_build_b200 import workloads as W
 from block_sparse_long_build_b200.session import DecodeSession
 
-from gpu_harness import ATOL, assert_status_clean, current_label, host, record_ties
+from gpu_harness import ATOL, assert_status_clean, current_label, host, record_err, record_ties
 
 pytestmark = pytest.mark.gpu
 
@@ -62,4 +62,5 @@ def test_semantic_decode_matches_oracle(cfg):
             rows = np.concatenate([pos, np.arange(L - loc, L + t + 1)])
             ref, _ = oracle.attend(qg, Kpos[0, g], Vpos[0, g], rows, 1 / math.sqrt(cfg.D))
             err = np.abs(out[0, g * cfg.G:(g + 1) * cfg.G] - ref).max()
+            record_err(current_label(), err)
             assert err <= ATOL, f"step {t} head {g}: max |out - oracle| = {err:.3e}"
