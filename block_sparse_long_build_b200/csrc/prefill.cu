@@ -263,46 +263,60 @@ __global__ void __launch_bounds__(1024) prefill_tiles_kernel(PfArgs a) {
 //               lanes 32 (w % 4).. and the column quarter w / 4); each warp
 //               also converts its 2 KiB slice of every V tile to fp16 while
 //               the tile's S is computed
-//   warp 16     lane 0 issues every tcgen05.mma
-//   warp 17     lane 0 streams the K tiles, lane 1 the V tiles by TMA (no
+//   warp 16     lane 0 streams the K tiles, lane 1 the V tiles by TMA (no
 //               multicast); the two lanes wait on different barriers
-//   warps 18-19 describe work items, gather their Q rows into one of two Q
-//               buffers and publish the item (rows, positions, records)
-// S is double-buffered in TMEM by a running tile counter u that crosses
-// items, O and the Q buffer by item parity, the item descriptions four deep.
-// A Q buffer is refilled as soon as its item's last S = QK^T is done, an O
-// buffer once its item's epilogue has read it, so the producers run up to
-// two items ahead and each epilogue overlaps the next item.  O is rescaled only
-// when a row's running maximum grows by more than 2^8 (the exponentials then
-// stay below 256).
+//   warp 17     lane 0 issues every tcgen05.mma
+//   warps 18-19 describe work items (alternately, each one ahead), gather
+//               their Q rows into the Q buffer and publish them (rows,
+//               positions, records)
+// TMEM: S double-buffered by a running tile counter u that crosses items
+// (columns 0..127, 128..255), O (256..383), and Q double-buffered by item
+// parity (384..447, 448..511).  The MMA lane copies an item's Q rows from
+// shared memory into TMEM once (tcgen05.cp), so S = Q K^T reads only K from
+// shared memory, whose bandwidth the products otherwise saturate.  The one
+// shared-memory Q buffer is refilled as soon as it is copied, V has three
+// stages so that its loads start a tile earlier, and the item descriptions
+// run up to four deep.  An item's epilogue reads O out right after the
+// softmax of the next item's first tile, before that tile's P.V overwrites
+// it.  O is
+// rescaled only when a row's running maximum grows by more than 2^8 (the
+// exponentials then stay below 256).
 //
 // Barriers and their phases (every waiter derives the parity from an index):
 //   qready[m] item n (m = n & 3) described, Q gathered (32) parity (n >> 2) & 1
-//   qfree[b]  item n's last S complete (b = n & 1)          parity (n >> 1) & 1
-//   efree[b]  item n's epilogue done, 16 softmax warps      parity (n >> 1) & 1
-//   kfull/vfull[s] tile u (s = u & 1), TMA bytes (vfull also awaited by the
-//             softmax warps, which convert V)         parity (u >> 1) & 1
-//   kfree/vfree[s] S(u) / P.V(u) complete (tcgen05.commit) parity (u >> 1) & 1
+//   qfree[b]  item n's Q copied to TMEM (b = n & 1)         parity (n >> 1) & 1
+//   qtfree[b] item n's last S complete: TMEM Q[b] free      parity (n >> 1) & 1
+//   efree[b]  item n's O read out (16 warps)                parity (n >> 1) & 1
+//   slotfree[m] item n's rows read (16 warps)               parity (n >> 2) & 1
+//   kfull[s]  K(u) landed (s = u & 1)                       parity (u >> 1) & 1
+//   vfull[s]  V(u) landed (s = u % 3; also awaited by the softmax warps,
+//             which convert it)                           parity (u / 3) & 1
+//   kfree[s]  S(u) complete (tcgen05.commit)                parity (u >> 1) & 1
+//   vfree[s]  P.V(u) complete (s = u % 3)                   parity (u / 3) & 1
 //   sfull[s]  S(u) complete; pfull[s] P(u) in TMEM and V(u) in fp16 (16
 //             warps); odone[s] P.V(u) complete
 constexpr int kPfSoftWarps = 16;
-constexpr int kPfMmaWarp = 16, kPfLoadWarp = 17, kPfProdWarp = 18;
+constexpr int kPfLoadWarp = 16, kPfMmaWarp = 17, kPfProdWarp = 18;
+constexpr int kPfVStages = 3;
 constexpr int kPfAttThreads = 32 * 20;
+// warps 0-15 softmax, 16 loads, 17 MMA, 18-19 producers
+static_assert(kPfSoftWarps == 16 && kPfProdWarp + 2 == kPfAttThreads / 32, "warp roles");
 constexpr float kPfRescale = 8.0f;   // log2 of the largest exponential kept without rescaling
 constexpr int kPfPrefixCap = 4097;   // tile prefix entries staged in shared memory
 
 struct PfSmem {
-    static constexpr int kQ = 0;                          // 2 items x 2 boxes x 16 KiB
-    static constexpr int kK = 65536;                      // 2 stages x 32 KiB
-    static constexpr int kV = kK + 65536;                 // 2 stages x 32 KiB
-    static constexpr int kRowPos = kV + 65536;            // int [4][128] query position
+    static constexpr int kQ = 0;                          // 2 boxes x 16 KiB
+    static constexpr int kK = 32768;                      // 2 stages x 32 KiB
+    static constexpr int kV = kK + 65536;                 // 3 stages x 32 KiB
+    static constexpr int kRowPos = kV + kPfVStages * 32768;   // int [4][128] query position
     static constexpr int kRowQ = kRowPos + 4 * kTile * 4; // int [4][128] row of Q (-1: none)
     static constexpr int kRowRec = kRowQ + 4 * kTile * 4; // int [4][128] partial record (-1: none)
     static constexpr int kDesc = kRowRec + 4 * kTile * 4; // int [4][8]: g, kbeg, kend, T, local, end
     static constexpr int kPair = kDesc + 4 * 8 * 4;       // float [3][4][128]: quarter-row maxima (by
                                                           // tile parity), quarter-row sums
-    static constexpr int kBars = kPair + 3 * 4 * kTile * 4;   // u64 [23]
-    static constexpr int kMisc = kBars + 23 * 8;          // tmem base
+    static constexpr int kBars = kPair + 3 * 4 * kTile * 4;   // u64 [31]
+    static_assert(kBars % 8 == 0, "barrier alignment");
+    static constexpr int kMisc = kBars + 31 * 8;          // tmem base
     static constexpr int kPrefix = kMisc + 32;            // int [kPfPrefixCap]
     static constexpr int kBytes = kPrefix + kPfPrefixCap * 4 + 1024;
 };
@@ -394,8 +408,8 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
     float *pairv = reinterpret_cast<float *>(sm + PfSmem::kPair);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PfSmem::kBars);
     uint64_t *qready = bars, *qfree = bars + 4, *efree = bars + 6, *kfull = bars + 8, *vfull = bars + 10,
-             *kfree = bars + 12, *vfree = bars + 14, *sfull = bars + 16, *pfull = bars + 18, *odone = bars + 20,
-             *drain = bars + 22;
+             *kfree = bars + 13, *vfree = bars + 15, *sfull = bars + 18, *pfull = bars + 20, *odone = bars + 22,
+             *drain = bars + 24, *qtfree = bars + 25, *slotfree = bars + 27;
     uint32_t *tmem_sh = reinterpret_cast<uint32_t *>(sm + PfSmem::kMisc);
     int *prefix_s = reinterpret_cast<int *>(sm + PfSmem::kPrefix);
 
@@ -408,17 +422,23 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
     }
     if (tid == 0) {
         prefetch_tmap(&tmKp); prefetch_tmap(&tmVp); prefetch_tmap(&tmKl); prefetch_tmap(&tmVl);
-        for (int i = 0; i < 4; ++i) mbar_init(&qready[i], 32);   // one producer warp per item
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&qready[i], 32);   // the producer warp
+            mbar_init(&slotfree[i], kPfSoftWarps);
+        }
+        for (int i = 0; i < kPfVStages; ++i) {
+            mbar_init(&vfull[i], 1);
+            mbar_init(&vfree[i], 1);
+        }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&qfree[i], 1);
             mbar_init(&efree[i], kPfSoftWarps);
             mbar_init(&kfull[i], 1);
-            mbar_init(&vfull[i], 1);
             mbar_init(&kfree[i], 1);
-            mbar_init(&vfree[i], 1);
             mbar_init(&sfull[i], 1);
             mbar_init(&pfull[i], kPfSoftWarps);
             mbar_init(&odone[i], 1);
+            mbar_init(&qtfree[i], 1);
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -442,13 +462,13 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
         if (!timed_out && !mbar_wait_bounded(bar, parity)) timed_out = true;
     };
 
-    if (warp >= kPfProdWarp) {
+    if (warp == kPfProdWarp || warp == kPfProdWarp + 1) {
         // ================= producers.  The CTA's n-th item is blockIdx.x +
-        // n gridDim.x; warp kPfProdWarp + p takes the items with n = p (mod 2),
-        // i.e. Q buffer p.  A warp describes its next item (rows, positions,
-        // records: two rounds of dependent loads) as soon as it has published
-        // the current one, so only the Q copies sit between a free buffer and
-        // the next item.
+        // n gridDim.x; warp kPfProdWarp + p takes the items with n = p (mod 2).
+        // A warp describes its next item (rows, positions, records: two
+        // rounds of dependent loads) as soon as it has published the current
+        // one, so only the Q copies sit between the free Q buffer and the next
+        // item.
         const int pt = lane;
         // item n's description into slot n & 3; false for the end marker
         auto describe = [&](int n) -> bool {
@@ -517,7 +537,7 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
         // asynchronous 16-byte copies (a row with no query is zero-filled)
         auto gather = [&](int n) {
             const int m = n & 3;
-            unsigned char *Qs = sm + PfSmem::kQ + (n & 1) * 32768;
+            unsigned char *Qs = sm + PfSmem::kQ;
 #pragma unroll 4
             for (int c = pt; c < kTile * 16; c += 32) {
                 const int r = c >> 4, ch = c & 15, half = ch >> 3, cc = ch & 7;
@@ -533,22 +553,26 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
         int n = warp - kPfProdWarp;
         bool valid = describe(n);
         for (;;) {
-            const int b = n & 1, m = n & 3;
+            const int m = n & 3;
             if (!valid) {   // end marker: nothing to gather
                 mbar_arrive(&qready[m]);
                 break;
             }
-            if (n >= 2) wait(&qfree[b], ((n - 2) >> 1) & 1);   // item n-2's Q buffer is free
+            // item n-1 (the other warp's) has been copied out of the buffer;
+            // one barrier per item parity, so that this wait is never two
+            // phases behind
+            if (n >= 1) wait(&qfree[(n - 1) & 1], ((n - 1) >> 1) & 1);
             if (timed_out) break;
             gather(n);
             asm volatile("cp.async.wait_group 0;" ::: "memory");
             fence_proxy_async_smem();
             __syncwarp();
             mbar_arrive(&qready[m]);
-            // the next item's rows go to slot (n + 2) & 3 once item n-2's
-            // epilogue has read them; its dependent loads then overlap the
+            // this warp's next item goes to slot (n + 2) & 3 once item n-2's
+            // epilogue has read it; its dependent loads then overlap the
             // consumption of items n-1 and n
-            if (n >= 2) wait(&efree[b], ((n - 2) >> 1) & 1);
+            if (n >= 2) wait(&slotfree[(n + 2) & 3], ((n - 2) >> 2) & 1);
+            if (timed_out) break;
             valid = describe(n + 2);
             n += 2;
         }
@@ -557,6 +581,7 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
         // ================= K loader (lane 0) and V loader (lane 1)
         if (lane < 2) {
             const bool isk = lane == 0;
+            const int nst = isk ? 2 : kPfVStages;   // stages: tile u in stage u % nst
             uint64_t *full = isk ? kfull : vfull, *freeb = isk ? kfree : vfree;
             unsigned char *base = sm + (isk ? PfSmem::kK : PfSmem::kV);
             int u = 0;
@@ -570,8 +595,8 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                 const int kbeg = desc[1] - (desc[4] ? a.pos_base : 0);
                 const CUtensorMap *map = desc[4] ? (isk ? &tmKl : &tmVl) : (isk ? &tmKp : &tmVp);
                 for (int t = 0; t < T; ++t, ++u) {
-                    const int st = u & 1;
-                    if (u >= 2) wait(&freeb[st], ((u - 2) >> 1) & 1);
+                    const int st = u % nst;
+                    if (u >= nst) wait(&freeb[st], ((u - nst) / nst) & 1);
                     unsigned char *dst = base + st * 32768;
                     mbar_arrive_expect_tx(&full[st], 32768);
                     tma_load_4d(dst, map, &full[st], 0, kbeg + t * kTile, g, 0);
@@ -581,7 +606,7 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
             // the last loads of each stage have landed before the CTA can exit
             const bool to = timed_out;
             timed_out = false;
-            for (int v = max(0, u - 2); v < u; ++v) wait(&full[v & 1], (v >> 1) & 1);
+            for (int v = max(0, u - nst); v < u; ++v) wait(&full[v % nst], (v / nst) & 1);
             timed_out = timed_out || to;
         }
         __syncwarp();
@@ -592,21 +617,22 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
             constexpr uint32_t kIdescPV = umma_idesc_f16(128, 128, 0, 1);   // P and V in fp16
             int pend_u = -1, pend_n = 0;
             bool pend_first = false;
-            auto pv = [&](int v, int pn, bool first) {   // O[pn & 1] (+)= P(v) V(v)
-                const int st = v & 1, b = pn & 1;
-                if (first && pn >= 2) wait(&efree[b], ((pn - 2) >> 1) & 1);   // O[b] read out
-                wait(&pfull[st], (v >> 1) & 1);
-                wait(&vfull[st], (v >> 1) & 1);
+            auto pv = [&](int v, int pn, bool first) {   // O (+)= P(v) V(v)
+                const int st = v & 1;
+                // O has been read out by the previous item's epilogue
+                if (first && pn >= 1) wait(&efree[(pn - 1) & 1], ((pn - 1) >> 1) & 1);
+                wait(&pfull[st], (v >> 1) & 1);   // also: every warp's slice of V(v) in fp16
+                const int vs = v % kPfVStages;
                 tc_fence_after();
-                const uint32_t v0 = smem_u32(sm + PfSmem::kV + st * 32768);
-                const uint32_t tP = tmem + st * 128, tO = tmem + 256 + b * 128;
+                const uint32_t v0 = smem_u32(sm + PfSmem::kV + vs * 32768);
+                const uint32_t tP = tmem + st * 128, tO = tmem + 256;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint64_t vd = umma_sdesc_sw128(v0 + k * 2048, 16384, 1024);
                     umma_ts(tO, tP + k * 8, vd, kIdescPV, (!first || k > 0) ? 1u : 0u);
                 }
                 umma_commit(&odone[st]);
-                umma_commit(&vfree[st]);
+                umma_commit(&vfree[vs]);
             };
             int u = 0;
             for (int n = 0;; ++n) {
@@ -615,7 +641,17 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                 const int *desc = desc_s + m * 8;
                 if (timed_out || desc[5]) break;
                 const int T = desc[3];
-                const uint32_t q0 = smem_u32(sm + PfSmem::kQ + b * 32768);
+                // the item's Q rows from shared memory into TMEM buffer b, once
+                // the S products of its previous user (item n - 2) are done;
+                // tcgen05.cp and the products that read it run in issue order
+                if (n >= 2) wait(&qtfree[b], ((n - 2) >> 1) & 1);
+                tc_fence_after();
+                const uint32_t q0 = smem_u32(sm + PfSmem::kQ);
+                const uint32_t tQ = tmem + 384 + b * 64;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    tmem_cp_128x256b(tQ + k * 8, umma_sdesc_sw128(q0 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024));
+                umma_commit(&qfree[b]);   // the shared-memory Q buffer is copied
                 for (int t = 0; t < T; ++t, ++u) {
                     const int st = u & 1;
                     wait(&kfull[st], (u >> 1) & 1);
@@ -623,15 +659,14 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                     tc_fence_after();
                     const uint32_t k0 = smem_u32(sm + PfSmem::kK + st * 32768);
                     const uint32_t tS = tmem + st * 128;
+                    const uint64_t kd = umma_sdesc_sw128(k0, 16, 1024);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                        umma_ss(tS, umma_sdesc_sw128(q0 + off, 16, 1024), umma_sdesc_sw128(k0 + off, 16, 1024),
-                                kIdescQK, k > 0);
-                    }
+                    for (int k = 0; k < 8; ++k)
+                        umma_ts(tS, tQ + k * 8, kd + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4), kIdescQK,
+                                k > 0);
                     umma_commit(&sfull[st]);
                     umma_commit(&kfree[st]);
-                    if (t == T - 1) umma_commit(&qfree[b]);   // the item's Q buffer is read
+                    if (t == T - 1) umma_commit(&qtfree[b]);   // TMEM Q buffer b is read
                     if (pend_u >= 0) pv(pend_u, pend_n, pend_first);
                     pend_u = u;
                     pend_n = n;
@@ -647,7 +682,7 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
             timed_out = timed_out || to;
         }
         __syncwarp();
-    } else {
+    } else if (warp < kPfSoftWarps) {
         // ================= softmax warps
         const int q = warp & 3, cq = warp >> 2;      // row quarter (TMEM lanes), key quarter
         const int r = q * 32 + lane;                 // this thread's row
@@ -670,8 +705,15 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
             const int rec = rowrec_s[pend_m4 * kTile + r];
             float *po = rec >= 0 ? a.part_o + (int64_t)rec * D + cq * 32 : nullptr;
             uint32_t ov[32];
-            tmem_ld32(tmem + 256 + pend_b * 128 + lane_base + cq * 32, ov);
+            tmem_ld32(tmem + 256 + lane_base + cq * 32, ov);
             tmem_ld_wait();
+            // O and the item's shared-memory rows may be reused
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&efree[pend_b]);
+                mbar_arrive(&slotfree[pend_m4]);
+            }
             if (po) {
 #pragma unroll
                 for (int e = 0; e < 32; e += 4)
@@ -680,28 +722,25 @@ __global__ void __launch_bounds__(kPfAttThreads, 1)
                                     __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
             }
             if (rec >= 0 && cq == 0) a.part_ml[rec] = make_float2(pend_m, l_row);
-            // O[pend_b] and the item's shared-memory rows may be reused
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&efree[pend_b]);
             pend = false;
         };
         int u = 0;
         for (int n = 0;; ++n) {
-            const int b = n & 1, m = n & 3;
+            const int m = n & 3;
             wait(&qready[m], (n >> 2) & 1);
             const int *desc = desc_s + m * 8;
             if (timed_out || desc[5]) break;
             const int kbeg = desc[1], kend = desc[2], T = desc[3];
             const int my_pos = rowpos_s[m * kTile + r];
-            const uint32_t tO = tmem + 256 + b * 128;
+            const uint32_t tO = tmem + 256;
             float m_used = kPfNegInf, l_part = 0.0f;
             for (int t = 0; t < T; ++t, ++u) {
                 const int st = u & 1;
-                // V(u) to fp16, while S(u) is computed; P(u)'s arrival below
-                // also tells the MMA lane that this warp's slice is converted
-                wait(&vfull[st], (u >> 1) & 1);
-                v_to_f16(sm + PfSmem::kV + st * 32768, warp, lane);
+                // V(u) to fp16 (this warp's slice), while S(u) is computed;
+                // P(u)'s arrival below also tells the MMA lane that the slice
+                // is converted
+                wait(&vfull[u % kPfVStages], (u / kPfVStages) & 1);
+                v_to_f16(sm + PfSmem::kV + (u % kPfVStages) * 32768, warp, lane);
                 fence_proxy_async_smem();
                 wait(&sfull[st], (u >> 1) & 1);
                 tc_fence_after();
