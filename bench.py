@@ -907,8 +907,9 @@ def run_case(args, device):
       select      Quest workload: bsa_select three times, L2 flushed before each
       select_lb   large-batch workload cut to --case-batch sequences: bsa_select
                   three times
-      prefill     semantic workload at a 65,536-token context: the last chunk of
-                  1,024 queries three times"""
+      prefill     semantic workload at a 65,536-token context (--case-context),
+                  256 blocks (--case-blocks): the last chunk of 1,024 queries
+                  (--case-chunk) three times"""
     from block_sparse_long_build_b200 import build as Bld
     from block_sparse_long_build_b200 import workloads as W
     from block_sparse_long_build_b200.session import DecodeSession
@@ -939,8 +940,8 @@ def run_case(args, device):
             e1.record()
             ev.append((e0, e1))
     elif args.case == "prefill":
-        L, Tq = 65536, 1024
-        cfg = W.semantic(0).scaled(L=L, budget_tokens=L // 16, chunk=Tq)
+        L, Tq = args.case_context, args.case_chunk
+        cfg = W.semantic(0).scaled(L=L, budget_tokens=L // 16, chunk=Tq, n_blocks=args.case_blocks)
         wl = W.Workload(cfg, device)
         sess = DecodeSession(wl)
         sess.build_summaries()
@@ -1000,6 +1001,9 @@ def main():
                     default=None, help="run one small profiling case instead of the bench (for ncu)")
     ap.add_argument("--case-batch", type=int, default=8,
                     help="sequences of the large-batch profiling cases")
+    ap.add_argument("--case-context", type=int, default=65536, help="prefill case: context length")
+    ap.add_argument("--case-chunk", type=int, default=1024, help="prefill case: queries per chunk")
+    ap.add_argument("--case-blocks", type=int, default=256, help="prefill case: semantic blocks")
     ap.add_argument("--case-fp8", action="store_true",
                     help="the decode and select profiling cases on an FP8 cache")
     args = ap.parse_args()
