@@ -91,3 +91,26 @@ def test_prefill_ragged_chunk():
     cfg, wl, sess = _setup(L=12288 + 5, n_blocks=24, Tq=700, dense_below=2048, Hkv=1, Hq=8)
     p = 9000
     _check_chunk(cfg, wl, sess, p, 700, [0, 5, 99, 350, 511, 699])
+
+
+def test_prefill_single_query_chunk():
+    """A chunk of one query at a sparse position: each KV head's local item
+    holds G rows, the rest of the item and every grouped item's other rows
+    are empty."""
+    cfg, wl, sess = _setup(L=16384, n_blocks=32, Tq=1, dense_below=4096)
+    _check_chunk(cfg, wl, sess, 12345, 1, [0])
+
+
+def test_prefill_budget_admits_no_block():
+    """Two blocks of ~8k positions and the first sparse chunk at 2,048: the
+    budget (128 tokens) is smaller than any block's visible prefix, so every
+    query attends only its own chunk and no grouped item exists."""
+    cfg, wl, sess = _setup(L=16384, n_blocks=2, Tq=512, dense_below=2048)
+    _check_chunk(cfg, wl, sess, 2048, 512, [0, 1, 127, 128, 255, 511])
+
+
+def test_prefill_first_sparse_chunk():
+    """The chunk that starts exactly at the dense limit: the first one whose
+    queries select blocks."""
+    cfg, wl, sess = _setup(L=16384, n_blocks=32, Tq=1024, dense_below=4096)
+    _check_chunk(cfg, wl, sess, 4096, 1024, [0, 1, 63, 64, 511, 1023])
