@@ -51,7 +51,7 @@
  *    word that kernels set and never clear: bit 0 a decode wait for a tile
  *    copy gave up, bit 1 a selection wait gave up, bit 3 a prefill wait gave
  *    up (each BSA_ERR_TIMEOUT; the call finished with partial data), bit 2 a
- *    prefill query had more blocks within its budget than the 64 this build
+ *    prefill query had more blocks within its budget than the 64 the library
  *    keeps (BSA_ERR_CAPACITY; that query's block list was cut at 64).  Read
  *    and clear it with bsa_workspace_status().
  */
@@ -76,11 +76,11 @@ typedef struct CUstream_st *bsa_stream_t;   /* == cudaStream_t */
 typedef enum {
     BSA_OK = 0,
     BSA_ERR_ARG = -1,          /* invalid argument; nothing launched            */
-    BSA_ERR_UNSUPPORTED = -2,  /* valid, but a shape this build does not cover  */
+    BSA_ERR_UNSUPPORTED = -2,  /* valid, but a shape the library does not cover */
     BSA_ERR_CUDA = -3,         /* a CUDA call or launch failed                  */
     BSA_ERR_WORKSPACE = -4,    /* workspace missing, misaligned or too small    */
     BSA_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up            */
-    BSA_ERR_CAPACITY = -6      /* a per-query limit of this build was reached
+    BSA_ERR_CAPACITY = -6      /* a per-query limit of the library was reached
                                   and the result was truncated                 */
 } bsa_status;
 
