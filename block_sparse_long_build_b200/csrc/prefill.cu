@@ -278,12 +278,12 @@ __global__ void __launch_bounds__(1024) prefill_tiles_kernel(PfArgs a) {
 // stages so that its loads start a tile earlier, and the item descriptions
 // run up to four deep.  An item's epilogue reads O out right after the
 // softmax of the next item's first tile, before that tile's P.V overwrites
-// it.  O is
-// rescaled only when a row's running maximum grows by more than 2^8 (the
-// exponentials then stay below 256).
+// it.  O is rescaled only when a row's running maximum grows by more than 2^8
+// (the exponentials then stay below 256).
 //
 // Barriers and their phases (every waiter derives the parity from an index):
-//   qready[m] item n (m = n & 3) described, Q gathered (32) parity (n >> 2) & 1
+//   qready[m] item n (m = n & 3) described, Q gathered (32 lanes of its producer)
+//                                                         parity (n >> 2) & 1
 //   qfree[b]  item n's Q copied to TMEM (b = n & 1)         parity (n >> 1) & 1
 //   qtfree[b] item n's last S complete: TMEM Q[b] free      parity (n >> 1) & 1
 //   efree[b]  item n's O read out (16 warps)                parity (n >> 1) & 1
