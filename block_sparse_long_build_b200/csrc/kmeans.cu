@@ -11,6 +11,9 @@
 //          position order) / n_j; an empty cluster keeps its centre.
 //   `iters` rounds of assignment, iters - 1 updates between them.
 //
+// The unit keys u_r are computed once per build (km_unit_kernel) into the
+// workspace; the rounds read them instead of dividing again.
+//
 // Kernels, per round (every segment at once):
 //   km_assign_tiled_kernel  (k <= 256) a CTA per 1,024 keys of a segment, 64
 //                       keys at a time: unit keys and centres transposed in
@@ -44,6 +47,7 @@ struct KmArgs {
     int32_t *offsets;      // [nseg][k + 1]
     int32_t *order;        // [nseg][L]
     float *norms;          // [nseg][L]
+    float *U;              // [nseg][L][D]: unit keys
     int32_t *chist;        // [nseg][nchunk][k]: counts, then first slots
 };
 
@@ -67,6 +71,19 @@ __global__ void __launch_bounds__(256) km_norms_kernel(KmArgs a) {
         acc = __fmaf_rn(v, v, acc);
     }
     a.norms[(int64_t)s * a.L + r] = __fsqrt_rn(acc);
+}
+
+// u_r = k_r / ||k_r|| (zero stays zero), one element per thread.
+template <typename T>
+__global__ void __launch_bounds__(256) km_unit_kernel(KmArgs a) {
+    const int s = blockIdx.y;
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= a.L * a.D) return;
+    const int64_t r = e / a.D;
+    const int i = (int)(e % a.D);
+    const float nr = a.norms[(int64_t)s * a.L + r];
+    const float v = load_elem(km_row<T>(a, s, r), i);
+    a.U[(int64_t)s * a.L * a.D + e] = nr > 0.0f ? __fdiv_rn(v, nr) : 0.0f;
 }
 
 // c_j = u_{init[j]}: CTA (j, segment), thread i.
@@ -95,13 +112,12 @@ __global__ void __launch_bounds__(kKmAssignThreads) km_assign_kernel(KmArgs a) {
     for (int t = 0; t < kKmChunk / kKmAssignThreads; ++t) {
         const int64_t r = (int64_t)c * kKmChunk + t * kKmAssignThreads + threadIdx.x;
         if (r < a.L) {
-            const T *row = km_row<T>(a, s, r);
-            const float nr = a.norms[(int64_t)s * a.L + r];
+            const float *ur = a.U + ((int64_t)s * a.L + r) * D;
             float u[D];
 #pragma unroll
-            for (int i = 0; i < D; ++i) {
-                const float v = load_elem(row, i);
-                u[i] = nr > 0.0f ? __fdiv_rn(v, nr) : 0.0f;
+            for (int i = 0; i < D; i += 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(ur + i);
+                u[i] = v.x; u[i + 1] = v.y; u[i + 2] = v.z; u[i + 3] = v.w;
             }
             float best = -__builtin_huge_valf();
             int lab = 0;
@@ -160,23 +176,20 @@ __global__ void __launch_bounds__(256) km_assign_tiled_kernel(KmArgs a) {
     }
     for (int j = tid; j < k; j += blockDim.x) hist[j] = 0;
     const int64_t key0 = (int64_t)c * kKmChunk;
-    // the tile's rows: thread = (key kk, quarter part of D); the next tile's
-    // raw rows are fetched (16-byte loads) while the current tile computes
-    constexpr int Q = D / 4, EPV = 16 / (int)sizeof(T), NV = Q / EPV;
+    // the tile's unit rows: thread = (key kk, quarter part of D); the next
+    // tile's rows are fetched (16-byte loads) while the current tile computes
+    constexpr int Q = D / 4, NV = Q / 4;
     const int kk = tid >> 2, part = tid & 3;
     uint4 raw[NV];
-    float nrr = 0.0f;
     auto fetch = [&](int t0) {
         const int64_t r = key0 + t0 + kk;
         if (r < a.L) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(km_row<T>(a, s, r) + part * Q);
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.U + ((int64_t)s * a.L + r) * D + part * Q);
 #pragma unroll
             for (int v = 0; v < NV; ++v) raw[v] = __ldg(src + v);
-            nrr = a.norms[(int64_t)s * a.L + r];
         } else {
 #pragma unroll
             for (int v = 0; v < NV; ++v) raw[v] = make_uint4(0u, 0u, 0u, 0u);
-            nrr = 0.0f;
         }
     };
     fetch(0);
@@ -187,15 +200,7 @@ __global__ void __launch_bounds__(256) km_assign_tiled_kernel(KmArgs a) {
             for (int v = 0; v < NV; ++v) {
                 const uint32_t w[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
 #pragma unroll
-                for (int e = 0; e < EPV; ++e) {
-                    float x;
-                    if constexpr (sizeof(T) == 2)
-                        x = __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
-                    else
-                        x = __uint_as_float(w[e]);
-                    const int d = part * Q + v * EPV + e;
-                    uT[d * kKmTile + kk] = nrr > 0.0f ? __fdiv_rn(x, nrr) : 0.0f;
-                }
+                for (int e = 0; e < 4; ++e) uT[(part * Q + v * 4 + e) * kKmTile + kk] = __uint_as_float(w[e]);
             }
         }
         __syncthreads();
@@ -335,29 +340,22 @@ __global__ void __launch_bounds__(128) km_update_kernel(KmArgs a) {
     const int beg = off[j], end = off[j + 1];
     if (end <= beg) return;
     const int32_t *ord = a.order + (int64_t)s * a.L;
-    const float *nrm = a.norms + (int64_t)s * a.L;
+    const float *Us = a.U + (int64_t)s * a.L * D;
     float acc = 0.0f;
     if (i < D) {
         int p = beg;
         constexpr int kB = 16;   // rows in flight; the adds stay in order
         for (; p + kB <= end; p += kB) {
             int r[kB];
-            float v[kB], n[kB];
+            float v[kB];
 #pragma unroll
             for (int q = 0; q < kB; ++q) r[q] = ord[p + q];
 #pragma unroll
-            for (int q = 0; q < kB; ++q) {
-                v[q] = load_elem(km_row<T>(a, s, r[q]), i);
-                n[q] = nrm[r[q]];
-            }
+            for (int q = 0; q < kB; ++q) v[q] = Us[(int64_t)r[q] * D + i];
 #pragma unroll
-            for (int q = 0; q < kB; ++q) acc = __fadd_rn(acc, n[q] > 0.0f ? __fdiv_rn(v[q], n[q]) : 0.0f);
+            for (int q = 0; q < kB; ++q) acc = __fadd_rn(acc, v[q]);
         }
-        for (; p < end; ++p) {
-            const int r0 = ord[p];
-            const float v0 = load_elem(km_row<T>(a, s, r0), i), n0 = nrm[r0];
-            acc = __fadd_rn(acc, n0 > 0.0f ? __fdiv_rn(v0, n0) : 0.0f);
-        }
+        for (; p < end; ++p) acc = __fadd_rn(acc, Us[(int64_t)ord[p] * D + i]);
         m[i] = __fdiv_rn(acc, (float)(end - beg));
     }
     __syncthreads();
@@ -376,7 +374,8 @@ __global__ void __launch_bounds__(128) km_update_kernel(KmArgs a) {
 size_t kmeans_ws_bytes(const bsa_kv_desc *d, int64_t L, int k) {
     const size_t nseg = (size_t)d->B * d->Hkv;
     const size_t nchunk = (size_t)div_up(L, kKmChunk);
-    return align_up(nseg * (size_t)L * 4, 256) + align_up(nseg * nchunk * (size_t)k * 4, 256);
+    return align_up(nseg * (size_t)L * 4, 256) + align_up(nseg * nchunk * (size_t)k * 4, 256) +
+           align_up(nseg * (size_t)L * d->D * 4, 256);
 }
 
 bool kmeans_supported(const bsa_kv_desc *d, int k) {
@@ -395,6 +394,8 @@ bsa_status launch_kmeans(const bsa_kv_desc *d, const void *K, int64_t L, int k, 
     const size_t nseg = (size_t)d->B * d->Hkv;
     a.norms = static_cast<float *>(ws);
     a.chist = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + align_up(nseg * (size_t)L * 4, 256));
+    a.U = reinterpret_cast<float *>(static_cast<char *>(ws) + align_up(nseg * (size_t)L * 4, 256) +
+                                    align_up(nseg * (size_t)a.nchunk * k * 4, 256));
     const dim3 gkeys((unsigned)div_up(L, 256), (unsigned)nseg);
     const dim3 gchunks((unsigned)a.nchunk, (unsigned)nseg), gclusters((unsigned)k, (unsigned)nseg);
     const size_t smem_assign = (size_t)((k + 3) & ~3) * d->D * 4 + (size_t)k * 4;
@@ -409,6 +410,8 @@ bsa_status launch_kmeans(const bsa_kv_desc *d, const void *K, int64_t L, int k, 
         BSA_CUDA_TRY(cudaFuncSetAttribute(km_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)smem_scatter));
         km_norms_kernel<T><<<gkeys, 256, 0, st>>>(a);
+        BSA_LAUNCH_CHECK();
+        km_unit_kernel<T><<<dim3((unsigned)div_up(L * DD, 256), (unsigned)nseg), 256, 0, st>>>(a);
         BSA_LAUNCH_CHECK();
         km_init_kernel<T><<<gclusters, DD, 0, st>>>(a);
         BSA_LAUNCH_CHECK();

@@ -352,8 +352,9 @@ BSA_API bsa_status bsa_prefill_grouped(const bsa_kv_desc *desc, const void *K, c
  * positions ascending), which is the kv_pos a grouped prefill takes and the
  * row list bsa_gather_rows takes.  init [B*Hkv][k]: starting rows (entries
  * outside [0, L) are clamped).  1 <= k <= min(L, 1024) and k * D <= 49,152;
- * the workspace (bsa_index_workspace_size bytes, 16-byte aligned) needs no
- * zeroing.  BSA_ERR_ARG / BSA_ERR_UNSUPPORTED / BSA_ERR_WORKSPACE before any
+ * the workspace (bsa_index_workspace_size bytes, 16-byte aligned; it holds
+ * every key's unit vector in fp32, L * D * 4 bytes per segment, computed once
+ * per call) needs no zeroing.  BSA_ERR_ARG / BSA_ERR_UNSUPPORTED / BSA_ERR_WORKSPACE before any
  * launch. */
 BSA_API size_t bsa_index_workspace_size(const bsa_kv_desc *desc, int64_t L, int32_t n_clusters);
 BSA_API bsa_status bsa_build_semantic_index(const bsa_kv_desc *desc, const void *K, int64_t L,
