@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(128) km_update_kernel(KmArgs a) {
     float acc = 0.0f;
     if (i < D) {
         int p = beg;
-        constexpr int kB = 16;   // rows in flight; the adds stay in order
+        constexpr int kB = 64;   // rows in flight; the adds stay in order
         for (; p + kB <= end; p += kB) {
             int r[kB];
             float v[kB];
