@@ -308,20 +308,32 @@ __global__ void __launch_bounds__(kSelThreads * score_tpb(GT), 3)
 constexpr int kPairRows = BSA_SCORE_PAIR_ROWS;   // rows per tile = threads per CTA
 static_assert(kPairRows == 64 || kPairRows == 128, "tile of 64 or 128 rows");
 
+// dynamic shared memory of score_pair_kernel: nst tile stages and query
+// buffers, the bound selectors and nst barriers (no alignment slack)
+inline size_t pair_smem_bytes(int nst, uint32_t tile_bytes, size_t qbytes) {
+    return (size_t)nst * (tile_bytes + qbytes) + qbytes + (size_t)nst * 8;
+}
+
 template <int SK, int G, int D>
 __global__ void __launch_bounds__(kPairRows, 384 / kPairRows)
     score_pair_kernel(const __grid_constant__ CUtensorMap tmS, SelArgs a) {
     constexpr int HPT = G / 2;
     static_assert(G % 2 == 0 && G <= kSelMaxG, "pairs of head slices");
-    extern __shared__ unsigned char dsm_raw[];
-    unsigned char *ring = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    // No static shared memory and no alignment slack: the dynamic block
+    // starts 1024-byte aligned, so the ring sits at its start and the query
+    // rows, selectors and barriers after it (sizes in pair_smem_bytes).
+    extern __shared__ __align__(1024) unsigned char dsm_raw[];
+    unsigned char *ring = dsm_raw;
     const int nb = a.nb_total;
     constexpr int QS = D + 4;                                                       // floats per head row
     float *qbuf = reinterpret_cast<float *>(ring + (size_t)a.nst * a.tile_bytes);   // [nst][G][D+4]
     uint32_t *selb = reinterpret_cast<uint32_t *>(qbuf + (size_t)a.nst * G * QS);   // [G][D+4]
-    __shared__ uint64_t full[kSelMaxStages];
+    uint64_t *full = reinterpret_cast<uint64_t *>(selb + G * QS);                  // [nst]
     const int tid = threadIdx.x;
+    if (smem_u32(dsm_raw) & 1023u) {   // the swizzled TMA boxes need it: report, touch nothing
+        if (tid == 0) atomicOr(a.status, 2u);
+        return;
+    }
     const int pr = tid >> 1, part = tid & 1;   // row pair (rows pr, pr + 64), head half
     const int my_items =
         a.n_items > (int)blockIdx.x ? (a.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
@@ -940,7 +952,8 @@ bsa_status launch_select(const bsa_kv_desc *d, const float *q, const void *summ,
     a.nst = (int)std::min<size_t>(pair ? BSA_SCORE_PAIR_STAGES : kScoreStages,
                                   (cap - qbytes) / (a.tile_bytes + qbytes));
     if (a.nst < 1) return BSA_ERR_UNSUPPORTED;
-    const size_t smem1 = 1024 + (size_t)a.nst * (a.tile_bytes + qbytes) + qbytes;   // + selectors
+    const size_t smem1 = pair ? pair_smem_bytes(a.nst, a.tile_bytes, qbytes)
+                              : 1024 + (size_t)a.nst * (a.tile_bytes + qbytes) + qbytes;   // + selectors
     const size_t smem2 = PickSmem::bytes(nb_total, max_sel);
     if (smem2 > cap) return BSA_ERR_UNSUPPORTED;
     a.tiles_per_seg = (int)div_up(nb_total, tile_rows);

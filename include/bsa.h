@@ -49,8 +49,10 @@
  *    may overlap on the GPU need separate workspaces.
  *  - Device-side errors: the first 4 bytes of a workspace are a sticky status
  *    word that kernels set and never clear: bit 0 a decode wait for a tile
- *    copy gave up, bit 1 a selection wait gave up, bit 3 a prefill wait gave
- *    up (each BSA_ERR_TIMEOUT; the call finished with partial data), bit 2 a
+ *    copy gave up, bit 1 a selection wait gave up (or a scoring CTA found
+ *    its shared memory misaligned for the swizzled copies and scored
+ *    nothing), bit 3 a prefill wait gave up (each BSA_ERR_TIMEOUT; the call
+ *    finished with partial data), bit 2 a
  *    prefill query had more blocks within its budget than the 64 the library
  *    keeps (BSA_ERR_CAPACITY; that query's block list was cut at 64).  Read
  *    and clear it with bsa_workspace_status().
