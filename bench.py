@@ -960,12 +960,14 @@ def run_reference(args):
 def run_case(args, device):
     """A small, fixed invocation of one library call for a profiler to capture
     (a few launches on a workload of a few GB at most); prints one line.
-      decode      Quest workload: two steps (the second a fused append + decode),
+      decode      Quest workload (another with --case-config): two steps (the
+                  second a fused append + decode where the workload fuses),
                   then bsa_decode five times, L2 flushed before each
       decode_lb   large-batch workload cut to --case-batch sequences (default
                   8: 1.1 GB of cache): one step, then bsa_decode five times, L2
                   flushed before each
-      select      Quest workload: bsa_select three times, L2 flushed before each
+      select      Quest workload (another with --case-config): bsa_select three
+                  times, L2 flushed before each
       select_lb   large-batch workload cut to --case-batch sequences: bsa_select
                   three times
       prefill     semantic workload at a 65,536-token context (--case-context),
@@ -978,7 +980,7 @@ def run_case(args, device):
     flush = _flusher(device)
     ev = []
     if args.case in ("decode", "select", "decode_lb", "select_lb"):
-        cfg = (W.quest(0) if args.case in ("decode", "select")
+        cfg = (W.CONFIGS[args.case_config](0) if args.case in ("decode", "select")
                else W.largebatch(0).scaled(B=args.case_batch))
         if args.case_fp8:
             cfg = cfg.scaled(kv_dtype=torch.float8_e4m3fn)
@@ -1060,6 +1062,9 @@ def main():
                     help="keys per KV head for --index (a smaller case for profiling)")
     ap.add_argument("--case", choices=["decode", "select", "decode_lb", "select_lb", "prefill"],
                     default=None, help="run one small profiling case instead of the bench (for ncu)")
+    ap.add_argument("--case-config", default="quest",
+                    help="decode / select cases: the decode configuration (quest, moba, msa, "
+                         "semantic, ...)")
     ap.add_argument("--case-batch", type=int, default=8,
                     help="sequences of the large-batch profiling cases")
     ap.add_argument("--case-context", type=int, default=65536, help="prefill case: context length")
